@@ -1,0 +1,206 @@
+/*
+ * mk.h -- C ABI of the B200 decode megakernel library (libmk.so).
+ *
+ * One call of mk_decode_step computes the next token of every sequence in a
+ * small batch from the previous token, the weights and the KV cache -- the
+ * workload of "Look Ma, No Bubbles! Designing a Low-Latency Megakernel for
+ * Llama-1B" (Hazy Research), introduction: a single sequence generated with
+ * Llama-3.2-1B, bound by how fast the weights stream from HBM.  It runs as one
+ * persistent kernel whose dependent operations start as soon as the tiles
+ * they read are ready ("MegaOps: A Kernel Overlapping Framework ...",
+ * "In plain words" and "Keep kernels separate": a consumer starts once the
+ * particular input tiles it needs are ready), or, for comparison, as the same
+ * operations launched as separate kernels inside one CUDA graph (the
+ * megakernel-versus-graph argument of "Megakernel Debate Sparks CUDA
+ * Infrastructure Community Feud", "Confirmed").
+ *
+ * Conventions
+ *  - Every call returns an mk_status.  MK_OK is 0; errors are negative.
+ *    mk_last_error() gives a one-line reason for the last failure on a ctx.
+ *  - All device memory is owned by the caller (for example allocated through
+ *    PyTorch) and passed as raw device pointers; the library allocates host
+ *    memory only and never frees caller memory.  mk_swiglu_stage1 is
+ *    stateless and allocates nothing.
+ *  - `stream` arguments are cudaStream_t values passed as void* (NULL = the
+ *    legacy default stream).  Calls are asynchronous on that stream unless
+ *    stated otherwise.
+ *  - All sequences of a context sit at the same position; mk_prefill_kv sets
+ *    it to T and every decode step advances it by one.
+ *  - Not thread-safe per context.  Different contexts are independent.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MK_OK = 0,
+    MK_ERR_INVALID = -1,     /* bad argument: null pointer, size or position out of range */
+    MK_ERR_CUDA = -2,        /* a CUDA runtime call failed (message in mk_last_error) */
+    MK_ERR_TIMEOUT = -3,     /* a device-side dependency wait ran past its time limit */
+    MK_ERR_UNSUPPORTED = -4, /* a shape the kernels do not handle (see mk_create) */
+    MK_ERR_STATE = -5        /* call out of order (e.g. decode before load), or the
+                                context is poisoned by an earlier device error */
+} mk_status;
+
+enum { MK_BF16 = 0 };
+/* Execution variants of one decode step. */
+enum {
+    MK_MEGAKERNEL = 0, /* one persistent launch, tile-ready counters between ops */
+    MK_GRAPH = 1,      /* the same ops as one launch per op, replayed from a CUDA graph */
+    MK_GRAPH_PDL = 2   /* as MK_GRAPH, launches chained by programmatic dependent launch so
+                          each op streams its weights while the previous op finishes */
+};
+/* Tilings of the fused SwiGLU first stage ("Deep Kernel Fusion for
+ * Transformers", Key points, "Fusion scope": row-major tiling reuses the
+ * activations, column-major tiling reuses the weights). */
+enum { MK_SWIGLU_AUTO = 0, MK_SWIGLU_ROW = 1, MK_SWIGLU_COL = 2 };
+
+/* Architecture and limits of one context. */
+typedef struct {
+    int n_layers, hidden, n_heads, n_kv_heads, head_dim, intermediate, vocab;
+    float rms_eps, rope_theta;
+    int tied_embeddings; /* 1: the LM head is the embedding table */
+    int qk_norm;         /* 1: per-head RMSNorm of q and k before RoPE (Qwen3) */
+    int batch;           /* sequences decoded together, 1..64 */
+    int max_seq;         /* KV cache positions per sequence */
+    int dtype;           /* MK_BF16 (the only one) */
+    int variant;         /* MK_MEGAKERNEL | MK_GRAPH | MK_GRAPH_PDL */
+    int num_sms;         /* CTAs of the persistent kernel; 0 = the device's SM count */
+} mk_config;
+
+/* Device pointers to the caller's bf16 weights in nn.Linear layout
+ * [out_features, in_features], row-major.  The per-layer members are HOST
+ * arrays of n_layers DEVICE pointers.  q_norm/k_norm are read only when
+ * qk_norm is set; lm_head is ignored when tied_embeddings is set. */
+typedef struct {
+    const void *embed;      /* [vocab, hidden]; must stay alive while the ctx decodes */
+    const void *final_norm; /* [hidden] */
+    const void *lm_head;    /* [vocab, hidden] */
+    const void *const *attn_norm; /* [hidden] */
+    const void *const *wq;  /* [n_heads*head_dim, hidden] */
+    const void *const *wk;  /* [n_kv_heads*head_dim, hidden] */
+    const void *const *wv;  /* [n_kv_heads*head_dim, hidden] */
+    const void *const *wo;  /* [hidden, n_heads*head_dim] */
+    const void *const *q_norm; /* [head_dim] */
+    const void *const *k_norm; /* [head_dim] */
+    const void *const *mlp_norm; /* [hidden] */
+    const void *const *wg;  /* [intermediate, hidden] (gate) */
+    const void *const *wu;  /* [intermediate, hidden] (up) */
+    const void *const *wd;  /* [hidden, intermediate] (down) */
+} mk_weights;
+
+typedef struct mk_ctx mk_ctx;
+
+/* Validate `cfg`, build the per-SM instruction lists and counter targets on
+ * the host, and check that schedule for deadlock and producer/consumer count
+ * mismatches.  `device` is the CUDA device ordinal, or -1 to plan without a
+ * device (then cfg->num_sms must be > 0; only the planning calls below work).
+ * Shapes handled: head_dim 64 or 128, n_heads a multiple of n_kv_heads with at
+ * most 8 query heads per KV head, hidden/intermediate multiples of 8,
+ * hidden <= 8192.  Errors: MK_ERR_INVALID (null/negative), MK_ERR_UNSUPPORTED. */
+mk_status mk_create(const mk_config *cfg, int device, mk_ctx **out);
+mk_status mk_destroy(mk_ctx *ctx);
+const char *mk_last_error(const mk_ctx *ctx);
+
+/* Bytes of the caller-allocated device workspace (256-byte aligned base):
+ * repacked weights, activations, partial sums, counters, instruction lists. */
+mk_status mk_workspace_bytes(const mk_ctx *ctx, size_t *bytes);
+/* Bytes of the caller-allocated KV cache: bf16 K then V, each
+ * [n_layers][batch][n_kv_heads][max_seq][head_dim]. */
+mk_status mk_kv_cache_bytes(const mk_ctx *ctx, size_t *bytes);
+
+/* Repack the weights into the workspace in the tile order the kernels stream
+ * (one pass, synchronous on `stream`), upload the instruction lists, zero the
+ * counters and the KV cache, and set the position to 0.  The caller's weight
+ * buffers other than `embed` may be freed afterwards. */
+mk_status mk_load_weights(mk_ctx *ctx, const mk_weights *w, void *workspace, void *kv_cache, void *stream);
+
+/* Fill the KV cache from a prompt: `d_tokens` is a device int32 [batch, T]
+ * row-major array; positions restart at 0 and end at T.  Runs T decode steps
+ * whose outputs are discarded.  MK_ERR_INVALID if T < 1 or T > max_seq. */
+mk_status mk_prefill_kv(mk_ctx *ctx, const int32_t *d_tokens, int batch, int T, void *stream);
+
+/* One decode step at the current position p: `d_tokens` is a device int32
+ * [batch]; the K/V rows of those tokens are written at position p, every
+ * sequence attends to positions 0..p, and the argmax over the vocabulary
+ * (lowest index on ties) goes to `d_next` (device int32 [batch], may be NULL).
+ * If `d_logits` is not NULL it receives the fp32 logits [batch, vocab] the
+ * argmax was taken over.  Advances the position.  MK_ERR_INVALID if p ==
+ * max_seq.  A token outside [0, vocab) is clamped to the range on the device;
+ * a device wait timeout is reported by mk_get_status. */
+mk_status mk_decode_step(mk_ctx *ctx, const int32_t *d_tokens, int32_t *d_next, float *d_logits, void *stream);
+
+/* Synchronize `stream` and return MK_ERR_TIMEOUT if a device wait gave up
+ * during any earlier step (the context is then poisoned until mk_reset),
+ * MK_ERR_CUDA on a CUDA error, else MK_OK. */
+mk_status mk_get_status(mk_ctx *ctx, void *stream);
+/* Clear counters, error word and position (KV cache contents are kept). */
+mk_status mk_reset(mk_ctx *ctx, void *stream);
+mk_status mk_get_position(const mk_ctx *ctx, int *pos);
+/* Rewind (or advance) the position to `pos` (0 <= pos <= max_seq), for
+ * example to decode another continuation of a shared prompt.  KV slots at
+ * and after `pos` are treated as free and are overwritten by later steps;
+ * slots before it must have been written.  One tiny kernel on `stream`. */
+mk_status mk_set_position(mk_ctx *ctx, int pos, void *stream);
+
+/* Select the execution variant for later decode steps (MK_MEGAKERNEL,
+ * MK_GRAPH or MK_GRAPH_PDL). */
+mk_status mk_set_variant(mk_ctx *ctx, int variant);
+
+/* One-time profiling pass ("Deep Kernel Fusion for Transformers", Summary and
+ * Key points: a profiler-based scheduler benchmarks the tiling variants on
+ * the target GPU before inference and keeps the fastest, with no dispatch
+ * cost at run time).  Times the row-tiled and column-tiled forms of the fused
+ * gate/up stage inside the step and keeps the faster; the KV cache and the
+ * position are restored afterwards.  Synchronous.  *chosen (may be NULL)
+ * receives MK_SWIGLU_ROW or MK_SWIGLU_COL. */
+mk_status mk_tune(mk_ctx *ctx, void *stream, int *chosen);
+
+/* Device wait limit in nanoseconds (default 1e9).  A wait that runs out sets
+ * the context's error word and makes every CTA return early. */
+mk_status mk_set_timeout_ns(mk_ctx *ctx, unsigned long long ns);
+
+/* Test hook: when set, the instruction at index `instr` of the flattened
+ * schedule does its work but does not signal its counter, so its consumers'
+ * waits run out; -1 clears it.  Used to test timeout reporting. */
+mk_status mk_debug_drop_signal(mk_ctx *ctx, int instr);
+
+/* Introspection of the host-built schedule (CPU-testable with device -1).
+ * info[] receives, in order: n_instructions, n_ctas, n_counters, n_phases,
+ * batch_rows_per_instruction, attention_chunks, ring_stages,
+ * act_bytes, swiglu_variant, down_k_splits.  `n` is the capacity of info[]. */
+mk_status mk_schedule_info(const mk_ctx *ctx, long long *info, int n);
+/* Re-run the host-side schedule check: simulates every CTA executing its list
+ * in order against the counters and fails (MK_ERR_STATE, reason in
+ * mk_last_error) on a deadlock, a counter whose producers do not match its
+ * consumers' expected count, or an index outside its buffer. */
+mk_status mk_validate_schedule(const mk_ctx *ctx);
+
+/* Fused SwiGLU first stage on its own ("Deep Kernel Fusion for
+ * Transformers", Summary and Key points, "Fusion scope"):
+ *   out[b][n] = SiLU(sum_k x[b][k] w_gate[k][n]) * sum_k x[b][k] w_up[k][n]
+ * x: device fp16 [B, K] row-major; w_gate, w_up: device fp16 [K, N] row-major
+ * (N contiguous); out: device fp16 [B, N].  fp32 accumulation, SiLU in fp32,
+ * one rounding to fp16 at the end.  variant: MK_SWIGLU_ROW, MK_SWIGLU_COL or
+ * MK_SWIGLU_AUTO (the variant mk_swiglu_tune picked for this (B, K, N), else
+ * COL for B <= 8 and ROW above).  Needs K % 64 == 0, N % 64 == 0, 1 <= B <= 64,
+ * all pointers 16-byte aligned; MK_ERR_INVALID otherwise.  Allocates nothing. */
+mk_status mk_swiglu_stage1(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K, int N,
+                           int variant, void *stream);
+/* Time both variants on the given buffers (synchronous; `out` is
+ * overwritten), remember the faster for (B, K, N) in a process-wide table and
+ * return it in *chosen.  Per-variant mean microseconds go to us_row/us_col
+ * (may be NULL). */
+mk_status mk_swiglu_tune(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K, int N,
+                         void *stream, int *chosen, float *us_row, float *us_col);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H */

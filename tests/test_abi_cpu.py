@@ -1,0 +1,109 @@
+"""Host-side checks of the C-ABI library (no GPU): it builds, loads, exports
+every symbol include/mk.h declares, and its native scheduler produces valid,
+deadlock-free plans for every workload shape."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+import synth
+import tile_synchronised_b200 as mkpy
+from tile_synchronised_b200 import _lib
+from tile_synchronised_b200 import build as mkbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mk.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mk_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_builds_for_sm100a():
+    path = mkbuild.build()
+    assert os.path.exists(path)
+    assert "arch=compute_100a,code=sm_100a" in " ".join(mkbuild.NVCC_FLAGS)
+
+
+def test_every_declared_symbol_is_exported():
+    syms = declared_symbols()
+    assert len(syms) >= 19
+    assert set(syms) == set(_lib.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", mkbuild.LIB], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (mk_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [s for s in syms if s not in exported]
+    assert not missing, missing
+    L = _lib.load()
+    for s in syms:
+        assert getattr(L, s) is not None
+
+
+WORKLOADS = [(synth.TINY, 1), (synth.TINY, 3), (synth.LLAMA1B, 1), (synth.LLAMA8B, 1), (synth.LLAMA8B, 8),
+             (synth.LLAMA8B, 32), (synth.QWEN3_8B, 16)]
+
+
+@pytest.mark.parametrize("shape,batch", WORKLOADS, ids=[f"{s.name}-b{b}" for s, b in WORKLOADS])
+def test_plans_validate(shape, batch):
+    p = mkpy.Plan(shape, batch, shape.max_seq, num_sms=148)
+    p.validate()
+    info = p.info()
+    assert info["n_ctas"] == 148
+    assert 2 <= info["ring_stages"] <= 8
+    # the workspace holds at least every streamed weight once (repacked, padded)
+    assert p.workspace_bytes() >= shape.replace(batch=batch).weight_bytes() * 0.99
+    s = shape
+    assert p.kv_cache_bytes() == 2 * s.n_layers * batch * s.n_kv_heads * s.max_seq * s.head_dim * 2
+
+
+@pytest.mark.parametrize("n_ctas", [1, 7, 132, 148])
+def test_plans_validate_for_any_cta_count(n_ctas):
+    p = mkpy.Plan(synth.TINY, 2, synth.TINY.max_seq, num_sms=n_ctas)
+    p.validate()
+    assert p.info()["n_ctas"] == n_ctas
+
+
+def _create(shape, batch=1, **kw):
+    lib = _lib.load()
+    cfg = mkpy.make_config(shape, batch, shape.max_seq, "megakernel", 148)
+    for k, v in kw.items():
+        setattr(cfg, k, v)
+    ctx = C.c_void_p()
+    st = lib.mk_create(C.byref(cfg), -1, C.byref(ctx))
+    if st == 0:
+        lib.mk_destroy(ctx)
+    return st
+
+
+def test_create_rejects_bad_configs():
+    assert _create(synth.TINY) == _lib.MK_OK
+    assert _create(synth.TINY, head_dim=96) == _lib.MK_ERR_UNSUPPORTED
+    assert _create(synth.TINY, n_kv_heads=3) == _lib.MK_ERR_UNSUPPORTED
+    assert _create(synth.TINY, batch=0) == _lib.MK_ERR_INVALID
+    assert _create(synth.TINY, batch=65) == _lib.MK_ERR_UNSUPPORTED
+    assert _create(synth.TINY, hidden=260) == _lib.MK_ERR_UNSUPPORTED
+    assert _create(synth.TINY, dtype=1) == _lib.MK_ERR_UNSUPPORTED
+    assert _create(synth.TINY, num_sms=0) == _lib.MK_ERR_INVALID  # no device to ask
+
+
+def test_device_calls_refuse_without_device():
+    lib = _lib.load()
+    p = mkpy.Plan(synth.TINY, 1, synth.TINY.max_seq)
+    w = _lib.MkWeights()
+    assert lib.mk_load_weights(p.ctx, C.byref(w), None, None, None) == _lib.MK_ERR_STATE
+    assert lib.mk_decode_step(p.ctx, None, None, None, None) == _lib.MK_ERR_STATE
+    assert "mk_load_weights" in lib.mk_last_error(p.ctx).decode() or lib.mk_last_error(p.ctx)
+
+
+def test_swiglu_argument_checks_need_no_device():
+    lib = _lib.load()
+    dummy = C.c_void_p(256)
+    # misaligned pointer, bad sizes, null: all refused before any launch
+    assert lib.mk_swiglu_stage1(C.c_void_p(8), dummy, dummy, dummy, 1, 8192, 7168, 0, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_swiglu_stage1(dummy, dummy, dummy, dummy, 0, 8192, 7168, 0, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_swiglu_stage1(dummy, dummy, dummy, dummy, 65, 8192, 7168, 0, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_swiglu_stage1(dummy, dummy, dummy, dummy, 1, 8200, 7168, 0, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_swiglu_stage1(None, dummy, dummy, dummy, 1, 8192, 7168, 0, None) == _lib.MK_ERR_INVALID

@@ -1,0 +1,270 @@
+"""Parity of the CUDA decode step with the CPU oracle (needs a B200).
+
+Small workloads run whole teacher-forced trajectories through both sides;
+the full-size workloads run the GPU trajectory and hand the GPU's KV cache to
+the oracle for single steps ("state handoff"), plus sampled layer-0 cache rows
+recomputed from the embedding.  The comparison rules live in gpu_common.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_common import build_pair, check_argmax, logits_close, widen_bf16
+
+pytestmark = pytest.mark.gpu
+
+needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="no CUDA device")
+
+
+def run_trajectory(model, orc, tokens, prefill, steps, check_every=1):
+    """Prefill both sides, then teacher-force `steps` tokens; compare logits/argmax."""
+    B = model.batch
+    model.prefill(tokens[:, :prefill].cuda())
+    orc.prefill(tokens[:, :prefill].numpy())
+    logits = torch.empty((B, model.shape.vocab), dtype=torch.float32, device="cuda")
+    worst, undecided = 0.0, 0
+    for s in range(steps):
+        tok = tokens[:, prefill + s].contiguous()
+        nxt = model.decode(tok.cuda(), logits=logits)
+        ref, ref_next = orc.step(tok.numpy())
+        if s % check_every == 0 or s == steps - 1:
+            g = logits.cpu().numpy()
+            d = logits_close(g, ref)
+            worst = max(worst, d)
+            undecided += check_argmax(nxt.cpu().numpy(), g, ref, d)
+    assert model.status() == 0
+    return worst, undecided
+
+
+@needs_cuda
+def test_tiny_trajectory_and_kv_indexing():
+    s = synth.TINY
+    tw, model, orc = build_pair(s)
+    k, v = model.kv_views()
+    k.view(torch.int16).fill_(-1)  # 0xFFFF: a NaN pattern in bf16
+    v.view(torch.int16).fill_(-1)
+    tokens = synth.make_tokens(s, s.prefill + s.steps)
+    worst, undecided = run_trajectory(model, orc, tokens, s.prefill, s.steps)
+    assert undecided <= 2
+    p_final = s.prefill + s.steps
+    assert model.position == p_final
+    # every written slot matches the oracle's cache; every other slot keeps the poison bits
+    for cache, ref in ((k, orc.kc), (v, orc.vc)):
+        got = widen_bf16(cache[:, :, :, :p_final])
+        want = ref[:, :, :, :p_final]
+        assert np.all(np.isfinite(got))
+        for l in range(s.n_layers):
+            assert np.max(np.abs(got[l] - want[l])) <= 2e-2 * np.max(np.abs(want[l]))
+        rest = cache[:, :, :, p_final:].contiguous().view(torch.int16)
+        assert bool((rest == -1).all())
+
+
+@needs_cuda
+@pytest.mark.parametrize("variant", ["graph", "graph_pdl"])
+def test_separate_kernel_variants_bit_equal_megakernel(variant):
+    s = synth.TINY
+    tw = synth.make_weights(s, device="cuda")
+    import tile_synchronised_b200 as mk
+    a = mk.Model(s, tw, variant="megakernel")
+    b = mk.Model(s, tw, variant=variant)
+    tokens = synth.make_tokens(s, 24)
+    a.prefill(tokens[:, :16].cuda())
+    b.prefill(tokens[:, :16].cuda())
+    la = torch.empty((1, s.vocab), device="cuda")
+    lb = torch.empty((1, s.vocab), device="cuda")
+    tok = torch.empty(1, dtype=torch.int32, device="cuda")
+    for i in range(16, 24):
+        tok.copy_(tokens[:, i])
+        na = a.decode(tok, logits=la).clone()
+        nb = b.decode(tok, logits=lb).clone()
+        assert torch.equal(la, lb), f"step {i}: max|delta| {(la - lb).abs().max().item()}"
+        assert torch.equal(na, nb)
+    assert a.status() == 0 and b.status() == 0
+    ka, va = a.kv_views()
+    kb, vb = b.kv_views()
+    assert torch.equal(ka[:, :, :, :24], kb[:, :, :, :24]) and torch.equal(va[:, :, :, :24], vb[:, :, :, :24])
+
+
+@needs_cuda
+@pytest.mark.parametrize("case", ["batch3", "qknorm_tied", "d128", "group8"])
+def test_tiny_shape_variants(case):
+    s = synth.TINY
+    batch = 1
+    if case == "batch3":
+        batch = 3
+    elif case == "qknorm_tied":
+        s = s.replace(qk_norm=True, tied=True, rms_eps=1e-6, rope_theta=1e6)
+    elif case == "d128":
+        s = s.replace(head_dim=128, n_heads=4, n_kv_heads=1)
+    elif case == "group8":
+        s = s.replace(n_heads=8, n_kv_heads=1, head_dim=64, hidden=512, intermediate=1024)
+    s = s.replace(batch=batch)
+    tw, model, orc = build_pair(s, batch=batch)
+    tokens = synth.make_tokens(s, 40, batch=batch)
+    worst, undecided = run_trajectory(model, orc, tokens, 24, 16)
+    assert undecided <= 2 * batch
+
+
+@needs_cuda
+def test_split_kv_chunk_count_does_not_change_results():
+    s = synth.TINY
+    tw = synth.make_weights(s, device="cuda")
+    import tile_synchronised_b200 as mk
+    outs = []
+    for n in (148, 17, 2):
+        m = mk.Model(s, tw, num_sms=n)
+        tokens = synth.make_tokens(s, 80)
+        m.prefill(tokens[:, :79].cuda())
+        lg = torch.empty((1, s.vocab), device="cuda")
+        m.decode(tokens[:, 79].contiguous().cuda(), logits=lg)
+        assert m.status() == 0
+        outs.append(lg.cpu().numpy())
+    for o in outs[1:]:
+        assert np.max(np.abs(o - outs[0])) <= 1e-3 * np.max(np.abs(outs[0]))
+
+
+@needs_cuda
+def test_wait_timeout_is_reported_and_context_recovers():
+    s = synth.TINY
+    tw = synth.make_weights(s, device="cuda")
+    import tile_synchronised_b200 as mk
+    from tile_synchronised_b200 import _lib
+    m = mk.Model(s, tw)
+    m.set_timeout_ns(20_000_000)  # 20 ms
+    # instruction 0 of CTA 0 is a layer-0 QKV tile: without its signal the
+    # attention instructions of layer 0 can never start
+    m.drop_signal(0)
+    tok = torch.zeros(1, dtype=torch.int32, device="cuda")
+    m.decode(tok)
+    assert m.status() == _lib.MK_ERR_TIMEOUT
+    assert "gave up" in m.last_error()
+    with pytest.raises(mk.MkError):
+        m.decode(tok)  # poisoned until reset
+    m.drop_signal(-1)
+    m.reset()
+    tokens = synth.make_tokens(s, 8)
+    m.prefill(tokens[:, :7].cuda())
+    lg = torch.empty((1, s.vocab), device="cuda")
+    m.decode(tokens[:, 7].contiguous().cuda(), logits=lg)
+    assert m.status() == 0
+    orc = oracle.OracleModel.from_torch(s, tw)
+    orc.prefill(tokens[:, :7].numpy())
+    ref, _ = orc.step(tokens[:, 7].numpy())
+    logits_close(lg.cpu().numpy(), ref)
+
+
+@needs_cuda
+def test_position_bounds():
+    s = synth.TINY.replace(max_seq=8)
+    tw = synth.make_weights(s, device="cuda")
+    import tile_synchronised_b200 as mk
+    m = mk.Model(s, tw, max_seq=8)
+    tokens = synth.make_tokens(s, 8)
+    m.prefill(tokens[:, :6].cuda())
+    assert m.position == 6
+    tok = torch.zeros(1, dtype=torch.int32, device="cuda")
+    m.decode(tok)
+    m.decode(tok)
+    assert m.position == 8
+    with pytest.raises(mk.MkError):
+        m.decode(tok)
+    with pytest.raises(mk.MkError):
+        m.prefill(torch.zeros((1, 9), dtype=torch.int32))
+    assert m.status() == 0
+
+
+# ---------------------------------------------------------------- full-size workloads (state handoff)
+def sampled_layer0_rows(shape, tw, k, v, tokens_np, b, positions):
+    L0 = tw["layers"][0]
+    wk = synth.to_u16(L0["wk"])
+    wv = synth.to_u16(L0["wv"])
+    emb = tw["embed"]
+    ones = synth.to_u16(L0["attn_norm"])
+    for p in positions:
+        x = emb[int(tokens_np[b, p])].float().cpu().numpy()
+        h = oracle.rmsnorm(x, ones, shape.rms_eps)
+        kk = oracle.gemv_bf16(wk, h).reshape(shape.n_kv_heads, shape.head_dim)
+        vv = oracle.gemv_bf16(wv, h).reshape(shape.n_kv_heads, shape.head_dim)
+        for g in range(shape.n_kv_heads):
+            kh = kk[g]
+            if shape.qk_norm:
+                kh = oracle.rmsnorm(kh, synth.to_u16(L0["k_norm"]), shape.rms_eps)
+            want_k = oracle.rope(kh, p, shape.rope_theta)
+            got_k = k[0, b, g, p].float().cpu().numpy()
+            got_v = v[0, b, g, p].float().cpu().numpy()
+            assert np.max(np.abs(got_k - want_k)) <= 2e-2 * np.max(np.abs(want_k))
+            assert np.max(np.abs(got_v - vv[g])) <= 2e-2 * np.max(np.abs(vv[g]))
+
+
+def full_size_case(shape, batch, prefill, extra_steps, seqs, max_seq=None):
+    import tile_synchronised_b200 as mk
+    ms = max_seq or shape.max_seq
+    tw = synth.make_weights(shape, device="cuda")
+    model = mk.Model(shape, tw, batch=batch, max_seq=ms)
+    tokens = synth.make_tokens(shape, prefill + extra_steps + 1, batch=batch)
+    tnp = tokens.numpy()
+    model.prefill(tokens[:, :prefill].cuda())
+    for s in range(extra_steps):
+        model.decode(tokens[:, prefill + s].contiguous().cuda())
+    pos = prefill + extra_steps
+    assert model.position == pos
+    k, v = model.kv_views()
+    sampled_layer0_rows(shape, tw, k, v, tnp, seqs[0], [0, 1, pos // 2, pos - 1])
+    lg = torch.empty((batch, shape.vocab), dtype=torch.float32, device="cuda")
+    nxt = model.decode(tokens[:, pos].contiguous().cuda(), logits=lg).cpu().numpy()
+    assert model.status() == 0
+    g = lg.cpu().numpy()
+    host = {kk: (None if tw[kk] is None else synth.to_u16(tw[kk])) for kk in ("embed", "final_norm", "lm_head")}
+    host["layers"] = [{a: (None if t is None else synth.to_u16(t)) for a, t in lw.items()} for lw in tw["layers"]]
+    del tw
+    for b in seqs:
+        orc = oracle.OracleModel(shape, host, batch=1, max_seq=pos + 1)
+        orc.kc[:, 0, :, :pos] = k[:, b, :, :pos].float().cpu().numpy()
+        orc.vc[:, 0, :, :pos] = v[:, b, :, :pos].float().cpu().numpy()
+        orc.pos[0] = pos
+        ref, _ = orc.step([int(tnp[b, pos])])
+        d = logits_close(g[b:b + 1], ref)
+        check_argmax(nxt[b:b + 1], g[b:b + 1], ref, d)
+        # the cache row this step appended agrees with the oracle's
+        for l in (0, shape.n_layers - 1):
+            gk = k[l, b, :, pos].float().cpu().numpy()
+            assert np.max(np.abs(gk - orc.kc[l, 0, :, pos])) <= 2e-2 * np.max(np.abs(orc.kc[l, 0, :, pos]))
+
+
+@needs_cuda
+def test_llama1b_full_size_handoff():
+    s = synth.LLAMA1B
+    full_size_case(s, 1, s.prefill, 8, [0])
+
+
+@needs_cuda
+@pytest.mark.parametrize("batch,seqs", [(1, [0]), (8, [0, 7])])
+def test_llama8b_full_size_handoff(batch, seqs):
+    s = synth.LLAMA8B
+    full_size_case(s, batch, s.prefill, 4, seqs)
+
+
+@needs_cuda
+def test_qwen3_8b_handoff_at_1k():
+    s = synth.QWEN3_8B
+    full_size_case(s, 16, 1024, 2, [0, 15], max_seq=1040)
+
+
+# ---------------------------------------------------------------- the fused SwiGLU first stage
+@needs_cuda
+@pytest.mark.parametrize("B", synth.SWIGLU_BATCHES)
+def test_swiglu_stage1_full_size(B):
+    import tile_synchronised_b200 as mk
+    x, wg, wu = synth.make_swiglu_inputs(B, device="cuda")
+    ref = oracle.swiglu_stage1_f16(synth.to_u16(x), synth.to_u16(wg), synth.to_u16(wu))
+    amax = float(np.max(np.abs(ref)))
+    for variant in (mk.MK_SWIGLU_ROW, mk.MK_SWIGLU_COL, mk.MK_SWIGLU_AUTO):
+        out = mk.swiglu_stage1(x, wg, wu, variant=variant)
+        torch.cuda.synchronize()
+        got = out.float().cpu().numpy()
+        # fp16 output rounding (2^-11 relative) plus fp32 accumulation over K = 8192
+        assert np.all(np.abs(got - ref) <= 2e-3 * np.abs(ref) + 1e-4 * amax), variant
+    chosen, us_row, us_col = mk.swiglu_tune(x, wg, wu, out)
+    assert chosen in (mk.MK_SWIGLU_ROW, mk.MK_SWIGLU_COL) and us_row > 0 and us_col > 0

@@ -1,0 +1,186 @@
+"""B200 decode megakernel: one small-batch decode step of a dense
+Llama-architecture decoder as a persistent, tile-synchronised kernel.
+
+The work happens in libmk.so (CUDA for sm_100a, C ABI in include/mk.h).  This
+module only marshals arguments: PyTorch provides device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import torch
+
+from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW,
+                   MkConfig, MkError, MkWeights, check, load)
+
+__all__ = ["Model", "swiglu_stage1", "swiglu_tune", "MkError", "VARIANTS", "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW",
+           "MK_SWIGLU_COL", "load"]
+
+VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL}
+SCHEDULE_FIELDS = ("n_instructions", "n_ctas", "n_counters", "n_phases", "batch_rows", "attention_chunks",
+                   "ring_stages", "act_bytes", "swiglu_variant", "down_k_splits")
+
+
+def _stream(stream) -> C.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def make_config(shape, batch: int, max_seq: int, variant: str = "megakernel", num_sms: int = 0) -> MkConfig:
+    return MkConfig(shape.n_layers, shape.hidden, shape.n_heads, shape.n_kv_heads, shape.head_dim,
+                    shape.intermediate, shape.vocab, shape.rms_eps, shape.rope_theta, int(shape.tied),
+                    int(shape.qk_norm), batch, max_seq, 0, VARIANTS[variant], num_sms)
+
+
+class Plan:
+    """A host-only schedule (no device): for inspecting and validating plans on CPU."""
+
+    def __init__(self, shape, batch: int, max_seq: int, num_sms: int = 148):
+        self.lib = load()
+        self.ctx = C.c_void_p()
+        cfg = make_config(shape, batch, max_seq, "megakernel", num_sms)
+        check(self.lib.mk_create(C.byref(cfg), -1, C.byref(self.ctx)), None, "mk_create")
+
+    def info(self) -> dict:
+        arr = (C.c_longlong * len(SCHEDULE_FIELDS))()
+        check(self.lib.mk_schedule_info(self.ctx, arr, len(arr)), self.ctx, "mk_schedule_info")
+        return dict(zip(SCHEDULE_FIELDS, list(arr)))
+
+    def workspace_bytes(self) -> int:
+        n = C.c_size_t()
+        check(self.lib.mk_workspace_bytes(self.ctx, C.byref(n)), self.ctx, "mk_workspace_bytes")
+        return n.value
+
+    def kv_cache_bytes(self) -> int:
+        n = C.c_size_t()
+        check(self.lib.mk_kv_cache_bytes(self.ctx, C.byref(n)), self.ctx, "mk_kv_cache_bytes")
+        return n.value
+
+    def validate(self) -> None:
+        check(self.lib.mk_validate_schedule(self.ctx), self.ctx, "mk_validate_schedule")
+
+    def close(self):
+        if self.ctx:
+            self.lib.mk_destroy(self.ctx)
+            self.ctx = C.c_void_p()
+
+    __del__ = close
+
+
+class Model(Plan):
+    """A decoder bound to device weights (``synth.make_weights`` structure, bf16 on CUDA)."""
+
+    def __init__(self, shape, weights: dict, batch: int | None = None, max_seq: int | None = None,
+                 variant: str = "megakernel", device: int | None = None, num_sms: int = 0, stream=None):
+        self.lib = load()
+        self.shape = shape
+        self.batch = shape.batch if batch is None else batch
+        self.max_seq = shape.max_seq if max_seq is None else max_seq
+        dev = torch.cuda.current_device() if device is None else device
+        self.device = torch.device("cuda", dev)
+        self.ctx = C.c_void_p()
+        cfg = make_config(shape, self.batch, self.max_seq, variant, num_sms)
+        check(self.lib.mk_create(C.byref(cfg), dev, C.byref(self.ctx)), None, "mk_create")
+        self.workspace = torch.empty(self.workspace_bytes(), dtype=torch.uint8, device=self.device)
+        self.kv = torch.empty(self.kv_cache_bytes(), dtype=torch.uint8, device=self.device)
+        self._weights = weights  # the embedding table must stay alive
+        L = shape.n_layers
+
+        def ptr(t):
+            return None if t is None else t.data_ptr()
+
+        def arr(name):
+            a = (C.c_void_p * L)(*[ptr(lw[name]) for lw in weights["layers"]])
+            self._keep.append(a)
+            return C.cast(a, C.POINTER(C.c_void_p))
+
+        self._keep = []
+        w = MkWeights(ptr(weights["embed"]), ptr(weights["final_norm"]), ptr(weights.get("lm_head")),
+                      *[arr(n) for n in ("attn_norm", "wq", "wk", "wv", "wo", "q_norm", "k_norm", "mlp_norm",
+                                         "wg", "wu", "wd")])
+        check(self.lib.mk_load_weights(self.ctx, C.byref(w), C.c_void_p(self.workspace.data_ptr()),
+                                       C.c_void_p(self.kv.data_ptr()), _stream(stream)), self.ctx, "mk_load_weights")
+        self._next = torch.empty(self.batch, dtype=torch.int32, device=self.device)
+
+    # ---------------------------------------------------------------- views
+    def kv_views(self):
+        """(K, V) bf16 views of the cache, each [L, B, nkv, max_seq, d]."""
+        s = self.shape
+        shp = (s.n_layers, self.batch, s.n_kv_heads, self.max_seq, s.head_dim)
+        half = self.kv.numel() // 2
+        k = self.kv[:half].view(torch.bfloat16).view(shp)
+        v = self.kv[half:].view(torch.bfloat16).view(shp)
+        return k, v
+
+    @property
+    def position(self) -> int:
+        p = C.c_int()
+        check(self.lib.mk_get_position(self.ctx, C.byref(p)), self.ctx, "mk_get_position")
+        return p.value
+
+    def set_position(self, pos: int, stream=None) -> None:
+        check(self.lib.mk_set_position(self.ctx, int(pos), _stream(stream)), self.ctx, "mk_set_position")
+
+    # ---------------------------------------------------------------- calls
+    def prefill(self, tokens: torch.Tensor, stream=None) -> None:
+        t = tokens.to(device=self.device, dtype=torch.int32).contiguous()
+        assert t.dim() == 2 and t.shape[0] == self.batch
+        check(self.lib.mk_prefill_kv(self.ctx, C.c_void_p(t.data_ptr()), self.batch, t.shape[1], _stream(stream)),
+              self.ctx, "mk_prefill_kv")
+
+    def decode(self, tokens: torch.Tensor, logits: torch.Tensor | None = None, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+        """One step; returns the next-token tensor (int32 [B]); fills `logits` if given (fp32 [B, V])."""
+        assert tokens.dtype == torch.int32 and tokens.is_cuda and tokens.is_contiguous()
+        nxt = self._next if out is None else out
+        lp = C.c_void_p(logits.data_ptr()) if logits is not None else None
+        check(self.lib.mk_decode_step(self.ctx, C.c_void_p(tokens.data_ptr()), C.c_void_p(nxt.data_ptr()), lp,
+                                      _stream(stream)), self.ctx, "mk_decode_step")
+        return nxt
+
+    def status(self, stream=None) -> int:
+        return self.lib.mk_get_status(self.ctx, _stream(stream))
+
+    def reset(self, stream=None) -> None:
+        check(self.lib.mk_reset(self.ctx, _stream(stream)), self.ctx, "mk_reset")
+
+    def set_variant(self, name: str) -> None:
+        check(self.lib.mk_set_variant(self.ctx, VARIANTS[name]), self.ctx, "mk_set_variant")
+
+    def set_timeout_ns(self, ns: int) -> None:
+        check(self.lib.mk_set_timeout_ns(self.ctx, int(ns)), self.ctx, "mk_set_timeout_ns")
+
+    def drop_signal(self, instr: int) -> None:
+        check(self.lib.mk_debug_drop_signal(self.ctx, int(instr)), self.ctx, "mk_debug_drop_signal")
+
+    def tune(self, stream=None) -> int:
+        ch = C.c_int()
+        check(self.lib.mk_tune(self.ctx, _stream(stream), C.byref(ch)), self.ctx, "mk_tune")
+        return ch.value
+
+    def last_error(self) -> str:
+        return self.lib.mk_last_error(self.ctx).decode()
+
+
+def swiglu_stage1(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor, out: torch.Tensor | None = None,
+                  variant: int = MK_SWIGLU_AUTO, stream=None) -> torch.Tensor:
+    """out = SiLU(x @ w_gate) * (x @ w_up); fp16 x [B,K], w [K,N] -> out fp16 [B,N]."""
+    B, K = x.shape
+    N = w_gate.shape[1]
+    if out is None:
+        out = torch.empty((B, N), dtype=torch.float16, device=x.device)
+    check(load().mk_swiglu_stage1(C.c_void_p(x.data_ptr()), C.c_void_p(w_gate.data_ptr()),
+                                  C.c_void_p(w_up.data_ptr()), C.c_void_p(out.data_ptr()), B, K, N, variant,
+                                  _stream(stream)), None, "mk_swiglu_stage1")
+    return out
+
+
+def swiglu_tune(x, w_gate, w_up, out, stream=None):
+    """Time both tilings once and remember the faster; returns (chosen, us_row, us_col)."""
+    B, K = x.shape
+    N = w_gate.shape[1]
+    ch, ur, uc = C.c_int(), C.c_float(), C.c_float()
+    check(load().mk_swiglu_tune(C.c_void_p(x.data_ptr()), C.c_void_p(w_gate.data_ptr()), C.c_void_p(w_up.data_ptr()),
+                                C.c_void_p(out.data_ptr()), B, K, N, _stream(stream), C.byref(ch), C.byref(ur),
+                                C.byref(uc)), None, "mk_swiglu_tune")
+    return ch.value, ur.value, uc.value

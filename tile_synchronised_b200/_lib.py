@@ -1,0 +1,104 @@
+"""ctypes binding of libmk.so: the C ABI declared in include/mk.h, nothing else.
+
+Loading fails loudly (RuntimeError) when the shared library is missing and
+cannot be built: there is no CPU fallback anywhere on this path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+from . import build as _build
+
+MK_OK, MK_ERR_INVALID, MK_ERR_CUDA, MK_ERR_TIMEOUT, MK_ERR_UNSUPPORTED, MK_ERR_STATE = 0, -1, -2, -3, -4, -5
+MK_BF16 = 0
+MK_MEGAKERNEL, MK_GRAPH, MK_GRAPH_PDL = 0, 1, 2
+MK_SWIGLU_AUTO, MK_SWIGLU_ROW, MK_SWIGLU_COL = 0, 1, 2
+
+STATUS_NAMES = {0: "MK_OK", -1: "MK_ERR_INVALID", -2: "MK_ERR_CUDA", -3: "MK_ERR_TIMEOUT",
+                -4: "MK_ERR_UNSUPPORTED", -5: "MK_ERR_STATE"}
+
+# Every symbol include/mk.h declares.
+EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk_kv_cache_bytes",
+           "mk_load_weights", "mk_prefill_kv", "mk_decode_step", "mk_get_status", "mk_reset",
+           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_timeout_ns", "mk_debug_drop_signal",
+           "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1", "mk_swiglu_tune")
+
+
+class MkConfig(C.Structure):
+    _fields_ = [(n, C.c_int) for n in ("n_layers", "hidden", "n_heads", "n_kv_heads", "head_dim",
+                                       "intermediate", "vocab")] + \
+               [("rms_eps", C.c_float), ("rope_theta", C.c_float)] + \
+               [(n, C.c_int) for n in ("tied_embeddings", "qk_norm", "batch", "max_seq", "dtype", "variant",
+                                       "num_sms")]
+
+
+_PP = C.POINTER(C.c_void_p)
+
+
+class MkWeights(C.Structure):
+    _fields_ = [("embed", C.c_void_p), ("final_norm", C.c_void_p), ("lm_head", C.c_void_p)] + \
+               [(n, _PP) for n in ("attn_norm", "wq", "wk", "wv", "wo", "q_norm", "k_norm", "mlp_norm",
+                                   "wg", "wu", "wd")]
+
+
+class MkError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load() -> C.CDLL:
+    """Load libmk.so (building it first only if it is absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.LIB
+    if not os.path.exists(path):
+        try:
+            _build.build()
+        except Exception as e:  # noqa: BLE001 - re-raised with context
+            raise RuntimeError(f"libmk.so is missing and could not be built: {e}") from e
+    L = C.CDLL(path)
+    vp, i32, sz = C.c_void_p, C.c_int, C.c_size_t
+    st = C.c_int
+    sig = {
+        "mk_create": ([C.POINTER(MkConfig), i32, C.POINTER(vp)], st),
+        "mk_destroy": ([vp], st),
+        "mk_last_error": ([vp], C.c_char_p),
+        "mk_workspace_bytes": ([vp, C.POINTER(sz)], st),
+        "mk_kv_cache_bytes": ([vp, C.POINTER(sz)], st),
+        "mk_load_weights": ([vp, C.POINTER(MkWeights), vp, vp, vp], st),
+        "mk_prefill_kv": ([vp, vp, i32, i32, vp], st),
+        "mk_decode_step": ([vp, vp, vp, vp, vp], st),
+        "mk_get_status": ([vp, vp], st),
+        "mk_reset": ([vp, vp], st),
+        "mk_get_position": ([vp, C.POINTER(i32)], st),
+        "mk_set_position": ([vp, i32, vp], st),
+        "mk_set_variant": ([vp, i32], st),
+        "mk_tune": ([vp, vp, C.POINTER(i32)], st),
+        "mk_set_timeout_ns": ([vp, C.c_ulonglong], st),
+        "mk_debug_drop_signal": ([vp, i32], st),
+        "mk_schedule_info": ([vp, C.POINTER(C.c_longlong), i32], st),
+        "mk_validate_schedule": ([vp], st),
+        "mk_swiglu_stage1": ([vp, vp, vp, vp, i32, i32, i32, i32, vp], st),
+        "mk_swiglu_tune": ([vp, vp, vp, vp, i32, i32, i32, vp, C.POINTER(i32), C.POINTER(C.c_float),
+                            C.POINTER(C.c_float)], st),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def check(status: int, ctx=None, what: str = "") -> None:
+    if status != MK_OK:
+        msg = what
+        if ctx is not None:
+            msg = f"{what}: {load().mk_last_error(ctx).decode()}"
+        raise MkError(status, msg)

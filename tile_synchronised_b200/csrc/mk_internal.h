@@ -1,0 +1,133 @@
+// mk_internal.h -- structures shared by the host scheduler and the device
+// interpreter of the decode megakernel.  Plain C++ (no CUDA types) so the
+// scheduler compiles with the host compiler as well.
+#pragma once
+#include <stdint.h>
+
+namespace mk {
+
+// ---------------------------------------------------------------- constants
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;   // 256
+constexpr int kThreads = kConsumerThreads + 32;         // + one producer warp
+constexpr int kStageBytes = 32768;                      // one ring slot
+constexpr int kMaxStages = 8;
+constexpr int kTileRows = 8;                            // weight rows per GEMV tile
+constexpr int kMaxBatchRows = 8;                        // batch rows one GEMV instruction carries
+constexpr int kMaxSmem = 232448;                        // opt-in dynamic smem per CTA on sm_100
+constexpr int kSmemReserve = 8192;                      // barriers, reductions, attention scratch
+constexpr int kMaxAttnChunks = 64;
+constexpr int kMaxGroup = 8;                            // query heads per KV head
+constexpr uint16_t kNoCounter = 0xFFFF;
+
+// ---------------------------------------------------------------- opcodes
+enum Op : uint8_t {
+    OP_QKV = 1,     // RMSNorm(x) . W_qkv^T            -> qkv (fp32)
+    OP_ATTN = 2,    // RoPE/qk-norm, split-KV partials, KV append, LSE combine by last arriver
+    OP_OPROJ = 3,   // x += attn . W_o^T
+    OP_GATEUP = 4,  // RMSNorm(x) . [W_g;W_u]^T, SiLU(g)*u -> a (bf16)
+    OP_DOWN = 5,    // x += a . W_d^T
+    OP_LMHEAD = 6,  // RMSNorm(x) . W_head^T -> logits, running argmax; last arriver picks the token
+};
+
+enum Flags : uint8_t {
+    F_EMBED_X = 1,    // layer 0: the residual stream is the embedding row
+    F_LAST_LM = 2,    // last LM-head instruction of this CTA: publish the CTA's best
+    F_ATOMIC = 4,     // K-split residual update (red.add into x)
+    F_DROP_SIGNAL = 8 // test hook: skip the signal
+};
+
+// One instruction: 32 bytes, read by both the producer and the consumer warps.
+struct Instr {
+    uint8_t op;
+    uint8_t flags;
+    uint16_t layer;
+    uint32_t tile;        // GEMV: row tile; ATTN: (b * nkv + g) * chunks + c
+    uint16_t kb0, kb1;    // K block range [kb0, kb1)
+    uint16_t b0, nb;      // batch rows [b0, b0 + nb)
+    uint16_t wait_ctr;    // counter to wait on (kNoCounter: none)
+    uint16_t signal_ctr;  // counter to increment when done (ATTN: arrival counter)
+    uint32_t wait_count;  // increments the waited counter receives per step
+    uint16_t signal2_ctr; // ATTN/LM: counter the last arriver signals
+    uint16_t pad0;
+    uint32_t arrive_count;// ATTN/LM: arrivals per step on signal_ctr
+};
+static_assert(sizeof(Instr) == 32, "Instr must be 32 bytes");
+
+// A weight matrix repacked into tiles of kTileRows rows x kc columns; the
+// (tile, kblock) blocks are contiguous, kblock fastest, each block row-major.
+struct PackedMat {
+    uint64_t offset;   // byte offset in the workspace
+    int32_t n_rows;    // logical rows (N)
+    int32_t k;         // logical columns (K)
+    int32_t kc;        // block width (columns)
+    int32_t nkb;       // blocks along K
+    int32_t tiles;     // row tiles
+    int32_t pad;
+};
+
+// Per-layer device pointers (in the workspace; filled by the host after packing).
+struct LayerW {
+    const void *qkv;       // packed [(nq+2nkv)d, H]
+    const void *o;         // packed [H, nq d]
+    const void *gu;        // packed, tile t = gate rows 4t..4t+3 then up rows 4t..4t+3
+    const void *down;      // packed [H, I]
+    const void *attn_norm; // bf16 [H]
+    const void *mlp_norm;  // bf16 [H]
+    const void *q_norm;    // bf16 [d] or null
+    const void *k_norm;    // bf16 [d] or null
+};
+
+// Device-resident step state.
+struct State {
+    uint32_t gen;      // steps completed since the last reset
+    int32_t pos;       // position of the token decoded by the next step
+    uint32_t err;      // 0 or an error code (1 = wait timeout)
+    uint32_t err_cta;
+    uint32_t err_instr;
+    uint32_t err_ctr;
+    uint32_t pad[2];
+};
+
+struct LmBest {
+    float value;
+    int32_t index;
+    uint32_t gen;
+    uint32_t pad;
+};
+
+// Kernel parameters (passed by value).
+struct KParams {
+    const Instr *instrs;
+    const int32_t *cta_begin;   // [n_ctas] first instruction of each CTA in this launch
+    const int32_t *cta_end;     // [n_ctas] one past the last
+    const LayerW *layers;
+    const void *lm_w;           // packed LM head
+    const void *final_norm;     // bf16 [H]
+    const void *embed;          // bf16 [V, H] (caller's)
+    const double *rope_inv_freq;// [d/2]
+    float *x;                   // [B, H] residual stream
+    float *qkv;                 // [B, qkv_rows]
+    uint16_t *attn;             // bf16 [B, nq d]
+    uint16_t *act_a;            // bf16 [B, I_pad]
+    float *partials;            // [B, nq, chunks, d + 2]
+    uint16_t *kcache;           // bf16 [L, B, nkv, max_seq, d]
+    uint16_t *vcache;
+    uint32_t *counters;
+    State *state;
+    LmBest *lm_best;            // [B, n_ctas]
+    const int32_t *tokens;      // token of sequence b at tokens[b * tok_stride]
+    int32_t *next;              // [B] or null
+    float *logits;              // [B, V] or null
+    int64_t tok_stride;
+    unsigned long long timeout_ns;
+    // shapes
+    int32_t n_layers, hidden, n_heads, n_kv_heads, head_dim, intermediate, vocab, batch, max_seq;
+    int32_t qkv_rows, i_pad, chunks, n_ctas, stages, act_bytes, qk_norm;
+    float rms_eps;
+    int32_t qkv_kc, qkv_nkb, o_kc, o_nkb, gu_kc, gu_nkb, down_kc, down_nkb, lm_kc, lm_nkb;
+    int32_t use_waits;          // 0 in the separate-kernels variant (kernel boundaries order the ops)
+    int32_t pdl;                // 1: wait on the previous grid before reading activations
+};
+
+}  // namespace mk

@@ -1,0 +1,18 @@
+// mk_kernel.h -- host entry points of the device code.
+#pragma once
+#include <cuda_runtime.h>
+
+#include "mk_internal.h"
+
+namespace mk {
+int smem_bytes(const KParams &P);
+// Launch the interpreter over P.cta_begin/cta_end; bs = batch rows per GEMV instruction.
+cudaError_t launch_step(const KParams &P, int bs, int n_ctas, cudaStream_t s, bool cooperative, bool pdl_attr);
+const void *step_kernel_func(int bs);
+cudaError_t launch_pack(const void *src, const void *src2, void *dst, int n_rows, int k, int kc, int nkb, int tiles,
+                        int mode, cudaStream_t s);
+cudaError_t launch_set_position(State *state, int pos, cudaStream_t s);
+// Fused SwiGLU first stage (fp16): variant MK_SWIGLU_ROW or MK_SWIGLU_COL.
+cudaError_t launch_swiglu(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N, int variant,
+                          cudaStream_t s);
+}  // namespace mk

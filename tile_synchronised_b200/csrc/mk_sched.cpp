@@ -1,0 +1,359 @@
+// mk_sched.cpp -- host-side planner of the decode megakernel.
+//
+// The step is a fixed sequence of phases per layer -- QKV, attention, O-proj,
+// gate/up, down -- and a final LM-head phase.  Each phase is cut into
+// instructions (a GEMV row tile over a K range and a batch range, or one
+// split-KV attention chunk); every instruction is handed to one CTA, and each
+// CTA runs its instructions in phase order.  Instead of a kernel boundary
+// between phases, a consumer instruction waits on one global counter until it
+// has received the number of increments its producers make per step; the
+// counters only grow (the target is (step + 1) * count), so nothing is reset
+// between steps.  This is the tile-level producer/consumer synchronisation of
+// "MegaOps: A Kernel Overlapping Framework ..." ("In plain words", "Keep
+// kernels separate"), here inside one persistent kernel.
+//
+// Deadlock freedom: instructions only wait on counters fed by earlier phases
+// and every CTA runs its list in phase order, so with all CTAs resident the
+// earliest unfinished phase always makes progress.  validate_plan() checks
+// this, and every count, by simulating the lists.
+#include "mk_sched.h"
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <queue>
+
+namespace mk {
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static int block_width(int k) {
+    int kc = 256;
+    while (kc < k && kc < 2048) kc *= 2;
+    return kc;
+}
+
+static PackedMat make_mat(int n_rows, int k, int tiles_override = -1) {
+    PackedMat m{};
+    m.n_rows = n_rows;
+    m.k = k;
+    m.kc = block_width(k);
+    m.nkb = (k + m.kc - 1) / m.kc;
+    m.tiles = tiles_override > 0 ? tiles_override : (n_rows + kTileRows - 1) / kTileRows;
+    return m;
+}
+
+static size_t mat_bytes(const PackedMat &m) { return (size_t)m.tiles * m.nkb * kTileRows * m.kc * 2; }
+
+mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p, std::string &err) {
+    p = Plan();
+    p.cfg = c;
+    auto bad = [&](mk_status s, const char *msg) {
+        err = msg;
+        return s;
+    };
+    if (c.n_layers < 1 || c.hidden < 8 || c.n_heads < 1 || c.n_kv_heads < 1 || c.intermediate < 4 ||
+        c.vocab < 1 || c.batch < 1 || c.max_seq < 1 || n_ctas < 1)
+        return bad(MK_ERR_INVALID, "mk_config: sizes must be positive");
+    if (!(c.rms_eps >= 0.0f) || !(c.rope_theta > 0.0f)) return bad(MK_ERR_INVALID, "mk_config: bad eps/theta");
+    if (c.dtype != MK_BF16) return bad(MK_ERR_UNSUPPORTED, "only MK_BF16 weights are supported");
+    if (c.head_dim != 64 && c.head_dim != 128) return bad(MK_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (c.n_heads % c.n_kv_heads) return bad(MK_ERR_UNSUPPORTED, "n_heads must be a multiple of n_kv_heads");
+    if (c.n_heads / c.n_kv_heads > kMaxGroup) return bad(MK_ERR_UNSUPPORTED, "more than 8 query heads per KV head");
+    if (c.hidden % 8 || c.intermediate % 8) return bad(MK_ERR_UNSUPPORTED, "hidden and intermediate must be multiples of 8");
+    if (c.hidden > 8192) return bad(MK_ERR_UNSUPPORTED, "hidden above 8192");
+    if (c.batch > 64) return bad(MK_ERR_UNSUPPORTED, "batch above 64");
+    if (c.max_seq > (1 << 20)) return bad(MK_ERR_UNSUPPORTED, "max_seq above 2^20");
+    if (n_ctas > 1024) return bad(MK_ERR_UNSUPPORTED, "more than 1024 CTAs");
+    if (c.variant < MK_MEGAKERNEL || c.variant > MK_GRAPH_PDL) return bad(MK_ERR_INVALID, "unknown variant");
+
+    const int L = c.n_layers, H = c.hidden, nq = c.n_heads, nkv = c.n_kv_heads, d = c.head_dim;
+    const int I = c.intermediate, V = c.vocab, B = c.batch;
+    p.n_ctas = n_ctas;
+    p.B = B;
+    p.swiglu_variant = swiglu_variant;
+    p.qkv_rows = (nq + 2 * nkv) * d;
+    p.qkv = make_mat(p.qkv_rows, H);
+    p.o = make_mat(H, nq * d);
+    p.gu = make_mat(2 * I, H, (I + 3) / 4);
+    p.down = make_mat(H, I);
+    p.lm = make_mat(V, H);
+    p.i_pad = p.down.nkb * p.down.kc;
+
+    // Batch rows per instruction and the activation region.
+    const int kActMax = 65536;
+    p.bs = std::min(B, kMaxBatchRows);
+    auto fit_bs = [&](const PackedMat &m) { return std::max(1, std::min(p.bs, kActMax / (m.nkb * m.kc * 2))); };
+    int bs_norm = std::min({fit_bs(p.qkv), fit_bs(p.gu), fit_bs(p.lm), fit_bs(p.o)});
+    p.bs = bs_norm;
+    if ((size_t)p.bs * p.qkv.nkb * p.qkv.kc * 2 > (size_t)kActMax) return bad(MK_ERR_UNSUPPORTED, "hidden too large");
+    p.gu_bs = p.bs;
+    if (swiglu_variant == MK_SWIGLU_ROW && B > 1) p.gu_bs = std::max(1, (std::min(B, p.bs) + 1) / 2);
+    int down_blocks_per_range = std::max(1, kActMax / (p.bs * p.down.kc * 2));
+    down_blocks_per_range = std::min(down_blocks_per_range, p.down.nkb);
+    p.down_ksplit = (p.down.nkb + down_blocks_per_range - 1) / down_blocks_per_range;
+    int act = 0;
+    act = std::max(act, p.bs * p.qkv.nkb * p.qkv.kc * 2);
+    act = std::max(act, p.bs * p.o.nkb * p.o.kc * 2);
+    act = std::max(act, p.bs * p.lm.nkb * p.lm.kc * 2);
+    act = std::max(act, p.gu_bs * p.gu.nkb * p.gu.kc * 2);
+    act = std::max(act, p.bs * down_blocks_per_range * p.down.kc * 2);
+    const int G = nq / nkv;
+    const int sp = kStageBytes / (4 * d);  // positions per attention ring slot (K and V halves)
+    int attn_scratch = G * d * 4 + G * sp * 4 + 2 * d * 4 + 2 * kMaxGroup * 4 * 4;
+    act = std::max(act, attn_scratch);
+    p.act_bytes = (int)align_up(act, 128);
+    p.stages = std::min(kMaxStages, (kMaxSmem - p.act_bytes - kSmemReserve) / kStageBytes);
+    if (p.stages < 2) return bad(MK_ERR_UNSUPPORTED, "not enough shared memory for the ring");
+
+    // Split-KV chunks: enough attention instructions to cover the CTAs once.
+    p.chunks = std::max(1, std::min(kMaxAttnChunks, (n_ctas + B * nkv - 1) / (B * nkv)));
+    p.chunks = std::min(p.chunks, std::max(1, c.max_seq / 16));
+
+    // Counters.
+    const int n_arr_att = L * B * nkv;
+    p.n_counters = 5 * L + n_arr_att + 1;
+    if (p.n_counters >= kNoCounter) return bad(MK_ERR_UNSUPPORTED, "too many counters");
+    auto arr_att = [&](int l, int b, int g) { return 5 * L + (l * B + b) * nkv + g; };
+    const int arr_lm = 5 * L + n_arr_att;
+    p.counter_count.assign(p.n_counters, 0);
+
+    // ---------------------------------------------------------- instructions per phase
+    std::vector<std::vector<Instr>> phases;
+    std::vector<std::vector<double>> costs;
+    auto gemv_phase = [&](uint8_t op, int l, const PackedMat &m, int bs, int ksplit, uint8_t flags, int wait,
+                          int signal) {
+        std::vector<Instr> v;
+        std::vector<double> cost;
+        int per = (m.nkb + ksplit - 1) / ksplit;
+        for (int t = 0; t < m.tiles; ++t)
+            for (int kb = 0; kb < m.nkb; kb += per)
+                for (int b0 = 0; b0 < B; b0 += bs) {
+                    Instr in{};
+                    in.op = op;
+                    in.flags = flags | (ksplit > 1 ? F_ATOMIC : 0);
+                    in.layer = (uint16_t)l;
+                    in.tile = (uint32_t)t;
+                    in.kb0 = (uint16_t)kb;
+                    in.kb1 = (uint16_t)std::min(m.nkb, kb + per);
+                    in.b0 = (uint16_t)b0;
+                    in.nb = (uint16_t)std::min(bs, B - b0);
+                    in.wait_ctr = wait < 0 ? kNoCounter : (uint16_t)wait;
+                    in.signal_ctr = signal < 0 ? kNoCounter : (uint16_t)signal;
+                    in.signal2_ctr = kNoCounter;
+                    v.push_back(in);
+                    cost.push_back((double)(in.kb1 - in.kb0) * kTileRows * m.kc * 2 + 4096.0);
+                }
+        if (signal >= 0) p.counter_count[signal] += (uint32_t)v.size();
+        phases.push_back(v);
+        costs.push_back(cost);
+    };
+    const double typical_ctx = std::max(1.0, 0.75 * c.max_seq);
+    for (int l = 0; l < L; ++l) {
+        gemv_phase(OP_QKV, l, p.qkv, p.bs, 1, l == 0 ? F_EMBED_X : 0, l == 0 ? -1 : counter_down(l - 1),
+                   counter_qkv(l));
+        {
+            std::vector<Instr> v;
+            std::vector<double> cost;
+            for (int b = 0; b < B; ++b)
+                for (int g = 0; g < nkv; ++g)
+                    for (int ch = 0; ch < p.chunks; ++ch) {
+                        Instr in{};
+                        in.op = OP_ATTN;
+                        in.layer = (uint16_t)l;
+                        in.tile = (uint32_t)((b * nkv + g) * p.chunks + ch);
+                        in.b0 = (uint16_t)b;
+                        in.nb = 1;
+                        in.wait_ctr = (uint16_t)counter_qkv(l);
+                        in.signal_ctr = (uint16_t)arr_att(l, b, g);
+                        in.arrive_count = (uint32_t)p.chunks;
+                        in.signal2_ctr = (uint16_t)counter_att(l);
+                        v.push_back(in);
+                        cost.push_back(typical_ctx / p.chunks * d * 4 + 8192.0);
+                    }
+            p.counter_count[counter_att(l)] += (uint32_t)(B * nkv);
+            phases.push_back(v);
+            costs.push_back(cost);
+        }
+        gemv_phase(OP_OPROJ, l, p.o, p.bs, 1, l == 0 ? F_EMBED_X : 0, counter_att(l), counter_o(l));
+        gemv_phase(OP_GATEUP, l, p.gu, p.gu_bs, 1, 0, counter_o(l), counter_gu(l));
+        gemv_phase(OP_DOWN, l, p.down, p.bs, p.down_ksplit, 0, counter_gu(l), counter_down(l));
+    }
+    gemv_phase(OP_LMHEAD, L - 1, p.lm, p.bs, 1, 0, counter_down(L - 1), -1);
+    p.n_phases = (int)phases.size();
+
+    // Fill wait counts now that every producer is known.
+    for (auto &ph : phases)
+        for (auto &in : ph)
+            if (in.wait_ctr != kNoCounter) in.wait_count = p.counter_count[in.wait_ctr];
+
+    // ---------------------------------------------------------- assignment to CTAs
+    // Greedy least-loaded by cumulative streamed bytes: each phase's
+    // instructions go, in order, to the CTA with the least work so far, which
+    // keeps every SM's total bytes per step within one instruction of the mean.
+    std::vector<std::vector<std::vector<Instr>>> per(n_ctas, std::vector<std::vector<Instr>>(p.n_phases));
+    using Item = std::pair<double, int>;
+    std::priority_queue<Item, std::vector<Item>, std::greater<Item>> heap;
+    for (int i = 0; i < n_ctas; ++i) heap.push({0.0, i});
+    for (int ph = 0; ph < p.n_phases; ++ph) {
+        for (size_t j = 0; j < phases[ph].size(); ++j) {
+            Item it = heap.top();
+            heap.pop();
+            per[it.second][ph].push_back(phases[ph][j]);
+            it.first += costs[ph][j];
+            heap.push(it);
+        }
+    }
+    // LM-head arrivals: one per CTA that has LM work; its last LM instruction publishes.
+    int lm_ctas = 0;
+    const int lm_phase = p.n_phases - 1;
+    for (int i = 0; i < n_ctas; ++i)
+        if (!per[i][lm_phase].empty()) {
+            ++lm_ctas;
+            per[i][lm_phase].back().flags |= F_LAST_LM;
+        }
+    for (int i = 0; i < n_ctas; ++i)
+        for (auto &in : per[i][lm_phase]) {
+            in.signal_ctr = (uint16_t)arr_lm;
+            in.arrive_count = (uint32_t)lm_ctas;
+        }
+
+    // Flatten.
+    p.cta_base.assign(n_ctas + 1, 0);
+    p.phase_begin.assign((size_t)(p.n_phases + 1) * n_ctas, 0);
+    for (int i = 0; i < n_ctas; ++i) {
+        p.cta_base[i] = (int32_t)p.instrs.size();
+        for (int ph = 0; ph < p.n_phases; ++ph) {
+            p.phase_begin[(size_t)ph * n_ctas + i] = (int32_t)p.instrs.size();
+            for (auto &in : per[i][ph]) p.instrs.push_back(in);
+        }
+        p.phase_begin[(size_t)p.n_phases * n_ctas + i] = (int32_t)p.instrs.size();
+    }
+    p.cta_base[n_ctas] = (int32_t)p.instrs.size();
+
+    // ---------------------------------------------------------- workspace layout
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = align_up(o, 256);
+        o = at + bytes;
+        return at;
+    };
+    p.off_state = take(sizeof(State));
+    p.off_counters = take((size_t)p.n_counters * 4);
+    p.off_instrs = take(p.instrs.size() * sizeof(Instr));
+    p.off_ranges = take((size_t)(p.n_phases + 2) * 2 * n_ctas * 4);
+    p.off_layers = take((size_t)L * sizeof(LayerW));
+    p.off_rope = take((size_t)(d / 2) * 8);
+    p.off_x = take((size_t)B * H * 4);
+    p.off_qkv = take((size_t)B * p.qkv_rows * 4);
+    p.off_attn = take((size_t)B * p.o.nkb * p.o.kc * 2);
+    p.off_act_a = take((size_t)B * p.i_pad * 2);
+    p.off_partials = take((size_t)B * nq * p.chunks * (d + 2) * 4);
+    p.off_lm_best = take((size_t)B * n_ctas * sizeof(LmBest));
+    p.off_next_scratch = take((size_t)B * 4);
+    p.off_norms = take((size_t)(L * (2 * H + 2 * d) + H) * 2);
+    p.layer_weight_bytes = align_up(mat_bytes(p.qkv), 256) + align_up(mat_bytes(p.o), 256) +
+                           align_up(mat_bytes(p.gu), 256) + align_up(mat_bytes(p.down), 256);
+    p.off_weights = take((size_t)L * p.layer_weight_bytes);
+    p.off_lm = take(mat_bytes(p.lm));
+    p.qkv.offset = 0;
+    p.o.offset = align_up(mat_bytes(p.qkv), 256);
+    p.gu.offset = p.o.offset + align_up(mat_bytes(p.o), 256);
+    p.down.offset = p.gu.offset + align_up(mat_bytes(p.gu), 256);
+    p.lm.offset = p.off_lm;
+    p.workspace_bytes = align_up(o, 256);
+    p.kv_bytes = (size_t)2 * L * B * nkv * (size_t)c.max_seq * d * 2;
+    return MK_OK;
+}
+
+mk_status validate_plan(const Plan &p, std::string &err) {
+    const mk_config &c = p.cfg;
+    char buf[256];
+    auto fail = [&](const char *msg) {
+        err = msg;
+        return MK_ERR_STATE;
+    };
+    // Index ranges.
+    for (size_t i = 0; i < p.instrs.size(); ++i) {
+        const Instr &in = p.instrs[i];
+        const PackedMat *m = nullptr;
+        switch (in.op) {
+            case OP_QKV: m = &p.qkv; break;
+            case OP_OPROJ: m = &p.o; break;
+            case OP_GATEUP: m = &p.gu; break;
+            case OP_DOWN: m = &p.down; break;
+            case OP_LMHEAD: m = &p.lm; break;
+            case OP_ATTN: break;
+            default:
+                snprintf(buf, sizeof buf, "instruction %zu: bad opcode %d", i, in.op);
+                return fail(buf);
+        }
+        if (in.layer >= c.n_layers) return fail("instruction layer out of range");
+        if (in.b0 + in.nb > p.B || in.nb < 1) return fail("instruction batch range out of range");
+        if (m) {
+            if (in.tile >= (uint32_t)m->tiles || in.kb0 >= in.kb1 || in.kb1 > m->nkb)
+                return fail("GEMV instruction tile/K range out of range");
+            if (in.nb > kMaxBatchRows) return fail("GEMV instruction carries too many batch rows");
+            if ((size_t)in.nb * (in.kb1 - in.kb0) * m->kc * 2 > (size_t)p.act_bytes)
+                return fail("GEMV activation range does not fit the shared-memory region");
+            if ((in.flags & F_ATOMIC) && in.op != OP_DOWN) return fail("K-split only allowed for down");
+        } else {
+            if (in.tile >= (uint32_t)(p.B * c.n_kv_heads * p.chunks)) return fail("attention unit out of range");
+        }
+        if (in.wait_ctr != kNoCounter && in.wait_ctr >= p.n_counters) return fail("wait counter out of range");
+        if (in.signal_ctr != kNoCounter && in.signal_ctr >= p.n_counters) return fail("signal counter out of range");
+        if (in.signal2_ctr != kNoCounter && in.signal2_ctr >= p.n_counters) return fail("signal2 out of range");
+    }
+    // Simulate one step: every CTA executes its list in order.
+    std::vector<uint32_t> ctr(p.n_counters, 0);
+    std::vector<int32_t> ptr(p.n_ctas);
+    for (int i = 0; i < p.n_ctas; ++i) ptr[i] = p.cta_base[i];
+    bool progress = true;
+    size_t done = 0;
+    while (progress) {
+        progress = false;
+        for (int i = 0; i < p.n_ctas; ++i) {
+            while (ptr[i] < p.cta_base[i + 1]) {
+                const Instr &in = p.instrs[ptr[i]];
+                if (in.wait_ctr != kNoCounter && ctr[in.wait_ctr] < in.wait_count) break;
+                if (in.op == OP_ATTN || in.op == OP_LMHEAD) {
+                    if (in.op == OP_ATTN || (in.flags & F_LAST_LM)) {
+                        uint32_t a = ++ctr[in.signal_ctr];
+                        if (a == in.arrive_count && in.signal2_ctr != kNoCounter) ++ctr[in.signal2_ctr];
+                        if (a > in.arrive_count) return fail("more arrivals than expected");
+                    }
+                } else if (in.signal_ctr != kNoCounter) {
+                    ++ctr[in.signal_ctr];
+                }
+                ++ptr[i];
+                ++done;
+                progress = true;
+            }
+        }
+    }
+    if (done != p.instrs.size()) {
+        for (int i = 0; i < p.n_ctas; ++i)
+            if (ptr[i] < p.cta_base[i + 1]) {
+                const Instr &in = p.instrs[ptr[i]];
+                snprintf(buf, sizeof buf, "deadlock: CTA %d stuck at instruction %d (op %d layer %d) waiting on counter %d (%u of %u)",
+                         i, ptr[i], in.op, in.layer, in.wait_ctr, ctr[in.wait_ctr], in.wait_count);
+                return fail(buf);
+            }
+    }
+    for (size_t i = 0; i < p.instrs.size(); ++i) {
+        const Instr &in = p.instrs[i];
+        if (in.wait_ctr != kNoCounter && ctr[in.wait_ctr] != in.wait_count) {
+            snprintf(buf, sizeof buf, "counter %d receives %u increments per step but instruction %zu expects %u",
+                     in.wait_ctr, ctr[in.wait_ctr], i, in.wait_count);
+            return fail(buf);
+        }
+        if ((in.op == OP_ATTN || (in.op == OP_LMHEAD && (in.flags & F_LAST_LM))) && ctr[in.signal_ctr] != in.arrive_count) {
+            snprintf(buf, sizeof buf, "arrival counter %d gets %u arrivals, expected %u", in.signal_ctr,
+                     ctr[in.signal_ctr], in.arrive_count);
+            return fail(buf);
+        }
+    }
+    return MK_OK;
+}
+
+}  // namespace mk
