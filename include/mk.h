@@ -171,6 +171,23 @@ mk_status mk_set_timeout_ns(mk_ctx *ctx, unsigned long long ns);
  * waits run out; -1 clears it.  Used to test timeout reporting. */
 mk_status mk_debug_drop_signal(mk_ctx *ctx, int instr);
 
+/* Per-instruction timing trace for the following steps: `d_trace` is a
+ * device buffer of at least 8 * n_instructions uint64 (64 bytes per
+ * instruction; see mk_schedule_info).  For instruction i of the flattened
+ * schedule, entries [8i..8i+7] receive, in %globaltimer nanoseconds: when its
+ * CTA starts it, when its dependency wait is satisfied, when it is done, when
+ * the producer issued its first copy (0 if it streams nothing), the time the
+ * consumer spent waiting for ring data, the time the producer spent waiting
+ * for a free ring slot, and when the producer issued its last copy.  Each step
+ * overwrites the buffer.  NULL turns tracing off.  MK_ERR_INVALID if the
+ * buffer is too small. */
+mk_status mk_set_trace(mk_ctx *ctx, void *d_trace, size_t bytes);
+/* Copy the flattened schedule to host memory: 32 bytes per instruction
+ * (uint8 op, uint8 flags, uint16 layer, uint32 tile, uint16 kb0, kb1, b0, nb,
+ * then counter fields), CTA-major; `cta_base` (may be NULL) receives
+ * n_ctas + 1 int32 offsets of each CTA's first instruction. */
+mk_status mk_get_schedule(const mk_ctx *ctx, void *host_instrs, size_t bytes, int32_t *cta_base);
+
 /* Introspection of the host-built schedule (CPU-testable with device -1).
  * info[] receives, in order: n_instructions, n_ctas, n_counters, n_phases,
  * batch_rows_per_instruction, attention_chunks, ring_stages,

@@ -56,6 +56,19 @@ class Plan:
         check(self.lib.mk_kv_cache_bytes(self.ctx, C.byref(n)), self.ctx, "mk_kv_cache_bytes")
         return n.value
 
+    def schedule(self):
+        """The flattened instruction list as a numpy structured array, and CTA offsets."""
+        import numpy as np
+        n = self.info()["n_instructions"]
+        dt = np.dtype([("op", "u1"), ("flags", "u1"), ("layer", "<u2"), ("tile", "<u4"), ("kb0", "<u2"),
+                       ("kb1", "<u2"), ("b0", "<u2"), ("nb", "<u2"), ("wait_ctr", "<u2"), ("signal_ctr", "<u2"),
+                       ("wait_count", "<u4"), ("signal2_ctr", "<u2"), ("pad0", "<u2"), ("arrive_count", "<u4")])
+        arr = np.zeros(n, dt)
+        base = np.zeros(self.info()["n_ctas"] + 1, np.int32)
+        check(self.lib.mk_get_schedule(self.ctx, C.c_void_p(arr.ctypes.data), arr.nbytes,
+                                       C.c_void_p(base.ctypes.data)), self.ctx, "mk_get_schedule")
+        return arr, base
+
     def validate(self) -> None:
         check(self.lib.mk_validate_schedule(self.ctx), self.ctx, "mk_validate_schedule")
 
@@ -117,6 +130,14 @@ class Model(Plan):
         p = C.c_int()
         check(self.lib.mk_get_position(self.ctx, C.byref(p)), self.ctx, "mk_get_position")
         return p.value
+
+    def set_trace(self, buf: torch.Tensor | None) -> None:
+        """Trace into `buf` (int64 CUDA tensor of >= 8 * n_instructions), or None to stop."""
+        if buf is None:
+            check(self.lib.mk_set_trace(self.ctx, None, 0), self.ctx, "mk_set_trace")
+        else:
+            check(self.lib.mk_set_trace(self.ctx, C.c_void_p(buf.data_ptr()), buf.numel() * buf.element_size()),
+                  self.ctx, "mk_set_trace")
 
     def set_position(self, pos: int, stream=None) -> None:
         check(self.lib.mk_set_position(self.ctx, int(pos), _stream(stream)), self.ctx, "mk_set_position")

@@ -26,6 +26,7 @@ struct mk_ctx {
     int variant = MK_MEGAKERNEL;
     unsigned long long timeout_ns = 1000000000ull;
     int drop_instr = -1;
+    unsigned long long *trace = nullptr;
     const void *embed = nullptr;
     // captured graph of the separate-kernels variant
     cudaGraph_t graph = nullptr;
@@ -173,6 +174,23 @@ mk_status mk_schedule_info(const mk_ctx *c, long long *info, int n) {
     return MK_OK;
 }
 
+mk_status mk_set_trace(mk_ctx *c, void *d_trace, size_t bytes) {
+    if (!c) return MK_ERR_INVALID;
+    if (d_trace && bytes < c->plan.instrs.size() * 64) return fail(c, MK_ERR_INVALID, "trace buffer too small");
+    c->trace = static_cast<unsigned long long *>(d_trace);
+    drop_graph(c);
+    return MK_OK;
+}
+
+mk_status mk_get_schedule(const mk_ctx *c, void *host_instrs, size_t bytes, int32_t *cta_base) {
+    if (!c || !host_instrs) return MK_ERR_INVALID;
+    const Plan &p = c->plan;
+    if (bytes < p.instrs.size() * sizeof(Instr)) return MK_ERR_INVALID;
+    memcpy(host_instrs, p.instrs.data(), p.instrs.size() * sizeof(Instr));
+    if (cta_base) memcpy(cta_base, p.cta_base.data(), p.cta_base.size() * sizeof(int32_t));
+    return MK_OK;
+}
+
 mk_status mk_validate_schedule(const mk_ctx *c) {
     if (!c) return MK_ERR_INVALID;
     return validate_plan(c->plan, const_cast<mk_ctx *>(c)->err);
@@ -191,8 +209,8 @@ static KParams make_params(mk_ctx *c, const int32_t *tokens, int64_t tok_stride,
     P.rope_inv_freq = reinterpret_cast<const double *>(ws + p.off_rope);
     P.x = reinterpret_cast<float *>(ws + p.off_x);
     P.qkv = reinterpret_cast<float *>(ws + p.off_qkv);
-    P.attn = reinterpret_cast<uint16_t *>(ws + p.off_attn);
-    P.act_a = reinterpret_cast<uint16_t *>(ws + p.off_act_a);
+    P.attn = reinterpret_cast<float *>(ws + p.off_attn);
+    P.act_a = reinterpret_cast<float *>(ws + p.off_act_a);
     P.partials = reinterpret_cast<float *>(ws + p.off_partials);
     P.kcache = reinterpret_cast<uint16_t *>(c->kv);
     P.vcache = reinterpret_cast<uint16_t *>(c->kv + p.kv_bytes / 2);
@@ -204,6 +222,7 @@ static KParams make_params(mk_ctx *c, const int32_t *tokens, int64_t tok_stride,
     P.logits = logits;
     P.tok_stride = tok_stride;
     P.timeout_ns = c->timeout_ns;
+    P.trace = c->trace;
     P.n_layers = g.n_layers;
     P.hidden = g.hidden;
     P.n_heads = g.n_heads;
@@ -220,6 +239,7 @@ static KParams make_params(mk_ctx *c, const int32_t *tokens, int64_t tok_stride,
     P.stages = p.stages;
     P.act_bytes = p.act_bytes;
     P.qk_norm = g.qk_norm;
+    P.bs = p.bs;
     P.rms_eps = g.rms_eps;
     P.qkv_kc = p.qkv.kc; P.qkv_nkb = p.qkv.nkb;
     P.o_kc = p.o.kc; P.o_nkb = p.o.nkb;

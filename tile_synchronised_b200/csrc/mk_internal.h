@@ -15,9 +15,22 @@ constexpr int kMaxStages = 8;
 constexpr int kTileRows = 8;                            // weight rows per GEMV tile
 constexpr int kMaxBatchRows = 8;                        // batch rows one GEMV instruction carries
 constexpr int kMaxSmem = 232448;                        // opt-in dynamic smem per CTA on sm_100
-constexpr int kSmemReserve = 8192;                      // barriers, reductions, attention scratch
+// shared memory after the ring and the activations: barriers, flags, two reduction buffers
+// Batch rows of the kernel instance that runs a plan carrying `bs` rows per
+// instruction (instances exist for 1, 2, 4 and 8).
+constexpr int kernel_bs(int bs) { return bs <= 1 ? 1 : (bs <= 2 ? 2 : (bs <= 4 ? 4 : 8)); }
+// Rotating reduction slots per CTA: a warp can run at most `stages` ring blocks
+// (so at most `stages` instructions) ahead of another, so stages + 2 slots
+// never hand a slot to a new instruction while an older one still uses it.
+constexpr int reduce_slots(int stages) { return stages + 2; }
+// Bytes after the ring and the activation region: barriers, flags and small
+// arrays (1536 B), then the per-warp partial sums [slots][8 warps][8 rows][bs].
+constexpr int misc_bytes(int bs, int stages) { return 1536 + reduce_slots(stages) * 256 * kernel_bs(bs); }
 constexpr int kMaxAttnChunks = 64;
 constexpr int kMaxGroup = 8;                            // query heads per KV head
+// Row stride (floats) of the attention score buffer: one slot of positions plus
+// this step's position, padded so every later scratch array stays 16-byte aligned.
+constexpr int score_stride(int head_dim) { return ((kStageBytes / (4 * head_dim)) + 1 + 3) & ~3; }
 constexpr uint16_t kNoCounter = 0xFFFF;
 
 // ---------------------------------------------------------------- opcodes
@@ -108,8 +121,8 @@ struct KParams {
     const double *rope_inv_freq;// [d/2]
     float *x;                   // [B, H] residual stream
     float *qkv;                 // [B, qkv_rows]
-    uint16_t *attn;             // bf16 [B, nq d]
-    uint16_t *act_a;            // bf16 [B, I_pad]
+    float *attn;                // [B, nq d padded] attention output
+    float *act_a;               // [B, I_pad] SwiGLU product
     float *partials;            // [B, nq, chunks, d + 2]
     uint16_t *kcache;           // bf16 [L, B, nkv, max_seq, d]
     uint16_t *vcache;
@@ -123,11 +136,12 @@ struct KParams {
     unsigned long long timeout_ns;
     // shapes
     int32_t n_layers, hidden, n_heads, n_kv_heads, head_dim, intermediate, vocab, batch, max_seq;
-    int32_t qkv_rows, i_pad, chunks, n_ctas, stages, act_bytes, qk_norm;
+    int32_t qkv_rows, i_pad, chunks, n_ctas, stages, act_bytes, qk_norm, bs;
     float rms_eps;
     int32_t qkv_kc, qkv_nkb, o_kc, o_nkb, gu_kc, gu_nkb, down_kc, down_nkb, lm_kc, lm_nkb;
     int32_t use_waits;          // 0 in the separate-kernels variant (kernel boundaries order the ops)
     int32_t pdl;                // 1: wait on the previous grid before reading activations
+    unsigned long long *trace;  // [n_instr][8] globaltimer stamps and waits, or null
 };
 
 }  // namespace mk

@@ -80,35 +80,43 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     p.lm = make_mat(V, H);
     p.i_pad = p.down.nkb * p.down.kc;
 
-    // Batch rows per instruction and the activation region.
+    // Split-KV chunks: enough attention instructions to cover the CTAs once.
+    // Batch rows per instruction and the activation region.  Activations are
+    // staged in shared memory as fp32 [rows][K range]; the region is capped at
+    // 64 KB so at least five 32 KB ring slots remain.  A GEMV whose rows do not
+    // fit carries fewer batch rows (its weights stream once per row group); the
+    // down projection splits K instead (atomic residual update).
     const int kActMax = 65536;
     p.bs = std::min(B, kMaxBatchRows);
-    auto fit_bs = [&](const PackedMat &m) { return std::max(1, std::min(p.bs, kActMax / (m.nkb * m.kc * 2))); };
-    int bs_norm = std::min({fit_bs(p.qkv), fit_bs(p.gu), fit_bs(p.lm), fit_bs(p.o)});
-    p.bs = bs_norm;
-    if ((size_t)p.bs * p.qkv.nkb * p.qkv.kc * 2 > (size_t)kActMax) return bad(MK_ERR_UNSUPPORTED, "hidden too large");
+    auto fit_bs = [&](const PackedMat &m) { return std::max(1, std::min(p.bs, kActMax / (m.nkb * m.kc * 4))); };
+    p.bs = std::min({fit_bs(p.qkv), fit_bs(p.gu), fit_bs(p.lm), fit_bs(p.o)});
+    if ((size_t)p.bs * p.qkv.nkb * p.qkv.kc * 4 > (size_t)kActMax) return bad(MK_ERR_UNSUPPORTED, "hidden too large");
+    if ((size_t)p.bs * p.o.nkb * p.o.kc * 4 > (size_t)kActMax) return bad(MK_ERR_UNSUPPORTED, "n_heads*head_dim too large");
     p.gu_bs = p.bs;
     if (swiglu_variant == MK_SWIGLU_ROW && B > 1) p.gu_bs = std::max(1, (std::min(B, p.bs) + 1) / 2);
-    int down_blocks_per_range = std::max(1, kActMax / (p.bs * p.down.kc * 2));
+    int down_blocks_per_range = std::max(1, kActMax / (p.bs * p.down.kc * 4));
     down_blocks_per_range = std::min(down_blocks_per_range, p.down.nkb);
     p.down_ksplit = (p.down.nkb + down_blocks_per_range - 1) / down_blocks_per_range;
     int act = 0;
-    act = std::max(act, p.bs * p.qkv.nkb * p.qkv.kc * 2);
-    act = std::max(act, p.bs * p.o.nkb * p.o.kc * 2);
-    act = std::max(act, p.bs * p.lm.nkb * p.lm.kc * 2);
-    act = std::max(act, p.gu_bs * p.gu.nkb * p.gu.kc * 2);
-    act = std::max(act, p.bs * down_blocks_per_range * p.down.kc * 2);
+    act = std::max(act, p.bs * p.qkv.nkb * p.qkv.kc * 4);
+    act = std::max(act, p.bs * p.o.nkb * p.o.kc * 4);
+    act = std::max(act, p.bs * p.lm.nkb * p.lm.kc * 4);
+    act = std::max(act, p.gu_bs * p.gu.nkb * p.gu.kc * 4);
+    act = std::max(act, p.bs * down_blocks_per_range * p.down.kc * 4);
     const int G = nq / nkv;
-    const int sp = kStageBytes / (4 * d);  // positions per attention ring slot (K and V halves)
-    int attn_scratch = G * d * 4 + G * sp * 4 + 2 * d * 4 + 2 * kMaxGroup * 4 * 4;
-    act = std::max(act, attn_scratch);
-    p.act_bytes = (int)align_up(act, 128);
-    p.stages = std::min(kMaxStages, (kMaxSmem - p.act_bytes - kSmemReserve) / kStageBytes);
-    if (p.stages < 2) return bad(MK_ERR_UNSUPPORTED, "not enough shared memory for the ring");
-
-    // Split-KV chunks: enough attention instructions to cover the CTAs once.
     p.chunks = std::max(1, std::min(kMaxAttnChunks, (n_ctas + B * nkv - 1) / (B * nkv)));
     p.chunks = std::min(p.chunks, std::max(1, c.max_seq / 16));
+    // the combine gathers every chunk's partial output [G][chunks][d] into shared memory
+    p.chunks = std::min(p.chunks, std::max(1, kActMax / (G * d * 4)));
+    int attn_scratch = G * d * 4 + G * score_stride(d) * 4 + 2 * d * 4 + 2 * G * p.chunks * 4;
+    attn_scratch = std::max(attn_scratch, G * p.chunks * d * 4 + 2 * G * p.chunks * 4);
+    act = std::max(act, attn_scratch);
+    p.act_bytes = (int)align_up(act, 128);
+    p.stages = kMaxStages;
+    while (p.stages >= 2 && (size_t)p.stages * kStageBytes + p.act_bytes + misc_bytes(p.bs, p.stages) > (size_t)kMaxSmem)
+        --p.stages;
+    if (p.stages < 2) return bad(MK_ERR_UNSUPPORTED, "not enough shared memory for the ring");
+
 
     // Counters.
     const int n_arr_att = L * B * nkv;
@@ -188,20 +196,26 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
             if (in.wait_ctr != kNoCounter) in.wait_count = p.counter_count[in.wait_ctr];
 
     // ---------------------------------------------------------- assignment to CTAs
-    // Greedy least-loaded by cumulative streamed bytes: each phase's
-    // instructions go, in order, to the CTA with the least work so far, which
-    // keeps every SM's total bytes per step within one instruction of the mean.
+    // Greedy least-loaded by cumulative streamed bytes, with at most
+    // ceil(n / n_ctas) instructions of one phase per CTA: every SM's total
+    // bytes per step stay within one instruction of the mean, and no phase
+    // (attention in particular, whose units are cheap) piles several of its
+    // instructions onto the same few CTAs and lengthens its critical path.
     std::vector<std::vector<std::vector<Instr>>> per(n_ctas, std::vector<std::vector<Instr>>(p.n_phases));
+    std::vector<double> load(n_ctas, 0.0);
     using Item = std::pair<double, int>;
-    std::priority_queue<Item, std::vector<Item>, std::greater<Item>> heap;
-    for (int i = 0; i < n_ctas; ++i) heap.push({0.0, i});
     for (int ph = 0; ph < p.n_phases; ++ph) {
-        for (size_t j = 0; j < phases[ph].size(); ++j) {
+        const size_t n = phases[ph].size();
+        const size_t cap = (n + n_ctas - 1) / n_ctas;
+        std::priority_queue<Item, std::vector<Item>, std::greater<Item>> heap;
+        for (int i = 0; i < n_ctas; ++i) heap.push({load[i], i});
+        std::vector<size_t> taken(n_ctas, 0);
+        for (size_t j = 0; j < n; ++j) {
             Item it = heap.top();
             heap.pop();
             per[it.second][ph].push_back(phases[ph][j]);
-            it.first += costs[ph][j];
-            heap.push(it);
+            load[it.second] += costs[ph][j];
+            if (++taken[it.second] < cap) heap.push({load[it.second], it.second});
         }
     }
     // LM-head arrivals: one per CTA that has LM work; its last LM instruction publishes.
@@ -246,8 +260,8 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     p.off_rope = take((size_t)(d / 2) * 8);
     p.off_x = take((size_t)B * H * 4);
     p.off_qkv = take((size_t)B * p.qkv_rows * 4);
-    p.off_attn = take((size_t)B * p.o.nkb * p.o.kc * 2);
-    p.off_act_a = take((size_t)B * p.i_pad * 2);
+    p.off_attn = take((size_t)B * p.o.nkb * p.o.kc * 4);
+    p.off_act_a = take((size_t)B * p.i_pad * 4);
     p.off_partials = take((size_t)B * nq * p.chunks * (d + 2) * 4);
     p.off_lm_best = take((size_t)B * n_ctas * sizeof(LmBest));
     p.off_next_scratch = take((size_t)B * 4);
@@ -273,6 +287,9 @@ mk_status validate_plan(const Plan &p, std::string &err) {
         err = msg;
         return MK_ERR_STATE;
     };
+    // Shared memory: ring + activations + misc (sized for the kernel instance).
+    if ((size_t)p.stages * kStageBytes + p.act_bytes + misc_bytes(p.bs, p.stages) > (size_t)kMaxSmem)
+        return fail("shared-memory layout exceeds the per-CTA limit");
     // Index ranges.
     for (size_t i = 0; i < p.instrs.size(); ++i) {
         const Instr &in = p.instrs[i];
@@ -294,7 +311,7 @@ mk_status validate_plan(const Plan &p, std::string &err) {
             if (in.tile >= (uint32_t)m->tiles || in.kb0 >= in.kb1 || in.kb1 > m->nkb)
                 return fail("GEMV instruction tile/K range out of range");
             if (in.nb > kMaxBatchRows) return fail("GEMV instruction carries too many batch rows");
-            if ((size_t)in.nb * (in.kb1 - in.kb0) * m->kc * 2 > (size_t)p.act_bytes)
+            if ((size_t)in.nb * (in.kb1 - in.kb0) * m->kc * 4 > (size_t)p.act_bytes)
                 return fail("GEMV activation range does not fit the shared-memory region");
             if ((in.flags & F_ATOMIC) && in.op != OP_DOWN) return fail("K-split only allowed for down");
         } else {

@@ -1,0 +1,116 @@
+"""Profiling driver: run a few decode steps of a workload, optionally with the
+per-instruction device trace, and summarise where the step's time goes.
+
+    python -m tile_synchronised_b200.profile [--workload llama1b] [--batch 1]
+        [--prefill 1024] [--steps 3] [--variant megakernel] [--trace out.json]
+
+Used as the command under ncu (small --prefill keeps the capture short) and
+for trace summaries: per phase (op, layer) the span from the first dependency
+satisfied to the last instruction done, per op the mean instruction time, the
+time spent waiting on counters, and how far the producer ran ahead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import sys
+
+import numpy as np
+import torch
+
+OPS = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead"}
+
+
+def summarise(sched, base, tr):
+    """sched: structured instruction array; tr: int64 [n, 8] stamps and waits (ns)."""
+    t0, t1, t2, tp = (tr[:, k].astype(np.float64) for k in range(4))
+    cwait, pwait = tr[:, 4].astype(np.float64), tr[:, 5].astype(np.float64)
+    origin = t0[t0 > 0].min()
+    t0, t1, t2 = t0 - origin, t1 - origin, t2 - origin
+    tp = np.where(tp > 0, tp - origin, np.nan)
+    out = {"step_us": float((t2.max()) / 1e3)}
+    per_op = {}
+    for code, name in OPS.items():
+        m = sched["op"] == code
+        if not m.any():
+            continue
+        dur = (t2[m] - t1[m]) / 1e3
+        wait = (t1[m] - t0[m]) / 1e3
+        lead = (t1[m] - tp[m]) / 1e3
+        per_op[name] = {"n": int(m.sum()), "mean_us": float(dur.mean()), "p90_us": float(np.percentile(dur, 90)),
+                        "sum_us_per_cta": float(dur.sum() / (len(base) - 1)),
+                        "wait_sum_us_per_cta": float(wait.sum() / (len(base) - 1)),
+                        "producer_lead_us": float(np.nanmean(lead)) if np.isfinite(lead).any() else None,
+                        "consumer_data_wait_us": float(cwait[m].mean() / 1e3),
+                        "producer_slot_wait_us": float(pwait[m].mean() / 1e3)}
+    out["per_op"] = per_op
+    phases = []
+    keys = sched["op"].astype(np.int64) * 100000 + sched["layer"].astype(np.int64)
+    for k in np.unique(keys):
+        m = keys == k
+        phases.append((float(t1[m].min() / 1e3), float(t2[m].max() / 1e3), OPS[int(k // 100000)], int(k % 100000)))
+    phases.sort()
+    out["phases"] = [{"op": o, "layer": l, "start_us": round(a, 2), "end_us": round(b, 2)} for a, b, o, l in phases]
+    # per-CTA: total busy (sum of instruction durations) vs span
+    busy = []
+    for c in range(len(base) - 1):
+        s, e = base[c], base[c + 1]
+        if e > s:
+            busy.append(float((t2[s:e] - t1[s:e]).sum() / max(1.0, t2[s:e].max())))
+    out["cta_busy_frac_mean"] = float(np.mean(busy))
+    return out
+
+
+def main(argv=None):
+    import os
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import synth
+    import tile_synchronised_b200 as mk
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="llama1b", choices=sorted(synth.MODELS))
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--prefill", type=int, default=None)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--variant", default="megakernel", choices=sorted(mk.VARIANTS))
+    ap.add_argument("--trace", default=None, help="write a trace summary (JSON) of the last step here")
+    ap.add_argument("--max-seq", type=int, default=None)
+    a = ap.parse_args(argv)
+    shape = synth.MODELS[a.workload]
+    B = a.batch or shape.batch
+    prefill = shape.prefill if a.prefill is None else a.prefill
+    max_seq = a.max_seq or max(prefill + a.steps + 1, 16)
+    tw = synth.make_weights(shape, device="cuda")
+    model = mk.Model(shape, tw, batch=B, max_seq=max_seq, variant=a.variant)
+    tokens = synth.make_tokens(shape, prefill + a.steps, batch=B)
+    if prefill:
+        model.prefill(tokens[:, :prefill].cuda())
+    d_tok = tokens[:, prefill:].t().contiguous().cuda()  # [steps, B]
+    for s in range(a.steps - 1):
+        model.decode(d_tok[s])
+    tr = None
+    if a.trace:
+        n = model.info()["n_instructions"]
+        tr = torch.zeros((n, 8), dtype=torch.int64, device="cuda")
+        model.set_trace(tr)
+    model.decode(d_tok[a.steps - 1])
+    torch.cuda.synchronize()
+    st = model.status()
+    if st != 0:
+        raise SystemExit(f"device status {st}: {model.last_error()}")
+    if a.trace:
+        sched, base = model.schedule()
+        summ = summarise(sched, base, tr.cpu().numpy())
+        summ.update({"workload": a.workload, "batch": B, "prefill": prefill, "variant": a.variant,
+                     "schedule": model.info()})
+        np.save(a.trace.replace(".json", "") + "_raw.npy", tr.cpu().numpy())
+        with open(a.trace, "w") as f:
+            json.dump(summ, f, indent=1)
+        print(json.dumps({k: v for k, v in summ.items() if k != "phases"}, indent=1))
+        print("first phases:", summ["phases"][:12])
+        print("last phases:", summ["phases"][-6:])
+    print("profile run ok")
+
+
+if __name__ == "__main__":
+    main()
