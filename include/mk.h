@@ -162,6 +162,10 @@ mk_status mk_set_variant(mk_ctx *ctx, int variant);
  * receives MK_SWIGLU_ROW or MK_SWIGLU_COL. */
 mk_status mk_tune(mk_ctx *ctx, void *stream, int *chosen);
 
+/* Distance, in 32 KB ring blocks, by which the producer's L2 prefetches run
+ * ahead of its shared-memory loads (default 8; 0 disables prefetching). 0..64. */
+mk_status mk_set_prefetch(mk_ctx *ctx, int blocks);
+
 /* Device wait limit in nanoseconds (default 1e9).  A wait that runs out sets
  * the context's error word and makes every CTA return early. */
 mk_status mk_set_timeout_ns(mk_ctx *ctx, unsigned long long ns);

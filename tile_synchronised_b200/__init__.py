@@ -168,6 +168,9 @@ class Model(Plan):
     def set_variant(self, name: str) -> None:
         check(self.lib.mk_set_variant(self.ctx, VARIANTS[name]), self.ctx, "mk_set_variant")
 
+    def set_prefetch(self, blocks: int) -> None:
+        check(self.lib.mk_set_prefetch(self.ctx, int(blocks)), self.ctx, "mk_set_prefetch")
+
     def set_timeout_ns(self, ns: int) -> None:
         check(self.lib.mk_set_timeout_ns(self.ctx, int(ns)), self.ctx, "mk_set_timeout_ns")
 

@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "MK_OK", -1: "MK_ERR_INVALID", -2: "MK_ERR_CUDA", -3: "MK_ERR
 # Every symbol include/mk.h declares.
 EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk_kv_cache_bytes",
            "mk_load_weights", "mk_prefill_kv", "mk_decode_step", "mk_get_status", "mk_reset",
-           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_timeout_ns", "mk_debug_drop_signal",
+           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch", "mk_set_timeout_ns", "mk_debug_drop_signal",
            "mk_set_trace", "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1", "mk_swiglu_tune")
 
 
@@ -80,6 +80,7 @@ def load() -> C.CDLL:
         "mk_set_position": ([vp, i32, vp], st),
         "mk_set_variant": ([vp, i32], st),
         "mk_tune": ([vp, vp, C.POINTER(i32)], st),
+        "mk_set_prefetch": ([vp, i32], st),
         "mk_set_timeout_ns": ([vp, C.c_ulonglong], st),
         "mk_debug_drop_signal": ([vp, i32], st),
         "mk_set_trace": ([vp, vp, sz], st),

@@ -27,6 +27,7 @@ struct mk_ctx {
     unsigned long long timeout_ns = 1000000000ull;
     int drop_instr = -1;
     unsigned long long *trace = nullptr;
+    int prefetch = 8;  // L2 prefetch distance in ring blocks
     const void *embed = nullptr;
     // captured graph of the separate-kernels variant
     cudaGraph_t graph = nullptr;
@@ -206,7 +207,7 @@ static KParams make_params(mk_ctx *c, const int32_t *tokens, int64_t tok_stride,
     P.lm_w = ws + p.lm.offset;
     P.final_norm = ws + p.off_norms + (size_t)g.n_layers * (2 * g.hidden + 2 * g.head_dim) * 2;
     P.embed = c->embed;
-    P.rope_inv_freq = reinterpret_cast<const double *>(ws + p.off_rope);
+    for (int i = 0; i < g.head_dim / 2 && i < 64; ++i) P.rope_inv_freq[i] = std::pow((double)g.rope_theta, -2.0 * i / g.head_dim);
     P.x = reinterpret_cast<float *>(ws + p.off_x);
     P.qkv = reinterpret_cast<float *>(ws + p.off_qkv);
     P.attn = reinterpret_cast<float *>(ws + p.off_attn);
@@ -223,6 +224,7 @@ static KParams make_params(mk_ctx *c, const int32_t *tokens, int64_t tok_stride,
     P.tok_stride = tok_stride;
     P.timeout_ns = c->timeout_ns;
     P.trace = c->trace;
+    P.prefetch = c->prefetch;
     P.n_layers = g.n_layers;
     P.hidden = g.hidden;
     P.n_heads = g.n_heads;
@@ -407,7 +409,7 @@ static mk_status retarget_graph(mk_ctx *c, const int32_t *tok, int32_t *next, fl
         KParams P = phase_params(c, k, tok, next, logits, pdl);
         void *args[1] = {&P};
         cudaKernelNodeParams np = {};
-        np.func = const_cast<void *>(step_kernel_func(p.bs));
+        np.func = const_cast<void *>(step_kernel_func(P));
         np.gridDim = dim3(p.n_ctas);
         np.blockDim = dim3(kThreads);
         np.sharedMemBytes = smem_bytes(P);
@@ -538,6 +540,13 @@ mk_status mk_set_variant(mk_ctx *c, int variant) {
     if (!c) return MK_ERR_INVALID;
     if (variant < MK_MEGAKERNEL || variant > MK_GRAPH_PDL) return fail(c, MK_ERR_INVALID, "unknown variant");
     c->variant = variant;
+    return MK_OK;
+}
+
+mk_status mk_set_prefetch(mk_ctx *c, int blocks) {
+    if (!c || blocks < 0 || blocks > 64) return MK_ERR_INVALID;
+    c->prefetch = blocks;
+    drop_graph(c);
     return MK_OK;
 }
 

@@ -24,13 +24,10 @@ constexpr int kernel_bs(int bs) { return bs <= 1 ? 1 : (bs <= 2 ? 2 : (bs <= 4 ?
 // never hand a slot to a new instruction while an older one still uses it.
 constexpr int reduce_slots(int stages) { return stages + 2; }
 // Bytes after the ring and the activation region: barriers, flags and small
-// arrays (1536 B), then the per-warp partial sums [slots][8 warps][8 rows][bs].
-constexpr int misc_bytes(int bs, int stages) { return 1536 + reduce_slots(stages) * 256 * kernel_bs(bs); }
+// arrays and the RoPE table (2048 B), then the per-warp partial sums [slots][8 warps][8 rows][bs].
+constexpr int misc_bytes(int bs, int stages) { return 2048 + reduce_slots(stages) * 256 * kernel_bs(bs); }
 constexpr int kMaxAttnChunks = 64;
 constexpr int kMaxGroup = 8;                            // query heads per KV head
-// Row stride (floats) of the attention score buffer: one slot of positions plus
-// this step's position, padded so every later scratch array stays 16-byte aligned.
-constexpr int score_stride(int head_dim) { return ((kStageBytes / (4 * head_dim)) + 1 + 3) & ~3; }
 constexpr uint16_t kNoCounter = 0xFFFF;
 
 // ---------------------------------------------------------------- opcodes
@@ -118,7 +115,6 @@ struct KParams {
     const void *lm_w;           // packed LM head
     const void *final_norm;     // bf16 [H]
     const void *embed;          // bf16 [V, H] (caller's)
-    const double *rope_inv_freq;// [d/2]
     float *x;                   // [B, H] residual stream
     float *qkv;                 // [B, qkv_rows]
     float *attn;                // [B, nq d padded] attention output
@@ -142,6 +138,8 @@ struct KParams {
     int32_t use_waits;          // 0 in the separate-kernels variant (kernel boundaries order the ops)
     int32_t pdl;                // 1: wait on the previous grid before reading activations
     unsigned long long *trace;  // [n_instr][8] globaltimer stamps and waits, or null
+    int32_t prefetch;           // ring blocks the L2 prefetch cursor runs ahead of the TMA loads
+    double rope_inv_freq[64];   // theta^(-2i/d), i < d/2
 };
 
 }  // namespace mk

@@ -37,6 +37,7 @@ struct SmemLayout {
     unsigned long long *best; // [64] argmax keys per batch row
     int *rcnt;                // [slots][8] warps that delivered each output
     float *rsum;              // [slots][8 warps][8 rows][bs] per-warp partial dot products
+    double *rope;             // [64] RoPE inverse frequencies theta^(-2i/d)
 };
 
 __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &P) {
@@ -53,7 +54,8 @@ __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &
     S.ssq = reinterpret_cast<float *>(misc + 320);
     S.best = reinterpret_cast<unsigned long long *>(misc + 576);
     S.rcnt = reinterpret_cast<int *>(misc + 1088);
-    S.rsum = reinterpret_cast<float *>(misc + 1536);
+    S.rope = reinterpret_cast<double *>(misc + 1536);
+    S.rsum = reinterpret_cast<float *>(misc + 2048);
     return S;
 }
 
@@ -61,11 +63,25 @@ __host__ int smem_bytes(const KParams &P) { return P.stages * kStageBytes + P.ac
 
 // ------------------------------------------------------------------ helpers
 __device__ __forceinline__ Instr load_instr(const KParams &P, int i) {
+    // field-by-field from two 16-byte loads (no address-taken copy, so the
+    // instruction stays in registers)
     const uint4 *p = reinterpret_cast<const uint4 *>(P.instrs + i);
-    uint4 a = __ldg(p), b = __ldg(p + 1);
+    const uint4 a = __ldg(p), b = __ldg(p + 1);
     Instr in;
-    memcpy(reinterpret_cast<uint8_t *>(&in), &a, 16);
-    memcpy(reinterpret_cast<uint8_t *>(&in) + 16, &b, 16);
+    in.op = (uint8_t)(a.x & 0xFFu);
+    in.flags = (uint8_t)((a.x >> 8) & 0xFFu);
+    in.layer = (uint16_t)(a.x >> 16);
+    in.tile = a.y;
+    in.kb0 = (uint16_t)(a.z & 0xFFFFu);
+    in.kb1 = (uint16_t)(a.z >> 16);
+    in.b0 = (uint16_t)(a.w & 0xFFFFu);
+    in.nb = (uint16_t)(a.w >> 16);
+    in.wait_ctr = (uint16_t)(b.x & 0xFFFFu);
+    in.signal_ctr = (uint16_t)(b.x >> 16);
+    in.wait_count = b.y;
+    in.signal2_ctr = (uint16_t)(b.z & 0xFFFFu);
+    in.pad0 = 0;
+    in.arrive_count = b.w;
     return in;
 }
 
@@ -86,6 +102,7 @@ __device__ bool wait_counter(const KParams &P, uint32_t ctr, uint32_t target, ui
     for (uint32_t it = 1;; ++it) {
         uint32_t v = ld_acquire_gpu(p);
         if (static_cast<int32_t>(v - target) >= 0) return true;
+        __nanosleep(32);
         if ((it & 15u) == 0u) {
             if (ld_relaxed_gpu(&P.state->err) != 0u) return false;
             uint64_t now = globaltimer_ns();
@@ -98,12 +115,15 @@ __device__ bool wait_counter(const KParams &P, uint32_t ctr, uint32_t target, ui
     }
 }
 
-// Bounded wait on a ring barrier; also returns false once the CTA aborts.
+// Bounded wait on a ring barrier; also returns false once the CTA aborts.  The
+// thread sleeps in hardware between checks (woken when the phase completes),
+// so a waiting producer does not take issue slots from the consumer warps.
 __device__ bool wait_bar(const KParams &P, uint64_t *bar, uint32_t parity, volatile int *abort, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = 0;
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 7u) == 0u) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if ((it & 3u) == 0u) {
             if (*abort) return false;
             uint64_t now = globaltimer_ns();
             if (t0 == 0) t0 = now;
@@ -168,57 +188,116 @@ __device__ __forceinline__ size_t kv_off(const KParams &P, int l, int b, int g, 
 }
 
 // ------------------------------------------------------------------ producer (one lane)
+// A cursor over the ring blocks of a CTA's instruction list: GEMV weight
+// blocks, or (K, V) chunks of one split-KV unit.  Instructions that stream
+// nothing are skipped.
+struct BlockCursor {
+    int i, end, j, n;
+    Instr in;
+    AttnGeom a;
+    MatRef m;
+};
+
+__device__ __forceinline__ void cursor_settle(const KParams &P, BlockCursor &c, int pos) {
+    while (c.i < c.end) {
+        c.in = load_instr(P, c.i);
+        c.j = 0;
+        if (c.in.op == OP_ATTN) {
+            c.a = attn_geom(P, c.in, pos);
+            c.n = c.a.nstages;
+        } else {
+            c.m = mat_of(P, c.in);
+            c.n = c.in.kb1 - c.in.kb0;
+        }
+        if (c.n > 0) return;
+        ++c.i;
+    }
+}
+
+__device__ __forceinline__ void cursor_next(const KParams &P, BlockCursor &c, int pos) {
+    if (++c.j >= c.n) {
+        ++c.i;
+        cursor_settle(P, c, pos);
+    }
+}
+
+// Source of the cursor's block: src2 is the V half of an attention chunk
+// (null for weights); `bytes` is per half.
+__device__ __forceinline__ void cursor_block(const KParams &P, const BlockCursor &c, const void *&src1,
+                                             const void *&src2, uint32_t &bytes) {
+    if (c.in.op == OP_ATTN) {
+        const int d = P.head_dim, sp = kStageBytes / (4 * d);
+        const int p = c.a.p0 + c.j * sp;
+        const int n = min(sp, c.a.tma_end - p);
+        bytes = (uint32_t)(n * d * 2);
+        src1 = P.kcache + kv_off(P, c.in.layer, c.a.b, c.a.g, p);
+        src2 = P.vcache + kv_off(P, c.in.layer, c.a.b, c.a.g, p);
+    } else {
+        bytes = (uint32_t)(kTileRows * c.m.kc * 2);
+        src1 = c.m.base + ((size_t)c.in.tile * c.m.nkb + c.in.kb0 + c.j) * bytes;
+        src2 = nullptr;
+    }
+}
+
+// The producer fills the ring in instruction order.  A second cursor runs
+// P.prefetch blocks ahead and pulls those blocks into L2, so the ring's TMA
+// loads hit L2 and the bytes in flight per SM are not limited to the ring.
 __device__ void producer(const KParams &P, const SmemLayout &S, int begin, int end, int pos) {
     const uint64_t pol = policy_evict_first();
+    const uint64_t pol_pf = policy_evict_normal();
     int slot = 0;
     uint32_t phase = 0, issued = 0, issued_par = 0;
     const uint64_t limit = 2ull * P.timeout_ns + 1000000ull;
     bool ok = true;
-    for (int i = begin; i < end && ok; ++i) {
-        const Instr in = load_instr(P, i);
-        unsigned long long pw = 0;
-        if (P.trace) P.trace[8 * (size_t)i + 3] = 0ull;
-        if (in.op == OP_ATTN) {
-            const AttnGeom a = attn_geom(P, in, pos);
-            const int d = P.head_dim, sp = kStageBytes / (4 * d);
-            const uint16_t *kb = P.kcache + kv_off(P, in.layer, a.b, a.g, 0);
-            const uint16_t *vb = P.vcache + kv_off(P, in.layer, a.b, a.g, 0);
-            for (int s = 0; s < a.nstages; ++s) {
-                const int p = a.p0 + s * sp;
-                const int n = min(sp, a.tma_end - p);
-                const unsigned long long w0 = P.trace ? globaltimer_ns() : 0ull;
-                if (!wait_bar(P, &S.empty[slot], phase ^ 1u, S.abort, limit)) { ok = false; break; }
-                if (P.trace) pw += globaltimer_ns() - w0;
-                const uint32_t bytes = (uint32_t)(n * d * 2);
-                if (P.trace && s == 0) P.trace[8 * (size_t)i + 3] = globaltimer_ns();
-                mbar_arrive_expect_tx(&S.full[slot], 2u * bytes);
-                uint8_t *dst = S.ring + (size_t)slot * kStageBytes;
-                bulk_g2s(dst, kb + (size_t)p * d, bytes, &S.full[slot], pol);
-                bulk_g2s(dst + kStageBytes / 2, vb + (size_t)p * d, bytes, &S.full[slot], pol);
-                issued |= 1u << slot;
-                issued_par = (issued_par & ~(1u << slot)) | (phase << slot);
-                if (++slot == P.stages) { slot = 0; phase ^= 1u; }
-            }
-        } else {
-            const MatRef m = mat_of(P, in);
-            const uint32_t bytes = (uint32_t)(kTileRows * m.kc * 2);
-            for (int kb = in.kb0; kb < in.kb1; ++kb) {
-                const unsigned long long w0 = P.trace ? globaltimer_ns() : 0ull;
-                if (!wait_bar(P, &S.empty[slot], phase ^ 1u, S.abort, limit)) { ok = false; break; }
-                if (P.trace) pw += globaltimer_ns() - w0;
-                if (P.trace && kb == in.kb0) P.trace[8 * (size_t)i + 3] = globaltimer_ns();
-                mbar_arrive_expect_tx(&S.full[slot], bytes);
-                const uint8_t *src = m.base + ((size_t)in.tile * m.nkb + kb) * bytes;
-                bulk_g2s(S.ring + (size_t)slot * kStageBytes, src, bytes, &S.full[slot], pol);
-                issued |= 1u << slot;
-                issued_par = (issued_par & ~(1u << slot)) | (phase << slot);
-                if (++slot == P.stages) { slot = 0; phase ^= 1u; }
-            }
+    BlockCursor cur{begin, end, 0, 0}, pf{begin, end, 0, 0};
+    cursor_settle(P, cur, pos);
+    cursor_settle(P, pf, pos);
+    for (int k = 0; k < P.prefetch && pf.i < end; ++k) {  // prime the prefetch distance
+        const void *s1, *s2;
+        uint32_t bytes;
+        cursor_block(P, pf, s1, s2, bytes);
+        bulk_prefetch_l2(s1, bytes, pol_pf);
+        if (s2) bulk_prefetch_l2(s2, bytes, pol_pf);
+        cursor_next(P, pf, pos);
+    }
+    unsigned long long pw = 0;
+    while (cur.i < end) {
+        const void *s1, *s2;
+        uint32_t bytes;
+        cursor_block(P, cur, s1, s2, bytes);
+        const unsigned long long w0 = P.trace ? globaltimer_ns() : 0ull;
+        if (!wait_bar(P, &S.empty[slot], phase ^ 1u, S.abort, limit)) {
+            ok = false;
+            break;
         }
         if (P.trace) {
-            P.trace[8 * (size_t)i + 5] = pw;
-            P.trace[8 * (size_t)i + 6] = globaltimer_ns();
+            pw += globaltimer_ns() - w0;
+            if (cur.j == 0) P.trace[8 * (size_t)cur.i + 3] = globaltimer_ns();
         }
+        uint8_t *dst = S.ring + (size_t)slot * kStageBytes;
+        mbar_arrive_expect_tx(&S.full[slot], s2 ? 2u * bytes : bytes);
+        bulk_g2s(dst, s1, bytes, &S.full[slot], pol);
+        if (s2) bulk_g2s(dst + kStageBytes / 2, s2, bytes, &S.full[slot], pol);
+        issued |= 1u << slot;
+        issued_par = (issued_par & ~(1u << slot)) | (phase << slot);
+        if (++slot == P.stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+        if (pf.i < end) {
+            const void *p1, *p2;
+            uint32_t pb;
+            cursor_block(P, pf, p1, p2, pb);
+            bulk_prefetch_l2(p1, pb, pol_pf);
+            if (p2) bulk_prefetch_l2(p2, pb, pol_pf);
+            cursor_next(P, pf, pos);
+        }
+        if (P.trace && cur.j == cur.n - 1) {
+            P.trace[8 * (size_t)cur.i + 5] = pw;
+            P.trace[8 * (size_t)cur.i + 6] = globaltimer_ns();
+            pw = 0;
+        }
+        cursor_next(P, cur, pos);
     }
     if (!ok && !*S.abort) {
         set_error(P, 3u, (uint32_t)begin, 0u);
@@ -266,8 +345,8 @@ __device__ __forceinline__ void c_release(const KParams &P, const SmemLayout &S,
 // [nb][klen] into shared memory: RMSNorm(x) * gain for QKV / gate-up / LM head,
 // a plain copy of the attention output or of the SwiGLU product otherwise.
 template <int BS>
-__device__ void stage_act(const KParams &P, const SmemLayout &S, const Instr &in, const MatRef &m, int klen,
-                          float *red) {
+__device__ __forceinline__ void stage_act(const KParams &P, const SmemLayout &S, const Instr &in, const MatRef &m,
+                                       int klen, float *red) {
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int nb = in.nb;
     float *act = reinterpret_cast<float *>(S.act);
@@ -546,10 +625,54 @@ __device__ __forceinline__ void gemv_tile(const KParams &P, const SmemLayout &S,
     gemv_epilogue<BS>(P, S, in, r0, v0, v1);
 }
 
-template <int BS>
-__device__ void gemv_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in, uint64_t &act_tag,
-                           uint32_t gen, int pos, int q) {
+// Publish this CTA's best (value, index) per sequence; the last CTA to do so
+// picks the token and advances the step state.
+__device__ __forceinline__ void lm_publish(const KParams &P, const SmemLayout &S, const Instr &in, uint32_t gen, int pos) {
     const int t = threadIdx.x;
+    consumer_sync();  // every row of every LM tile of this CTA is folded into best[]
+    if (t < P.batch) {
+        const unsigned long long k = S.best[t];
+        LmBest e;
+        e.value = key_value(k);
+        e.index = key_index(k);
+        e.gen = gen;
+        e.pad = 0;
+        P.lm_best[(size_t)t * P.n_ctas + blockIdx.x] = e;
+    }
+    consumer_sync();
+    if (t == 0) {
+        __threadfence();
+        const uint32_t old = atom_acq_rel_add(P.counters + in.signal_ctr, 1u);
+        *S.flag = (old + 1u == (gen + 1u) * in.arrive_count) ? 1 : 0;
+    }
+    consumer_sync();
+    if (*S.flag) {
+        if (t < P.batch) {
+            float bv = -CUDART_INF_F;
+            int bi = 0x7fffffff;
+            for (int c = 0; c < P.n_ctas; ++c) {
+                const uint4 raw = __ldcg(reinterpret_cast<const uint4 *>(P.lm_best + (size_t)t * P.n_ctas + c));
+                if (raw.z == gen && better(__uint_as_float(raw.x), (int)raw.y, bv, bi)) {
+                    bv = __uint_as_float(raw.x);
+                    bi = (int)raw.y;
+                }
+            }
+            if (P.next) P.next[t] = bi;
+        }
+        consumer_sync();
+        if (t == 0) {
+            P.state->pos = pos + 1;
+            P.state->gen = gen + 1u;
+            __threadfence();
+        }
+    }
+}
+
+// One GEMV instruction.  WIDE: every matrix of the plan uses 2048-column
+// blocks, so only that tile shape is compiled into the hot loop.
+template <int BS, bool WIDE>
+__device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
+                                           uint64_t &act_tag, uint32_t gen, int pos, int q) {
     const MatRef m = mat_of(P, in);
     const int nblocks = in.kb1 - in.kb0, klen = nblocks * m.kc;
     const uint64_t tag = ((uint64_t)in.op << 56) | ((uint64_t)in.layer << 40) | ((uint64_t)in.b0 << 24) |
@@ -560,58 +683,24 @@ __device__ void gemv_instr(const KParams &P, const SmemLayout &S, CRing &ring, c
         act_tag = tag;
         consumer_sync();
     }
-    switch (m.kc) {
-        case 256: gemv_tile<BS, 1>(P, S, ring, in, m, nblocks, klen, q); break;
-        case 512: gemv_tile<BS, 2>(P, S, ring, in, m, nblocks, klen, q); break;
-        case 1024: gemv_tile<BS, 4>(P, S, ring, in, m, nblocks, klen, q); break;
-        default: gemv_tile<BS, 8>(P, S, ring, in, m, nblocks, klen, q); break;
-    }
-    if (in.op == OP_LMHEAD && (in.flags & F_LAST_LM)) {
-        consumer_sync();  // every row of every LM tile of this CTA is folded into best[]
-        if (t < P.batch) {
-            const unsigned long long k = S.best[t];
-            LmBest e;
-            e.value = key_value(k);
-            e.index = key_index(k);
-            e.gen = gen;
-            e.pad = 0;
-            P.lm_best[(size_t)t * P.n_ctas + blockIdx.x] = e;
-        }
-        consumer_sync();
-        if (t == 0) {
-            __threadfence();
-            const uint32_t old = atom_acq_rel_add(P.counters + in.signal_ctr, 1u);
-            *S.flag = (old + 1u == (gen + 1u) * in.arrive_count) ? 1 : 0;
-        }
-        consumer_sync();
-        if (*S.flag) {
-            if (t < P.batch) {
-                float bv = -CUDART_INF_F;
-                int bi = 0x7fffffff;
-                for (int c = 0; c < P.n_ctas; ++c) {
-                    const uint4 raw = __ldcg(reinterpret_cast<const uint4 *>(P.lm_best + (size_t)t * P.n_ctas + c));
-                    if (raw.z == gen && better(__uint_as_float(raw.x), (int)raw.y, bv, bi)) {
-                        bv = __uint_as_float(raw.x);
-                        bi = (int)raw.y;
-                    }
-                }
-                if (P.next) P.next[t] = bi;
-            }
-            consumer_sync();
-            if (t == 0) {
-                P.state->pos = pos + 1;
-                P.state->gen = gen + 1u;
-                __threadfence();
-            }
+    if constexpr (WIDE) {
+        gemv_tile<BS, 8>(P, S, ring, in, m, nblocks, klen, q);
+    } else {
+        switch (m.kc) {
+            case 256: gemv_tile<BS, 1>(P, S, ring, in, m, nblocks, klen, q); break;
+            case 512: gemv_tile<BS, 2>(P, S, ring, in, m, nblocks, klen, q); break;
+            case 1024: gemv_tile<BS, 4>(P, S, ring, in, m, nblocks, klen, q); break;
+            default: gemv_tile<BS, 8>(P, S, ring, in, m, nblocks, klen, q); break;
         }
     }
+    if (in.op == OP_LMHEAD && (in.flags & F_LAST_LM)) lm_publish(P, S, in, gen, pos);
 }
 
 // ------------------------------------------------------------------ attention
 // One warp prepares one head: optional per-head RMSNorm, rotate-half RoPE at
 // `pos` (angles in double, reduced mod 2*pi before the fp32 sin/cos), scale.
-__device__ void prep_head(const KParams &P, const float *src, const uint16_t *gain, int pos, float scale,
-                          float *dst, uint16_t *cache_row) {
+__device__ __forceinline__ void prep_head(const KParams &P, const SmemLayout &S, const float *src, const uint16_t *gain,
+                                          int pos, float scale, float *dst, uint16_t *cache_row) {
     const int lane = threadIdx.x & 31, d = P.head_dim, nj = d / 32, jh = nj / 2;
     float v[4];
 #pragma unroll
@@ -626,18 +715,21 @@ __device__ void prep_head(const KParams &P, const float *src, const uint16_t *ga
         for (int j = 0; j < 4; ++j)
             if (j < nj) v[j] = v[j] * r * bf2f(gain[lane + 32 * j]);
     }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        if (j < jh) {
-            const int i = lane + 32 * j;
-            double ang = (double)pos * P.rope_inv_freq[i];
-            ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
-            float sn, cs;
-            sincosf((float)ang, &sn, &cs);
-            const float a = v[j], b = v[j + jh];
-            v[j] = a * cs - b * sn;
-            v[j + jh] = b * cs + a * sn;
-        }
+    // rotate-half pairs (i, i + d/2): d = 64 -> (v0, v1); d = 128 -> (v0, v2), (v1, v3)
+    auto rot = [&](float &x, float &y, int i) {
+        double ang = (double)pos * S.rope[i];
+        ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
+        float sn, cs;
+        __sincosf((float)ang, &sn, &cs);  // |ang| <= pi here
+        const float a = x, b = y;
+        x = a * cs - b * sn;
+        y = b * cs + a * sn;
+    };
+    if (jh == 1) {
+        rot(v[0], v[1], lane);
+    } else {
+        rot(v[0], v[2], lane);
+        rot(v[1], v[3], lane + 32);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -667,162 +759,157 @@ __device__ __forceinline__ void load8<float>(const float *p, float *f) {
 __device__ __forceinline__ float ld1(const uint16_t *p) { return bf2f(*p); }
 __device__ __forceinline__ float ld1(const float *p) { return *p; }
 
-// Online-softmax update of the G heads of one KV head over n positions from a
-// ring slot (bf16 K rows, then V rows 16 KB further), plus, when `extra`, the
-// position decoded in this step from fp32 rows kx / vx.
-__device__ void attn_block(const KParams &P, const SmemLayout &S, const uint16_t *K, const uint16_t *V, int n,
-                           const float *kx, const float *vx, bool extra, int G, const float *qs, float *sc, int scs,
-                           float (&o)[4]) {
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31, d = P.head_dim, CH = d / 8;
-    float *mrun = S.mlc, *lrun = S.mlc + 8, *corr = S.mlc + 16;
-    const int rows = n + (extra ? 1 : 0);
-    for (int base = 0; base < rows * CH; base += kConsumerThreads) {
-        const int idx = base + t, j = idx / CH, ch = idx % CH;
-        float kf[8];
-        if (j < n) {
-            unpack8(*reinterpret_cast<const uint4 *>(K + (size_t)j * d + ch * 8), kf);
-        } else if (j < rows) {
-            const float4 a = *reinterpret_cast<const float4 *>(kx + ch * 8);
-            const float4 b = *reinterpret_cast<const float4 *>(kx + ch * 8 + 4);
-            kf[0] = a.x; kf[1] = a.y; kf[2] = a.z; kf[3] = a.w; kf[4] = b.x; kf[5] = b.y; kf[6] = b.z; kf[7] = b.w;
-        } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) kf[q] = 0.f;
-        }
-        float part[kMaxGroup];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            part[h] = 0.f;
-            if (h < G) {
-                const float *qh = qs + h * d + ch * 8;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) part[h] = fmaf(qh[q], kf[q], part[h]);
-            }
-        }
-        for (int off = 1; off < CH; off <<= 1)
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h)
-                if (h < G) part[h] += __shfl_xor_sync(0xFFFFFFFFu, part[h], off);
-        if (j < rows && ch == 0)
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h)
-                if (h < G) sc[h * scs + j] = part[h];
-    }
-    consumer_sync();
-    if (warp < G) {
-        float *sh = sc + warp * scs;
-        float ml = -CUDART_INF_F;
-        for (int j = lane; j < rows; j += 32) ml = fmaxf(ml, sh[j]);
-        ml = warp_max(ml);
-        const float mold = mrun[warp];
-        const float mnew = fmaxf(mold, ml);
-        float s = 0.f;
-        for (int j = lane; j < rows; j += 32) {
-            const float p = exp2f(sh[j] - mnew);
-            sh[j] = p;
-            s += p;
-        }
-        s = warp_sum(s);
-        if (lane == 0) {
-            const float cf = exp2f(mold - mnew);
-            corr[warp] = cf;
-            lrun[warp] = lrun[warp] * cf + s;
-            mrun[warp] = mnew;
-        }
-    }
-    consumer_sync();
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int oi = t + kConsumerThreads * k;
-        if (oi < G * d) {
-            const int h = oi / d, e = oi % d;
-            const float *ph = sc + h * scs;
-            float acc = o[k] * corr[h];
-            float a2 = 0.f;
-            int j = 0;
-            for (; j + 1 < n; j += 2) {
-                acc = fmaf(ph[j], bf2f(V[(size_t)j * d + e]), acc);
-                a2 = fmaf(ph[j + 1], bf2f(V[(size_t)(j + 1) * d + e]), a2);
-            }
-            for (; j < n; ++j) acc = fmaf(ph[j], bf2f(V[(size_t)j * d + e]), acc);
-            if (extra) acc = fmaf(ph[n], vx[e], acc);
-            o[k] = acc + a2;
-        }
-    }
-    consumer_sync();
-}
-
-__device__ bool attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in, uint32_t gen, int pos) {
-    const int t = threadIdx.x, warp = t >> 5;
+// One split-KV unit: the G query heads of KV head g over positions [p0, p1).
+// Warps are split into G groups of wph = 8 / G; warp (h, s) takes positions
+// s*32 + k*wph*32 + lane of every ring stage, one position per lane, and keeps
+// its own online-softmax state (running max m, sum l, unnormalised output o)
+// in registers, so a stage needs no CTA barrier.  The warps of a head merge at
+// the end; the last chunk of a (sequence, KV head) to finish combines the
+// chunks' partials with their log-sum-exp weights.
+__device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
+                                           uint32_t gen, int pos) {
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int d = P.head_dim, nkv = P.n_kv_heads, G = P.n_heads / nkv, l = in.layer;
     const int NC = P.chunks, nq = P.n_heads;
     const AttnGeom a = attn_geom(P, in, pos);
     const int sp = kStageBytes / (4 * d);
+    const int wph = kConsumerWarps / G, h = warp / wph, sl = warp % wph;
+    const bool active = h < G;
+    const int dpl = d / 32;  // output dimensions per lane: lane*dpl .. lane*dpl + dpl - 1
     float *qs = reinterpret_cast<float *>(S.act);  // [G][d] rotated, scaled queries
-    const int scs = score_stride(d);
-    float *sc = qs + G * d;                         // [G][scs] scores / probabilities
-    float *kpos = sc + G * scs;                     // [d] key of this step's position
+    float *kpos = qs + G * d;                       // [d] key of this step's position
     float *vpos = kpos + d;                         // [d] value of this step's position
-    float *mrun = S.mlc, *lrun = S.mlc + 8;
+    float *mrg = vpos + d;                          // [8 warps][d + 2] per-warp states
     const float *qkv_b = P.qkv + (size_t)a.b * P.qkv_rows;
     const LayerW *LW = P.layers + l;
     const float qscale = 1.4426950408889634f * rsqrtf((float)d);  // log2(e)/sqrt(d): scores in the exp2 domain
     consumer_sync();  // the previous instruction's readers of the activation region are done
     if (warp < G) {
-        const int h = a.g * G + warp;
-        prep_head(P, qkv_b + h * d, P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->q_norm) : nullptr, pos, qscale,
-                  qs + warp * d, nullptr);
+        prep_head(P, S, qkv_b + (a.g * G + warp) * d,
+                  P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->q_norm) : nullptr, pos, qscale, qs + warp * d,
+                  nullptr);
     } else if (a.has_cur && warp == G) {
-        prep_head(P, qkv_b + nq * d + a.g * d, P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->k_norm) : nullptr,
+        prep_head(P, S, qkv_b + nq * d + a.g * d, P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->k_norm) : nullptr,
                   pos, 1.0f, kpos, P.kcache + kv_off(P, l, a.b, a.g, pos));
     }
     if (a.has_cur && warp == kConsumerWarps - 1) {
-        // with G == 8 every warp holds a query head; the key then follows below
         const float *vs = qkv_b + (nq + nkv) * d + a.g * d;
         uint16_t *vrow = P.vcache + kv_off(P, l, a.b, a.g, pos);
-        for (int e = t & 31; e < d; e += 32) {
-            const uint16_t h = f2bf(__ldcg(vs + e));
-            vrow[e] = h;
-            vpos[e] = bf2f(h);
+        for (int e = lane; e < d; e += 32) {
+            const uint16_t hv = f2bf(__ldcg(vs + e));
+            vrow[e] = hv;
+            vpos[e] = bf2f(hv);
         }
-    }
-    if (t < 8) {
-        mrun[t] = -CUDART_INF_F;
-        lrun[t] = 0.f;
     }
     consumer_sync();
-    if (a.has_cur && G == kConsumerWarps) {
+    if (a.has_cur && G == kConsumerWarps) {  // every warp held a query head: the key comes now
         if (warp == 0)
-            prep_head(P, qkv_b + nq * d + a.g * d, P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->k_norm) : nullptr,
-                      pos, 1.0f, kpos, P.kcache + kv_off(P, l, a.b, a.g, pos));
+            prep_head(P, S, qkv_b + nq * d + a.g * d,
+                      P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->k_norm) : nullptr, pos, 1.0f, kpos,
+                      P.kcache + kv_off(P, l, a.b, a.g, pos));
         consumer_sync();
     }
-    float o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < a.nstages; ++s) {
-        const int n = min(sp, a.tma_end - (a.p0 + s * sp));
+    float m = -CUDART_INF_F, lsum = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+    const float *qh = qs + (active ? h : 0) * d;
+    const int nch = d / 8;
+    for (int st = 0; st < a.nstages; ++st) {
+        const int n = min(sp, a.tma_end - (a.p0 + st * sp));
         const uint8_t *slot = c_wait(P, S, ring);
-        const bool last = s == a.nstages - 1;
-        attn_block(P, S, reinterpret_cast<const uint16_t *>(slot), reinterpret_cast<const uint16_t *>(slot + kStageBytes / 2),
-                   n, kpos, vpos, last && a.has_cur, G, qs, sc, scs, o);
+        if (active) {
+            const uint16_t *K = reinterpret_cast<const uint16_t *>(slot);
+            const uint16_t *V = reinterpret_cast<const uint16_t *>(slot + kStageBytes / 2);
+            for (int base = sl * 32; base < n; base += wph * 32) {
+                const int j = base + lane;
+                const bool valid = j < n;
+                float sc = 0.f;
+                if (valid) {
+                    for (int k = 0; k < nch; ++k) {
+                        const int cc = (k + lane) % nch;  // rotated chunk order: no bank conflicts across lanes
+                        float kf[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(K + (size_t)j * d + cc * 8), kf);
+                        const float4 q0 = *reinterpret_cast<const float4 *>(qh + cc * 8);
+                        const float4 q1 = *reinterpret_cast<const float4 *>(qh + cc * 8 + 4);
+                        sc = fmaf(q0.x, kf[0], fmaf(q0.y, kf[1], fmaf(q0.z, kf[2], fmaf(q0.w, kf[3], sc))));
+                        sc = fmaf(q1.x, kf[4], fmaf(q1.y, kf[5], fmaf(q1.z, kf[6], fmaf(q1.w, kf[7], sc))));
+                    }
+                } else {
+                    sc = -CUDART_INF_F;
+                }
+                const float mb = warp_max(sc);
+                const float mnew = fmaxf(m, mb);
+                const float corr = exp2f(m - mnew);
+                const float p = valid ? exp2f(sc - mnew) : 0.f;
+                lsum = lsum * corr + warp_sum(p);
+                m = mnew;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[e] *= corr;
+                const int cnt = min(32, n - base);
+                for (int jj = 0; jj < cnt; ++jj) {
+                    const float pj = __shfl_sync(0xFFFFFFFFu, p, jj);
+                    const uint16_t *vr = V + (size_t)(base + jj) * d + lane * dpl;
+                    if (dpl == 2) {
+                        const uint32_t w = *reinterpret_cast<const uint32_t *>(vr);
+                        o[0] = fmaf(pj, bf_lo(w), o[0]);
+                        o[1] = fmaf(pj, bf_hi(w), o[1]);
+                    } else {
+                        const uint2 w = *reinterpret_cast<const uint2 *>(vr);
+                        o[0] = fmaf(pj, bf_lo(w.x), o[0]);
+                        o[1] = fmaf(pj, bf_hi(w.x), o[1]);
+                        o[2] = fmaf(pj, bf_lo(w.y), o[2]);
+                        o[3] = fmaf(pj, bf_hi(w.y), o[3]);
+                    }
+                }
+            }
+        }
         c_release(P, S, ring);
     }
-    if (a.nstages == 0 && a.has_cur) attn_block(P, S, nullptr, nullptr, 0, kpos, vpos, true, G, qs, sc, scs, o);
-
-    // Partial result of this chunk: unnormalised o, running max m (log2 domain), sum l.
-    float *part = P.partials;
+    if (a.has_cur && active && sl == 0) {  // this step's own position, from fp32 rows
+        float part = 0.f;
+        for (int e = lane; e < d; e += 32) part = fmaf(qh[e], kpos[e], part);
+        const float sc = warp_sum(part);
+        const float mnew = fmaxf(m, sc);
+        const float corr = exp2f(m - mnew);
+        const float p = exp2f(sc - mnew);
+        lsum = lsum * corr + p;
+        m = mnew;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int oi = t + kConsumerThreads * k;
-        if (oi < G * d) {
-            const int h = oi / d, e = oi % d, hg = a.g * G + h;
-            __stcg(part + (((size_t)a.b * nq + hg) * NC + a.c) * (d + 2) + e, o[k]);
+        for (int e = 0; e < 4; ++e)
+            if (e < dpl) o[e] = o[e] * corr + p * vpos[lane * dpl + e];
+    }
+    // merge the warps of each head
+    if (active) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (e < dpl) mrg[warp * (d + 2) + lane * dpl + e] = o[e];
+        if (lane == 0) {
+            mrg[warp * (d + 2) + d] = m;
+            mrg[warp * (d + 2) + d + 1] = lsum;
         }
     }
-    if (t < G) {
-        const int hg = a.g * G + t;
-        float *pm = part + (((size_t)a.b * nq + hg) * NC + a.c) * (d + 2) + d;
-        __stcg(pm, mrun[t]);
-        __stcg(pm + 1, lrun[t]);
+    consumer_sync();
+    float *part = P.partials;
+    if (active && sl == 0) {
+        const int w0 = h * wph;
+        float M = -CUDART_INF_F;
+        for (int k = 0; k < wph; ++k) M = fmaxf(M, mrg[(w0 + k) * (d + 2) + d]);
+        float L = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < wph; ++k) {
+            const float mk = mrg[(w0 + k) * (d + 2) + d];
+            const float wk = (mk == -CUDART_INF_F) ? 0.f : exp2f(mk - M);
+            L = fmaf(wk, mrg[(w0 + k) * (d + 2) + d + 1], L);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (e < dpl) O[e] = fmaf(wk, mrg[(w0 + k) * (d + 2) + lane * dpl + e], O[e]);
+        }
+        const int hg = a.g * G + h;
+        float *pd = part + (((size_t)a.b * nq + hg) * NC + a.c) * (d + 2);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (e < dpl) __stcg(pd + lane * dpl + e, O[e]);
+        if (lane == 0) {
+            __stcg(pd + d, M);
+            __stcg(pd + d + 1, L);
+        }
     }
     consumer_sync();
     if (t == 0) {
@@ -834,19 +921,29 @@ __device__ bool attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, c
     if (*S.flag) {
         // Last chunk to finish for this (sequence, KV head): log-sum-exp combine.
         // The group's partials are one contiguous [G][NC][d + 2] range: gather it
-        // into shared memory with independent loads, then reduce there.
+        // into shared memory with independent loads (all in flight), then reduce.
         float *co = reinterpret_cast<float *>(S.act);  // [G][NC][d]
         float *cm = co + G * NC * d;                    // [G][NC] chunk maxima -> weights
         float *cl = cm + G * NC;                        // [G][NC] chunk sums; cl[h*NC] <- 1 / L
         const float *src = part + ((size_t)a.b * nq + a.g * G) * NC * (d + 2);
         const int total = G * NC * (d + 2);
-#pragma unroll 4
-        for (int i = t; i < total; i += kConsumerThreads) {
-            const float val = __ldcg(src + i);
-            const int hc = i / (d + 2), e = i % (d + 2);
-            if (e < d) co[hc * d + e] = val;
-            else if (e == d) cm[hc] = val;
-            else cl[hc] = val;
+        for (int i0 = 0; i0 < total; i0 += 16 * kConsumerThreads) {
+            float val[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int i = i0 + k * kConsumerThreads + t;
+                val[k] = i < total ? __ldcg(src + i) : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int i = i0 + k * kConsumerThreads + t;
+                if (i < total) {
+                    const int hc = i / (d + 2), e = i % (d + 2);
+                    if (e < d) co[hc * d + e] = val[k];
+                    else if (e == d) cm[hc] = val[k];
+                    else cl[hc] = val[k];
+                }
+            }
         }
         consumer_sync();
         if (t < G) {  // per head: M = max_c m_c, w_c = 2^(m_c - M), L = sum_c w_c l_c
@@ -863,11 +960,11 @@ __device__ bool attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, c
         consumer_sync();
         const int ostride = P.o_nkb * P.o_kc;
         for (int oi = t; oi < G * d; oi += kConsumerThreads) {
-            const int h = oi / d, e = oi % d, hg = a.g * G + h;
-            const float *ph = co + (size_t)h * NC * d + e;
+            const int hh = oi / d, e = oi % d, hg = a.g * G + hh;
+            const float *ph = co + (size_t)hh * NC * d + e;
             float acc = 0.f;
-            for (int c = 0; c < NC; ++c) acc = fmaf(cm[h * NC + c], ph[(size_t)c * d], acc);
-            __stcg(P.attn + (size_t)a.b * ostride + hg * d + e, acc * cl[h * NC]);
+            for (int c = 0; c < NC; ++c) acc = fmaf(cm[hh * NC + c], ph[(size_t)c * d], acc);
+            __stcg(P.attn + (size_t)a.b * ostride + hg * d + e, acc * cl[hh * NC]);
         }
         consumer_sync();
         if (t == 0 && !(in.flags & F_DROP_SIGNAL)) red_release_add(P.counters + in.signal2_ctr, 1u);
@@ -881,7 +978,7 @@ __device__ bool attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, c
 // before it blocks on a wait, so it never holds back a signal it (through
 // others) might be waiting for.  A wait already satisfied for this step is not
 // re-checked.  Every stop decision comes out of an OR-reducing barrier.
-template <int BS>
+template <int BS, bool WIDE>
 __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int end, uint32_t gen, int pos) {
     const int t = threadIdx.x;
     CRing ring{0, 0u, 0ull};
@@ -892,11 +989,17 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
     bool stop = false;
     if (P.pdl) pdl_wait();
     consumer_sync();
-    Instr nxt;
-    if (begin < end) nxt = load_instr(P, begin);
+    // instructions are fetched three ahead: an L2 round trip is longer than
+    // one instruction's work, and L1 is nearly all given to shared memory
+    Instr q1, q2, q3;
+    if (begin < end) q1 = load_instr(P, begin);
+    if (begin + 1 < end) q2 = load_instr(P, begin + 1);
+    if (begin + 2 < end) q3 = load_instr(P, begin + 2);
     for (int i = begin; i < end && !stop; ++i) {
-        const Instr in = nxt;
-        if (i + 1 < end) nxt = load_instr(P, i + 1);
+        const Instr in = q1;
+        q1 = q2;
+        q2 = q3;
+        if (i + 3 < end) q3 = load_instr(P, i + 3);
         unsigned long long t_start = 0;
         if (P.trace && t == 0) t_start = globaltimer_ns();
         if (P.use_waits && in.wait_ctr != kNoCounter) {
@@ -922,7 +1025,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
             stop = attn_instr(P, S, ring, in, gen, pos);
             act_tag = ~0ull;
         } else {
-            gemv_instr<BS>(P, S, ring, in, act_tag, gen, pos, q);
+            gemv_instr<BS, WIDE>(P, S, ring, in, act_tag, gen, pos, q);
             if (++q == reduce_slots(P.stages)) q = 0;
             if (in.op != OP_LMHEAD && !(in.flags & F_DROP_SIGNAL)) {
                 if (pend_ctr != in.signal_ctr) {
@@ -948,7 +1051,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
     }
 }
 
-template <int BS>
+template <int BS, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant__ KParams P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const SmemLayout S = smem_layout(smem_raw, P);
@@ -964,6 +1067,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
         fence_barrier_init();
     }
     for (int i = t; i < reduce_slots(P.stages) * 8; i += kThreads) S.rcnt[i] = 0;
+    for (int i = t; i < P.head_dim / 2; i += kThreads) S.rope[i] = P.rope_inv_freq[i];
     if (t < 64) S.best[t] = argmax_key(-CUDART_INF_F, 0x7fffffff);
     __syncthreads();
     const int begin = P.cta_begin[blockIdx.x], end = P.cta_end[blockIdx.x];
@@ -973,7 +1077,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
         if ((t & 31) == 0) producer(P, S, begin, end, pos);
         __syncwarp();
     } else {
-        consumer<BS>(P, S, begin, end, gen, pos);
+        consumer<BS, WIDE>(P, S, begin, end, gen, pos);
     }
     __syncthreads();
 }
@@ -1008,12 +1112,16 @@ __global__ void pack_kernel(const uint16_t *src, const uint16_t *src2, uint16_t 
 }
 
 // ------------------------------------------------------------------ host launchers
-template <int BS>
+static bool all_wide(const KParams &P) {
+    return P.qkv_kc == 2048 && P.o_kc == 2048 && P.gu_kc == 2048 && P.down_kc == 2048 && P.lm_kc == 2048;
+}
+
+template <int BS, bool WIDE>
 static cudaError_t launch_bs(const KParams &P, int n_ctas, cudaStream_t s, bool cooperative, bool pdl_attr) {
     const int smem = smem_bytes(P);
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(step_kernel<BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+        cudaError_t e = cudaFuncSetAttribute(step_kernel<BS, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -1036,21 +1144,30 @@ static cudaError_t launch_bs(const KParams &P, int n_ctas, cudaStream_t s, bool 
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, step_kernel<BS>, P);
+    return cudaLaunchKernelEx(&cfg, step_kernel<BS, WIDE>, P);
 }
 
-const void *step_kernel_func(int bs) {
-    if (bs <= 1) return reinterpret_cast<const void *>(step_kernel<1>);
-    if (bs <= 2) return reinterpret_cast<const void *>(step_kernel<2>);
-    if (bs <= 4) return reinterpret_cast<const void *>(step_kernel<4>);
-    return reinterpret_cast<const void *>(step_kernel<8>);
+template <bool WIDE>
+static const void *func_of(int bs) {
+    if (bs <= 1) return reinterpret_cast<const void *>(step_kernel<1, WIDE>);
+    if (bs <= 2) return reinterpret_cast<const void *>(step_kernel<2, WIDE>);
+    if (bs <= 4) return reinterpret_cast<const void *>(step_kernel<4, WIDE>);
+    return reinterpret_cast<const void *>(step_kernel<8, WIDE>);
+}
+
+const void *step_kernel_func(const KParams &P) { return all_wide(P) ? func_of<true>(P.bs) : func_of<false>(P.bs); }
+
+template <bool WIDE>
+static cudaError_t launch_w(const KParams &P, int bs, int n_ctas, cudaStream_t s, bool coop, bool pdl) {
+    if (bs <= 1) return launch_bs<1, WIDE>(P, n_ctas, s, coop, pdl);
+    if (bs <= 2) return launch_bs<2, WIDE>(P, n_ctas, s, coop, pdl);
+    if (bs <= 4) return launch_bs<4, WIDE>(P, n_ctas, s, coop, pdl);
+    return launch_bs<8, WIDE>(P, n_ctas, s, coop, pdl);
 }
 
 cudaError_t launch_step(const KParams &P, int bs, int n_ctas, cudaStream_t s, bool cooperative, bool pdl_attr) {
-    if (bs <= 1) return launch_bs<1>(P, n_ctas, s, cooperative, pdl_attr);
-    if (bs <= 2) return launch_bs<2>(P, n_ctas, s, cooperative, pdl_attr);
-    if (bs <= 4) return launch_bs<4>(P, n_ctas, s, cooperative, pdl_attr);
-    return launch_bs<8>(P, n_ctas, s, cooperative, pdl_attr);
+    return all_wide(P) ? launch_w<true>(P, bs, n_ctas, s, cooperative, pdl_attr)
+                       : launch_w<false>(P, bs, n_ctas, s, cooperative, pdl_attr);
 }
 
 __global__ void set_position_kernel(State *state, int pos) { state->pos = pos; }

@@ -8,7 +8,7 @@ namespace mk {
 int smem_bytes(const KParams &P);
 // Launch the interpreter over P.cta_begin/cta_end; bs = batch rows per GEMV instruction.
 cudaError_t launch_step(const KParams &P, int bs, int n_ctas, cudaStream_t s, bool cooperative, bool pdl_attr);
-const void *step_kernel_func(int bs);
+const void *step_kernel_func(const KParams &P);
 cudaError_t launch_pack(const void *src, const void *src2, void *dst, int n_rows, int k, int kc, int nkb, int tiles,
                         int mode, cudaStream_t s);
 cudaError_t launch_set_position(State *state, int pos, cudaStream_t s);

@@ -80,10 +80,9 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     p.lm = make_mat(V, H);
     p.i_pad = p.down.nkb * p.down.kc;
 
-    // Split-KV chunks: enough attention instructions to cover the CTAs once.
     // Batch rows per instruction and the activation region.  Activations are
     // staged in shared memory as fp32 [rows][K range]; the region is capped at
-    // 64 KB so at least five 32 KB ring slots remain.  A GEMV whose rows do not
+    // 64 KB so at least four 32 KB ring slots remain.  A GEMV whose rows do not
     // fit carries fewer batch rows (its weights stream once per row group); the
     // down projection splits K instead (atomic residual update).
     const int kActMax = 65536;
@@ -104,11 +103,13 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     act = std::max(act, p.gu_bs * p.gu.nkb * p.gu.kc * 4);
     act = std::max(act, p.bs * down_blocks_per_range * p.down.kc * 4);
     const int G = nq / nkv;
-    p.chunks = std::max(1, std::min(kMaxAttnChunks, (n_ctas + B * nkv - 1) / (B * nkv)));
+    // Split-KV chunks: as many units as fit one per CTA, so an attention phase
+    // is one unit deep.  The last unit of a (sequence, KV head) gathers every
+    // chunk's partial output [G][chunks][d] into shared memory.
+    p.chunks = std::max(1, std::min(kMaxAttnChunks, n_ctas / (B * nkv)));
     p.chunks = std::min(p.chunks, std::max(1, c.max_seq / 16));
-    // the combine gathers every chunk's partial output [G][chunks][d] into shared memory
     p.chunks = std::min(p.chunks, std::max(1, kActMax / (G * d * 4)));
-    int attn_scratch = G * d * 4 + G * score_stride(d) * 4 + 2 * d * 4 + 2 * G * p.chunks * 4;
+    int attn_scratch = G * d * 4 + 2 * d * 4 + kConsumerWarps * (d + 2) * 4;
     attn_scratch = std::max(attn_scratch, G * p.chunks * d * 4 + 2 * G * p.chunks * 4);
     act = std::max(act, attn_scratch);
     p.act_bytes = (int)align_up(act, 128);
@@ -116,7 +117,6 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     while (p.stages >= 2 && (size_t)p.stages * kStageBytes + p.act_bytes + misc_bytes(p.bs, p.stages) > (size_t)kMaxSmem)
         --p.stages;
     if (p.stages < 2) return bad(MK_ERR_UNSUPPORTED, "not enough shared memory for the ring");
-
 
     // Counters.
     const int n_arr_att = L * B * nkv;

@@ -75,6 +75,8 @@ def main(argv=None):
     ap.add_argument("--variant", default="megakernel", choices=sorted(mk.VARIANTS))
     ap.add_argument("--trace", default=None, help="write a trace summary (JSON) of the last step here")
     ap.add_argument("--max-seq", type=int, default=None)
+    ap.add_argument("--prefetch", type=int, default=None, help="L2 prefetch distance (ring blocks)")
+    ap.add_argument("--time", type=int, default=0, help="also time this many steps (CUDA events)")
     a = ap.parse_args(argv)
     shape = synth.MODELS[a.workload]
     B = a.batch or shape.batch
@@ -83,11 +85,25 @@ def main(argv=None):
     tw = synth.make_weights(shape, device="cuda")
     model = mk.Model(shape, tw, batch=B, max_seq=max_seq, variant=a.variant)
     tokens = synth.make_tokens(shape, prefill + a.steps, batch=B)
+    if a.prefetch is not None:
+        model.set_prefetch(a.prefetch)
     if prefill:
         model.prefill(tokens[:, :prefill].cuda())
     d_tok = tokens[:, prefill:].t().contiguous().cuda()  # [steps, B]
     for s in range(a.steps - 1):
         model.decode(d_tok[s])
+    if a.time:
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for r in range(a.time):
+            model.set_position(prefill + a.steps - 1)
+            model.decode(d_tok[a.steps - 2 if a.steps > 1 else 0])
+        e1.record()
+        torch.cuda.synchronize()
+        print(json.dumps({"timed_steps": a.time, "us_per_step": round(1e3 * e0.elapsed_time(e1) / a.time, 2),
+                          "prefetch": a.prefetch}))
+        model.set_position(prefill + a.steps - 1)
     tr = None
     if a.trace:
         n = model.info()["n_instructions"]
@@ -103,7 +119,10 @@ def main(argv=None):
         summ = summarise(sched, base, tr.cpu().numpy())
         summ.update({"workload": a.workload, "batch": B, "prefill": prefill, "variant": a.variant,
                      "schedule": model.info()})
-        np.save(a.trace.replace(".json", "") + "_raw.npy", tr.cpu().numpy())
+        stem = a.trace.replace(".json", "")
+        np.save(stem + "_raw.npy", tr.cpu().numpy())
+        np.save(stem + "_sched.npy", sched)
+        np.save(stem + "_base.npy", base)
         with open(a.trace, "w") as f:
             json.dump(summ, f, indent=1)
         print(json.dumps({k: v for k, v in summ.items() if k != "phases"}, indent=1))
