@@ -26,7 +26,9 @@ constexpr int reduce_slots(int stages) { return stages + 2; }
 // Bytes after the ring and the activation region: barriers, flags and small
 // arrays and the RoPE table (2048 B), then the per-warp partial sums [slots][8 warps][8 rows][bs].
 constexpr int misc_bytes(int bs, int stages) { return 2048 + reduce_slots(stages) * 256 * kernel_bs(bs); }
-constexpr int kMaxAttnChunks = 64;
+constexpr int kMaxAttnChunks = 16;  // split-KV chunks per (sequence, KV head); the O-projection gathers them all
+// Floats per split-KV partial record: o[d], m, l, padding to a 16-byte multiple.
+constexpr int partial_stride(int head_dim) { return head_dim + 4; }
 constexpr int kMaxGroup = 8;                            // query heads per KV head
 constexpr uint16_t kNoCounter = 0xFFFF;
 
@@ -52,15 +54,15 @@ struct Instr {
     uint8_t op;
     uint8_t flags;
     uint16_t layer;
-    uint32_t tile;        // GEMV: row tile; ATTN: (b * nkv + g) * chunks + c
+    uint32_t tile;        // GEMV: first row tile of the run; ATTN: (b * nkv + g) * chunks + c
     uint16_t kb0, kb1;    // K block range [kb0, kb1)
     uint16_t b0, nb;      // batch rows [b0, b0 + nb)
     uint16_t wait_ctr;    // counter to wait on (kNoCounter: none)
-    uint16_t signal_ctr;  // counter to increment when done (ATTN: arrival counter)
+    uint16_t signal_ctr;  // counter to increment when done
     uint32_t wait_count;  // increments the waited counter receives per step
-    uint16_t signal2_ctr; // ATTN/LM: counter the last arriver signals
-    uint16_t pad0;
-    uint32_t arrive_count;// ATTN/LM: arrivals per step on signal_ctr
+    uint16_t signal2_ctr; // LM: counter the last arriver signals (unused)
+    uint16_t ntiles;      // GEMV: consecutive row tiles in this run (>= 1)
+    uint32_t arrive_count;// LM: arrivals per step on signal_ctr
 };
 static_assert(sizeof(Instr) == 32, "Instr must be 32 bytes");
 
@@ -117,9 +119,9 @@ struct KParams {
     const void *embed;          // bf16 [V, H] (caller's)
     float *x;                   // [B, H] residual stream
     float *qkv;                 // [B, qkv_rows]
-    float *attn;                // [B, nq d padded] attention output
+    float *attn;                // unused (the O-projection combines the split-KV partials itself)
     float *act_a;               // [B, I_pad] SwiGLU product
-    float *partials;            // [B, nq, chunks, d + 2]
+    float *partials;            // [B, nq, chunks, d + 4]: o[d], m, l, pad
     uint16_t *kcache;           // bf16 [L, B, nkv, max_seq, d]
     uint16_t *vcache;
     uint32_t *counters;

@@ -80,7 +80,7 @@ __device__ __forceinline__ Instr load_instr(const KParams &P, int i) {
     in.signal_ctr = (uint16_t)(b.x >> 16);
     in.wait_count = b.y;
     in.signal2_ctr = (uint16_t)(b.z & 0xFFFFu);
-    in.pad0 = 0;
+    in.ntiles = (uint16_t)(b.z >> 16);
     in.arrive_count = b.w;
     return in;
 }
@@ -207,7 +207,7 @@ __device__ __forceinline__ void cursor_settle(const KParams &P, BlockCursor &c, 
             c.n = c.a.nstages;
         } else {
             c.m = mat_of(P, c.in);
-            c.n = c.in.kb1 - c.in.kb0;
+            c.n = (c.in.kb1 - c.in.kb0) * c.in.ntiles;
         }
         if (c.n > 0) return;
         ++c.i;
@@ -233,8 +233,9 @@ __device__ __forceinline__ void cursor_block(const KParams &P, const BlockCursor
         src1 = P.kcache + kv_off(P, c.in.layer, c.a.b, c.a.g, p);
         src2 = P.vcache + kv_off(P, c.in.layer, c.a.b, c.a.g, p);
     } else {
+        const int nkr = c.in.kb1 - c.in.kb0;  // blocks of one tile in this run
         bytes = (uint32_t)(kTileRows * c.m.kc * 2);
-        src1 = c.m.base + ((size_t)c.in.tile * c.m.nkb + c.in.kb0 + c.j) * bytes;
+        src1 = c.m.base + ((size_t)(c.in.tile + c.j / nkr) * c.m.nkb + c.in.kb0 + c.j % nkr) * bytes;
         src2 = nullptr;
     }
 }
@@ -346,86 +347,161 @@ __device__ __forceinline__ void c_release(const KParams &P, const SmemLayout &S,
 // a plain copy of the attention output or of the SwiGLU product otherwise.
 template <int BS>
 __device__ __forceinline__ void stage_act(const KParams &P, const SmemLayout &S, const Instr &in, const MatRef &m,
-                                       int klen, float *red) {
+                                          int klen, float *red) {
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int nb = in.nb;
     float *act = reinterpret_cast<float *>(S.act);
-    if (in.op == OP_OPROJ || in.op == OP_DOWN) {
-        const float *src = in.op == OP_OPROJ ? P.attn : P.act_a;
-        const int stride = in.op == OP_OPROJ ? P.o_nkb * P.o_kc : P.i_pad;
-        const int k0 = in.kb0 * m.kc;
-        for (int b = 0; b < nb; ++b) {
-            const float4 *s = reinterpret_cast<const float4 *>(src + (size_t)(in.b0 + b) * stride + k0);
-            float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen);
-            for (int v = t; v < klen / 4; v += kConsumerThreads) dst[v] = __ldcg(s + v);
+    if (in.op == OP_OPROJ) {
+        // Log-sum-exp combine of the split-KV partials of every head:
+        // attn[b][h*d + e] = sum_c 2^(m_c - M) o_c[e] / sum_c 2^(m_c - M) l_c.
+        const int d = P.head_dim, nq = P.n_heads, NC = P.chunks, hd = nq * d, ps = partial_stride(d);
+        float *wts = act + (size_t)nb * klen;  // [nb][nq][NC] normalised chunk weights
+        for (int i = t; i < nb * nq; i += kConsumerThreads) {
+            const int b = i / nq, h = i % nq;
+            const float *pc = P.partials + (((size_t)(in.b0 + b) * nq + h) * NC) * ps + d;
+            float2 ml[kMaxAttnChunks];
+#pragma unroll
+            for (int c = 0; c < kMaxAttnChunks; ++c)
+                ml[c] = c < NC ? __ldcg(reinterpret_cast<const float2 *>(pc + (size_t)c * ps)) : make_float2(-CUDART_INF_F, 0.f);
+            float M = -CUDART_INF_F;
+#pragma unroll
+            for (int c = 0; c < kMaxAttnChunks; ++c) M = fmaxf(M, ml[c].x);
+            float L = 0.f;
+#pragma unroll
+            for (int c = 0; c < kMaxAttnChunks; ++c) {
+                ml[c].x = exp2f(ml[c].x - M);
+                L = fmaf(ml[c].x, ml[c].y, L);
+            }
+            const float inv = 1.0f / L;
+#pragma unroll
+            for (int c = 0; c < kMaxAttnChunks; ++c)
+                if (c < NC) wts[(size_t)i * NC + c] = ml[c].x * inv;
+        }
+        consumer_sync();
+        // four consecutive outputs per thread: one float4 per chunk, all loads in flight
+        for (int i4 = t; i4 < nb * klen / 4; i4 += kConsumerThreads) {
+            const int b = (4 * i4) / klen, k = (4 * i4) % klen;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (k < hd) {
+                const int h = k / d, e = k % d;
+                const float4 *pc = reinterpret_cast<const float4 *>(
+                    P.partials + (((size_t)(in.b0 + b) * nq + h) * NC) * ps + e);
+                const float *w = wts + ((size_t)b * nq + h) * NC;
+                float4 v[kMaxAttnChunks];
+#pragma unroll
+                for (int c = 0; c < kMaxAttnChunks; ++c)
+                    v[c] = c < NC ? __ldcg(pc + (size_t)c * (ps / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < kMaxAttnChunks; ++c) {
+                    if (c < NC) {
+                        acc.x = fmaf(w[c], v[c].x, acc.x);
+                        acc.y = fmaf(w[c], v[c].y, acc.y);
+                        acc.z = fmaf(w[c], v[c].z, acc.z);
+                        acc.w = fmaf(w[c], v[c].w, acc.w);
+                    }
+                }
+            }
+            reinterpret_cast<float4 *>(act)[i4] = acc;
         }
         return;
     }
+    if (in.op == OP_DOWN) {
+        // plain copy of the SwiGLU product, eight 16-byte loads in flight per thread
+        const int k0 = in.kb0 * m.kc, n4 = klen / 4;
+        for (int b = 0; b < nb; ++b) {
+            const float4 *s4 = reinterpret_cast<const float4 *>(P.act_a + (size_t)(in.b0 + b) * P.i_pad + k0);
+            float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen);
+            for (int v0 = t; v0 < n4; v0 += 8 * kConsumerThreads) {
+                float4 r[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int v = v0 + u * kConsumerThreads;
+                    r[u] = v < n4 ? __ldcg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int v = v0 + u * kConsumerThreads;
+                    if (v < n4) dst[v] = r[u];
+                }
+            }
+        }
+        return;
+    }
+    // RMSNorm(x) * gain with one pass over global memory: every thread loads
+    // its chunks of x (all batch rows) together with the gains, accumulates
+    // sum(x^2) and keeps x * gain in shared memory, then multiplies by the
+    // per-row 1/rms once the sums are known (the gain and 1/rms commute).
     const int H = P.hidden;
     const uint16_t *gain = reinterpret_cast<const uint16_t *>(
         in.op == OP_QKV ? P.layers[in.layer].attn_norm
                         : (in.op == OP_GATEUP ? P.layers[in.layer].mlp_norm : P.final_norm));
     const bool from_embed = (in.flags & F_EMBED_X) && in.op == OP_QKV;
     const uint16_t *emb = reinterpret_cast<const uint16_t *>(P.embed);
-    // pass 1: sum of squares per row
     float ss[BS];
 #pragma unroll
-    for (int b = 0; b < BS; ++b) {
-        ss[b] = 0.f;
-        if (b < nb) {
-            const int row = in.b0 + b;
-            if (from_embed) {
-                const uint4 *e = reinterpret_cast<const uint4 *>(emb + (size_t)token_of(P, row) * H);
-                for (int v = t; v < H / 8; v += kConsumerThreads) {
-                    float f[8];
-                    unpack8(__ldg(e + v), f);
+    for (int b = 0; b < BS; ++b) ss[b] = 0.f;
+    const int nch = klen / 8;
+    const uint4 *g8 = reinterpret_cast<const uint4 *>(gain);
+    for (int c = t; c < nch; c += kConsumerThreads) {
+        const bool in_range = c * 8 < H;
+        float g[8];
+        if (in_range) unpack8(__ldg(g8 + c), g);
+        float f[BS][8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) ss[b] = fmaf(f[q], f[q], ss[b]);
-                }
+        for (int b = 0; b < BS; ++b) {
+            const int row = in.b0 + (b < nb ? b : 0);
+            if (!in_range || b >= nb) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) f[b][q] = 0.f;
+            } else if (from_embed) {
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(emb + (size_t)token_of(P, row) * H) + c), f[b]);
             } else {
-                const float4 *x = reinterpret_cast<const float4 *>(P.x + (size_t)row * H);
-                for (int v = t; v < H / 4; v += kConsumerThreads) {
-                    float4 f = __ldcg(x + v);
-                    ss[b] = fmaf(f.x, f.x, fmaf(f.y, f.y, fmaf(f.z, f.z, fmaf(f.w, f.w, ss[b]))));
+                const float4 *x = reinterpret_cast<const float4 *>(P.x + (size_t)row * H) + 2 * c;
+                const float4 x0 = __ldcg(x), x1 = __ldcg(x + 1);
+                f[b][0] = x0.x; f[b][1] = x0.y; f[b][2] = x0.z; f[b][3] = x0.w;
+                f[b][4] = x1.x; f[b][5] = x1.y; f[b][6] = x1.z; f[b][7] = x1.w;
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < BS; ++b) {
+            if (b < nb) {
+                float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen + c * 8);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) ss[b] = fmaf(f[b][q], f[b][q], ss[b]);
+                if (in_range) {
+                    dst[0] = make_float4(f[b][0] * g[0], f[b][1] * g[1], f[b][2] * g[2], f[b][3] * g[3]);
+                    dst[1] = make_float4(f[b][4] * g[4], f[b][5] * g[5], f[b][6] * g[6], f[b][7] * g[7]);
+                } else {
+                    dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    dst[1] = dst[0];
                 }
             }
         }
     }
 #pragma unroll
     for (int b = 0; b < BS; ++b) {
-        float s = warp_sum(ss[b]);
+        const float s = warp_sum(ss[b]);
         if (lane == 0) red[warp * BS + b] = s;
     }
     consumer_sync();
-    if (t < nb) {
+    float rs[BS];
+#pragma unroll
+    for (int b = 0; b < BS; ++b) {
         float s = 0.f;
-        for (int w = 0; w < kConsumerWarps; ++w) s += red[w * BS + t];
-        S.rstd[t] = rsqrtf(s / (float)H + P.rms_eps);
+        for (int w = 0; w < kConsumerWarps; ++w) s += red[w * BS + b];
+        rs[b] = rsqrtf(s / (float)H + P.rms_eps);
     }
-    consumer_sync();
-    // pass 2: normalise and apply the gain (fp32)
-    const uint4 *g8 = reinterpret_cast<const uint4 *>(gain);
-    for (int b = 0; b < nb; ++b) {
-        const int row = in.b0 + b;
-        const float r = S.rstd[b];
-        float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen);
-        for (int v = t; v < klen / 8; v += kConsumerThreads) {
-            float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;
-            if (v * 8 < H) {
-                float f[8], g[8];
-                if (from_embed) {
-                    unpack8(__ldg(reinterpret_cast<const uint4 *>(emb + (size_t)token_of(P, row) * H) + v), f);
-                } else {
-                    const float4 *x = reinterpret_cast<const float4 *>(P.x + (size_t)row * H) + 2 * v;
-                    float4 a = __ldcg(x), c = __ldcg(x + 1);
-                    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = c.x; f[5] = c.y; f[6] = c.z; f[7] = c.w;
-                }
-                unpack8(__ldg(g8 + v), g);
-                o0 = make_float4(f[0] * r * g[0], f[1] * r * g[1], f[2] * r * g[2], f[3] * r * g[3]);
-                o1 = make_float4(f[4] * r * g[4], f[5] * r * g[5], f[6] * r * g[6], f[7] * r * g[7]);
+    for (int c = t; c < nch; c += kConsumerThreads) {
+        if (c * 8 >= H) continue;
+#pragma unroll
+        for (int b = 0; b < BS; ++b) {
+            if (b < nb) {
+                float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen + c * 8);
+                const float4 x0 = dst[0], x1 = dst[1];
+                const float r = rs[b];
+                dst[0] = make_float4(x0.x * r, x0.y * r, x0.z * r, x0.w * r);
+                dst[1] = make_float4(x1.x * r, x1.y * r, x1.z * r, x1.w * r);
             }
-            dst[2 * v] = o0;
-            dst[2 * v + 1] = o1;
         }
     }
 }
@@ -504,12 +580,12 @@ __device__ __forceinline__ int key_index(unsigned long long k) { return (int)(0x
 // Epilogue of one finished output (tile row r, or gate/up pair r) for all
 // batch rows: v0 = the row's dot products, v1 = the up row's for gate/up.
 template <int BS>
-__device__ void gemv_epilogue(const KParams &P, const SmemLayout &S, const Instr &in, int r, const float (&v0)[BS],
-                              const float (&v1)[BS]) {
+__device__ void gemv_epilogue(const KParams &P, const SmemLayout &S, const Instr &in, int tile, int r,
+                              const float (&v0)[BS], const float (&v1)[BS]) {
     const int H = P.hidden, nb = in.nb;
     switch (in.op) {
         case OP_QKV: {
-            const int n = (int)in.tile * 8 + r;
+            const int n = tile * 8 + r;
             if (n < P.qkv_rows)
 #pragma unroll
                 for (int b = 0; b < BS; ++b)
@@ -517,7 +593,7 @@ __device__ void gemv_epilogue(const KParams &P, const SmemLayout &S, const Instr
         } break;
         case OP_OPROJ:
         case OP_DOWN: {
-            const int n = (int)in.tile * 8 + r;
+            const int n = tile * 8 + r;
             if (n < H)
 #pragma unroll
                 for (int b = 0; b < BS; ++b) {
@@ -536,7 +612,7 @@ __device__ void gemv_epilogue(const KParams &P, const SmemLayout &S, const Instr
                 }
         } break;
         case OP_GATEUP: {
-            const int j = (int)in.tile * 4 + r;
+            const int j = tile * 4 + r;
             if (j < P.intermediate)
 #pragma unroll
                 for (int b = 0; b < BS; ++b)
@@ -544,7 +620,7 @@ __device__ void gemv_epilogue(const KParams &P, const SmemLayout &S, const Instr
                         __stcg(P.act_a + (size_t)(in.b0 + b) * P.i_pad + j, v0[b] / (1.0f + __expf(-v0[b])) * v1[b]);
         } break;
         default: {  // OP_LMHEAD
-            const int n = (int)in.tile * 8 + r;
+            const int n = tile * 8 + r;
             if (n < P.vocab)
 #pragma unroll
                 for (int b = 0; b < BS; ++b) {
@@ -565,7 +641,7 @@ __device__ void gemv_epilogue(const KParams &P, const SmemLayout &S, const Instr
 // than there are slots.
 template <int BS, int RPT>
 __device__ __forceinline__ void gemv_tile(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                          const MatRef &m, int nblocks, int klen, int q) {
+                                          const MatRef &m, int tile, int nblocks, int klen, int q) {
     constexpr int NRG = 8 / RPT;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     float acc[8][BS];
@@ -622,7 +698,7 @@ __device__ __forceinline__ void gemv_tile(const KParams &P, const SmemLayout &S,
             v0[b] += vpart[((w0 + k) * 8 + r0) * BS + b];
             if (pair) v1[b] += vpart[((w1 + k) * 8 + r0 + 4) * BS + b];
         }
-    gemv_epilogue<BS>(P, S, in, r0, v0, v1);
+    gemv_epilogue<BS>(P, S, in, tile, r0, v0, v1);
 }
 
 // Publish this CTA's best (value, index) per sequence; the last CTA to do so
@@ -672,7 +748,7 @@ __device__ __forceinline__ void lm_publish(const KParams &P, const SmemLayout &S
 // blocks, so only that tile shape is compiled into the hot loop.
 template <int BS, bool WIDE>
 __device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                           uint64_t &act_tag, uint32_t gen, int pos, int q) {
+                                           uint64_t &act_tag, uint32_t gen, int pos, int &q) {
     const MatRef m = mat_of(P, in);
     const int nblocks = in.kb1 - in.kb0, klen = nblocks * m.kc;
     const uint64_t tag = ((uint64_t)in.op << 56) | ((uint64_t)in.layer << 40) | ((uint64_t)in.b0 << 24) |
@@ -683,15 +759,20 @@ __device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S
         act_tag = tag;
         consumer_sync();
     }
-    if constexpr (WIDE) {
-        gemv_tile<BS, 8>(P, S, ring, in, m, nblocks, klen, q);
-    } else {
-        switch (m.kc) {
-            case 256: gemv_tile<BS, 1>(P, S, ring, in, m, nblocks, klen, q); break;
-            case 512: gemv_tile<BS, 2>(P, S, ring, in, m, nblocks, klen, q); break;
-            case 1024: gemv_tile<BS, 4>(P, S, ring, in, m, nblocks, klen, q); break;
-            default: gemv_tile<BS, 8>(P, S, ring, in, m, nblocks, klen, q); break;
+    const int nslots = reduce_slots(P.stages);
+    for (int k = 0; k < (int)in.ntiles; ++k) {
+        const int tile = (int)in.tile + k;
+        if constexpr (WIDE) {
+            gemv_tile<BS, 8>(P, S, ring, in, m, tile, nblocks, klen, q);
+        } else {
+            switch (m.kc) {
+                case 256: gemv_tile<BS, 1>(P, S, ring, in, m, tile, nblocks, klen, q); break;
+                case 512: gemv_tile<BS, 2>(P, S, ring, in, m, tile, nblocks, klen, q); break;
+                case 1024: gemv_tile<BS, 4>(P, S, ring, in, m, tile, nblocks, klen, q); break;
+                default: gemv_tile<BS, 8>(P, S, ring, in, m, tile, nblocks, klen, q); break;
+            }
         }
+        if (++q == nslots) q = 0;
     }
     if (in.op == OP_LMHEAD && (in.flags & F_LAST_LM)) lm_publish(P, S, in, gen, pos);
 }
@@ -764,10 +845,10 @@ __device__ __forceinline__ float ld1(const float *p) { return *p; }
 // s*32 + k*wph*32 + lane of every ring stage, one position per lane, and keeps
 // its own online-softmax state (running max m, sum l, unnormalised output o)
 // in registers, so a stage needs no CTA barrier.  The warps of a head merge at
-// the end; the last chunk of a (sequence, KV head) to finish combines the
-// chunks' partials with their log-sum-exp weights.
+// the end and write the chunk's partial (o, m, l); the O-projection combines
+// the chunks of each head with their log-sum-exp weights.
 __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                           uint32_t gen, int pos) {
+                                           int pos) {
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int d = P.head_dim, nkv = P.n_kv_heads, G = P.n_heads / nkv, l = in.layer;
     const int NC = P.chunks, nq = P.n_heads;
@@ -902,7 +983,7 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
                 if (e < dpl) O[e] = fmaf(wk, mrg[(w0 + k) * (d + 2) + lane * dpl + e], O[e]);
         }
         const int hg = a.g * G + h;
-        float *pd = part + (((size_t)a.b * nq + hg) * NC + a.c) * (d + 2);
+        float *pd = part + (((size_t)a.b * nq + hg) * NC + a.c) * partial_stride(d);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             if (e < dpl) __stcg(pd + lane * dpl + e, O[e]);
@@ -911,64 +992,8 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
             __stcg(pd + d + 1, L);
         }
     }
-    consumer_sync();
-    if (t == 0) {
-        __threadfence();
-        const uint32_t old = atom_acq_rel_add(P.counters + in.signal_ctr, 1u);
-        *S.flag = (old + 1u == (gen + 1u) * in.arrive_count) ? 1 : 0;
-    }
-    consumer_sync();
-    if (*S.flag) {
-        // Last chunk to finish for this (sequence, KV head): log-sum-exp combine.
-        // The group's partials are one contiguous [G][NC][d + 2] range: gather it
-        // into shared memory with independent loads (all in flight), then reduce.
-        float *co = reinterpret_cast<float *>(S.act);  // [G][NC][d]
-        float *cm = co + G * NC * d;                    // [G][NC] chunk maxima -> weights
-        float *cl = cm + G * NC;                        // [G][NC] chunk sums; cl[h*NC] <- 1 / L
-        const float *src = part + ((size_t)a.b * nq + a.g * G) * NC * (d + 2);
-        const int total = G * NC * (d + 2);
-        for (int i0 = 0; i0 < total; i0 += 16 * kConsumerThreads) {
-            float val[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int i = i0 + k * kConsumerThreads + t;
-                val[k] = i < total ? __ldcg(src + i) : 0.f;
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int i = i0 + k * kConsumerThreads + t;
-                if (i < total) {
-                    const int hc = i / (d + 2), e = i % (d + 2);
-                    if (e < d) co[hc * d + e] = val[k];
-                    else if (e == d) cm[hc] = val[k];
-                    else cl[hc] = val[k];
-                }
-            }
-        }
-        consumer_sync();
-        if (t < G) {  // per head: M = max_c m_c, w_c = 2^(m_c - M), L = sum_c w_c l_c
-            float M = -CUDART_INF_F;
-            for (int c = 0; c < NC; ++c) M = fmaxf(M, cm[t * NC + c]);
-            float L = 0.f;
-            for (int c = 0; c < NC; ++c) {
-                const float w = exp2f(cm[t * NC + c] - M);
-                cm[t * NC + c] = w;
-                L = fmaf(w, cl[t * NC + c], L);
-            }
-            cl[t * NC] = 1.0f / L;
-        }
-        consumer_sync();
-        const int ostride = P.o_nkb * P.o_kc;
-        for (int oi = t; oi < G * d; oi += kConsumerThreads) {
-            const int hh = oi / d, e = oi % d, hg = a.g * G + hh;
-            const float *ph = co + (size_t)hh * NC * d + e;
-            float acc = 0.f;
-            for (int c = 0; c < NC; ++c) acc = fmaf(cm[hh * NC + c], ph[(size_t)c * d], acc);
-            __stcg(P.attn + (size_t)a.b * ostride + hg * d + e, acc * cl[hh * NC]);
-        }
-        consumer_sync();
-        if (t == 0 && !(in.flags & F_DROP_SIGNAL)) red_release_add(P.counters + in.signal2_ctr, 1u);
-    }
+    // the partial is published with the CTA's batched counter signal; the
+    // O-projection combines the chunks
     return consumer_sync_or(*S.abort != 0);
 }
 
@@ -1022,11 +1047,12 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
             P.trace[8 * (size_t)i + 1] = globaltimer_ns();
         }
         if (in.op == OP_ATTN) {
-            stop = attn_instr(P, S, ring, in, gen, pos);
+            stop = attn_instr(P, S, ring, in, pos);
             act_tag = ~0ull;
         } else {
             gemv_instr<BS, WIDE>(P, S, ring, in, act_tag, gen, pos, q);
-            if (++q == reduce_slots(P.stages)) q = 0;
+        }
+        if (!stop) {
             if (in.op != OP_LMHEAD && !(in.flags & F_DROP_SIGNAL)) {
                 if (pend_ctr != in.signal_ctr) {
                     if (pend_n) {

@@ -103,14 +103,15 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     act = std::max(act, p.gu_bs * p.gu.nkb * p.gu.kc * 4);
     act = std::max(act, p.bs * down_blocks_per_range * p.down.kc * 4);
     const int G = nq / nkv;
-    // Split-KV chunks: as many units as fit one per CTA, so an attention phase
-    // is one unit deep.  The last unit of a (sequence, KV head) gathers every
-    // chunk's partial output [G][chunks][d] into shared memory.
+    // Split-KV chunks: as many units as fit one per CTA (an attention phase is
+    // one unit deep), at most kMaxAttnChunks per (sequence, KV head) since every
+    // O-projection CTA gathers all of a sequence's chunk partials.
     p.chunks = std::max(1, std::min(kMaxAttnChunks, n_ctas / (B * nkv)));
     p.chunks = std::min(p.chunks, std::max(1, c.max_seq / 16));
-    p.chunks = std::min(p.chunks, std::max(1, kActMax / (G * d * 4)));
-    int attn_scratch = G * d * 4 + 2 * d * 4 + kConsumerWarps * (d + 2) * 4;
-    attn_scratch = std::max(attn_scratch, G * p.chunks * d * 4 + 2 * G * p.chunks * 4);
+    const int attn_scratch = G * d * 4 + 2 * d * 4 + kConsumerWarps * (d + 2) * 4;
+    // the O-projection stages its input by combining every chunk's partial:
+    // fp32 [rows][nq*d] plus the per-(row, head, chunk) weights
+    act = std::max(act, p.bs * (p.o.nkb * p.o.kc + nq * p.chunks) * 4);
     act = std::max(act, attn_scratch);
     p.act_bytes = (int)align_up(act, 128);
     p.stages = kMaxStages;
@@ -118,30 +119,38 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
         --p.stages;
     if (p.stages < 2) return bad(MK_ERR_UNSUPPORTED, "not enough shared memory for the ring");
 
-    // Counters.
-    const int n_arr_att = L * B * nkv;
-    p.n_counters = 5 * L + n_arr_att + 1;
+    // Counters: five per layer (QKV, attention, O, gate/up, down), then the
+    // LM-head arrival counter.
+    p.n_counters = 5 * L + 1;
     if (p.n_counters >= kNoCounter) return bad(MK_ERR_UNSUPPORTED, "too many counters");
-    auto arr_att = [&](int l, int b, int g) { return 5 * L + (l * B + b) * nkv + g; };
-    const int arr_lm = 5 * L + n_arr_att;
+    const int arr_lm = 5 * L;
     p.counter_count.assign(p.n_counters, 0);
 
     // ---------------------------------------------------------- instructions per phase
     std::vector<std::vector<Instr>> phases;
     std::vector<std::vector<double>> costs;
+    // A GEMV phase is cut into runs of consecutive row tiles, about one run
+    // per CTA for every (K range, batch range) combination, so each CTA streams
+    // contiguous weights and pays the per-instruction cost once per run.
     auto gemv_phase = [&](uint8_t op, int l, const PackedMat &m, int bs, int ksplit, uint8_t flags, int wait,
                           int signal) {
         std::vector<Instr> v;
         std::vector<double> cost;
-        int per = (m.nkb + ksplit - 1) / ksplit;
-        for (int t = 0; t < m.tiles; ++t)
+        const int per = (m.nkb + ksplit - 1) / ksplit;
+        const int nk = (m.nkb + per - 1) / per, nbr = (B + bs - 1) / bs;
+        const int combos = nk * nbr;
+        const int runs = std::max(1, std::min(m.tiles, (n_ctas + combos - 1) / combos));
+        for (int r = 0; r < runs; ++r) {
+            const int t0 = (int)((long long)r * m.tiles / runs), t1 = (int)((long long)(r + 1) * m.tiles / runs);
+            if (t1 <= t0) continue;
             for (int kb = 0; kb < m.nkb; kb += per)
                 for (int b0 = 0; b0 < B; b0 += bs) {
                     Instr in{};
                     in.op = op;
                     in.flags = flags | (ksplit > 1 ? F_ATOMIC : 0);
                     in.layer = (uint16_t)l;
-                    in.tile = (uint32_t)t;
+                    in.tile = (uint32_t)t0;
+                    in.ntiles = (uint16_t)(t1 - t0);
                     in.kb0 = (uint16_t)kb;
                     in.kb1 = (uint16_t)std::min(m.nkb, kb + per);
                     in.b0 = (uint16_t)b0;
@@ -150,8 +159,9 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
                     in.signal_ctr = signal < 0 ? kNoCounter : (uint16_t)signal;
                     in.signal2_ctr = kNoCounter;
                     v.push_back(in);
-                    cost.push_back((double)(in.kb1 - in.kb0) * kTileRows * m.kc * 2 + 4096.0);
+                    cost.push_back((double)(t1 - t0) * (in.kb1 - in.kb0) * kTileRows * m.kc * 2 + 4096.0);
                 }
+        }
         if (signal >= 0) p.counter_count[signal] += (uint32_t)v.size();
         phases.push_back(v);
         costs.push_back(cost);
@@ -173,13 +183,12 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
                         in.b0 = (uint16_t)b;
                         in.nb = 1;
                         in.wait_ctr = (uint16_t)counter_qkv(l);
-                        in.signal_ctr = (uint16_t)arr_att(l, b, g);
-                        in.arrive_count = (uint32_t)p.chunks;
-                        in.signal2_ctr = (uint16_t)counter_att(l);
+                        in.signal_ctr = (uint16_t)counter_att(l);
+                        in.signal2_ctr = kNoCounter;
                         v.push_back(in);
                         cost.push_back(typical_ctx / p.chunks * d * 4 + 8192.0);
                     }
-            p.counter_count[counter_att(l)] += (uint32_t)(B * nkv);
+            p.counter_count[counter_att(l)] += (uint32_t)v.size();
             phases.push_back(v);
             costs.push_back(cost);
         }
@@ -262,7 +271,7 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     p.off_qkv = take((size_t)B * p.qkv_rows * 4);
     p.off_attn = take((size_t)B * p.o.nkb * p.o.kc * 4);
     p.off_act_a = take((size_t)B * p.i_pad * 4);
-    p.off_partials = take((size_t)B * nq * p.chunks * (d + 2) * 4);
+    p.off_partials = take((size_t)B * nq * p.chunks * partial_stride(d) * 4);
     p.off_lm_best = take((size_t)B * n_ctas * sizeof(LmBest));
     p.off_next_scratch = take((size_t)B * 4);
     p.off_norms = take((size_t)(L * (2 * H + 2 * d) + H) * 2);
@@ -308,7 +317,7 @@ mk_status validate_plan(const Plan &p, std::string &err) {
         if (in.layer >= c.n_layers) return fail("instruction layer out of range");
         if (in.b0 + in.nb > p.B || in.nb < 1) return fail("instruction batch range out of range");
         if (m) {
-            if (in.tile >= (uint32_t)m->tiles || in.kb0 >= in.kb1 || in.kb1 > m->nkb)
+            if (in.ntiles < 1 || in.tile + in.ntiles > (uint32_t)m->tiles || in.kb0 >= in.kb1 || in.kb1 > m->nkb)
                 return fail("GEMV instruction tile/K range out of range");
             if (in.nb > kMaxBatchRows) return fail("GEMV instruction carries too many batch rows");
             if ((size_t)in.nb * (in.kb1 - in.kb0) * m->kc * 4 > (size_t)p.act_bytes)
@@ -333,10 +342,9 @@ mk_status validate_plan(const Plan &p, std::string &err) {
             while (ptr[i] < p.cta_base[i + 1]) {
                 const Instr &in = p.instrs[ptr[i]];
                 if (in.wait_ctr != kNoCounter && ctr[in.wait_ctr] < in.wait_count) break;
-                if (in.op == OP_ATTN || in.op == OP_LMHEAD) {
-                    if (in.op == OP_ATTN || (in.flags & F_LAST_LM)) {
-                        uint32_t a = ++ctr[in.signal_ctr];
-                        if (a == in.arrive_count && in.signal2_ctr != kNoCounter) ++ctr[in.signal2_ctr];
+                if (in.op == OP_LMHEAD) {
+                    if (in.flags & F_LAST_LM) {
+                        const uint32_t a = ++ctr[in.signal_ctr];
                         if (a > in.arrive_count) return fail("more arrivals than expected");
                     }
                 } else if (in.signal_ctr != kNoCounter) {
@@ -364,7 +372,7 @@ mk_status validate_plan(const Plan &p, std::string &err) {
                      in.wait_ctr, ctr[in.wait_ctr], i, in.wait_count);
             return fail(buf);
         }
-        if ((in.op == OP_ATTN || (in.op == OP_LMHEAD && (in.flags & F_LAST_LM))) && ctr[in.signal_ctr] != in.arrive_count) {
+        if (in.op == OP_LMHEAD && (in.flags & F_LAST_LM) && ctr[in.signal_ctr] != in.arrive_count) {
             snprintf(buf, sizeof buf, "arrival counter %d gets %u arrivals, expected %u", in.signal_ctr,
                      ctr[in.signal_ctr], in.arrive_count);
             return fail(buf);
