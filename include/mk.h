@@ -180,8 +180,8 @@ mk_status mk_debug_drop_signal(mk_ctx *ctx, int instr);
  * instruction; see mk_schedule_info).  For instruction i of the flattened
  * schedule, entries [8i..8i+7] receive, in %globaltimer nanoseconds: when its
  * CTA starts it, when its dependency wait is satisfied, when it is done, when
- * the producer issued its first copy (0 if it streams nothing), the time the
- * consumer spent waiting for ring data, the time the producer spent waiting
+ * the producer issued its first copy (0 if it streams nothing), the SM clock
+ * cycles the consumer spent waiting for ring data, the time the producer spent waiting
  * for a free ring slot, and when the producer issued its last copy.  Each step
  * overwrites the buffer.  NULL turns tracing off.  MK_ERR_INVALID if the
  * buffer is too small. */

@@ -62,7 +62,7 @@ class Plan:
         n = self.info()["n_instructions"]
         dt = np.dtype([("op", "u1"), ("flags", "u1"), ("layer", "<u2"), ("tile", "<u4"), ("kb0", "<u2"),
                        ("kb1", "<u2"), ("b0", "<u2"), ("nb", "<u2"), ("wait_ctr", "<u2"), ("signal_ctr", "<u2"),
-                       ("wait_count", "<u4"), ("signal2_ctr", "<u2"), ("pad0", "<u2"), ("arrive_count", "<u4")])
+                       ("wait_count", "<u4"), ("signal2_ctr", "<u2"), ("ntiles", "<u2"), ("arrive_count", "<u4")])
         arr = np.zeros(n, dt)
         base = np.zeros(self.info()["n_ctas"] + 1, np.int32)
         check(self.lib.mk_get_schedule(self.ctx, C.c_void_p(arr.ctypes.data), arr.nbytes,

@@ -248,6 +248,7 @@ static KParams make_params(mk_ctx *c, const int32_t *tokens, int64_t tok_stride,
     P.gu_kc = p.gu.kc; P.gu_nkb = p.gu.nkb;
     P.down_kc = p.down.kc; P.down_nkb = p.down.nkb;
     P.lm_kc = p.lm.kc; P.lm_nkb = p.lm.nkb;
+    P.qkv_rt = p.qkv.rows; P.o_rt = p.o.rows; P.gu_rt = p.gu.rows; P.down_rt = p.down.rows; P.lm_rt = p.lm.rows;
     return P;
 }
 
@@ -306,19 +307,19 @@ mk_status mk_load_weights(mk_ctx *c, const mk_weights *w, void *workspace, void 
             !w->attn_norm[l] || !w->mlp_norm[l] || (g.qk_norm && (!w->q_norm[l] || !w->k_norm[l])))
             return fail(c, MK_ERR_INVALID, "mk_load_weights: null per-layer pointer");
         uint8_t *base = c->ws + p.off_weights + (size_t)l * p.layer_weight_bytes;
-        // QKV: concatenate q, k, v rows into a staging area of the packed region? Pack each source
-        // separately into its row range: rows of q, k and v are tile-aligned because (nq, nkv) * d
-        // are multiples of 8.
+        // QKV: q, k and v rows packed into consecutive tile ranges (each count
+        // is a multiple of the tile height)
         const int nqd = g.n_heads * d, nkd = g.n_kv_heads * d;
-        const size_t tile_bytes = (size_t)p.qkv.nkb * kTileRows * p.qkv.kc * 2;
-        CK(launch_pack(w->wq[l], nullptr, base + p.qkv.offset, nqd, H, p.qkv.kc, p.qkv.nkb, nqd / kTileRows, 0, s));
-        CK(launch_pack(w->wk[l], nullptr, base + p.qkv.offset + tile_bytes * (nqd / kTileRows), nkd, H, p.qkv.kc,
-                       p.qkv.nkb, nkd / kTileRows, 0, s));
-        CK(launch_pack(w->wv[l], nullptr, base + p.qkv.offset + tile_bytes * ((nqd + nkd) / kTileRows), nkd, H,
-                       p.qkv.kc, p.qkv.nkb, nkd / kTileRows, 0, s));
-        CK(launch_pack(w->wo[l], nullptr, base + p.o.offset, H, nqd, p.o.kc, p.o.nkb, p.o.tiles, 0, s));
-        CK(launch_pack(w->wg[l], w->wu[l], base + p.gu.offset, I, H, p.gu.kc, p.gu.nkb, p.gu.tiles, 1, s));
-        CK(launch_pack(w->wd[l], nullptr, base + p.down.offset, H, I, p.down.kc, p.down.nkb, p.down.tiles, 0, s));
+        const PackedMat &Q = p.qkv;
+        const size_t tile_bytes = (size_t)Q.nkb * Q.rows * Q.kc * 2;
+        CK(launch_pack(w->wq[l], nullptr, base + Q.offset, nqd, H, Q.kc, Q.nkb, nqd / Q.rows, Q.rows, 0, s));
+        CK(launch_pack(w->wk[l], nullptr, base + Q.offset + tile_bytes * (nqd / Q.rows), nkd, H, Q.kc, Q.nkb,
+                       nkd / Q.rows, Q.rows, 0, s));
+        CK(launch_pack(w->wv[l], nullptr, base + Q.offset + tile_bytes * ((nqd + nkd) / Q.rows), nkd, H, Q.kc, Q.nkb,
+                       nkd / Q.rows, Q.rows, 0, s));
+        CK(launch_pack(w->wo[l], nullptr, base + p.o.offset, H, nqd, p.o.kc, p.o.nkb, p.o.tiles, p.o.rows, 0, s));
+        CK(launch_pack(w->wg[l], w->wu[l], base + p.gu.offset, I, H, p.gu.kc, p.gu.nkb, p.gu.tiles, p.gu.rows, 1, s));
+        CK(launch_pack(w->wd[l], nullptr, base + p.down.offset, H, I, p.down.kc, p.down.nkb, p.down.tiles, p.down.rows, 0, s));
         uint8_t *nl = norms + (size_t)l * (2 * H + 2 * d) * 2;
         CK(cudaMemcpyAsync(nl, w->attn_norm[l], (size_t)H * 2, cudaMemcpyDeviceToDevice, s));
         CK(cudaMemcpyAsync(nl + (size_t)H * 2, w->mlp_norm[l], (size_t)H * 2, cudaMemcpyDeviceToDevice, s));
@@ -336,7 +337,7 @@ mk_status mk_load_weights(mk_ctx *c, const mk_weights *w, void *workspace, void 
         lw[l].k_norm = g.qk_norm ? nl + (size_t)4 * H + 2 * d : nullptr;
     }
     const void *head = g.tied_embeddings ? w->embed : w->lm_head;
-    CK(launch_pack(head, nullptr, c->ws + p.lm.offset, g.vocab, H, p.lm.kc, p.lm.nkb, p.lm.tiles, 0, s));
+    CK(launch_pack(head, nullptr, c->ws + p.lm.offset, g.vocab, H, p.lm.kc, p.lm.nkb, p.lm.tiles, p.lm.rows, 0, s));
     CK(cudaMemcpyAsync(norms + (size_t)L * (2 * H + 2 * d) * 2, w->final_norm, (size_t)H * 2,
                        cudaMemcpyDeviceToDevice, s));
     CK(cudaMemcpyAsync(c->ws + p.off_layers, lw.data(), lw.size() * sizeof(LayerW), cudaMemcpyHostToDevice, s));
@@ -364,7 +365,17 @@ static mk_status launch_megakernel(mk_ctx *c, const int32_t *tok, int64_t stride
     P.cta_end = ranges + p.n_ctas;
     P.use_waits = 1;
     P.pdl = 0;
-    CK(launch_step(P, p.bs, p.n_ctas, s, true, false));
+    cudaError_t e = launch_step(P, p.bs, p.n_ctas, s, true, false);
+    if (e != cudaSuccess) {
+        int per_sm = -1;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel_func(P), kThreads, smem_bytes(P));
+        cudaFuncAttributes fa{};
+        cudaFuncGetAttributes(&fa, step_kernel_func(P));
+        char buf[256];
+        snprintf(buf, sizeof buf, "megakernel launch: %s (occupancy %d CTA/SM at %d threads, %d B smem, %d regs, max %d threads)",
+                 cudaGetErrorString(e), per_sm, kThreads, smem_bytes(P), fa.numRegs, fa.maxThreadsPerBlock);
+        return fail(c, MK_ERR_CUDA, buf);
+    }
     return MK_OK;
 }
 

@@ -12,20 +12,16 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;   // 256
 constexpr int kThreads = kConsumerThreads + 32;         // + one producer warp
 constexpr int kStageBytes = 32768;                      // one ring slot
 constexpr int kMaxStages = 8;
-constexpr int kTileRows = 8;                            // weight rows per GEMV tile
-constexpr int kMaxBatchRows = 8;                        // batch rows one GEMV instruction carries
+constexpr int kMaxTileRows = 8;                         // weight rows per GEMV tile (fewer for long rows)
+constexpr int kMaxBatchRows = 4;                        // batch rows one GEMV instruction carries
 constexpr int kMaxSmem = 232448;                        // opt-in dynamic smem per CTA on sm_100
 // shared memory after the ring and the activations: barriers, flags, two reduction buffers
 // Batch rows of the kernel instance that runs a plan carrying `bs` rows per
-// instruction (instances exist for 1, 2, 4 and 8).
-constexpr int kernel_bs(int bs) { return bs <= 1 ? 1 : (bs <= 2 ? 2 : (bs <= 4 ? 4 : 8)); }
-// Rotating reduction slots per CTA: a warp can run at most `stages` ring blocks
-// (so at most `stages` instructions) ahead of another, so stages + 2 slots
-// never hand a slot to a new instruction while an older one still uses it.
-constexpr int reduce_slots(int stages) { return stages + 2; }
-// Bytes after the ring and the activation region: barriers, flags and small
-// arrays and the RoPE table (2048 B), then the per-warp partial sums [slots][8 warps][8 rows][bs].
-constexpr int misc_bytes(int bs, int stages) { return 2048 + reduce_slots(stages) * 256 * kernel_bs(bs); }
+// instruction (instances exist for 1, 2 and 4).
+constexpr int kernel_bs(int bs) { return bs <= 1 ? 1 : (bs <= 2 ? 2 : 4); }
+// Bytes after the ring and the activation region: barriers, flags, small
+// arrays and the RoPE table.
+constexpr int misc_bytes(int bs, int stages) { return 2560 + 0 * bs * stages; }
 constexpr int kMaxAttnChunks = 16;  // split-KV chunks per (sequence, KV head); the O-projection gathers them all
 // Floats per split-KV partial record: o[d], m, l, padding to a 16-byte multiple.
 constexpr int partial_stride(int head_dim) { return head_dim + 4; }
@@ -66,16 +62,17 @@ struct Instr {
 };
 static_assert(sizeof(Instr) == 32, "Instr must be 32 bytes");
 
-// A weight matrix repacked into tiles of kTileRows rows x kc columns; the
+// A weight matrix repacked into tiles of `rows` rows x kc columns; the
 // (tile, kblock) blocks are contiguous, kblock fastest, each block row-major.
+// rows * kc * 2 <= 32 KB: one block fills at most one ring slot.
 struct PackedMat {
     uint64_t offset;   // byte offset in the workspace
     int32_t n_rows;    // logical rows (N)
     int32_t k;         // logical columns (K)
-    int32_t kc;        // block width (columns)
+    int32_t kc;        // block width (columns, a multiple of 256)
     int32_t nkb;       // blocks along K
     int32_t tiles;     // row tiles
-    int32_t pad;
+    int32_t rows;      // rows per tile (1, 2, 4 or 8)
 };
 
 // Per-layer device pointers (in the workspace; filled by the host after packing).
@@ -137,6 +134,7 @@ struct KParams {
     int32_t qkv_rows, i_pad, chunks, n_ctas, stages, act_bytes, qk_norm, bs;
     float rms_eps;
     int32_t qkv_kc, qkv_nkb, o_kc, o_nkb, gu_kc, gu_nkb, down_kc, down_nkb, lm_kc, lm_nkb;
+    int32_t qkv_rt, o_rt, gu_rt, down_rt, lm_rt;  // rows per tile
     int32_t use_waits;          // 0 in the separate-kernels variant (kernel boundaries order the ops)
     int32_t pdl;                // 1: wait on the previous grid before reading activations
     unsigned long long *trace;  // [n_instr][8] globaltimer stamps and waits, or null

@@ -33,10 +33,9 @@ struct SmemLayout {
     volatile int *flag;
     float *rstd;              // [8] RMSNorm scale per batch row
     float *mlc;               // [24] attention m, l, correction per head
-    float *ssq;               // [8 warps][8] sums of squares
+    volatile uint32_t *seq;   // [kMaxStages] ring block index each slot currently holds
+    float *ssq;               // [consumer warps][8] sums of squares
     unsigned long long *best; // [64] argmax keys per batch row
-    int *rcnt;                // [slots][8] warps that delivered each output
-    float *rsum;              // [slots][8 warps][8 rows][bs] per-warp partial dot products
     double *rope;             // [64] RoPE inverse frequencies theta^(-2i/d)
 };
 
@@ -51,11 +50,10 @@ __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &
     S.flag = reinterpret_cast<volatile int *>(misc + 132);
     S.rstd = reinterpret_cast<float *>(misc + 160);
     S.mlc = reinterpret_cast<float *>(misc + 192);
-    S.ssq = reinterpret_cast<float *>(misc + 320);
-    S.best = reinterpret_cast<unsigned long long *>(misc + 576);
-    S.rcnt = reinterpret_cast<int *>(misc + 1088);
-    S.rope = reinterpret_cast<double *>(misc + 1536);
-    S.rsum = reinterpret_cast<float *>(misc + 2048);
+    S.seq = reinterpret_cast<volatile uint32_t *>(misc + 384);  // 8 words
+    S.best = reinterpret_cast<unsigned long long *>(misc + 512);
+    S.ssq = reinterpret_cast<float *>(misc + 1024);   // [16 warps][8]
+    S.rope = reinterpret_cast<double *>(misc + 2048); // [64]
     return S;
 }
 
@@ -139,18 +137,18 @@ __device__ __forceinline__ int token_of(const KParams &P, int b) {
 
 struct MatRef {
     const uint8_t *base;
-    int kc, nkb;
+    int kc, nkb, rows;
 };
 
 __device__ __forceinline__ MatRef mat_of(const KParams &P, const Instr &in) {
     MatRef m;
     const LayerW *L = P.layers + in.layer;
     switch (in.op) {
-        case OP_QKV: m.base = (const uint8_t *)L->qkv; m.kc = P.qkv_kc; m.nkb = P.qkv_nkb; break;
-        case OP_OPROJ: m.base = (const uint8_t *)L->o; m.kc = P.o_kc; m.nkb = P.o_nkb; break;
-        case OP_GATEUP: m.base = (const uint8_t *)L->gu; m.kc = P.gu_kc; m.nkb = P.gu_nkb; break;
-        case OP_DOWN: m.base = (const uint8_t *)L->down; m.kc = P.down_kc; m.nkb = P.down_nkb; break;
-        default: m.base = (const uint8_t *)P.lm_w; m.kc = P.lm_kc; m.nkb = P.lm_nkb; break;
+        case OP_QKV: m.base = (const uint8_t *)L->qkv; m.kc = P.qkv_kc; m.nkb = P.qkv_nkb; m.rows = P.qkv_rt; break;
+        case OP_OPROJ: m.base = (const uint8_t *)L->o; m.kc = P.o_kc; m.nkb = P.o_nkb; m.rows = P.o_rt; break;
+        case OP_GATEUP: m.base = (const uint8_t *)L->gu; m.kc = P.gu_kc; m.nkb = P.gu_nkb; m.rows = P.gu_rt; break;
+        case OP_DOWN: m.base = (const uint8_t *)L->down; m.kc = P.down_kc; m.nkb = P.down_nkb; m.rows = P.down_rt; break;
+        default: m.base = (const uint8_t *)P.lm_w; m.kc = P.lm_kc; m.nkb = P.lm_nkb; m.rows = P.lm_rt; break;
     }
     return m;
 }
@@ -234,7 +232,7 @@ __device__ __forceinline__ void cursor_block(const KParams &P, const BlockCursor
         src2 = P.vcache + kv_off(P, c.in.layer, c.a.b, c.a.g, p);
     } else {
         const int nkr = c.in.kb1 - c.in.kb0;  // blocks of one tile in this run
-        bytes = (uint32_t)(kTileRows * c.m.kc * 2);
+        bytes = (uint32_t)(c.m.rows * c.m.kc * 2);
         src1 = c.m.base + ((size_t)(c.in.tile + c.j / nkr) * c.m.nkb + c.in.kb0 + c.j % nkr) * bytes;
         src2 = nullptr;
     }
@@ -247,7 +245,7 @@ __device__ void producer(const KParams &P, const SmemLayout &S, int begin, int e
     const uint64_t pol = policy_evict_first();
     const uint64_t pol_pf = policy_evict_normal();
     int slot = 0;
-    uint32_t phase = 0, issued = 0, issued_par = 0;
+    uint32_t phase = 0, issued = 0, issued_par = 0, bi = 0;
     const uint64_t limit = 2ull * P.timeout_ns + 1000000ull;
     bool ok = true;
     BlockCursor cur{begin, end, 0, 0}, pf{begin, end, 0, 0};
@@ -276,6 +274,7 @@ __device__ void producer(const KParams &P, const SmemLayout &S, int begin, int e
             if (cur.j == 0) P.trace[8 * (size_t)cur.i + 3] = globaltimer_ns();
         }
         uint8_t *dst = S.ring + (size_t)slot * kStageBytes;
+        S.seq[slot] = bi++;  // the slot is free: announce which block it will hold
         mbar_arrive_expect_tx(&S.full[slot], s2 ? 2u * bytes : bytes);
         bulk_g2s(dst, s1, bytes, &S.full[slot], pol);
         if (s2) bulk_g2s(dst + kStageBytes / 2, s2, bytes, &S.full[slot], pol);
@@ -312,33 +311,48 @@ __device__ void producer(const KParams &P, const SmemLayout &S, int begin, int e
         }
 }
 
-// ------------------------------------------------------------------ consumer ring cursor
+// ------------------------------------------------------------------ consumer side of the ring
+// Blocks are numbered per CTA in the order the producer loads them; block bi
+// sits in slot bi % stages during its (bi / stages)-th use of that slot.
 struct CRing {
-    int slot;
-    uint32_t phase;
-    unsigned long long waited;  // ns spent waiting for ring data (thread 0, tracing only)
+    unsigned long long waited;  // SM cycles spent waiting for ring data (thread 0, tracing only)
 };
 
-__device__ __forceinline__ const uint8_t *c_wait(const KParams &P, const SmemLayout &S, CRing &r) {
-    if (P.trace && threadIdx.x == 0 && !mbar_try_wait(&S.full[r.slot], r.phase)) {
-        const unsigned long long w0 = globaltimer_ns();
-        wait_bar(P, &S.full[r.slot], r.phase, S.abort, P.timeout_ns);
-        r.waited += globaltimer_ns() - w0;
+// Wait until block bi is in shared memory.  Warps consume blocks out of
+// order (each GEMV tile belongs to one warp), so a warp may reach slot s for
+// use u while s is still on use u - 1; the parity of u then matches the long
+// completed use u - 2.  So first wait until the producer has stamped the slot
+// with bi (it does so only after use u - 1 was released, i.e. its data phase
+// completed), and only then test the phase parity.
+__device__ __forceinline__ const uint8_t *ring_wait(const KParams &P, const SmemLayout &S, CRing &r, uint32_t bi) {
+    const uint32_t slot = bi % (uint32_t)P.stages, par = (bi / (uint32_t)P.stages) & 1u;
+    const long long c0 = (P.trace && threadIdx.x == 0) ? clock64() : 0;
+    bool ok = true;
+    if (S.seq[slot] != bi) {
+        uint64_t t0 = 0;
+        for (uint32_t it = 1; S.seq[slot] != bi; ++it) {
+            __nanosleep(20);
+            if ((it & 15u) == 0u) {
+                if (*S.abort) { ok = false; break; }
+                const uint64_t now = globaltimer_ns();
+                if (t0 == 0) t0 = now;
+                else if (now - t0 > P.timeout_ns) { ok = false; break; }
+            }
+        }
     }
-    if (!wait_bar(P, &S.full[r.slot], r.phase, S.abort, P.timeout_ns)) {
-        if (!*S.abort) set_error(P, 2u, blockIdx.x, 0u);
+    if (!ok || !wait_bar(P, &S.full[slot], par, S.abort, P.timeout_ns)) {
+        if (!*S.abort) set_error(P, 2u, blockIdx.x, bi);
         *S.abort = 1;
     }
-    return S.ring + (size_t)r.slot * kStageBytes;
+    if (P.trace && threadIdx.x == 0) r.waited += (unsigned long long)(clock64() - c0);
+    return S.ring + (size_t)slot * kStageBytes;
 }
 
-__device__ __forceinline__ void c_release(const KParams &P, const SmemLayout &S, CRing &r) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(&S.empty[r.slot]);
-    if (++r.slot == P.stages) {
-        r.slot = 0;
-        r.phase ^= 1u;
-    }
+// Hand block bi's slot back to the producer.  A slot is free once it has
+// kConsumerWarps arrivals: every warp arrives once for a block they all read
+// (attention), the one consuming warp arrives for all of them (GEMV tiles).
+__device__ __forceinline__ void ring_release(const SmemLayout &S, const KParams &P, uint32_t bi, uint32_t count) {
+    mbar_arrive_cnt(&S.empty[bi % (uint32_t)P.stages], count);
 }
 
 // ------------------------------------------------------------------ activation staging
@@ -506,47 +520,13 @@ __device__ __forceinline__ void stage_act(const KParams &P, const SmemLayout &S,
     }
 }
 
-// ------------------------------------------------------------------ GEMV over ring blocks
-// Block = kTileRows rows x KC columns (CB = KC/8 chunks of 8).  Thread t owns
-// chunk c = t % CB and rows rg + NRG*i (rg = t / CB), so one activation chunk
-// load serves RPT rows; fp32 accumulation across all K blocks of the tile.
-template <int BS, int RPT>
-__device__ __forceinline__ void gemv_blocks(const KParams &P, const SmemLayout &S, CRing &ring, const float *act,
-                                            int klen, int nb, int nblocks, float (&acc)[8][BS]) {
-    constexpr int CB = RPT * 32;
-    constexpr int NRG = 8 / RPT;
-    constexpr int KC = CB * 8;
-    const int t = threadIdx.x;
-    const int c = t % CB, rg = t / CB;
-    for (int j = 0; j < nblocks; ++j) {
-        const uint8_t *blk = c_wait(P, S, ring);
-        float af[BS][8];
-#pragma unroll
-        for (int b = 0; b < BS; ++b) {
-            if (b < nb) {
-                const float4 *a4 = reinterpret_cast<const float4 *>(act + (size_t)b * klen + j * KC + c * 8);
-                const float4 x0 = a4[0], x1 = a4[1];
-                af[b][0] = x0.x; af[b][1] = x0.y; af[b][2] = x0.z; af[b][3] = x0.w;
-                af[b][4] = x1.x; af[b][5] = x1.y; af[b][6] = x1.z; af[b][7] = x1.w;
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) af[b][q] = 0.f;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-            const int r = rg + NRG * i;
-            const uint4 w = *reinterpret_cast<const uint4 *>(blk + ((size_t)r * KC + c * 8) * 2);
-            float wf[8];
-            unpack8(w, wf);
-#pragma unroll
-            for (int b = 0; b < BS; ++b)
-#pragma unroll
-                for (int q = 0; q < 8; ++q) acc[i][b] = fmaf(wf[q], af[b][q], acc[i][b]);
-        }
-        c_release(P, S, ring);
-    }
-}
+// ------------------------------------------------------------------ GEMV: one warp per tile
+// A tile is RT rows x (nkr blocks of kc columns) of one matrix, one ring slot
+// per block.  Lane l owns columns c*256 + l*8 .. +8 of every block (kc/256
+// chunks), accumulates RT x BS fp32 dot products, then the warp folds the RT
+// rows across its lanes (log2(RT) halving steps, then butterflies) and the
+// lanes holding a row's total run its epilogue.  No other warp takes part, so
+// warps never wait for each other on GEMV work.
 
 // Fold N per-lane values across lanes `o` apart: each lane keeps half of them
 // (the upper half when its `o` bit is set), added to its partner's copy.
@@ -577,128 +557,125 @@ __device__ __forceinline__ float key_value(unsigned long long k) {
 }
 __device__ __forceinline__ int key_index(unsigned long long k) { return (int)(0xFFFFFFFFu - (uint32_t)k); }
 
-// Epilogue of one finished output (tile row r, or gate/up pair r) for all
-// batch rows: v0 = the row's dot products, v1 = the up row's for gate/up.
-template <int BS>
-__device__ void gemv_epilogue(const KParams &P, const SmemLayout &S, const Instr &in, int tile, int r,
-                              const float (&v0)[BS], const float (&v1)[BS]) {
-    const int H = P.hidden, nb = in.nb;
-    switch (in.op) {
-        case OP_QKV: {
-            const int n = tile * 8 + r;
-            if (n < P.qkv_rows)
+template <int BS, int RT>
+__device__ __forceinline__ void gemv_warp_tile(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
+                                               const MatRef &m, int tile, uint32_t bi0, int klen) {
+    const int lane = threadIdx.x & 31;
+    const int nkr = in.kb1 - in.kb0, kc = m.kc, nch = kc / 256, nb = in.nb;
+    const float *act = reinterpret_cast<const float *>(S.act);
+    float acc[RT][BS];
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int b = 0; b < BS; ++b) acc[r][b] = 0.f;
+    for (int j = 0; j < nkr; ++j) {
+        const uint8_t *blk = ring_wait(P, S, ring, bi0 + j);
+        for (int c = 0; c < nch; ++c) {
+            const int col = c * 256 + lane * 8;
+            float af[BS][8];
+#pragma unroll
+            for (int b = 0; b < BS; ++b) {
+                if (b < nb) {
+                    const float4 *a4 = reinterpret_cast<const float4 *>(act + (size_t)b * klen + j * kc + col);
+                    const float4 x0 = a4[0], x1 = a4[1];
+                    af[b][0] = x0.x; af[b][1] = x0.y; af[b][2] = x0.z; af[b][3] = x0.w;
+                    af[b][4] = x1.x; af[b][5] = x1.y; af[b][6] = x1.z; af[b][7] = x1.w;
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) af[b][q] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RT; ++r) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(blk + ((size_t)r * kc + col) * 2);
+                float wf[8];
+                unpack8(w, wf);
 #pragma unroll
                 for (int b = 0; b < BS; ++b)
-                    if (b < nb) __stcg(P.qkv + (size_t)(in.b0 + b) * P.qkv_rows + n, v0[b]);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) acc[r][b] = fmaf(wf[q], af[b][q], acc[r][b]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) ring_release(S, P, bi0 + j, kConsumerWarps);
+    }
+    float v[BS];
+#pragma unroll
+    for (int b = 0; b < BS; ++b) {
+        float w[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) w[r] = r < RT ? acc[r < RT ? r : 0][b] : 0.f;
+        int o = 16;
+        if constexpr (RT >= 8) { fold_rows<8>(w, lane, o); o >>= 1; }
+        if constexpr (RT >= 4) { fold_rows<4>(w, lane, o); o >>= 1; }
+        if constexpr (RT >= 2) { fold_rows<2>(w, lane, o); o >>= 1; }
+        for (; o >= 1; o >>= 1) w[0] += __shfl_xor_sync(0xFFFFFFFFu, w[0], o);
+        v[b] = w[0];
+    }
+    // row held by this lane: bit 4 is the top row bit, then bits 3, 2
+    int fr = 0;
+    if constexpr (RT == 8) fr = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+    if constexpr (RT == 4) fr = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+    if constexpr (RT == 2) fr = (lane >> 4) & 1;
+    const bool holder = (lane & (32 / RT - 1)) == 0;
+    const int H = P.hidden;
+    switch (in.op) {
+        case OP_QKV: {
+            const int n = tile * RT + fr;
+            if (holder && n < P.qkv_rows)
+#pragma unroll
+                for (int b = 0; b < BS; ++b)
+                    if (b < nb) __stcg(P.qkv + (size_t)(in.b0 + b) * P.qkv_rows + n, v[b]);
         } break;
         case OP_OPROJ:
         case OP_DOWN: {
-            const int n = tile * 8 + r;
-            if (n < H)
+            const int n = tile * RT + fr;
+            if (holder && n < H)
 #pragma unroll
                 for (int b = 0; b < BS; ++b) {
                     if (b >= nb) break;
                     const int row = in.b0 + b;
                     float *xp = P.x + (size_t)row * H + n;
                     if (in.flags & F_ATOMIC) {
-                        atomicAdd(xp, v0[b]);
+                        atomicAdd(xp, v[b]);
                     } else {
                         const float base =
                             (in.flags & F_EMBED_X)
                                 ? bf2f(reinterpret_cast<const uint16_t *>(P.embed)[(size_t)token_of(P, row) * H + n])
                                 : __ldcg(xp);
-                        __stcg(xp, base + v0[b]);
+                        __stcg(xp, base + v[b]);
                     }
                 }
         } break;
         case OP_GATEUP: {
-            const int j = tile * 4 + r;
-            if (j < P.intermediate)
+            // gate rows 0..RT/2-1, up rows RT/2..RT-1: the up partner is lane ^ 16
+            float up[BS];
+#pragma unroll
+            for (int b = 0; b < BS; ++b) up[b] = __shfl_xor_sync(0xFFFFFFFFu, v[b], 16);
+            const int j = tile * (RT / 2) + fr;
+            if (RT >= 2 && holder && (lane & 16) == 0 && j < P.intermediate)
 #pragma unroll
                 for (int b = 0; b < BS; ++b)
                     if (b < nb)
-                        __stcg(P.act_a + (size_t)(in.b0 + b) * P.i_pad + j, v0[b] / (1.0f + __expf(-v0[b])) * v1[b]);
+                        __stcg(P.act_a + (size_t)(in.b0 + b) * P.i_pad + j, v[b] / (1.0f + __expf(-v[b])) * up[b]);
         } break;
-        default: {  // OP_LMHEAD
-            const int n = tile * 8 + r;
-            if (n < P.vocab)
+        default: {  // OP_LMHEAD: logits, then the warp's best of this tile folded into the CTA's
+            const int n = tile * RT + fr;
+            const bool valid = holder && n < P.vocab;
 #pragma unroll
-                for (int b = 0; b < BS; ++b) {
-                    if (b >= nb) break;
-                    if (P.logits) __stcg(P.logits + (size_t)(in.b0 + b) * P.vocab + n, v0[b]);
-                    atomicMax(S.best + in.b0 + b, argmax_key(v0[b], n));
+            for (int b = 0; b < BS; ++b) {
+                if (b >= nb) break;
+                if (valid && P.logits) __stcg(P.logits + (size_t)(in.b0 + b) * P.vocab + n, v[b]);
+                unsigned long long key = valid ? argmax_key(v[b], n) : 0ull;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, key, o);
+                    key = other > key ? other : key;
                 }
+                if (lane == 0) atomicMax(S.best + in.b0 + b, key);
+            }
         } break;
     }
-}
-
-// One GEMV tile.  No CTA-wide barrier on the common path: each warp folds its
-// row partials and stores them in its own entries of rotating slot q; the
-// warp whose store completes a row (or gate/up pair), counted with a
-// shared-memory atomic, adds the row's partials in fixed warp order -- so the
-// result does not depend on which warp came last -- and runs the epilogue.
-// Warps run ahead of each other by at most the ring depth, fewer instructions
-// than there are slots.
-template <int BS, int RPT>
-__device__ __forceinline__ void gemv_tile(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                          const MatRef &m, int tile, int nblocks, int klen, int q) {
-    constexpr int NRG = 8 / RPT;
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    float acc[8][BS];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int b = 0; b < BS; ++b) acc[i][b] = 0.f;
-    gemv_blocks<BS, RPT>(P, S, ring, reinterpret_cast<const float *>(S.act), klen, in.nb, nblocks, acc);
-    // warp sums of the RPT rows: log2(RPT) folding steps, then plain butterflies
-    float v[BS];
-#pragma unroll
-    for (int b = 0; b < BS; ++b) {
-        float w[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = acc[i][b];
-        int o = 16;
-        if constexpr (RPT >= 8) { fold_rows<8>(w, lane, o); o >>= 1; }
-        if constexpr (RPT >= 4) { fold_rows<4>(w, lane, o); o >>= 1; }
-        if constexpr (RPT >= 2) { fold_rows<2>(w, lane, o); o >>= 1; }
-        for (; o >= 1; o >>= 1) w[0] += __shfl_xor_sync(0xFFFFFFFFu, w[0], o);
-        v[b] = w[0];
-    }
-    int fi = 0;
-    if constexpr (RPT == 8) fi = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-    if constexpr (RPT == 4) fi = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-    if constexpr (RPT == 2) fi = (lane >> 4) & 1;
-    if ((lane & (32 / RPT - 1)) != 0) return;
-    const int rg = warp / RPT;
-    const int r = rg + NRG * fi;  // the tile row whose warp sum this lane holds
-    float *part = S.rsum + (size_t)q * 64 * BS;  // [warp][row][b]
-    volatile float *vpart = part;
-#pragma unroll
-    for (int b = 0; b < BS; ++b) vpart[(warp * 8 + r) * BS + b] = v[b];
-    __threadfence_block();
-    const bool pair = in.op == OP_GATEUP;
-    const int ci = pair ? (r & 3) : r;
-    int *cnt = S.rcnt + q * 8;
-    if (atomicAdd(cnt + ci, 1) != (pair ? 2 * RPT : RPT) - 1) return;
-    __threadfence_block();
-    cnt[ci] = 0;
-    const int r0 = ci;
-    float v0[BS], v1[BS];
-#pragma unroll
-    for (int b = 0; b < BS; ++b) {
-        v0[b] = 0.f;
-        v1[b] = 0.f;
-    }
-    // row x was delivered by the RPT warps of its row group x % NRG, in warp order
-    const int w0 = (r0 % NRG) * RPT, w1 = ((r0 + 4) % NRG) * RPT;
-#pragma unroll
-    for (int k = 0; k < RPT; ++k)
-#pragma unroll
-        for (int b = 0; b < BS; ++b) {
-            v0[b] += vpart[((w0 + k) * 8 + r0) * BS + b];
-            if (pair) v1[b] += vpart[((w1 + k) * 8 + r0 + 4) * BS + b];
-        }
-    gemv_epilogue<BS>(P, S, in, tile, r0, v0, v1);
 }
 
 // Publish this CTA's best (value, index) per sequence; the last CTA to do so
@@ -744,13 +721,15 @@ __device__ __forceinline__ void lm_publish(const KParams &P, const SmemLayout &S
     }
 }
 
-// One GEMV instruction.  WIDE: every matrix of the plan uses 2048-column
-// blocks, so only that tile shape is compiled into the hot loop.
-template <int BS, bool WIDE>
+// One GEMV instruction: a run of consecutive tiles.  Tile k goes to warp
+// (tc + k) % warps (tc counts this CTA's tiles so far) and uses ring blocks
+// bc + k*nkr .. bc + (k+1)*nkr - 1 (bc counts this CTA's ring blocks so far).
+template <int BS>
 __device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                           uint64_t &act_tag, uint32_t gen, int pos, int &q) {
+                                           uint64_t &act_tag, uint32_t gen, int pos, uint32_t &bc, uint32_t &tc) {
+    const int warp = threadIdx.x >> 5;
     const MatRef m = mat_of(P, in);
-    const int nblocks = in.kb1 - in.kb0, klen = nblocks * m.kc;
+    const int nkr = in.kb1 - in.kb0, klen = nkr * m.kc;
     const uint64_t tag = ((uint64_t)in.op << 56) | ((uint64_t)in.layer << 40) | ((uint64_t)in.b0 << 24) |
                          ((uint64_t)in.kb0 << 12) | (uint64_t)in.kb1;
     if (tag != act_tag) {
@@ -759,21 +738,18 @@ __device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S
         act_tag = tag;
         consumer_sync();
     }
-    const int nslots = reduce_slots(P.stages);
-    for (int k = 0; k < (int)in.ntiles; ++k) {
-        const int tile = (int)in.tile + k;
-        if constexpr (WIDE) {
-            gemv_tile<BS, 8>(P, S, ring, in, m, tile, nblocks, klen, q);
-        } else {
-            switch (m.kc) {
-                case 256: gemv_tile<BS, 1>(P, S, ring, in, m, tile, nblocks, klen, q); break;
-                case 512: gemv_tile<BS, 2>(P, S, ring, in, m, tile, nblocks, klen, q); break;
-                case 1024: gemv_tile<BS, 4>(P, S, ring, in, m, tile, nblocks, klen, q); break;
-                default: gemv_tile<BS, 8>(P, S, ring, in, m, tile, nblocks, klen, q); break;
-            }
+    const int T = (int)in.ntiles;
+    for (int k = (int)((warp - tc % kConsumerWarps + kConsumerWarps) % kConsumerWarps); k < T; k += kConsumerWarps) {
+        const uint32_t bi0 = bc + (uint32_t)(k * nkr);
+        switch (m.rows) {
+            case 8: gemv_warp_tile<BS, 8>(P, S, ring, in, m, (int)in.tile + k, bi0, klen); break;
+            case 4: gemv_warp_tile<BS, 4>(P, S, ring, in, m, (int)in.tile + k, bi0, klen); break;
+            case 2: gemv_warp_tile<BS, 2>(P, S, ring, in, m, (int)in.tile + k, bi0, klen); break;
+            default: gemv_warp_tile<BS, 1>(P, S, ring, in, m, (int)in.tile + k, bi0, klen); break;
         }
-        if (++q == nslots) q = 0;
     }
+    bc += (uint32_t)(T * nkr);
+    tc += (uint32_t)T;
     if (in.op == OP_LMHEAD && (in.flags & F_LAST_LM)) lm_publish(P, S, in, gen, pos);
 }
 
@@ -848,7 +824,7 @@ __device__ __forceinline__ float ld1(const float *p) { return *p; }
 // the end and write the chunk's partial (o, m, l); the O-projection combines
 // the chunks of each head with their log-sum-exp weights.
 __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                           int pos) {
+                                           int pos, uint32_t &bc) {
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int d = P.head_dim, nkv = P.n_kv_heads, G = P.n_heads / nkv, l = in.layer;
     const int NC = P.chunks, nq = P.n_heads;
@@ -895,7 +871,7 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
     const int nch = d / 8;
     for (int st = 0; st < a.nstages; ++st) {
         const int n = min(sp, a.tma_end - (a.p0 + st * sp));
-        const uint8_t *slot = c_wait(P, S, ring);
+        const uint8_t *slot = ring_wait(P, S, ring, bc + st);
         if (active) {
             const uint16_t *K = reinterpret_cast<const uint16_t *>(slot);
             const uint16_t *V = reinterpret_cast<const uint16_t *>(slot + kStageBytes / 2);
@@ -942,8 +918,10 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
                 }
             }
         }
-        c_release(P, S, ring);
+        __syncwarp();
+        if (lane == 0) ring_release(S, P, bc + st, 1);
     }
+    bc += (uint32_t)a.nstages;
     if (a.has_cur && active && sl == 0) {  // this step's own position, from fp32 rows
         float part = 0.f;
         for (int e = lane; e < d; e += 32) part = fmaf(qh[e], kpos[e], part);
@@ -1003,14 +981,14 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
 // before it blocks on a wait, so it never holds back a signal it (through
 // others) might be waiting for.  A wait already satisfied for this step is not
 // re-checked.  Every stop decision comes out of an OR-reducing barrier.
-template <int BS, bool WIDE>
+template <int BS>
 __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int end, uint32_t gen, int pos) {
     const int t = threadIdx.x;
-    CRing ring{0, 0u, 0ull};
+    CRing ring{0ull};
+    uint32_t bc = 0, tc = 0;  // ring blocks and GEMV tiles of this CTA consumed so far
     uint64_t act_tag = ~0ull;
     uint32_t sat_ctr = 0xFFFFFFFFu, sat_target = 0u;
     uint32_t pend_ctr = kNoCounter, pend_n = 0u;
-    int q = 0;
     bool stop = false;
     if (P.pdl) pdl_wait();
     consumer_sync();
@@ -1047,10 +1025,10 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
             P.trace[8 * (size_t)i + 1] = globaltimer_ns();
         }
         if (in.op == OP_ATTN) {
-            stop = attn_instr(P, S, ring, in, pos);
+            stop = attn_instr(P, S, ring, in, pos, bc);
             act_tag = ~0ull;
         } else {
-            gemv_instr<BS, WIDE>(P, S, ring, in, act_tag, gen, pos, q);
+            gemv_instr<BS>(P, S, ring, in, act_tag, gen, pos, bc, tc);
         }
         if (!stop) {
             if (in.op != OP_LMHEAD && !(in.flags & F_DROP_SIGNAL)) {
@@ -1077,7 +1055,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
     }
 }
 
-template <int BS, bool WIDE>
+template <int BS>
 __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant__ KParams P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const SmemLayout S = smem_layout(smem_raw, P);
@@ -1087,12 +1065,12 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
         for (int s = 0; s < P.stages; ++s) {
             mbar_init(&S.full[s], 1);
             mbar_init(&S.empty[s], kConsumerWarps);
+            S.seq[s] = 0xFFFFFFFFu;
         }
         *S.abort = 0;
         *S.flag = 0;
         fence_barrier_init();
     }
-    for (int i = t; i < reduce_slots(P.stages) * 8; i += kThreads) S.rcnt[i] = 0;
     for (int i = t; i < P.head_dim / 2; i += kThreads) S.rope[i] = P.rope_inv_freq[i];
     if (t < 64) S.best[t] = argmax_key(-CUDART_INF_F, 0x7fffffff);
     __syncthreads();
@@ -1103,32 +1081,33 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
         if ((t & 31) == 0) producer(P, S, begin, end, pos);
         __syncwarp();
     } else {
-        consumer<BS, WIDE>(P, S, begin, end, gen, pos);
+        consumer<BS>(P, S, begin, end, gen, pos);
     }
     __syncthreads();
 }
 
 // ------------------------------------------------------------------ packing
-// dst block (t, kb) row r column col  <-  source row, column kb*kc + col.
-// mode 0: source row t*8 + r of src; mode 1 (gate/up): rows r < 4 are gate
-// row 4t + r, rows r >= 4 are up row 4t + r - 4.
+// dst block (t, kb), row r, column col  <-  source row, column kb*kc + col.
+// mode 0: source row t*rows + r of src; mode 1 (gate/up): rows r < rows/2 are
+// gate row t*rows/2 + r, the others up row t*rows/2 + r - rows/2.
 __global__ void pack_kernel(const uint16_t *src, const uint16_t *src2, uint16_t *dst, int n_rows, int k, int kc,
-                            int nkb, int tiles, int mode) {
-    const size_t total8 = (size_t)tiles * nkb * kTileRows * kc / 8;
+                            int nkb, int tiles, int rows, int mode) {
+    const size_t total8 = (size_t)tiles * nkb * rows * kc / 8;
     for (size_t v = (size_t)blockIdx.x * blockDim.x + threadIdx.x; v < total8; v += (size_t)gridDim.x * blockDim.x) {
         const size_t e = v * 8;
         const int col = (int)(e % kc);
         size_t rest = e / kc;
-        const int r = (int)(rest % kTileRows);
-        rest /= kTileRows;
+        const int r = (int)(rest % rows);
+        rest /= rows;
         const int kb = (int)(rest % nkb);
         const int t = (int)(rest / nkb);
         const int kk = kb * kc + col;
         const uint16_t *s = src;
-        int row = t * kTileRows + r;
+        int row = t * rows + r;
         if (mode == 1) {
-            row = t * 4 + (r & 3);
-            s = r < 4 ? src : src2;
+            const int half = rows / 2;
+            row = t * half + (r % half);
+            s = r < half ? src : src2;
         }
         uint16_t out[8];
 #pragma unroll
@@ -1137,17 +1116,27 @@ __global__ void pack_kernel(const uint16_t *src, const uint16_t *src2, uint16_t 
     }
 }
 
-// ------------------------------------------------------------------ host launchers
-static bool all_wide(const KParams &P) {
-    return P.qkv_kc == 2048 && P.o_kc == 2048 && P.gu_kc == 2048 && P.down_kc == 2048 && P.lm_kc == 2048;
+__global__ void set_position_kernel(State *state, int pos) { state->pos = pos; }
+
+cudaError_t launch_set_position(State *state, int pos, cudaStream_t s) {
+    set_position_kernel<<<1, 1, 0, s>>>(state, pos);
+    return cudaGetLastError();
 }
 
-template <int BS, bool WIDE>
+cudaError_t launch_pack(const void *src, const void *src2, void *dst, int n_rows, int k, int kc, int nkb, int tiles,
+                        int rows, int mode, cudaStream_t s) {
+    pack_kernel<<<1184, 256, 0, s>>>(static_cast<const uint16_t *>(src), static_cast<const uint16_t *>(src2),
+                                     static_cast<uint16_t *>(dst), n_rows, k, kc, nkb, tiles, rows, mode);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ host launchers
+template <int BS>
 static cudaError_t launch_bs(const KParams &P, int n_ctas, cudaStream_t s, bool cooperative, bool pdl_attr) {
     const int smem = smem_bytes(P);
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(step_kernel<BS, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+        cudaError_t e = cudaFuncSetAttribute(step_kernel<BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -1170,44 +1159,19 @@ static cudaError_t launch_bs(const KParams &P, int n_ctas, cudaStream_t s, bool 
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, step_kernel<BS, WIDE>, P);
+    return cudaLaunchKernelEx(&cfg, step_kernel<BS>, P);
 }
 
-template <bool WIDE>
-static const void *func_of(int bs) {
-    if (bs <= 1) return reinterpret_cast<const void *>(step_kernel<1, WIDE>);
-    if (bs <= 2) return reinterpret_cast<const void *>(step_kernel<2, WIDE>);
-    if (bs <= 4) return reinterpret_cast<const void *>(step_kernel<4, WIDE>);
-    return reinterpret_cast<const void *>(step_kernel<8, WIDE>);
-}
-
-const void *step_kernel_func(const KParams &P) { return all_wide(P) ? func_of<true>(P.bs) : func_of<false>(P.bs); }
-
-template <bool WIDE>
-static cudaError_t launch_w(const KParams &P, int bs, int n_ctas, cudaStream_t s, bool coop, bool pdl) {
-    if (bs <= 1) return launch_bs<1, WIDE>(P, n_ctas, s, coop, pdl);
-    if (bs <= 2) return launch_bs<2, WIDE>(P, n_ctas, s, coop, pdl);
-    if (bs <= 4) return launch_bs<4, WIDE>(P, n_ctas, s, coop, pdl);
-    return launch_bs<8, WIDE>(P, n_ctas, s, coop, pdl);
+const void *step_kernel_func(const KParams &P) {
+    if (P.bs <= 1) return reinterpret_cast<const void *>(step_kernel<1>);
+    if (P.bs <= 2) return reinterpret_cast<const void *>(step_kernel<2>);
+    return reinterpret_cast<const void *>(step_kernel<4>);
 }
 
 cudaError_t launch_step(const KParams &P, int bs, int n_ctas, cudaStream_t s, bool cooperative, bool pdl_attr) {
-    return all_wide(P) ? launch_w<true>(P, bs, n_ctas, s, cooperative, pdl_attr)
-                       : launch_w<false>(P, bs, n_ctas, s, cooperative, pdl_attr);
-}
-
-__global__ void set_position_kernel(State *state, int pos) { state->pos = pos; }
-
-cudaError_t launch_set_position(State *state, int pos, cudaStream_t s) {
-    set_position_kernel<<<1, 1, 0, s>>>(state, pos);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_pack(const void *src, const void *src2, void *dst, int n_rows, int k, int kc, int nkb, int tiles,
-                        int mode, cudaStream_t s) {
-    pack_kernel<<<1184, 256, 0, s>>>(static_cast<const uint16_t *>(src), static_cast<const uint16_t *>(src2),
-                                     static_cast<uint16_t *>(dst), n_rows, k, kc, nkb, tiles, mode);
-    return cudaGetLastError();
+    if (bs <= 1) return launch_bs<1>(P, n_ctas, s, cooperative, pdl_attr);
+    if (bs <= 2) return launch_bs<2>(P, n_ctas, s, cooperative, pdl_attr);
+    return launch_bs<4>(P, n_ctas, s, cooperative, pdl_attr);
 }
 
 }  // namespace mk

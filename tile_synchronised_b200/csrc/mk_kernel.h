@@ -10,7 +10,7 @@ int smem_bytes(const KParams &P);
 cudaError_t launch_step(const KParams &P, int bs, int n_ctas, cudaStream_t s, bool cooperative, bool pdl_attr);
 const void *step_kernel_func(const KParams &P);
 cudaError_t launch_pack(const void *src, const void *src2, void *dst, int n_rows, int k, int kc, int nkb, int tiles,
-                        int mode, cudaStream_t s);
+                        int rows, int mode, cudaStream_t s);
 cudaError_t launch_set_position(State *state, int pos, cudaStream_t s);
 // Fused SwiGLU first stage (fp16): variant MK_SWIGLU_ROW or MK_SWIGLU_COL.
 cudaError_t launch_swiglu(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N, int variant,

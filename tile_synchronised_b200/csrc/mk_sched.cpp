@@ -27,23 +27,26 @@ namespace mk {
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-static int block_width(int k) {
-    int kc = 256;
-    while (kc < k && kc < 2048) kc *= 2;
-    return kc;
-}
-
-static PackedMat make_mat(int n_rows, int k, int tiles_override = -1) {
+// Tiles are `rows` x kc blocks with kc = K rounded up to 256 (one 8-column
+// chunk per lane of a warp) and rows the largest power of two <= 8 that keeps
+// a block within one 32 KB ring slot: K <= 2048 -> 8 rows, 4096 -> 4, 8192 -> 2,
+// up to 16384 -> 1.  `ksplit` cuts K into that many blocks (activation budget).
+// Gate/up tiles hold rows/2 gate rows then the matching rows/2 up rows.
+static PackedMat make_mat(int n_rows, int k, bool pair = false, int ksplit = 1) {
     PackedMat m{};
     m.n_rows = n_rows;
     m.k = k;
-    m.kc = block_width(k);
-    m.nkb = (k + m.kc - 1) / m.kc;
-    m.tiles = tiles_override > 0 ? tiles_override : (n_rows + kTileRows - 1) / kTileRows;
+    const int kpad = (k + 255) / 256 * 256;
+    m.nkb = std::max(1, ksplit);
+    m.kc = ((kpad + m.nkb - 1) / m.nkb + 255) / 256 * 256;
+    m.nkb = (kpad + m.kc - 1) / m.kc;
+    m.rows = kMaxTileRows;
+    while (m.rows > (pair ? 2 : 1) && m.rows * m.kc * 2 > kStageBytes) m.rows /= 2;
+    m.tiles = pair ? (n_rows / 2 + m.rows / 2 - 1) / (m.rows / 2) : (n_rows + m.rows - 1) / m.rows;
     return m;
 }
 
-static size_t mat_bytes(const PackedMat &m) { return (size_t)m.tiles * m.nkb * kTileRows * m.kc * 2; }
+static size_t mat_bytes(const PackedMat &m) { return (size_t)m.tiles * m.nkb * m.rows * m.kc * 2; }
 
 mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p, std::string &err) {
     p = Plan();
@@ -75,10 +78,12 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     p.qkv_rows = (nq + 2 * nkv) * d;
     p.qkv = make_mat(p.qkv_rows, H);
     p.o = make_mat(H, nq * d);
-    p.gu = make_mat(2 * I, H, (I + 3) / 4);
+    p.gu = make_mat(2 * I, H, true);
     p.down = make_mat(H, I);
     p.lm = make_mat(V, H);
-    p.i_pad = p.down.nkb * p.down.kc;
+    if (p.qkv.rows * p.qkv.kc * 2 > kStageBytes || p.gu.rows * p.gu.kc * 2 > kStageBytes)
+        return bad(MK_ERR_UNSUPPORTED, "hidden too large for one ring slot per tile row");
+    if ((nq * d) % p.qkv.rows || (nkv * d) % p.qkv.rows) return bad(MK_ERR_UNSUPPORTED, "q/k/v rows not tile-aligned");
 
     // Batch rows per instruction and the activation region.  Activations are
     // staged in shared memory as fp32 [rows][K range]; the region is capped at
@@ -93,9 +98,13 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     if ((size_t)p.bs * p.o.nkb * p.o.kc * 4 > (size_t)kActMax) return bad(MK_ERR_UNSUPPORTED, "n_heads*head_dim too large");
     p.gu_bs = p.bs;
     if (swiglu_variant == MK_SWIGLU_ROW && B > 1) p.gu_bs = std::max(1, (std::min(B, p.bs) + 1) / 2);
-    int down_blocks_per_range = std::max(1, kActMax / (p.bs * p.down.kc * 4));
-    down_blocks_per_range = std::min(down_blocks_per_range, p.down.nkb);
-    p.down_ksplit = (p.down.nkb + down_blocks_per_range - 1) / down_blocks_per_range;
+    // the down projection's K (= intermediate) is split so bs rows x kc fit the region
+    int down_split = 1;
+    while ((size_t)p.bs * (((I + 255) / 256 * 256 + down_split - 1) / down_split) * 4 > (size_t)kActMax) ++down_split;
+    p.down = make_mat(H, I, false, down_split);
+    p.down_ksplit = p.down.nkb;
+    p.i_pad = p.down.nkb * p.down.kc;
+    const int down_blocks_per_range = 1;
     int act = 0;
     act = std::max(act, p.bs * p.qkv.nkb * p.qkv.kc * 4);
     act = std::max(act, p.bs * p.o.nkb * p.o.kc * 4);
@@ -159,7 +168,7 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
                     in.signal_ctr = signal < 0 ? kNoCounter : (uint16_t)signal;
                     in.signal2_ctr = kNoCounter;
                     v.push_back(in);
-                    cost.push_back((double)(t1 - t0) * (in.kb1 - in.kb0) * kTileRows * m.kc * 2 + 4096.0);
+                    cost.push_back((double)(t1 - t0) * (in.kb1 - in.kb0) * m.rows * m.kc * 2 + 4096.0);
                 }
         }
         if (signal >= 0) p.counter_count[signal] += (uint32_t)v.size();

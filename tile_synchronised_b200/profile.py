@@ -41,7 +41,7 @@ def summarise(sched, base, tr):
                         "sum_us_per_cta": float(dur.sum() / (len(base) - 1)),
                         "wait_sum_us_per_cta": float(wait.sum() / (len(base) - 1)),
                         "producer_lead_us": float(np.nanmean(lead)) if np.isfinite(lead).any() else None,
-                        "consumer_data_wait_us": float(cwait[m].mean() / 1e3),
+                        "consumer_data_wait_us": float(cwait[m].mean() / 1965.0),  # SM cycles at 1965 MHz
                         "producer_slot_wait_us": float(pwait[m].mean() / 1e3)}
     out["per_op"] = per_op
     phases = []
