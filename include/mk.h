@@ -16,7 +16,9 @@
  *
  * Conventions
  *  - Every call returns an mk_status.  MK_OK is 0; errors are negative.
- *    mk_last_error() gives a one-line reason for the last failure on a ctx.
+ *    mk_last_error() gives a one-line reason for the last failure on a ctx;
+ *    mk_last_error(NULL) gives the calling thread's last failure of a
+ *    context-free call (mk_attention_decode and the like).
  *  - All device memory is owned by the caller (for example allocated through
  *    PyTorch) and passed as raw device pointers; the library allocates host
  *    memory only and never frees caller memory.  mk_swiglu_stage1 is
@@ -220,6 +222,39 @@ mk_status mk_swiglu_stage1(const void *x, const void *w_gate, const void *w_up, 
  * (may be NULL). */
 mk_status mk_swiglu_tune(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K, int N,
                          void *stream, int *chosen, float *us_row, float *us_col);
+
+/* Split-KV decode attention with a log-sum-exp combine, on its own: the
+ * attention of one layer of one decode step ("Look Ma, No Bubbles! Designing
+ * a Low-Latency Megakernel for Llama-1B", introduction: generating one
+ * sequence with Llama-3.2-1B; the megakernel runs the same split inside its
+ * interpreter).  For every sequence b and query head h (KV head
+ * g = h / (n_heads / n_kv_heads)):
+ *   out[b][h] = sum_j softmax_j(q[b][h] . K[b][g][j] / sqrt(d)) V[b][g][j],
+ *   j = 0 .. n_pos - 1.
+ * q: device fp32 [batch][n_heads][head_dim] (already rotated);
+ * k_cache, v_cache: device bf16 [batch][n_kv_heads][max_seq][head_dim], the
+ * layout of one layer of the decode cache; out: device fp32
+ * [batch][n_heads][head_dim].  The positions are cut into `chunks` equal
+ * ranges (0 = pick from the SM count, see mk_attention_chunks; at most n_pos);
+ * one CTA per (chunk, KV head, sequence) writes an unnormalised partial
+ * (o, max, sum) to `scratch`, and a second kernel combines them.  scratch is
+ * caller-owned device memory of at least mk_attention_scratch_bytes(batch,
+ * n_heads, head_dim, chunks) bytes; it needs no initialisation and is fully
+ * rewritten by every call, so calls that share a scratch buffer must not
+ * overlap.  head_dim in {64, 128, 256}; n_heads a multiple of n_kv_heads with at
+ * most 8 query heads per KV head; 1 <= n_pos <= max_seq; all pointers 16-byte
+ * aligned.  MK_ERR_INVALID / MK_ERR_UNSUPPORTED otherwise (reason in
+ * mk_last_error(NULL)).  fp32 accumulation, softmax in base 2.  Allocates
+ * nothing; asynchronous on `stream`. */
+mk_status mk_attention_decode(const float *q, const void *k_cache, const void *v_cache, int batch, int n_heads,
+                              int n_kv_heads, int head_dim, int max_seq, int n_pos, int chunks, float *out,
+                              void *scratch, size_t scratch_bytes, void *stream);
+/* Bytes of scratch mk_attention_decode needs (0 for non-positive arguments). */
+size_t mk_attention_scratch_bytes(int batch, int n_heads, int head_dim, int chunks);
+/* The chunk count mk_attention_decode picks for chunks = 0 on the current
+ * device: about one CTA per SM over (sequence, KV head) pairs, at most 64, and
+ * at least 16 positions per chunk. */
+int mk_attention_chunks(int batch, int n_kv_heads, int n_pos);
 
 #ifdef __cplusplus
 }

@@ -159,3 +159,16 @@ def to_u16(t: torch.Tensor):
     """Host numpy uint16 view of a 16-bit tensor's bytes (copies to CPU)."""
     import numpy as np
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def make_attention_inputs(batch: int, n_heads: int, n_kv_heads: int, head_dim: int, max_seq: int, n_pos: int,
+                          seed: int = 11, q_std: float = 1.0, device="cpu"):
+    """Decode-attention operands: q fp32 [B, nq, d] ~ N(0, q_std); K, V bf16
+    [B, nkv, max_seq, d] ~ N(0, 1) at positions < n_pos and the bf16 NaN
+    pattern 0xFFFF beyond, so that a read past n_pos poisons the result."""
+    q = _randn((batch, n_heads, head_dim), seed, device, torch.float32, q_std)
+    k = _randn((batch, n_kv_heads, max_seq, head_dim), seed + 1, device, torch.bfloat16, 1.0)
+    v = _randn((batch, n_kv_heads, max_seq, head_dim), seed + 2, device, torch.bfloat16, 1.0)
+    for t in (k, v):
+        t.view(torch.int16)[:, :, n_pos:] = -1  # 0xFFFF
+    return q, k, v

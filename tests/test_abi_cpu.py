@@ -107,3 +107,24 @@ def test_swiglu_argument_checks_need_no_device():
     assert lib.mk_swiglu_stage1(dummy, dummy, dummy, dummy, 65, 8192, 7168, 0, None) == _lib.MK_ERR_INVALID
     assert lib.mk_swiglu_stage1(dummy, dummy, dummy, dummy, 1, 8200, 7168, 0, None) == _lib.MK_ERR_INVALID
     assert lib.mk_swiglu_stage1(None, dummy, dummy, dummy, 1, 8192, 7168, 0, None) == _lib.MK_ERR_INVALID
+
+
+def test_attention_argument_checks_need_no_device():
+    lib = _lib.load()
+    d = C.c_void_p(256)
+    f = lib.mk_attention_decode
+    ok = (1, 32, 8, 64, 128, 100, 4)  # batch, nq, nkv, d, max_seq, n_pos, chunks
+    need = lib.mk_attention_scratch_bytes(1, 32, 64, 4)
+    assert need == 32 * 4 * 66 * 4
+    assert lib.mk_attention_scratch_bytes(0, 32, 64, 4) == 0
+    assert f(None, d, d, *ok, d, d, need, None) == _lib.MK_ERR_INVALID
+    assert "null" in lib.mk_last_error(None).decode()
+    assert f(C.c_void_p(8), d, d, *ok, d, d, need, None) == _lib.MK_ERR_INVALID
+    assert "aligned" in lib.mk_last_error(None).decode()
+    assert f(d, d, d, 1, 32, 8, 96, 128, 100, 4, d, d, need, None) == _lib.MK_ERR_UNSUPPORTED
+    assert f(d, d, d, 1, 32, 2, 64, 128, 100, 4, d, d, need, None) == _lib.MK_ERR_INVALID  # 16 heads per KV head
+    assert f(d, d, d, 1, 32, 8, 64, 128, 129, 4, d, d, need, None) == _lib.MK_ERR_INVALID  # n_pos > max_seq
+    assert f(d, d, d, 1, 32, 8, 64, 128, 3, 4, d, d, need, None) == _lib.MK_ERR_INVALID   # chunks > n_pos
+    assert "chunks" in lib.mk_last_error(None).decode()
+    assert f(d, d, d, *ok, d, d, need - 4, None) == _lib.MK_ERR_INVALID                  # scratch too small
+    assert "scratch" in lib.mk_last_error(None).decode()

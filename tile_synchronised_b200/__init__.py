@@ -208,3 +208,38 @@ def swiglu_tune(x, w_gate, w_up, out, stream=None):
                                 C.c_void_p(out.data_ptr()), B, K, N, _stream(stream), C.byref(ch), C.byref(ur),
                                 C.byref(uc)), None, "mk_swiglu_tune")
     return ch.value, ur.value, uc.value
+
+
+def _attn_shapes(q: torch.Tensor, k_cache: torch.Tensor):
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [batch, n_heads, head_dim] and the caches [batch, n_kv_heads, max_seq, head_dim]")
+    if q.dtype != torch.float32 or k_cache.dtype != torch.bfloat16:
+        raise TypeError("q must be float32 and the caches bfloat16")
+    B, nq, d = q.shape
+    return B, nq, k_cache.shape[1], d, k_cache.shape[2]
+
+
+def attention_chunks(batch: int, n_kv_heads: int, n_pos: int) -> int:
+    """The chunk count attention_decode picks for chunks=0 on the current device."""
+    return int(load().mk_attention_chunks(batch, n_kv_heads, n_pos))
+
+
+def attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, n_pos: int, chunks: int = 0,
+                     out: torch.Tensor | None = None, scratch: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Split-KV decode attention over positions 0..n_pos-1 of one layer's cache:
+    q fp32 [B, nq, d], caches bf16 [B, nkv, max_seq, d] -> out fp32 [B, nq, d]."""
+    B, nq, nkv, d, max_seq = _attn_shapes(q, k_cache)
+    if chunks == 0:
+        chunks = attention_chunks(B, nkv, n_pos)
+    if out is None:
+        out = torch.empty((B, nq, d), dtype=torch.float32, device=q.device)
+    need = int(load().mk_attention_scratch_bytes(B, nq, d, chunks))
+    if scratch is None:
+        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    check(load().mk_attention_decode(C.c_void_p(q.data_ptr()), C.c_void_p(k_cache.data_ptr()),
+                                     C.c_void_p(v_cache.data_ptr()), B, nq, nkv, d, max_seq, n_pos, chunks,
+                                     C.c_void_p(out.data_ptr()), C.c_void_p(scratch.data_ptr()),
+                                     scratch.numel() * scratch.element_size(), _stream(stream)),
+          None, "mk_attention_decode", op=True)
+    return out

@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "MK_OK", -1: "MK_ERR_INVALID", -2: "MK_ERR_CUDA", -3: "MK_ERR
 EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk_kv_cache_bytes",
            "mk_load_weights", "mk_prefill_kv", "mk_decode_step", "mk_get_status", "mk_reset",
            "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch", "mk_set_timeout_ns", "mk_debug_drop_signal",
-           "mk_set_trace", "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1", "mk_swiglu_tune")
+           "mk_set_trace", "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1", "mk_swiglu_tune",
+           "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks")
 
 
 class MkConfig(C.Structure):
@@ -90,6 +91,9 @@ def load() -> C.CDLL:
         "mk_swiglu_stage1": ([vp, vp, vp, vp, i32, i32, i32, i32, vp], st),
         "mk_swiglu_tune": ([vp, vp, vp, vp, i32, i32, i32, vp, C.POINTER(i32), C.POINTER(C.c_float),
                             C.POINTER(C.c_float)], st),
+        "mk_attention_decode": ([vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, sz, vp], st),
+        "mk_attention_scratch_bytes": ([i32, i32, i32, i32], sz),
+        "mk_attention_chunks": ([i32, i32, i32], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -99,9 +103,11 @@ def load() -> C.CDLL:
     return L
 
 
-def check(status: int, ctx=None, what: str = "") -> None:
+def check(status: int, ctx=None, what: str = "", op: bool = False) -> None:
+    """Raise MkError for a failed call; the reason comes from the context, or,
+    for a context-free call (op=True), from the calling thread's last error."""
     if status != MK_OK:
         msg = what
-        if ctx is not None:
+        if ctx is not None or op:
             msg = f"{what}: {load().mk_last_error(ctx).decode()}"
         raise MkError(status, msg)

@@ -152,7 +152,7 @@ mk_status mk_destroy(mk_ctx *c) {
     return MK_OK;
 }
 
-const char *mk_last_error(const mk_ctx *c) { return c ? c->err.c_str() : "null context"; }
+const char *mk_last_error(const mk_ctx *c) { return c ? c->err.c_str() : op_error(); }
 
 mk_status mk_workspace_bytes(const mk_ctx *c, size_t *bytes) {
     if (!c || !bytes) return MK_ERR_INVALID;

@@ -1,0 +1,260 @@
+// mk_attn.cu -- split-KV decode attention with a log-sum-exp combine, as an
+// operation of its own (the attention of one layer of one decode step).
+//
+// The decode step's attention reads every cached K/V position of a sequence
+// for a handful of query heads, so one (sequence, KV head) alone cannot keep
+// the GPU busy.  The positions are therefore cut into chunks; each CTA turns
+// one chunk into an unnormalised partial (o, m, l) for the G query heads that
+// share the KV head, and a second kernel combines the chunks:
+//     M = max_c m_c,   out = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c
+// (scores kept in the base-2 domain).  This is the split-KV attention plus
+// LSE combine of the decode step ("Look Ma, No Bubbles! Designing a
+// Low-Latency Megakernel for Llama-1B", introduction: one sequence generated
+// with Llama-3.2-1B; the megakernel runs the same split inside its
+// interpreter).
+//
+// Layouts: q fp32 [B][nq][d] (already rotated); K/V bf16 [B][nkv][max_seq][d]
+// (one layer of the model's KV cache); out fp32 [B][nq][d]; partial records
+// fp32 [B][nq][chunks][d + 2] = (o[0..d), m, l).
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include <cstdio>
+
+#include "../../include/mk.h"
+#include "mk_device.cuh"
+#include "mk_kernel.h"
+
+namespace mk {
+
+constexpr int kAttnThreads = 256;
+constexpr int kAttnWarps = kAttnThreads / 32;
+
+// Positions per shared-memory tile: K and V tiles together take 32 KB
+// (16 KB at d = 256), leaving the whole CTA under the 48 KB static limit.
+__host__ __device__ constexpr int attn_tile_positions(int d) { return d == 256 ? 16 : 8192 / d; }
+
+__host__ __device__ inline int attn_smem_bytes(int G, int d) {
+    return G * d * 4 + 2 * attn_tile_positions(d) * d * 2 + kAttnWarps * (d + 2) * 4;
+}
+
+struct AttnArgs {
+    const float *q;
+    const uint16_t *k, *v;
+    float *out, *part;
+    int B, nq, nkv, d, max_seq, n_pos, chunks;
+};
+
+// One CTA = one (chunk, KV head, sequence).  Warps split the G heads
+// (kAttnWarps / G warps per head, interleaving the tile's positions); each
+// keeps an online softmax over its positions with lane l owning dimensions
+// l*DPL .. l*DPL + DPL - 1.  The warps' states are merged in shared memory.
+template <int DPL>
+__global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) {
+    constexpr int d = 32 * DPL;
+    constexpr int TP = attn_tile_positions(d);
+    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int G = a.nq / a.nkv;
+    const int wph = G >= kAttnWarps ? 1 : kAttnWarps / G;
+    const int h = warp / wph, sl = warp % wph;
+    const bool active = h < G;
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *qs = reinterpret_cast<float *>(smem);                    // [G][d], scaled by log2(e)/sqrt(d)
+    uint16_t *kt = reinterpret_cast<uint16_t *>(qs + G * d);        // [TP][d]
+    uint16_t *vt = kt + TP * d;                                     // [TP][d]
+    float *mrg = reinterpret_cast<float *>(vt + TP * d);            // [warps][d + 2]
+    const long long p0 = (long long)c * a.n_pos / a.chunks, p1 = (long long)(c + 1) * a.n_pos / a.chunks;
+    const float qscale = 1.4426950408889634f * rsqrtf((float)d);
+    const float *qb = a.q + ((size_t)b * a.nq + (size_t)g * G) * d;
+    for (int i = t; i < G * d; i += kAttnThreads) qs[i] = qb[i] * qscale;
+    const size_t head = ((size_t)b * a.nkv + g) * (size_t)a.max_seq;
+    float m = -CUDART_INF_F, l = 0.f, o[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) o[e] = 0.f;
+    for (long long t0 = p0; t0 < p1; t0 += TP) {
+        const int n = (int)min((long long)TP, p1 - t0);
+        __syncthreads();  // the previous tile is consumed (and q is staged)
+        const uint4 *ks = reinterpret_cast<const uint4 *>(a.k + (head + t0) * d);
+        const uint4 *vs = reinterpret_cast<const uint4 *>(a.v + (head + t0) * d);
+        for (int i = t; i < n * d / 8; i += kAttnThreads) {
+            reinterpret_cast<uint4 *>(kt)[i] = __ldg(ks + i);
+            reinterpret_cast<uint4 *>(vt)[i] = __ldg(vs + i);
+        }
+        __syncthreads();
+        if (active) {
+            float qr[DPL];
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) qr[e] = qs[h * d + lane * DPL + e];
+            for (int j = sl; j < n; j += wph) {
+                const uint16_t *kr = kt + j * d + lane * DPL;
+                const uint16_t *vr = vt + j * d + lane * DPL;
+                float s = 0.f;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) s = fmaf(qr[e], bf2f(kr[e]), s);
+                s = warp_sum(s);
+                const float mn = fmaxf(m, s);
+                const float sc = exp2f(m - mn), p = exp2f(s - mn);
+                l = l * sc + p;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) o[e] = fmaf(p, bf2f(vr[e]), o[e] * sc);
+                m = mn;
+            }
+        }
+    }
+    __syncthreads();
+    if (active) {
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) mrg[warp * (d + 2) + lane * DPL + e] = o[e];
+        if (lane == 0) {
+            mrg[warp * (d + 2) + d] = m;
+            mrg[warp * (d + 2) + d + 1] = l;
+        }
+    }
+    __syncthreads();
+    for (int i = t; i < G * d; i += kAttnThreads) {
+        const int hh = i / d, e = i % d;
+        float M = -CUDART_INF_F;
+        for (int w = hh * wph; w < (hh + 1) * wph; ++w) M = fmaxf(M, mrg[w * (d + 2) + d]);
+        float O = 0.f, L = 0.f;
+        if (M != -CUDART_INF_F)
+            for (int w = hh * wph; w < (hh + 1) * wph; ++w) {
+                const float mw = mrg[w * (d + 2) + d];
+                if (mw == -CUDART_INF_F) continue;
+                const float f = exp2f(mw - M);
+                O = fmaf(f, mrg[w * (d + 2) + e], O);
+                L = fmaf(f, mrg[w * (d + 2) + d + 1], L);
+            }
+        float *rec = a.part + (((size_t)b * a.nq + (size_t)g * G + hh) * a.chunks + c) * (d + 2);
+        rec[e] = O;
+        if (e == 0) {
+            rec[d] = M;
+            rec[d + 1] = L;
+        }
+    }
+}
+
+// One CTA per (query head, sequence), one thread per output dimension.
+__global__ void attn_combine_kernel(AttnArgs a) {
+    const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x, d = a.d;
+    const float *rec = a.part + ((size_t)b * a.nq + h) * a.chunks * (size_t)(d + 2);
+    float M = -CUDART_INF_F;
+    for (int c = 0; c < a.chunks; ++c) M = fmaxf(M, rec[(size_t)c * (d + 2) + d]);
+    float O = 0.f, L = 0.f;
+    for (int c = 0; c < a.chunks; ++c) {
+        const float mc = rec[(size_t)c * (d + 2) + d];
+        if (mc == -CUDART_INF_F) continue;
+        const float f = exp2f(mc - M);
+        O = fmaf(f, rec[(size_t)c * (d + 2) + e], O);
+        L = fmaf(f, rec[(size_t)c * (d + 2) + d + 1], L);
+    }
+    a.out[((size_t)b * a.nq + h) * d + e] = O / L;
+}
+
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s) {
+    const int G = a.nq / a.nkv;
+    const dim3 grid(a.chunks, a.nkv, a.B);
+    const int smem = attn_smem_bytes(G, a.d);
+    switch (a.d) {
+        case 64: attn_partial_kernel<2><<<grid, kAttnThreads, smem, s>>>(a); break;
+        case 128: attn_partial_kernel<4><<<grid, kAttnThreads, smem, s>>>(a); break;
+        default: attn_partial_kernel<8><<<grid, kAttnThreads, smem, s>>>(a); break;
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_combine_kernel<<<dim3(a.nq, a.B), a.d, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ host side
+static thread_local char g_op_error[256] = "";
+
+void set_op_error(const char *msg) { snprintf(g_op_error, sizeof(g_op_error), "%s", msg); }
+const char *op_error() { return g_op_error[0] ? g_op_error : "null context"; }
+
+int attention_auto_chunks(int B, int nkv, int n_pos, int sms) {
+    int c = sms / (B * nkv);
+    if (c < 1) c = 1;
+    if (c > 64) c = 64;
+    const int by_len = n_pos / 16 > 0 ? n_pos / 16 : 1;  // at least 16 positions per chunk
+    return c < by_len ? c : by_len;
+}
+
+// Checks shared by every attention entry point; fills a.chunks when it is 0.
+mk_status attention_args(AttnArgs &a, const void *q, const void *k, const void *v, const float *out) {
+    char msg[200];
+    if (!q || !k || !v || !out) {
+        set_op_error("attention: null pointer");
+        return MK_ERR_INVALID;
+    }
+    if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out) & 15u) {
+        set_op_error("attention: q, k_cache, v_cache and out must be 16-byte aligned");
+        return MK_ERR_INVALID;
+    }
+    if (a.d != 64 && a.d != 128 && a.d != 256) {
+        snprintf(msg, sizeof msg, "attention: head_dim %d not in {64, 128, 256}", a.d);
+        set_op_error(msg);
+        return MK_ERR_UNSUPPORTED;
+    }
+    if (a.B < 1 || a.nkv < 1 || a.nq < a.nkv || a.nq % a.nkv || a.nq / a.nkv > kAttnWarps || a.max_seq < 1 ||
+        a.n_pos < 1 || a.n_pos > a.max_seq || a.chunks < 0 || a.B > 65535 || a.nkv > 65535 || a.nq > 65535) {
+        snprintf(msg, sizeof msg,
+                 "attention: bad sizes (batch %d, heads %d/%d, max_seq %d, n_pos %d, chunks %d)", a.B, a.nq, a.nkv,
+                 a.max_seq, a.n_pos, a.chunks);
+        set_op_error(msg);
+        return MK_ERR_INVALID;
+    }
+    if (a.chunks == 0) {
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        a.chunks = attention_auto_chunks(a.B, a.nkv, a.n_pos, sms);
+    }
+    if (a.chunks > a.n_pos || a.chunks > 65535) {
+        snprintf(msg, sizeof msg, "attention: %d chunks for %d positions", a.chunks, a.n_pos);
+        set_op_error(msg);
+        return MK_ERR_INVALID;
+    }
+    return MK_OK;
+}
+
+
+}  // namespace mk
+
+using namespace mk;
+
+extern "C" size_t mk_attention_scratch_bytes(int batch, int n_heads, int head_dim, int chunks) {
+    if (batch < 1 || n_heads < 1 || head_dim < 1 || chunks < 1) return 0;
+    return (size_t)batch * n_heads * chunks * (head_dim + 2) * sizeof(float);
+}
+
+extern "C" int mk_attention_chunks(int batch, int n_kv_heads, int n_pos) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (batch < 1 || n_kv_heads < 1 || n_pos < 1) return 0;
+    return attention_auto_chunks(batch, n_kv_heads, n_pos, sms);
+}
+
+extern "C" mk_status mk_attention_decode(const float *q, const void *k_cache, const void *v_cache, int batch,
+                                         int n_heads, int n_kv_heads, int head_dim, int max_seq, int n_pos,
+                                         int chunks, float *out, void *scratch, size_t scratch_bytes,
+                                         void *stream) {
+    AttnArgs a{q, static_cast<const uint16_t *>(k_cache), static_cast<const uint16_t *>(v_cache), out, nullptr,
+               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks};
+    mk_status st = attention_args(a, q, k_cache, v_cache, out);
+    if (st != MK_OK) return st;
+    const size_t need = mk_attention_scratch_bytes(batch, n_heads, head_dim, a.chunks);
+    if (!scratch || ((uintptr_t)scratch & 15u) || scratch_bytes < need) {
+        char msg[160];
+        snprintf(msg, sizeof msg, "attention: scratch must be 16-byte aligned and hold %zu bytes (got %zu)", need,
+                 scratch_bytes);
+        set_op_error(msg);
+        return MK_ERR_INVALID;
+    }
+    a.part = static_cast<float *>(scratch);
+    cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        set_op_error(cudaGetErrorString(e));
+        return MK_ERR_CUDA;
+    }
+    return MK_OK;
+}

@@ -15,4 +15,7 @@ cudaError_t launch_set_position(State *state, int pos, cudaStream_t s);
 // Fused SwiGLU first stage (fp16): variant MK_SWIGLU_ROW or MK_SWIGLU_COL.
 cudaError_t launch_swiglu(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N, int variant,
                           cudaStream_t s);
+// Last error of a context-free call (the isolated operations) on this thread.
+void set_op_error(const char *msg);
+const char *op_error();
 }  // namespace mk
