@@ -256,6 +256,32 @@ size_t mk_attention_scratch_bytes(int batch, int n_heads, int head_dim, int chun
  * at least 16 positions per chunk. */
 int mk_attention_chunks(int batch, int n_kv_heads, int n_pos);
 
+/* mk_attention_decode without a scratch argument: the partial records live in
+ * a fixed 4 MiB array of device memory inside libmk.so (one per device), so
+ * the call allocates nothing and needs no buffer from the caller.  It serves
+ * callers that cannot allocate or be handed scratch: code running after the
+ * allocator that owns the device's memory has reported it full, callbacks of
+ * that allocator (which may not re-enter it), and C callers without a device
+ * allocator.  The pages have no counterpart of this entry point.
+ *   Limit: batch * n_heads * chunks * (head_dim + 2) * 4 bytes must fit in
+ * mk_attention_noalloc_limit_bytes() (4 MiB).  With chunks = 0 the automatic
+ * count is lowered until it fits; an explicit `chunks`, or a shape where not
+ * even one chunk fits, is refused with MK_ERR_INVALID and the needed size in
+ * mk_last_error(NULL).  Other arguments as mk_attention_decode.
+ *   Set-up: the first call on a device looks up that device's copy of the
+ * array (cudaGetSymbolAddress, with the device current) and keeps it; make that
+ * first call before any stream capture on the device.
+ *   Nothing has to start at zero: every partial record is written by the
+ * first kernel of a call before the second kernel reads it.
+ *   Calls that overlap on the device (other streams or threads with work in
+ * flight at the same time) race on the one array and corrupt each other's
+ * results; calls issued in order on one stream are safe. */
+mk_status mk_attention_decode_noalloc(const float *q, const void *k_cache, const void *v_cache, int batch,
+                                      int n_heads, int n_kv_heads, int head_dim, int max_seq, int n_pos, int chunks,
+                                      float *out, void *stream);
+/* Bytes of the fixed scratch behind mk_attention_decode_noalloc (4 MiB). */
+size_t mk_attention_noalloc_limit_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif

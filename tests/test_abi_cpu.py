@@ -128,3 +128,13 @@ def test_attention_argument_checks_need_no_device():
     assert "chunks" in lib.mk_last_error(None).decode()
     assert f(d, d, d, *ok, d, d, need - 4, None) == _lib.MK_ERR_INVALID                  # scratch too small
     assert "scratch" in lib.mk_last_error(None).decode()
+
+
+def test_noalloc_attention_refuses_oversize_without_a_device():
+    lib = _lib.load()
+    d = C.c_void_p(256)
+    assert lib.mk_attention_noalloc_limit_bytes() == 4 << 20
+    # 16 x 32 heads x 16 chunks x 130 floats = 4259840 bytes > 4 MiB
+    st = lib.mk_attention_decode_noalloc(d, d, d, 16, 32, 8, 128, 1100, 1024, 16, d, None)
+    assert st == _lib.MK_ERR_INVALID
+    assert "4259840" in lib.mk_last_error(None).decode()

@@ -243,3 +243,15 @@ def attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
                                      scratch.numel() * scratch.element_size(), _stream(stream)),
           None, "mk_attention_decode", op=True)
     return out
+
+
+def attention_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, n_pos: int,
+                             out: torch.Tensor, chunks: int = 0, stream=None) -> torch.Tensor:
+    """attention_decode with the library's fixed device scratch instead of a
+    caller buffer; `out` (fp32 [B, nq, d]) must be given, nothing is allocated."""
+    B, nq, nkv, d, max_seq = _attn_shapes(q, k_cache)
+    check(load().mk_attention_decode_noalloc(C.c_void_p(q.data_ptr()), C.c_void_p(k_cache.data_ptr()),
+                                             C.c_void_p(v_cache.data_ptr()), B, nq, nkv, d, max_seq, n_pos, chunks,
+                                             C.c_void_p(out.data_ptr()), _stream(stream)),
+          None, "mk_attention_decode_noalloc", op=True)
+    return out

@@ -23,7 +23,8 @@ EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk
            "mk_load_weights", "mk_prefill_kv", "mk_decode_step", "mk_get_status", "mk_reset",
            "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch", "mk_set_timeout_ns", "mk_debug_drop_signal",
            "mk_set_trace", "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1", "mk_swiglu_tune",
-           "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks")
+           "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks",
+           "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes")
 
 
 class MkConfig(C.Structure):
@@ -94,6 +95,8 @@ def load() -> C.CDLL:
         "mk_attention_decode": ([vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, sz, vp], st),
         "mk_attention_scratch_bytes": ([i32, i32, i32, i32], sz),
         "mk_attention_chunks": ([i32, i32, i32], i32),
+        "mk_attention_decode_noalloc": ([vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp], st),
+        "mk_attention_noalloc_limit_bytes": ([], sz),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)

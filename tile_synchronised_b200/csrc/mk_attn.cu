@@ -20,6 +20,7 @@
 #include <math_constants.h>
 
 #include <cstdio>
+#include <mutex>
 
 #include "../../include/mk.h"
 #include "mk_device.cuh"
@@ -252,6 +253,77 @@ extern "C" mk_status mk_attention_decode(const float *q, const void *k_cache, co
     }
     a.part = static_cast<float *>(scratch);
     cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        set_op_error(cudaGetErrorString(e));
+        return MK_ERR_CUDA;
+    }
+    return MK_OK;
+}
+
+// ------------------------------------------------------------------ no-allocation variant
+// The same two kernels with their partials in a fixed array of device memory
+// owned by this library, for callers that cannot allocate, or be handed, a
+// scratch buffer: code that runs after the caching allocator that owns the
+// device's memory has reported it full (an out-of-memory handler that still
+// needs attention outputs), code that may not take the allocator's lock
+// (callbacks of the allocator itself), and C callers without an allocator of
+// their own.  The pages have no counterpart of this entry point.
+namespace mk {
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // 4 MiB of partial records
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_noalloc_mu;
+static void *g_noalloc_addr[kMaxDevices];  // device address of g_noalloc_partials, per device ordinal
+}  // namespace mk
+
+extern "C" size_t mk_attention_noalloc_limit_bytes(void) { return kNoAllocScratchBytes; }
+
+extern "C" mk_status mk_attention_decode_noalloc(const float *q, const void *k_cache, const void *v_cache, int batch,
+                                                 int n_heads, int n_kv_heads, int head_dim, int max_seq, int n_pos,
+                                                 int chunks, float *out, void *stream) {
+    AttnArgs a{q, static_cast<const uint16_t *>(k_cache), static_cast<const uint16_t *>(v_cache), out, nullptr,
+               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks};
+    const bool auto_chunks = chunks == 0;
+    mk_status st = attention_args(a, q, k_cache, v_cache, out);
+    if (st != MK_OK) return st;
+    char msg[200];
+    const size_t per_chunk = mk_attention_scratch_bytes(batch, n_heads, head_dim, 1);
+    if (auto_chunks && per_chunk * (size_t)a.chunks > kNoAllocScratchBytes)
+        a.chunks = (int)(kNoAllocScratchBytes / per_chunk);  // fewer chunks, if even one fits
+    if (a.chunks < 1 || per_chunk * (size_t)a.chunks > kNoAllocScratchBytes) {
+        snprintf(msg, sizeof msg,
+                 "attention (no-alloc): partials need %zu bytes (batch %d x %d heads x %d chunks x (d + 2) floats), "
+                 "above the fixed %zu-byte scratch",
+                 per_chunk * (size_t)(a.chunks < 1 ? 1 : a.chunks), batch, n_heads, a.chunks < 1 ? 1 : a.chunks,
+                 kNoAllocScratchBytes);
+        set_op_error(msg);
+        return MK_ERR_INVALID;
+    }
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        set_op_error(e != cudaSuccess ? cudaGetErrorString(e) : "attention (no-alloc): device ordinal out of range");
+        return e != cudaSuccess ? MK_ERR_CUDA : MK_ERR_UNSUPPORTED;
+    }
+    void *addr;
+    {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_addr[dev]) {  // first call on this device (which is current): look the array up once
+            void *p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+            if (e != cudaSuccess || !p) {
+                snprintf(msg, sizeof msg, "attention (no-alloc): cudaGetSymbolAddress: %s",
+                         e != cudaSuccess ? cudaGetErrorString(e) : "null address");
+                set_op_error(msg);
+                return MK_ERR_CUDA;
+            }
+            g_noalloc_addr[dev] = p;
+        }
+        addr = g_noalloc_addr[dev];
+    }
+    a.part = static_cast<float *>(addr);
+    e = launch_attention(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         set_op_error(cudaGetErrorString(e));
         return MK_ERR_CUDA;
