@@ -184,7 +184,10 @@ mk_status mk_debug_drop_signal(mk_ctx *ctx, int instr);
  * CTA starts it, when its dependency wait is satisfied, when it is done, when
  * the producer issued its first copy (0 if it streams nothing), the SM clock
  * cycles the consumer spent waiting for ring data, the time the producer spent waiting
- * for a free ring slot, and when the producer issued its last copy.  Each step
+ * for a free ring slot, when the producer issued its last copy, and when the
+ * instruction's inputs were in shared memory (activations staged, or
+ * attention heads rotated).  "Done" is taken after every consumer warp has
+ * finished, so tracing adds one CTA barrier per instruction.  Each step
  * overwrites the buffer.  NULL turns tracing off.  MK_ERR_INVALID if the
  * buffer is too small. */
 mk_status mk_set_trace(mk_ctx *ctx, void *d_trace, size_t bytes);

@@ -31,7 +31,7 @@ constexpr uint16_t kNoCounter = 0xFFFF;
 // ---------------------------------------------------------------- opcodes
 enum Op : uint8_t {
     OP_QKV = 1,     // RMSNorm(x) . W_qkv^T            -> qkv (fp32)
-    OP_ATTN = 2,    // RoPE/qk-norm, split-KV partials, KV append, LSE combine by last arriver
+    OP_ATTN = 2,    // RoPE/qk-norm, split-KV partial, KV append; the last unit of a group combines
     OP_OPROJ = 3,   // x += attn . W_o^T
     OP_GATEUP = 4,  // RMSNorm(x) . [W_g;W_u]^T, SiLU(g)*u -> a (bf16)
     OP_DOWN = 5,    // x += a . W_d^T
@@ -56,9 +56,9 @@ struct Instr {
     uint16_t wait_ctr;    // counter to wait on (kNoCounter: none)
     uint16_t signal_ctr;  // counter to increment when done
     uint32_t wait_count;  // increments the waited counter receives per step
-    uint16_t signal2_ctr; // LM: counter the last arriver signals (unused)
+    uint16_t signal2_ctr; // ATTN: split-KV arrival counter of its (sequence, KV head)
     uint16_t ntiles;      // GEMV: consecutive row tiles in this run (>= 1)
-    uint32_t arrive_count;// LM: arrivals per step on signal_ctr
+    uint32_t arrive_count;// LM: arrivals per step on signal_ctr; ATTN: chunks per (sequence, KV head)
 };
 static_assert(sizeof(Instr) == 32, "Instr must be 32 bytes");
 
@@ -116,7 +116,7 @@ struct KParams {
     const void *embed;          // bf16 [V, H] (caller's)
     float *x;                   // [B, H] residual stream
     float *qkv;                 // [B, qkv_rows]
-    float *attn;                // unused (the O-projection combines the split-KV partials itself)
+    float *attn;                // [B, o_nkb * o_kc] attention output (combined split-KV partials)
     float *act_a;               // [B, I_pad] SwiGLU product
     float *partials;            // [B, nq, chunks, d + 4]: o[d], m, l, pad
     uint16_t *kcache;           // bf16 [L, B, nkv, max_seq, d]

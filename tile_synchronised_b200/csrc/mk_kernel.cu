@@ -36,7 +36,7 @@ struct SmemLayout {
     volatile uint32_t *seq;   // [kMaxStages] ring block index each slot currently holds
     float *ssq;               // [consumer warps][8] sums of squares
     unsigned long long *best; // [64] argmax keys per batch row
-    double *rope;             // [64] RoPE inverse frequencies theta^(-2i/d)
+    float2 *rope;             // [64] (cos, sin) of the RoPE angles at this step's position
 };
 
 __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &P) {
@@ -53,7 +53,7 @@ __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &
     S.seq = reinterpret_cast<volatile uint32_t *>(misc + 384);  // 8 words
     S.best = reinterpret_cast<unsigned long long *>(misc + 512);
     S.ssq = reinterpret_cast<float *>(misc + 1024);   // [16 warps][8]
-    S.rope = reinterpret_cast<double *>(misc + 2048); // [64]
+    S.rope = reinterpret_cast<float2 *>(misc + 2048); // [64]
     return S;
 }
 
@@ -365,65 +365,14 @@ __device__ __forceinline__ void stage_act(const KParams &P, const SmemLayout &S,
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int nb = in.nb;
     float *act = reinterpret_cast<float *>(S.act);
-    if (in.op == OP_OPROJ) {
-        // Log-sum-exp combine of the split-KV partials of every head:
-        // attn[b][h*d + e] = sum_c 2^(m_c - M) o_c[e] / sum_c 2^(m_c - M) l_c.
-        const int d = P.head_dim, nq = P.n_heads, NC = P.chunks, hd = nq * d, ps = partial_stride(d);
-        float *wts = act + (size_t)nb * klen;  // [nb][nq][NC] normalised chunk weights
-        for (int i = t; i < nb * nq; i += kConsumerThreads) {
-            const int b = i / nq, h = i % nq;
-            const float *pc = P.partials + (((size_t)(in.b0 + b) * nq + h) * NC) * ps + d;
-            float2 ml[kMaxAttnChunks];
-#pragma unroll
-            for (int c = 0; c < kMaxAttnChunks; ++c)
-                ml[c] = c < NC ? __ldcg(reinterpret_cast<const float2 *>(pc + (size_t)c * ps)) : make_float2(-CUDART_INF_F, 0.f);
-            float M = -CUDART_INF_F;
-#pragma unroll
-            for (int c = 0; c < kMaxAttnChunks; ++c) M = fmaxf(M, ml[c].x);
-            float L = 0.f;
-#pragma unroll
-            for (int c = 0; c < kMaxAttnChunks; ++c) {
-                ml[c].x = exp2f(ml[c].x - M);
-                L = fmaf(ml[c].x, ml[c].y, L);
-            }
-            const float inv = 1.0f / L;
-#pragma unroll
-            for (int c = 0; c < kMaxAttnChunks; ++c)
-                if (c < NC) wts[(size_t)i * NC + c] = ml[c].x * inv;
-        }
-        consumer_sync();
-        // four consecutive outputs per thread: one float4 per chunk, all loads in flight
-        for (int i4 = t; i4 < nb * klen / 4; i4 += kConsumerThreads) {
-            const int b = (4 * i4) / klen, k = (4 * i4) % klen;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (k < hd) {
-                const int h = k / d, e = k % d;
-                const float4 *pc = reinterpret_cast<const float4 *>(
-                    P.partials + (((size_t)(in.b0 + b) * nq + h) * NC) * ps + e);
-                const float *w = wts + ((size_t)b * nq + h) * NC;
-                float4 v[kMaxAttnChunks];
-#pragma unroll
-                for (int c = 0; c < kMaxAttnChunks; ++c)
-                    v[c] = c < NC ? __ldcg(pc + (size_t)c * (ps / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int c = 0; c < kMaxAttnChunks; ++c) {
-                    if (c < NC) {
-                        acc.x = fmaf(w[c], v[c].x, acc.x);
-                        acc.y = fmaf(w[c], v[c].y, acc.y);
-                        acc.z = fmaf(w[c], v[c].z, acc.z);
-                        acc.w = fmaf(w[c], v[c].w, acc.w);
-                    }
-                }
-            }
-            reinterpret_cast<float4 *>(act)[i4] = acc;
-        }
-        return;
-    }
-    if (in.op == OP_DOWN) {
-        // plain copy of the SwiGLU product, eight 16-byte loads in flight per thread
+    if (in.op == OP_DOWN || in.op == OP_OPROJ) {
+        // plain copy of the SwiGLU product or of the attention output, eight
+        // 16-byte loads in flight per thread
         const int k0 = in.kb0 * m.kc, n4 = klen / 4;
+        const float *src = in.op == OP_DOWN ? P.act_a : P.attn;
+        const size_t rstride = in.op == OP_DOWN ? (size_t)P.i_pad : (size_t)P.o_nkb * P.o_kc;
         for (int b = 0; b < nb; ++b) {
-            const float4 *s4 = reinterpret_cast<const float4 *>(P.act_a + (size_t)(in.b0 + b) * P.i_pad + k0);
+            const float4 *s4 = reinterpret_cast<const float4 *>(src + (size_t)(in.b0 + b) * rstride + k0);
             float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen);
             for (int v0 = t; v0 < n4; v0 += 8 * kConsumerThreads) {
                 float4 r[8];
@@ -726,7 +675,8 @@ __device__ __forceinline__ void lm_publish(const KParams &P, const SmemLayout &S
 // bc + k*nkr .. bc + (k+1)*nkr - 1 (bc counts this CTA's ring blocks so far).
 template <int BS>
 __device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                           uint64_t &act_tag, uint32_t gen, int pos, uint32_t &bc, uint32_t &tc) {
+                                           uint64_t &act_tag, uint32_t gen, int pos, uint32_t &bc, uint32_t &tc,
+                                           int ii) {
     const int warp = threadIdx.x >> 5;
     const MatRef m = mat_of(P, in);
     const int nkr = in.kb1 - in.kb0, klen = nkr * m.kc;
@@ -738,6 +688,7 @@ __device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S
         act_tag = tag;
         consumer_sync();
     }
+    if (P.trace && threadIdx.x == 0) P.trace[8 * (size_t)ii + 7] = globaltimer_ns();  // activations staged
     const int T = (int)in.ntiles;
     for (int k = (int)((warp - tc % kConsumerWarps + kConsumerWarps) % kConsumerWarps); k < T; k += kConsumerWarps) {
         const uint32_t bi0 = bc + (uint32_t)(k * nkr);
@@ -755,7 +706,7 @@ __device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S
 
 // ------------------------------------------------------------------ attention
 // One warp prepares one head: optional per-head RMSNorm, rotate-half RoPE at
-// `pos` (angles in double, reduced mod 2*pi before the fp32 sin/cos), scale.
+// `pos` (from the step's cos/sin table), scale.
 __device__ __forceinline__ void prep_head(const KParams &P, const SmemLayout &S, const float *src, const uint16_t *gain,
                                           int pos, float scale, float *dst, uint16_t *cache_row) {
     const int lane = threadIdx.x & 31, d = P.head_dim, nj = d / 32, jh = nj / 2;
@@ -774,13 +725,10 @@ __device__ __forceinline__ void prep_head(const KParams &P, const SmemLayout &S,
     }
     // rotate-half pairs (i, i + d/2): d = 64 -> (v0, v1); d = 128 -> (v0, v2), (v1, v3)
     auto rot = [&](float &x, float &y, int i) {
-        double ang = (double)pos * S.rope[i];
-        ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
-        float sn, cs;
-        __sincosf((float)ang, &sn, &cs);  // |ang| <= pi here
+        const float2 cs = S.rope[i];
         const float a = x, b = y;
-        x = a * cs - b * sn;
-        y = b * cs + a * sn;
+        x = a * cs.x - b * cs.y;
+        y = b * cs.x + a * cs.y;
     };
     if (jh == 1) {
         rot(v[0], v[1], lane);
@@ -821,12 +769,33 @@ __device__ __forceinline__ float ld1(const float *p) { return *p; }
 // s*32 + k*wph*32 + lane of every ring stage, one position per lane, and keeps
 // its own online-softmax state (running max m, sum l, unnormalised output o)
 // in registers, so a stage needs no CTA barrier.  The warps of a head merge at
-// the end and write the chunk's partial (o, m, l); the O-projection combines
-// the chunks of each head with their log-sum-exp weights.
-__device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                           int pos, uint32_t &bc) {
+// the end and write the chunk's partial (o, m, l); the unit that completes its
+// (sequence, KV head) group combines the group's chunks with their
+// log-sum-exp weights into the attention output and signals the O-projection.
+constexpr int kAttnStop = 1, kAttnSignal = 2;
+
+// DPL consecutive bf16 values (2 or 4) of one V row, widened.
+template <int DPL>
+__device__ __forceinline__ void load_dpl(const uint16_t *p, float *v) {
+    if constexpr (DPL == 2) {
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+        v[0] = bf_lo(w);
+        v[1] = bf_hi(w);
+    } else {
+        const uint2 w = *reinterpret_cast<const uint2 *>(p);
+        v[0] = bf_lo(w.x);
+        v[1] = bf_hi(w.x);
+        v[2] = bf_lo(w.y);
+        v[3] = bf_hi(w.y);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ int attn_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
+                                          uint32_t gen, int pos, uint32_t &bc, int ii) {
+    constexpr int NCH = D / 8, DPL = D / 32;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    const int d = P.head_dim, nkv = P.n_kv_heads, G = P.n_heads / nkv, l = in.layer;
+    const int d = D, nkv = P.n_kv_heads, G = P.n_heads / nkv, l = in.layer;
     const int NC = P.chunks, nq = P.n_heads;
     const AttnGeom a = attn_geom(P, in, pos);
     const int sp = kStageBytes / (4 * d);
@@ -837,6 +806,7 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
     float *kpos = qs + G * d;                       // [d] key of this step's position
     float *vpos = kpos + d;                         // [d] value of this step's position
     float *mrg = vpos + d;                          // [8 warps][d + 2] per-warp states
+    float *pbuf = mrg + kConsumerWarps * (d + 2);   // [8 warps][32] probabilities
     const float *qkv_b = P.qkv + (size_t)a.b * P.qkv_rows;
     const LayerW *LW = P.layers + l;
     const float qscale = 1.4426950408889634f * rsqrtf((float)d);  // log2(e)/sqrt(d): scores in the exp2 domain
@@ -866,9 +836,10 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
                       P.kcache + kv_off(P, l, a.b, a.g, pos));
         consumer_sync();
     }
+    if (P.trace && t == 0) P.trace[8 * (size_t)ii + 7] = globaltimer_ns();  // heads prepared
     float m = -CUDART_INF_F, lsum = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
     const float *qh = qs + (active ? h : 0) * d;
-    const int nch = d / 8;
+    float *pw = pbuf + warp * 32;  // this warp's probabilities, broadcast to all lanes for P.V
     for (int st = 0; st < a.nstages; ++st) {
         const int n = min(sp, a.tma_end - (a.p0 + st * sp));
         const uint8_t *slot = ring_wait(P, S, ring, bc + st);
@@ -878,44 +849,70 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
             for (int base = sl * 32; base < n; base += wph * 32) {
                 const int j = base + lane;
                 const bool valid = j < n;
-                float sc = 0.f;
+                // score of position j: two interleaved FMA chains over the
+                // head's NCH 8-column chunks, visited in a per-lane rotated
+                // order so the lanes' 16-byte reads hit different banks
+                float s0 = 0.f, s1 = 0.f;
                 if (valid) {
-                    for (int k = 0; k < nch; ++k) {
-                        const int cc = (k + lane) % nch;  // rotated chunk order: no bank conflicts across lanes
+                    const uint16_t *kr = K + (size_t)j * D;
+#pragma unroll
+                    for (int k = 0; k < NCH; ++k) {
+                        const int cc = (k + lane) & (NCH - 1);
                         float kf[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(K + (size_t)j * d + cc * 8), kf);
+                        unpack8(*reinterpret_cast<const uint4 *>(kr + cc * 8), kf);
                         const float4 q0 = *reinterpret_cast<const float4 *>(qh + cc * 8);
                         const float4 q1 = *reinterpret_cast<const float4 *>(qh + cc * 8 + 4);
-                        sc = fmaf(q0.x, kf[0], fmaf(q0.y, kf[1], fmaf(q0.z, kf[2], fmaf(q0.w, kf[3], sc))));
-                        sc = fmaf(q1.x, kf[4], fmaf(q1.y, kf[5], fmaf(q1.z, kf[6], fmaf(q1.w, kf[7], sc))));
+                        s0 = fmaf(q0.x, kf[0], s0);
+                        s1 = fmaf(q0.y, kf[1], s1);
+                        s0 = fmaf(q0.z, kf[2], s0);
+                        s1 = fmaf(q0.w, kf[3], s1);
+                        s0 = fmaf(q1.x, kf[4], s0);
+                        s1 = fmaf(q1.y, kf[5], s1);
+                        s0 = fmaf(q1.z, kf[6], s0);
+                        s1 = fmaf(q1.w, kf[7], s1);
                     }
-                } else {
-                    sc = -CUDART_INF_F;
                 }
+                const float sc = valid ? s0 + s1 : -CUDART_INF_F;
                 const float mb = warp_max(sc);
                 const float mnew = fmaxf(m, mb);
                 const float corr = exp2f(m - mnew);
                 const float p = valid ? exp2f(sc - mnew) : 0.f;
                 lsum = lsum * corr + warp_sum(p);
                 m = mnew;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[e] *= corr;
+                pw[lane] = p;
+                __syncwarp();
+                // P.V: lane owns DPL dimensions; rows four at a time, two
+                // accumulator sets so consecutive FMAs do not depend on each other
                 const int cnt = min(32, n - base);
-                for (int jj = 0; jj < cnt; ++jj) {
-                    const float pj = __shfl_sync(0xFFFFFFFFu, p, jj);
-                    const uint16_t *vr = V + (size_t)(base + jj) * d + lane * dpl;
-                    if (dpl == 2) {
-                        const uint32_t w = *reinterpret_cast<const uint32_t *>(vr);
-                        o[0] = fmaf(pj, bf_lo(w), o[0]);
-                        o[1] = fmaf(pj, bf_hi(w), o[1]);
-                    } else {
-                        const uint2 w = *reinterpret_cast<const uint2 *>(vr);
-                        o[0] = fmaf(pj, bf_lo(w.x), o[0]);
-                        o[1] = fmaf(pj, bf_hi(w.x), o[1]);
-                        o[2] = fmaf(pj, bf_lo(w.y), o[2]);
-                        o[3] = fmaf(pj, bf_hi(w.y), o[3]);
+                float oa[DPL], ob[DPL];
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) oa[e] = ob[e] = 0.f;
+                const uint16_t *vb = V + (size_t)base * D + lane * DPL;
+                int jj = 0;
+                for (; jj + 4 <= cnt; jj += 4) {
+                    const float4 p4 = *reinterpret_cast<const float4 *>(pw + jj);
+                    float v0[DPL], v1[DPL], v2[DPL], v3[DPL];
+                    load_dpl<DPL>(vb + (size_t)(jj + 0) * D, v0);
+                    load_dpl<DPL>(vb + (size_t)(jj + 1) * D, v1);
+                    load_dpl<DPL>(vb + (size_t)(jj + 2) * D, v2);
+                    load_dpl<DPL>(vb + (size_t)(jj + 3) * D, v3);
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) {
+                        oa[e] = fmaf(p4.x, v0[e], oa[e]);
+                        ob[e] = fmaf(p4.y, v1[e], ob[e]);
+                        oa[e] = fmaf(p4.z, v2[e], oa[e]);
+                        ob[e] = fmaf(p4.w, v3[e], ob[e]);
                     }
                 }
+                for (; jj < cnt; ++jj) {
+                    float v0[DPL];
+                    load_dpl<DPL>(vb + (size_t)jj * D, v0);
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) oa[e] = fmaf(pw[jj], v0[e], oa[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) o[e] = fmaf(o[e], corr, oa[e] + ob[e]);
+                __syncwarp();  // pw is rewritten by the next 32 positions
             }
         }
         __syncwarp();
@@ -970,9 +967,86 @@ __device__ __forceinline__ bool attn_instr(const KParams &P, const SmemLayout &S
             __stcg(pd + d + 1, L);
         }
     }
-    // the partial is published with the CTA's batched counter signal; the
-    // O-projection combines the chunks
-    return consumer_sync_or(*S.abort != 0);
+    // Arrive on the group's counter; the unit that completes the group (all
+    // chunks of this sequence and KV head, this layer) combines the partials:
+    // attn[h*d + e] = sum_c 2^(m_c - M) o_c[e] / sum_c 2^(m_c - M) l_c.
+    consumer_sync();  // every partial store of this CTA is issued
+    if (t == 0) {
+        __threadfence();
+        const uint32_t target = (gen * (uint32_t)P.n_layers + (uint32_t)l + 1u) * in.arrive_count;
+        const uint32_t old = atom_acq_rel_add(P.counters + in.signal2_ctr, 1u);
+        *S.flag = (old + 1u == target) ? 1 : 0;
+    }
+    consumer_sync();
+    const bool last = *S.flag != 0;
+    if (last) {
+        // tpi threads (a power of two, same warp) share one float4 of output
+        // and take every tpi-th chunk, so each thread has at most four chunks'
+        // loads in flight; the group merges its (max, sum, vector) by shuffles
+        const int ps = partial_stride(d), items = G * d / 4;
+        int tpi = 1;
+        while (tpi < 16 && tpi < NC && 2 * tpi * items <= kConsumerThreads) tpi *= 2;
+        const int per_pass = kConsumerThreads / tpi, q = t % tpi;
+        float *dst = P.attn + (size_t)a.b * P.o_nkb * P.o_kc + (size_t)a.g * G * d;
+        for (int i0 = 0; i0 < items; i0 += per_pass) {
+            const int it = i0 + t / tpi;
+            const bool ok = it < items;
+            const int h = ok ? (4 * it) / d : 0, e = ok ? (4 * it) % d : 0;
+            const float *pc = part + (((size_t)a.b * nq + a.g * G + h) * NC) * ps;
+            float M = -CUDART_INF_F, L = 0.f;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int c0 = q; c0 < NC; c0 += 4 * tpi) {
+                float2 ml[4];
+                float4 ov[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u * tpi;
+                    const bool in_range = ok && c < NC;
+                    ml[u] = in_range ? __ldcg(reinterpret_cast<const float2 *>(pc + (size_t)c * ps + d))
+                                     : make_float2(-CUDART_INF_F, 0.f);
+                    ov[u] = in_range ? __ldcg(reinterpret_cast<const float4 *>(pc + (size_t)c * ps + e))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                float Mn = M;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) Mn = fmaxf(Mn, ml[u].x);
+                const float r = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mn);
+                L *= r;
+                acc.x *= r; acc.y *= r; acc.z *= r; acc.w *= r;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float w = (ml[u].x == -CUDART_INF_F) ? 0.f : exp2f(ml[u].x - Mn);
+                    L = fmaf(w, ml[u].y, L);
+                    acc.x = fmaf(w, ov[u].x, acc.x);
+                    acc.y = fmaf(w, ov[u].y, acc.y);
+                    acc.z = fmaf(w, ov[u].z, acc.z);
+                    acc.w = fmaf(w, ov[u].w, acc.w);
+                }
+                M = Mn;
+            }
+            // merge the tpi partial states of this float4 (lanes q = 0 .. tpi-1)
+            for (int o2 = 1; o2 < tpi; o2 <<= 1) {
+                const float Mo = __shfl_xor_sync(0xFFFFFFFFu, M, o2);
+                const float Lo = __shfl_xor_sync(0xFFFFFFFFu, L, o2);
+                const float4 Ao = make_float4(__shfl_xor_sync(0xFFFFFFFFu, acc.x, o2), __shfl_xor_sync(0xFFFFFFFFu, acc.y, o2),
+                                              __shfl_xor_sync(0xFFFFFFFFu, acc.z, o2), __shfl_xor_sync(0xFFFFFFFFu, acc.w, o2));
+                const float Mn = fmaxf(M, Mo);
+                const float ra = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mn);
+                const float rb = (Mo == -CUDART_INF_F) ? 0.f : exp2f(Mo - Mn);
+                L = L * ra + Lo * rb;
+                acc = make_float4(acc.x * ra + Ao.x * rb, acc.y * ra + Ao.y * rb, acc.z * ra + Ao.z * rb,
+                                  acc.w * ra + Ao.w * rb);
+                M = Mn;
+            }
+            if (ok && q == 0) {
+                const float inv = 1.0f / L;
+                __stcg(reinterpret_cast<float4 *>(dst + h * d + e),
+                       make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
+            }
+        }
+    }
+    const bool stop = consumer_sync_or(*S.abort != 0);
+    return (stop ? kAttnStop : 0) | (last ? kAttnSignal : 0);
 }
 
 // ------------------------------------------------------------------ consumer loop
@@ -1024,14 +1098,18 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
             P.trace[8 * (size_t)i + 0] = t_start;
             P.trace[8 * (size_t)i + 1] = globaltimer_ns();
         }
+        bool signal = in.op != OP_LMHEAD && !(in.flags & F_DROP_SIGNAL);
         if (in.op == OP_ATTN) {
-            stop = attn_instr(P, S, ring, in, pos, bc);
+            const int r = P.head_dim == 64 ? attn_instr<64>(P, S, ring, in, gen, pos, bc, i)
+                                           : attn_instr<128>(P, S, ring, in, gen, pos, bc, i);
+            stop = (r & kAttnStop) != 0;
+            signal = signal && (r & kAttnSignal) != 0;  // only the unit that completed its group
             act_tag = ~0ull;
         } else {
-            gemv_instr<BS>(P, S, ring, in, act_tag, gen, pos, bc, tc);
+            gemv_instr<BS>(P, S, ring, in, act_tag, gen, pos, bc, tc, i);
         }
         if (!stop) {
-            if (in.op != OP_LMHEAD && !(in.flags & F_DROP_SIGNAL)) {
+            if (signal) {
                 if (pend_ctr != in.signal_ctr) {
                     if (pend_n) {
                         consumer_sync();
@@ -1043,6 +1121,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
                 ++pend_n;
             }
         }
+        if (P.trace) consumer_sync();  // "done" means every warp is done (tracing only)
         if (P.trace && t == 0) {
             P.trace[8 * (size_t)i + 2] = globaltimer_ns();
             P.trace[8 * (size_t)i + 4] = ring.waited;
@@ -1071,12 +1150,22 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
         *S.flag = 0;
         fence_barrier_init();
     }
-    for (int i = t; i < P.head_dim / 2; i += kThreads) S.rope[i] = P.rope_inv_freq[i];
+    // Position and step of this launch (the step state changes only in the
+    // last phase of a step, after every other phase of it has finished).
+    const uint32_t gen = *reinterpret_cast<volatile const uint32_t *>(&P.state->gen);
+    const int pos = *reinterpret_cast<volatile const int32_t *>(&P.state->pos);
+    // RoPE angles pos * theta^(-2i/d) in double, reduced mod 2*pi, then the
+    // fp32 sine and cosine of the reduced angle (|angle| <= pi).
+    for (int i = t; i < P.head_dim / 2; i += kThreads) {
+        double ang = (double)pos * P.rope_inv_freq[i];
+        ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
+        float sn, cs;
+        __sincosf((float)ang, &sn, &cs);
+        S.rope[i] = make_float2(cs, sn);
+    }
     if (t < 64) S.best[t] = argmax_key(-CUDART_INF_F, 0x7fffffff);
     __syncthreads();
     const int begin = P.cta_begin[blockIdx.x], end = P.cta_end[blockIdx.x];
-    const uint32_t gen = *reinterpret_cast<volatile const uint32_t *>(&P.state->gen);
-    const int pos = *reinterpret_cast<volatile const int32_t *>(&P.state->pos);
     if (t >= kConsumerThreads) {
         if ((t & 31) == 0) producer(P, S, begin, end, pos);
         __syncwarp();

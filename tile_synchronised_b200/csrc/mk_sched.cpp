@@ -113,14 +113,11 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     act = std::max(act, p.bs * down_blocks_per_range * p.down.kc * 4);
     const int G = nq / nkv;
     // Split-KV chunks: as many units as fit one per CTA (an attention phase is
-    // one unit deep), at most kMaxAttnChunks per (sequence, KV head) since every
-    // O-projection CTA gathers all of a sequence's chunk partials.
+    // one unit deep), at most kMaxAttnChunks per (sequence, KV head) since the
+    // last unit of a (sequence, KV head) gathers every chunk's partial.
     p.chunks = std::max(1, std::min(kMaxAttnChunks, n_ctas / (B * nkv)));
     p.chunks = std::min(p.chunks, std::max(1, c.max_seq / 16));
-    const int attn_scratch = G * d * 4 + 2 * d * 4 + kConsumerWarps * (d + 2) * 4;
-    // the O-projection stages its input by combining every chunk's partial:
-    // fp32 [rows][nq*d] plus the per-(row, head, chunk) weights
-    act = std::max(act, p.bs * (p.o.nkb * p.o.kc + nq * p.chunks) * 4);
+    const int attn_scratch = G * d * 4 + 2 * d * 4 + kConsumerWarps * (d + 2) * 4 + kConsumerWarps * 32 * 4;
     act = std::max(act, attn_scratch);
     p.act_bytes = (int)align_up(act, 128);
     p.stages = kMaxStages;
@@ -128,9 +125,12 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
         --p.stages;
     if (p.stages < 2) return bad(MK_ERR_UNSUPPORTED, "not enough shared memory for the ring");
 
-    // Counters: five per layer (QKV, attention, O, gate/up, down), then the
-    // LM-head arrival counter.
-    p.n_counters = 5 * L + 1;
+    // Counters: five per layer (QKV, attention, O, gate/up, down), the LM-head
+    // arrival counter, then one split-KV arrival counter per (sequence, KV
+    // head), shared by all layers (a layer's units all arrive before the next
+    // layer's attention can start).
+    p.arr_attn = 5 * L + 1;
+    p.n_counters = p.arr_attn + B * nkv;
     if (p.n_counters >= kNoCounter) return bad(MK_ERR_UNSUPPORTED, "too many counters");
     const int arr_lm = 5 * L;
     p.counter_count.assign(p.n_counters, 0);
@@ -192,12 +192,13 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
                         in.b0 = (uint16_t)b;
                         in.nb = 1;
                         in.wait_ctr = (uint16_t)counter_qkv(l);
-                        in.signal_ctr = (uint16_t)counter_att(l);
-                        in.signal2_ctr = kNoCounter;
+                        in.signal_ctr = (uint16_t)counter_att(l);  // by the last unit of (b, g) only
+                        in.signal2_ctr = (uint16_t)(p.arr_attn + b * nkv + g);
+                        in.arrive_count = (uint32_t)p.chunks;
                         v.push_back(in);
                         cost.push_back(typical_ctx / p.chunks * d * 4 + 8192.0);
                     }
-            p.counter_count[counter_att(l)] += (uint32_t)v.size();
+            p.counter_count[counter_att(l)] += (uint32_t)(B * nkv);
             phases.push_back(v);
             costs.push_back(cost);
         }
@@ -356,6 +357,12 @@ mk_status validate_plan(const Plan &p, std::string &err) {
                         const uint32_t a = ++ctr[in.signal_ctr];
                         if (a > in.arrive_count) return fail("more arrivals than expected");
                     }
+                } else if (in.op == OP_ATTN) {
+                    // the unit that completes its (sequence, KV head) group signals
+                    const uint32_t a = ++ctr[in.signal2_ctr];
+                    if (in.arrive_count == 0 || a > (uint32_t)c.n_layers * in.arrive_count)
+                        return fail("more split-KV arrivals than expected");
+                    if (a % in.arrive_count == 0) ++ctr[in.signal_ctr];
                 } else if (in.signal_ctr != kNoCounter) {
                     ++ctr[in.signal_ctr];
                 }
@@ -379,6 +386,11 @@ mk_status validate_plan(const Plan &p, std::string &err) {
         if (in.wait_ctr != kNoCounter && ctr[in.wait_ctr] != in.wait_count) {
             snprintf(buf, sizeof buf, "counter %d receives %u increments per step but instruction %zu expects %u",
                      in.wait_ctr, ctr[in.wait_ctr], i, in.wait_count);
+            return fail(buf);
+        }
+        if (in.op == OP_ATTN && ctr[in.signal2_ctr] != (uint32_t)c.n_layers * in.arrive_count) {
+            snprintf(buf, sizeof buf, "split-KV arrival counter %d gets %u arrivals, expected %u", in.signal2_ctr,
+                     ctr[in.signal2_ctr], (uint32_t)c.n_layers * in.arrive_count);
             return fail(buf);
         }
         if (in.op == OP_LMHEAD && (in.flags & F_LAST_LM) && ctr[in.signal_ctr] != in.arrive_count) {

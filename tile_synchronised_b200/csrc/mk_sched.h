@@ -23,6 +23,7 @@ struct Plan {
     int stages = 0;          // ring slots
     int act_bytes = 0;       // shared-memory activation region
     int down_ksplit = 1;     // K ranges of the down projection (>1: atomic residual update)
+    int arr_attn = 0;        // first split-KV arrival counter (one per sequence and KV head)
     int qkv_rows = 0, i_pad = 0;
     PackedMat qkv{}, o{}, gu{}, down{}, lm{};
 
