@@ -58,6 +58,18 @@ enum {
     MK_GRAPH_PDL = 2   /* as MK_GRAPH, launches chained by programmatic dependent launch so
                           each op streams its weights while the previous op finishes */
 };
+/* How the megakernel's dependent instructions learn that their inputs are
+ * ready ("MegaOps: A Kernel Overlapping Framework ...", "In plain words": a
+ * consumer starts once the particular input tiles it needs are ready).  Every
+ * activation word carries the tag of the (step, layer) that wrote it in the
+ * same 64-bit store in both modes. */
+enum {
+    MK_SYNC_TAGS = 0,    /* readers spin on the tagged words they read (no fence,
+                            no separate flag; the default) */
+    MK_SYNC_COUNTERS = 1 /* tile-ready counters: each instruction release-increments
+                            its phase counter, consumers acquire-spin on it before
+                            reading (tags are then only verified) */
+};
 /* Tilings of the fused SwiGLU first stage ("Deep Kernel Fusion for
  * Transformers", Key points, "Fusion scope": row-major tiling reuses the
  * activations, column-major tiling reuses the weights). */
@@ -164,17 +176,24 @@ mk_status mk_set_variant(mk_ctx *ctx, int variant);
  * receives MK_SWIGLU_ROW or MK_SWIGLU_COL. */
 mk_status mk_tune(mk_ctx *ctx, void *stream, int *chosen);
 
-/* Distance, in 32 KB ring blocks, by which the producer's L2 prefetches run
- * ahead of its shared-memory loads (default 8; 0 disables prefetching). 0..64. */
+/* How far, in 32 KB ring blocks, the producer's L2 prefetches may run ahead of
+ * its shared-memory loads.  It keeps min(4, blocks) ahead at all times and
+ * runs on up to `blocks` while the ring is full (the consumers are waiting on
+ * an input).  Default 10; 0 disables prefetching.  0..64. */
 mk_status mk_set_prefetch(mk_ctx *ctx, int blocks);
 
 /* Device wait limit in nanoseconds (default 1e9).  A wait that runs out sets
  * the context's error word and makes every CTA return early. */
 mk_status mk_set_timeout_ns(mk_ctx *ctx, unsigned long long ns);
+/* Synchronisation of the megakernel variant: MK_SYNC_TAGS (default) or
+ * MK_SYNC_COUNTERS.  Results are bit-identical; only the waiting differs.
+ * Host-only, takes effect at the next launch.  MK_ERR_INVALID otherwise. */
+mk_status mk_set_sync(mk_ctx *ctx, int mode);
 
 /* Test hook: when set, the instruction at index `instr` of the flattened
- * schedule does its work but does not signal its counter, so its consumers'
- * waits run out; -1 clears it.  Used to test timeout reporting. */
+ * schedule does its work but publishes nothing (no counter signal, and its
+ * outputs keep a stale tag), so its consumers' waits run out in either sync
+ * mode; -1 clears it.  Used to test timeout reporting. */
 mk_status mk_debug_drop_signal(mk_ctx *ctx, int instr);
 
 /* Per-instruction timing trace for the following steps: `d_trace` is a

@@ -42,12 +42,14 @@ def widen_bf16(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy()
 
 
-def build_pair(shape, batch=None, max_seq=None, variant="megakernel", device="cuda", seed_tokens=synth.TOKEN_SEED):
+def build_pair(shape, batch=None, max_seq=None, variant="megakernel", device="cuda", seed_tokens=synth.TOKEN_SEED,
+               sync="tags"):
     """Weights on the GPU, the same bytes on the host for the oracle."""
     import tile_synchronised_b200 as mk
     b = shape.batch if batch is None else batch
     ms = shape.max_seq if max_seq is None else max_seq
     tw = synth.make_weights(shape, device=device)
     model = mk.Model(shape, tw, batch=b, max_seq=ms, variant=variant)
+    model.set_sync(sync)
     orc = oracle.OracleModel.from_torch(shape, tw, batch=b, max_seq=ms)
     return tw, model, orc

@@ -39,9 +39,10 @@ def run_trajectory(model, orc, tokens, prefill, steps, check_every=1):
 
 
 @needs_cuda
-def test_tiny_trajectory_and_kv_indexing():
+@pytest.mark.parametrize("sync", ["tags", "counters"])
+def test_tiny_trajectory_and_kv_indexing(sync):
     s = synth.TINY
-    tw, model, orc = build_pair(s)
+    tw, model, orc = build_pair(s, sync=sync)
     k, v = model.kv_views()
     k.view(torch.int16).fill_(-1)  # 0xFFFF: a NaN pattern in bf16
     v.view(torch.int16).fill_(-1)
@@ -63,13 +64,16 @@ def test_tiny_trajectory_and_kv_indexing():
 
 
 @needs_cuda
-@pytest.mark.parametrize("variant", ["graph", "graph_pdl"])
-def test_separate_kernel_variants_bit_equal_megakernel(variant):
+@pytest.mark.parametrize("variant,sync", [("graph", "tags"), ("graph_pdl", "tags"), ("megakernel", "counters")])
+def test_variants_and_sync_modes_bit_equal(variant, sync):
+    """The separate-kernel variants, and the counter-synchronised megakernel,
+    produce the same bits as the tag-synchronised megakernel."""
     s = synth.TINY
     tw = synth.make_weights(s, device="cuda")
     import tile_synchronised_b200 as mk
     a = mk.Model(s, tw, variant="megakernel")
     b = mk.Model(s, tw, variant=variant)
+    b.set_sync(sync)
     tokens = synth.make_tokens(s, 24)
     a.prefill(tokens[:, :16].cuda())
     b.prefill(tokens[:, :16].cuda())
@@ -127,15 +131,18 @@ def test_split_kv_chunk_count_does_not_change_results():
 
 
 @needs_cuda
-def test_wait_timeout_is_reported_and_context_recovers():
+@pytest.mark.parametrize("sync", ["tags", "counters"])
+def test_wait_timeout_is_reported_and_context_recovers(sync):
     s = synth.TINY
     tw = synth.make_weights(s, device="cuda")
     import tile_synchronised_b200 as mk
     from tile_synchronised_b200 import _lib
     m = mk.Model(s, tw)
+    m.set_sync(sync)
     m.set_timeout_ns(20_000_000)  # 20 ms
-    # instruction 0 of CTA 0 is a layer-0 QKV tile: without its signal the
-    # attention instructions of layer 0 can never start
+    # instruction 0 of CTA 0 is a layer-0 QKV tile: without its signal (or,
+    # with tags, with its outputs left stale) the attention instructions of
+    # layer 0 can never start
     m.drop_signal(0)
     tok = torch.zeros(1, dtype=torch.int32, device="cuda")
     m.decode(tok)

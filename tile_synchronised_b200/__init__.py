@@ -10,13 +10,15 @@ import ctypes as C
 
 import torch
 
-from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW,
+from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW, MK_SYNC_COUNTERS,
+                   MK_SYNC_TAGS,
                    MkConfig, MkError, MkWeights, check, load)
 
 __all__ = ["Model", "swiglu_stage1", "swiglu_tune", "MkError", "VARIANTS", "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW",
            "MK_SWIGLU_COL", "load"]
 
 VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL}
+SYNCS = {"tags": MK_SYNC_TAGS, "counters": MK_SYNC_COUNTERS}
 SCHEDULE_FIELDS = ("n_instructions", "n_ctas", "n_counters", "n_phases", "batch_rows", "attention_chunks",
                    "ring_stages", "act_bytes", "swiglu_variant", "down_k_splits")
 
@@ -170,6 +172,11 @@ class Model(Plan):
 
     def set_prefetch(self, blocks: int) -> None:
         check(self.lib.mk_set_prefetch(self.ctx, int(blocks)), self.ctx, "mk_set_prefetch")
+
+    def set_sync(self, name: str) -> None:
+        """Megakernel synchronisation: "tags" (readers spin on tagged
+        activations, the default) or "counters" (tile-ready counters)."""
+        check(self.lib.mk_set_sync(self.ctx, SYNCS[name]), self.ctx, "mk_set_sync")
 
     def set_timeout_ns(self, ns: int) -> None:
         check(self.lib.mk_set_timeout_ns(self.ctx, int(ns)), self.ctx, "mk_set_timeout_ns")

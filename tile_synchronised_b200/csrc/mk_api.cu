@@ -27,7 +27,8 @@ struct mk_ctx {
     unsigned long long timeout_ns = 1000000000ull;
     int drop_instr = -1;
     unsigned long long *trace = nullptr;
-    int prefetch = 8;  // L2 prefetch distance in ring blocks
+    int prefetch = 10;  // furthest L2 prefetch distance in ring blocks
+    int sync = MK_SYNC_TAGS;
     const void *embed = nullptr;
     // captured graph of the separate-kernels variant
     cudaGraph_t graph = nullptr;
@@ -73,7 +74,7 @@ static mk_status plan_both(mk_ctx *c, const mk_config &cfg, int n_ctas, int acti
         size_t have = p->off_ranges - p->off_instrs;
         size_t grow = need > have ? ((need - have + 255) / 256) * 256 : 0;
         if (grow) {
-            for (size_t *o : {&p->off_ranges, &p->off_layers, &p->off_rope, &p->off_x, &p->off_qkv, &p->off_attn,
+            for (size_t *o : {&p->off_ranges, &p->off_layers, &p->off_rope, &p->off_x, &p->off_xe, &p->off_dpart, &p->off_qkv, &p->off_attn,
                               &p->off_act_a, &p->off_partials, &p->off_lm_best, &p->off_next_scratch, &p->off_norms,
                               &p->off_weights, &p->off_lm, &p->workspace_bytes})
                 *o += grow;
@@ -85,7 +86,7 @@ static mk_status plan_both(mk_ctx *c, const mk_config &cfg, int n_ctas, int acti
         Plan &small = a.workspace_bytes < b.workspace_bytes ? a : b;
         const Plan &big = a.workspace_bytes < b.workspace_bytes ? b : a;
         small.off_ranges = big.off_ranges; small.off_layers = big.off_layers; small.off_rope = big.off_rope;
-        small.off_x = big.off_x; small.off_qkv = big.off_qkv; small.off_attn = big.off_attn;
+        small.off_x = big.off_x; small.off_xe = big.off_xe; small.off_dpart = big.off_dpart; small.off_qkv = big.off_qkv; small.off_attn = big.off_attn;
         small.off_act_a = big.off_act_a; small.off_partials = big.off_partials; small.off_lm_best = big.off_lm_best;
         small.off_next_scratch = big.off_next_scratch; small.off_norms = big.off_norms;
         small.off_weights = big.off_weights; small.off_lm = big.off_lm; small.lm.offset = big.lm.offset;
@@ -208,11 +209,15 @@ static KParams make_params(mk_ctx *c, const int32_t *tokens, int64_t tok_stride,
     P.final_norm = ws + p.off_norms + (size_t)g.n_layers * (2 * g.hidden + 2 * g.head_dim) * 2;
     P.embed = c->embed;
     for (int i = 0; i < g.head_dim / 2 && i < 64; ++i) P.rope_inv_freq[i] = std::pow((double)g.rope_theta, -2.0 * i / g.head_dim);
-    P.x = reinterpret_cast<float *>(ws + p.off_x);
-    P.qkv = reinterpret_cast<float *>(ws + p.off_qkv);
-    P.attn = reinterpret_cast<float *>(ws + p.off_attn);
-    P.act_a = reinterpret_cast<float *>(ws + p.off_act_a);
-    P.partials = reinterpret_cast<float *>(ws + p.off_partials);
+    P.xm = reinterpret_cast<uint64_t *>(ws + p.off_x);
+    P.xe = reinterpret_cast<uint64_t *>(ws + p.off_xe);
+    P.dpart = reinterpret_cast<uint64_t *>(ws + p.off_dpart);
+    P.qkv = reinterpret_cast<uint64_t *>(ws + p.off_qkv);
+    P.attn = reinterpret_cast<uint64_t *>(ws + p.off_attn);
+    P.act_a = reinterpret_cast<uint64_t *>(ws + p.off_act_a);
+    P.partials = reinterpret_cast<uint64_t *>(ws + p.off_partials);
+    P.down_ranges = p.down_ksplit;
+    P.down_per = p.down_per;
     P.kcache = reinterpret_cast<uint16_t *>(c->kv);
     P.vcache = reinterpret_cast<uint16_t *>(c->kv + p.kv_bytes / 2);
     P.counters = reinterpret_cast<uint32_t *>(ws + p.off_counters);
@@ -273,6 +278,9 @@ static mk_status upload_schedule(mk_ctx *c, cudaStream_t s) {
 
 static mk_status reset_device_state(mk_ctx *c, cudaStream_t s) {
     const Plan &p = c->plan;
+    // the step count restarts, so no tagged activation may keep a tag of the
+    // new count's range: zero them (tag 0 is never valid)
+    CK(cudaMemsetAsync(c->ws + p.off_x, 0, p.off_lm_best - p.off_x, s));
     CK(cudaMemsetAsync(c->ws + p.off_state, 0, sizeof(State), s));
     CK(cudaMemsetAsync(c->ws + p.off_counters, 0, (size_t)p.n_counters * 4, s));
     CK(cudaMemsetAsync(c->ws + p.off_lm_best, 0, (size_t)p.B * p.n_ctas * sizeof(LmBest), s));
@@ -344,8 +352,6 @@ mk_status mk_load_weights(mk_ctx *c, const mk_weights *w, void *workspace, void 
     std::vector<double> inv(d / 2);
     for (int i = 0; i < d / 2; ++i) inv[i] = std::pow((double)g.rope_theta, -2.0 * i / d);
     CK(cudaMemcpyAsync(c->ws + p.off_rope, inv.data(), inv.size() * 8, cudaMemcpyHostToDevice, s));
-    // activations and padding regions start at zero (padding must stay zero)
-    CK(cudaMemsetAsync(c->ws + p.off_x, 0, p.off_lm_best - p.off_x, s));
     CK(cudaStreamSynchronize(s));  // the host vectors above must outlive the copies
     mk_status st = upload_schedule(c, s);
     if (st != MK_OK) return st;
@@ -363,7 +369,10 @@ static mk_status launch_megakernel(mk_ctx *c, const int32_t *tok, int64_t stride
     const int32_t *ranges = reinterpret_cast<const int32_t *>(c->ws + p.off_ranges);
     P.cta_begin = ranges;
     P.cta_end = ranges + p.n_ctas;
-    P.use_waits = 1;
+    // tags: readers spin on the tagged activations themselves; counters:
+    // acquire-spin / release-increment per instruction, tags then only verify
+    P.use_waits = c->sync == MK_SYNC_COUNTERS ? 1 : 0;
+    P.use_signals = P.use_waits;
     P.pdl = 0;
     cudaError_t e = launch_step(P, p.bs, p.n_ctas, s, true, false);
     if (e != cudaSuccess) {
@@ -386,6 +395,7 @@ static KParams phase_params(mk_ctx *c, int k, const int32_t *tok, int32_t *next,
     const Plan &p = c->plan;
     const int32_t *ranges = reinterpret_cast<const int32_t *>(c->ws + p.off_ranges);
     P.use_waits = 0;
+    P.use_signals = 0;
     P.cta_begin = ranges + (size_t)(2 + k) * p.n_ctas;
     P.cta_end = ranges + (size_t)(3 + k) * p.n_ctas;
     P.pdl = (pdl && k > 0) ? 1 : 0;
@@ -411,12 +421,12 @@ static mk_status launch_phases(mk_ctx *c, const int32_t *tok, int32_t *next, flo
 }
 
 // Point the captured graph at new token / output buffers: only the phases
-// that read the tokens (layer-0 QKV and O-proj) or write the outputs (LM head)
-// are patched, so a new pointer costs three node updates, not a re-capture.
+// that read the tokens (layer-0 QKV and O-projection) or write the outputs (LM
+// head) are patched, so a new pointer costs three node updates, not a
+// re-capture.
 static mk_status retarget_graph(mk_ctx *c, const int32_t *tok, int32_t *next, float *logits, bool pdl) {
     const Plan &p = c->plan;
-    const int phases[3] = {0, 2, p.n_phases - 1};
-    for (int k : phases) {
+    for (int k : p.token_phases) {
         KParams P = phase_params(c, k, tok, next, logits, pdl);
         void *args[1] = {&P};
         cudaKernelNodeParams np = {};
@@ -561,6 +571,13 @@ mk_status mk_set_prefetch(mk_ctx *c, int blocks) {
     return MK_OK;
 }
 
+mk_status mk_set_sync(mk_ctx *c, int mode) {
+    if (!c) return MK_ERR_INVALID;
+    if (mode != MK_SYNC_TAGS && mode != MK_SYNC_COUNTERS) return fail(c, MK_ERR_INVALID, "unknown sync mode");
+    c->sync = mode;
+    return MK_OK;
+}
+
 mk_status mk_set_timeout_ns(mk_ctx *c, unsigned long long ns) {
     if (!c || ns == 0) return MK_ERR_INVALID;
     c->timeout_ns = ns;
@@ -587,6 +604,7 @@ static mk_status switch_plan(mk_ctx *c, cudaStream_t s) {
     mk_status st = upload_schedule(c, s);
     if (st != MK_OK) return st;
     const Plan &p = c->plan;
+    CK(cudaMemsetAsync(c->ws + p.off_x, 0, p.off_lm_best - p.off_x, s));  // the step count restarts
     CK(cudaMemsetAsync(c->ws + p.off_state, 0, sizeof(State), s));
     CK(cudaMemsetAsync(c->ws + p.off_counters, 0, (size_t)p.n_counters * 4, s));
     CK(cudaMemcpyAsync(c->ws + p.off_state + offsetof(State, pos), &pos, 4, cudaMemcpyHostToDevice, s));

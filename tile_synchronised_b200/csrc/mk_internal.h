@@ -22,28 +22,43 @@ constexpr int kernel_bs(int bs) { return bs <= 1 ? 1 : (bs <= 2 ? 2 : 4); }
 // Bytes after the ring and the activation region: barriers, flags, small
 // arrays and the RoPE table.
 constexpr int misc_bytes(int bs, int stages) { return 2560 + 0 * bs * stages; }
-constexpr int kMaxAttnChunks = 16;  // split-KV chunks per (sequence, KV head); the O-projection gathers them all
-// Floats per split-KV partial record: o[d], m, l, padding to a 16-byte multiple.
-constexpr int partial_stride(int head_dim) { return head_dim + 4; }
+constexpr int kMaxAttnChunks = 16;  // split-KV chunks per (sequence, KV head); one combine instruction gathers them
+// Tagged words per split-KV partial record: o[d], m, l.
+constexpr int partial_stride(int head_dim) { return head_dim + 2; }
 constexpr int kMaxGroup = 8;                            // query heads per KV head
 constexpr uint16_t kNoCounter = 0xFFFF;
 
 // ---------------------------------------------------------------- opcodes
+// Every activation that crosses an instruction boundary is a tagged word:
+// the fp32 value in the low half, the tag of the (step, layer) that wrote it in
+// the high half, stored and loaded as one 64-bit access.  A reader knows the
+// tag it expects, so a stale word can never pass for a fresh one.
 enum Op : uint8_t {
-    OP_QKV = 1,     // RMSNorm(x) . W_qkv^T            -> qkv (fp32)
-    OP_ATTN = 2,    // RoPE/qk-norm, split-KV partial, KV append; the last unit of a group combines
-    OP_OPROJ = 3,   // x += attn . W_o^T
-    OP_GATEUP = 4,  // RMSNorm(x) . [W_g;W_u]^T, SiLU(g)*u -> a (bf16)
-    OP_DOWN = 5,    // x += a . W_d^T
+    OP_QKV = 1,     // RMSNorm(x) . W_qkv^T                      -> qkv
+    OP_ATTN = 2,    // RoPE/qk-norm, KV append, one split-KV chunk -> partial (o, m, l)
+    OP_OPROJ = 3,   // x_mid = x + attn . W_o^T        (x = x_end + further down parts of the previous layer)
+    OP_GATEUP = 4,  // RMSNorm(x_mid) . [W_g;W_u]^T, SiLU(g)*u   -> a
+    OP_DOWN = 5,    // a . W_d^T over one K range: x_end = x_mid + range 0, further ranges -> down parts
     OP_LMHEAD = 6,  // RMSNorm(x) . W_head^T -> logits, running argmax; last arriver picks the token
+    OP_ACOMB = 7,   // log-sum-exp combine of one (sequence, KV head)'s chunk partials -> attn
 };
 
 enum Flags : uint8_t {
-    F_EMBED_X = 1,    // layer 0: the residual stream is the embedding row
+    F_EMBED_X = 1,    // layer 0: the residual stream before the O-projection is the embedding row
     F_LAST_LM = 2,    // last LM-head instruction of this CTA: publish the CTA's best
-    F_ATOMIC = 4,     // K-split residual update (red.add into x)
-    F_DROP_SIGNAL = 8 // test hook: skip the signal
+    F_DROP_SIGNAL = 8 // test hook: publish nothing (no counter signal, outputs keep a stale tag)
 };
+
+#ifdef __CUDACC__
+#define MK_HD __host__ __device__
+#else
+#define MK_HD
+#endif
+// Tag of every activation a layer writes in a step (never 0, so zeroed
+// buffers hold no valid word).
+MK_HD inline uint32_t act_tag(uint32_t gen, int n_layers, int layer) {
+    return gen * (uint32_t)n_layers + (uint32_t)layer + 1u;
+}
 
 // One instruction: 32 bytes, read by both the producer and the consumer warps.
 struct Instr {
@@ -114,11 +129,14 @@ struct KParams {
     const void *lm_w;           // packed LM head
     const void *final_norm;     // bf16 [H]
     const void *embed;          // bf16 [V, H] (caller's)
-    float *x;                   // [B, H] residual stream
-    float *qkv;                 // [B, qkv_rows]
-    float *attn;                // [B, o_nkb * o_kc] attention output (combined split-KV partials)
-    float *act_a;               // [B, I_pad] SwiGLU product
-    float *partials;            // [B, nq, chunks, d + 4]: o[d], m, l, pad
+    // tagged activations (see act_tag)
+    uint64_t *xm;               // [B, H] residual stream after the layer's O-projection
+    uint64_t *xe;               // [B, H] x_mid + the down projection's first K range
+    uint64_t *dpart;            // [down K ranges - 1, B, H] outputs of the further K ranges
+    uint64_t *qkv;              // [B, qkv_rows]
+    uint64_t *attn;             // [B, nq * d] attention output (combined split-KV partials)
+    uint64_t *act_a;            // [B, I] SwiGLU product
+    uint64_t *partials;         // [B, nq, chunks, d + 2]: o[d], m, l
     uint16_t *kcache;           // bf16 [L, B, nkv, max_seq, d]
     uint16_t *vcache;
     uint32_t *counters;
@@ -131,11 +149,12 @@ struct KParams {
     unsigned long long timeout_ns;
     // shapes
     int32_t n_layers, hidden, n_heads, n_kv_heads, head_dim, intermediate, vocab, batch, max_seq;
-    int32_t qkv_rows, i_pad, chunks, n_ctas, stages, act_bytes, qk_norm, bs;
+    int32_t qkv_rows, i_pad, chunks, n_ctas, stages, act_bytes, qk_norm, bs, down_ranges, down_per;
     float rms_eps;
     int32_t qkv_kc, qkv_nkb, o_kc, o_nkb, gu_kc, gu_nkb, down_kc, down_nkb, lm_kc, lm_nkb;
     int32_t qkv_rt, o_rt, gu_rt, down_rt, lm_rt;  // rows per tile
-    int32_t use_waits;          // 0 in the separate-kernels variant (kernel boundaries order the ops)
+    int32_t use_waits;          // 1: acquire-spin on the tile-ready counters before each instruction
+    int32_t use_signals;        // 1: release-increment the counters after each instruction
     int32_t pdl;                // 1: wait on the previous grid before reading activations
     unsigned long long *trace;  // [n_instr][8] globaltimer stamps and waits, or null
     int32_t prefetch;           // ring blocks the L2 prefetch cursor runs ahead of the TMA loads

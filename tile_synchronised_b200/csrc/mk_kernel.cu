@@ -238,9 +238,14 @@ __device__ __forceinline__ void cursor_block(const KParams &P, const BlockCursor
     }
 }
 
-// The producer fills the ring in instruction order.  A second cursor runs
-// P.prefetch blocks ahead and pulls those blocks into L2, so the ring's TMA
-// loads hit L2 and the bytes in flight per SM are not limited to the ring.
+// The producer fills the ring in instruction order.  A second cursor pulls
+// blocks further ahead into L2 with bulk prefetches: it always keeps a short
+// base distance, and while the next slot is still in use (the consumers are
+// waiting on an input, so HBM would otherwise idle) it runs on up to
+// P.prefetch blocks ahead.  Prefetching only while stalled keeps the far-ahead
+// traffic from competing with blocks the consumers need now.
+constexpr uint32_t kPrefetchBase = 4;
+
 __device__ void producer(const KParams &P, const SmemLayout &S, int begin, int end, int pos) {
     const uint64_t pol = policy_evict_first();
     const uint64_t pol_pf = policy_evict_normal();
@@ -251,23 +256,33 @@ __device__ void producer(const KParams &P, const SmemLayout &S, int begin, int e
     BlockCursor cur{begin, end, 0, 0}, pf{begin, end, 0, 0};
     cursor_settle(P, cur, pos);
     cursor_settle(P, pf, pos);
-    for (int k = 0; k < P.prefetch && pf.i < end; ++k) {  // prime the prefetch distance
-        const void *s1, *s2;
-        uint32_t bytes;
-        cursor_block(P, pf, s1, s2, bytes);
-        bulk_prefetch_l2(s1, bytes, pol_pf);
-        if (s2) bulk_prefetch_l2(s2, bytes, pol_pf);
+    const uint32_t maxd = (uint32_t)P.prefetch, base = maxd < kPrefetchBase ? maxd : kPrefetchBase;
+    uint32_t pf_n = 0;  // blocks from cur (included) to the prefetch cursor (excluded)
+    auto prefetch_one = [&]() {
+        const void *p1, *p2;
+        uint32_t pb;
+        cursor_block(P, pf, p1, p2, pb);
+        bulk_prefetch_l2(p1, pb, pol_pf);
+        if (p2) bulk_prefetch_l2(p2, pb, pol_pf);
         cursor_next(P, pf, pos);
-    }
+        ++pf_n;
+    };
+    while (pf_n < base && pf.i < end) prefetch_one();
     unsigned long long pw = 0;
     while (cur.i < end) {
         const void *s1, *s2;
         uint32_t bytes;
         cursor_block(P, cur, s1, s2, bytes);
         const unsigned long long w0 = P.trace ? globaltimer_ns() : 0ull;
-        if (!wait_bar(P, &S.empty[slot], phase ^ 1u, S.abort, limit)) {
-            ok = false;
-            break;
+        if (!mbar_try_wait(&S.empty[slot], phase ^ 1u)) {
+            while (pf_n < maxd && pf.i < end) {
+                prefetch_one();
+                if (mbar_try_wait(&S.empty[slot], phase ^ 1u)) break;
+            }
+            if (!wait_bar(P, &S.empty[slot], phase ^ 1u, S.abort, limit)) {
+                ok = false;
+                break;
+            }
         }
         if (P.trace) {
             pw += globaltimer_ns() - w0;
@@ -284,20 +299,17 @@ __device__ void producer(const KParams &P, const SmemLayout &S, int begin, int e
             slot = 0;
             phase ^= 1u;
         }
-        if (pf.i < end) {
-            const void *p1, *p2;
-            uint32_t pb;
-            cursor_block(P, pf, p1, p2, pb);
-            bulk_prefetch_l2(p1, pb, pol_pf);
-            if (p2) bulk_prefetch_l2(p2, pb, pol_pf);
-            cursor_next(P, pf, pos);
-        }
         if (P.trace && cur.j == cur.n - 1) {
             P.trace[8 * (size_t)cur.i + 5] = pw;
             P.trace[8 * (size_t)cur.i + 6] = globaltimer_ns();
             pw = 0;
         }
         cursor_next(P, cur, pos);
+        if (pf_n > 0)
+            --pf_n;  // cur moved into the prefetched window
+        else
+            cursor_next(P, pf, pos);  // the prefetch cursor never falls behind cur
+        while (pf_n < base && pf.i < end) prefetch_one();
     }
     if (!ok && !*S.abort) {
         set_error(P, 3u, (uint32_t)begin, 0u);
@@ -355,90 +367,224 @@ __device__ __forceinline__ void ring_release(const SmemLayout &S, const KParams 
     mbar_arrive_cnt(&S.empty[bi % (uint32_t)P.stages], count);
 }
 
+// ------------------------------------------------------------------ tagged reads
+// Bounded spin for a reader whose words do not carry the expected tag yet.
+struct LlSpin {
+    uint64_t t0;
+    uint32_t it;
+};
+__device__ __forceinline__ bool ll_spin(const KParams &P, const SmemLayout &S, LlSpin &sp, uint32_t who,
+                                        uint32_t tag) {
+    if ((++sp.it & 15u) == 0u) {
+        if (*S.abort) return false;
+        const uint64_t now = globaltimer_ns();
+        if (sp.t0 == 0) {
+            sp.t0 = now;
+        } else if (now - sp.t0 > P.timeout_ns) {
+            set_error(P, 4u, who, tag);
+            *S.abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// Slow path of the tagged reads: re-read the chunks (8 words each, chunk j
+// at base[j]) that did not all carry `tag` yet until they do.  Kept out of
+// line so the wait state costs the fast path no registers; it only runs while
+// a producer has not published yet.
+__device__ __noinline__ bool ll_spin_chunks(const KParams &P, const SmemLayout &S, const uint64_t *const *base,
+                                            int m, uint32_t pending, uint32_t tag, float *vals, uint32_t who) {
+    LlSpin sp{0ull, 0u};
+    while (pending) {
+        __nanosleep(16);
+        for (int j = 0; j < m; ++j) {
+            if (!((pending >> j) & 1u)) continue;
+            bool all = true;
+            for (int q = 0; q < 4; ++q) {
+                const ulonglong2 w = ll_ld2(base[j] + 2 * q);
+                all = all && ll_tag(w.x) == tag && ll_tag(w.y) == tag;
+                vals[8 * j + 2 * q] = ll_value(w.x);
+                vals[8 * j + 2 * q + 1] = ll_value(w.y);
+            }
+            if (all) pending &= ~(1u << j);
+        }
+        if (pending && !ll_spin(P, S, sp, who, tag)) return false;
+    }
+    return true;
+}
+
+// Read m <= M chunks of 8 tagged words (chunk j at ptr[j], 16-byte aligned),
+// all loads in flight together; if any word does not carry `tag` yet, spin
+// until all do.  The values go to f[j][0..7].  False when the wait gave up (f
+// is then junk).
+template <int M>
+__device__ __forceinline__ bool ll_chunks(const KParams &P, const SmemLayout &S, const uint64_t *const (&ptr)[M],
+                                          int m, uint32_t tag, float (&f)[M][8], uint32_t who) {
+    uint32_t pending = 0;
+#pragma unroll
+    for (int j = 0; j < M; ++j)
+        if (j < m) {
+            bool ok = true;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const ulonglong2 w = ll_ld2(ptr[j] + 2 * q);
+                ok = ok && ll_tag(w.x) == tag && ll_tag(w.y) == tag;
+                f[j][2 * q] = ll_value(w.x);
+                f[j][2 * q + 1] = ll_value(w.y);
+            }
+            if (!ok) pending |= 1u << j;
+        }
+    if (!pending) return true;
+    return ll_spin_chunks(P, S, ptr, m, pending, tag, &f[0][0], who);
+}
+
+// One tagged word, spinning until it carries `tag`.
+__device__ __forceinline__ bool ll_word(const KParams &P, const SmemLayout &S, const uint64_t *p, uint32_t tag,
+                                        float &v, uint32_t who) {
+    const uint64_t w = ll_ld(p);
+    if (ll_tag(w) == tag) {
+        v = ll_value(w);
+        return true;
+    }
+    LlSpin sp{0ull, 0u};
+    for (;;) {
+        __nanosleep(16);
+        if (!ll_spin(P, S, sp, who, tag)) return false;
+        const uint64_t w2 = ll_ld(p);
+        if (ll_tag(w2) == tag) {
+            v = ll_value(w2);
+            return true;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t who_of(const Instr &in) { return ((uint32_t)in.op << 16) | in.layer; }
+
+// The residual stream leaving layer l, x = x_end(l) + the outputs of the down
+// projection's further K ranges (only plans whose batch rows exceed the
+// activation budget have any), for 8 columns starting at col of sequence
+// `row`; the same additions, in the same order, wherever x is formed.
+__device__ __forceinline__ bool residual8(const KParams &P, const SmemLayout &S, int row, int col, uint32_t tag,
+                                          float (&x)[8], uint32_t who) {
+    const size_t H = (size_t)P.hidden, rows = (size_t)P.batch;
+    const uint64_t *ptr[1] = {P.xe + (size_t)row * H + col};
+    float f[1][8];
+    bool ok = ll_chunks<1>(P, S, ptr, 1, tag, f, who);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) x[q] = f[0][q];
+    for (int k = 1; k < P.down_ranges; ++k) {
+        ptr[0] = P.dpart + ((size_t)(k - 1) * rows + row) * H + col;
+        ok = ll_chunks<1>(P, S, ptr, 1, tag, f, who) && ok;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] += f[0][q];
+    }
+    return ok;
+}
+
 // ------------------------------------------------------------------ activation staging
 // Writes the instruction's activations for batch rows [b0, b0+nb) as fp32
 // [nb][klen] into shared memory: RMSNorm(x) * gain for QKV / gate-up / LM head,
 // a plain copy of the attention output or of the SwiGLU product otherwise.
+// Each thread reads tagged words and spins until they carry the producing
+// layer's tag.  Returns false if a wait gave up; every thread still reaches
+// every barrier.
 template <int BS>
-__device__ __forceinline__ void stage_act(const KParams &P, const SmemLayout &S, const Instr &in, const MatRef &m,
-                                          int klen, float *red) {
+__device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S, const Instr &in, const MatRef &m,
+                                          int klen, float *red, uint32_t gen) {
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int nb = in.nb;
     float *act = reinterpret_cast<float *>(S.act);
+    const uint32_t who = who_of(in);
+    bool ok = true;
     if (in.op == OP_DOWN || in.op == OP_OPROJ) {
-        // plain copy of the SwiGLU product or of the attention output, eight
-        // 16-byte loads in flight per thread
-        const int k0 = in.kb0 * m.kc, n4 = klen / 4;
-        const float *src = in.op == OP_DOWN ? P.act_a : P.attn;
-        const size_t rstride = in.op == OP_DOWN ? (size_t)P.i_pad : (size_t)P.o_nkb * P.o_kc;
+        // copy of the SwiGLU product or of the attention output; columns past
+        // the logical row (block padding) are zero
+        const int k0 = in.kb0 * m.kc, nch = klen / 8;
+        const uint64_t *src = in.op == OP_DOWN ? P.act_a : P.attn;
+        const int len = in.op == OP_DOWN ? P.intermediate : P.n_heads * P.head_dim;
+        const uint32_t tag = act_tag(gen, P.n_layers, in.layer);
         for (int b = 0; b < nb; ++b) {
-            const float4 *s4 = reinterpret_cast<const float4 *>(src + (size_t)(in.b0 + b) * rstride + k0);
-            float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen);
-            for (int v0 = t; v0 < n4; v0 += 8 * kConsumerThreads) {
-                float4 r[8];
+            const uint64_t *row = src + (size_t)(in.b0 + b) * len;
+            float *dst = act + (size_t)b * klen;
+            for (int c0 = t; c0 < nch; c0 += 2 * kConsumerThreads) {
+                const uint64_t *ptr[2];
+                int mm = 0;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int v = v0 + u * kConsumerThreads;
-                    r[u] = v < n4 ? __ldcg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int j = 0; j < 2; ++j) {
+                    const int c = c0 + j * kConsumerThreads;
+                    ptr[j] = row + k0 + (size_t)c * 8;
+                    if (c < nch && k0 + c * 8 < len) mm = j + 1;
                 }
+                float f[2][8];
+                ok = ll_chunks<2>(P, S, ptr, mm, tag, f, who) && ok;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int v = v0 + u * kConsumerThreads;
-                    if (v < n4) dst[v] = r[u];
+                for (int j = 0; j < 2; ++j) {
+                    const int c = c0 + j * kConsumerThreads;
+                    if (c < nch) {
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + (size_t)c * 8);
+                        if (j < mm) {
+                            d4[0] = make_float4(f[j][0], f[j][1], f[j][2], f[j][3]);
+                            d4[1] = make_float4(f[j][4], f[j][5], f[j][6], f[j][7]);
+                        } else {
+                            d4[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            d4[1] = d4[0];
+                        }
+                    }
                 }
             }
         }
-        return;
+        return ok;
     }
-    // RMSNorm(x) * gain with one pass over global memory: every thread loads
+    // RMSNorm(x) * gain with one pass over global memory: every thread reads
     // its chunks of x (all batch rows) together with the gains, accumulates
     // sum(x^2) and keeps x * gain in shared memory, then multiplies by the
     // per-row 1/rms once the sums are known (the gain and 1/rms commute).
+    // Gate/up reads x_mid of its own layer; QKV (layer > 0) and the LM head
+    // read x_mid plus the down parts of the previous layer.
     const int H = P.hidden;
     const uint16_t *gain = reinterpret_cast<const uint16_t *>(
         in.op == OP_QKV ? P.layers[in.layer].attn_norm
                         : (in.op == OP_GATEUP ? P.layers[in.layer].mlp_norm : P.final_norm));
     const bool from_embed = (in.flags & F_EMBED_X) && in.op == OP_QKV;
+    const bool with_down = in.op != OP_GATEUP;
+    const int xl = in.op == OP_GATEUP ? in.layer : (in.op == OP_LMHEAD ? P.n_layers - 1 : in.layer - 1);
+    const uint32_t xtag = act_tag(gen, P.n_layers, xl);
     const uint16_t *emb = reinterpret_cast<const uint16_t *>(P.embed);
     float ss[BS];
 #pragma unroll
     for (int b = 0; b < BS; ++b) ss[b] = 0.f;
     const int nch = klen / 8;
     const uint4 *g8 = reinterpret_cast<const uint4 *>(gain);
-    for (int c = t; c < nch; c += kConsumerThreads) {
-        const bool in_range = c * 8 < H;
-        float g[8];
-        if (in_range) unpack8(__ldg(g8 + c), g);
-        float f[BS][8];
+    // one batch row at a time keeps a single row's chunk in registers
 #pragma unroll
-        for (int b = 0; b < BS; ++b) {
-            const int row = in.b0 + (b < nb ? b : 0);
-            if (!in_range || b >= nb) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) f[b][q] = 0.f;
-            } else if (from_embed) {
-                unpack8(__ldg(reinterpret_cast<const uint4 *>(emb + (size_t)token_of(P, row) * H) + c), f[b]);
+    for (int b = 0; b < BS; ++b) {
+        if (b >= nb) break;
+        const int row = in.b0 + b;
+        for (int c = t; c < nch; c += kConsumerThreads) {
+            float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen + c * 8);
+            if (c * 8 >= H) {
+                dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                dst[1] = dst[0];
+                continue;
+            }
+            float f[8], g[8];
+            unpack8(__ldg(g8 + c), g);
+            if (from_embed) {
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(emb + (size_t)token_of(P, row) * H) + c), f);
+            } else if (with_down) {
+                ok = residual8(P, S, row, c * 8, xtag, f, who) && ok;
             } else {
-                const float4 *x = reinterpret_cast<const float4 *>(P.x + (size_t)row * H) + 2 * c;
-                const float4 x0 = __ldcg(x), x1 = __ldcg(x + 1);
-                f[b][0] = x0.x; f[b][1] = x0.y; f[b][2] = x0.z; f[b][3] = x0.w;
-                f[b][4] = x1.x; f[b][5] = x1.y; f[b][6] = x1.z; f[b][7] = x1.w;
-            }
-        }
+                const uint64_t *ptr[1] = {P.xm + (size_t)row * H + c * 8};
+                float f1[1][8];
+                ok = ll_chunks<1>(P, S, ptr, 1, xtag, f1, who) && ok;
 #pragma unroll
-        for (int b = 0; b < BS; ++b) {
-            if (b < nb) {
-                float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen + c * 8);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) ss[b] = fmaf(f[b][q], f[b][q], ss[b]);
-                if (in_range) {
-                    dst[0] = make_float4(f[b][0] * g[0], f[b][1] * g[1], f[b][2] * g[2], f[b][3] * g[3]);
-                    dst[1] = make_float4(f[b][4] * g[4], f[b][5] * g[5], f[b][6] * g[6], f[b][7] * g[7]);
-                } else {
-                    dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    dst[1] = dst[0];
-                }
+                for (int q = 0; q < 8; ++q) f[q] = f1[0][q];
             }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) ss[b] = fmaf(f[q], f[q], ss[b]);
+            dst[0] = make_float4(f[0] * g[0], f[1] * g[1], f[2] * g[2], f[3] * g[3]);
+            dst[1] = make_float4(f[4] * g[4], f[5] * g[5], f[6] * g[6], f[7] * g[7]);
         }
     }
 #pragma unroll
@@ -467,6 +613,7 @@ __device__ __forceinline__ void stage_act(const KParams &P, const SmemLayout &S,
             }
         }
     }
+    return ok;
 }
 
 // ------------------------------------------------------------------ GEMV: one warp per tile
@@ -507,11 +654,29 @@ __device__ __forceinline__ float key_value(unsigned long long k) {
 __device__ __forceinline__ int key_index(unsigned long long k) { return (int)(0xFFFFFFFFu - (uint32_t)k); }
 
 template <int BS, int RT>
-__device__ __forceinline__ void gemv_warp_tile(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                               const MatRef &m, int tile, uint32_t bi0, int klen) {
+__device__ __forceinline__ bool gemv_warp_tile(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
+                                               const MatRef &m, int tile, uint32_t bi0, int klen, uint32_t gen) {
     const int lane = threadIdx.x & 31;
     const int nkr = in.kb1 - in.kb0, kc = m.kc, nch = kc / 256, nb = in.nb;
     const float *act = reinterpret_cast<const float *>(S.act);
+    // row held by this lane after the fold: bit 4 is the top row bit, then bits 3, 2
+    int fr = 0;
+    if constexpr (RT == 8) fr = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+    if constexpr (RT == 4) fr = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+    if constexpr (RT == 2) fr = (lane >> 4) & 1;
+    const bool holder = (lane & (32 / RT - 1)) == 0;
+    const int H = P.hidden;
+    // The residual-stream word an epilogue adds to is read now, ahead of the
+    // dot products, so its round trip overlaps them: x_end of the previous
+    // layer for the O-projection, x_mid of this layer for the down
+    // projection's first K range.
+    const int n_out = tile * RT + fr;
+    const bool early = holder && n_out < H &&
+                       ((in.op == OP_OPROJ && !(in.flags & F_EMBED_X)) || (in.op == OP_DOWN && in.kb0 < P.down_per));
+    const uint64_t *early_src = in.op == OP_OPROJ ? P.xe : P.xm;
+    uint64_t pre[BS];
+#pragma unroll
+    for (int b = 0; b < BS; ++b) pre[b] = (early && b < nb) ? ll_ld(early_src + (size_t)(in.b0 + b) * H + n_out) : 0ull;
     float acc[RT][BS];
 #pragma unroll
     for (int r = 0; r < RT; ++r)
@@ -561,38 +726,60 @@ __device__ __forceinline__ void gemv_warp_tile(const KParams &P, const SmemLayou
         for (; o >= 1; o >>= 1) w[0] += __shfl_xor_sync(0xFFFFFFFFu, w[0], o);
         v[b] = w[0];
     }
-    // row held by this lane: bit 4 is the top row bit, then bits 3, 2
-    int fr = 0;
-    if constexpr (RT == 8) fr = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-    if constexpr (RT == 4) fr = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-    if constexpr (RT == 2) fr = (lane >> 4) & 1;
-    const bool holder = (lane & (32 / RT - 1)) == 0;
-    const int H = P.hidden;
+    // outputs carry this layer's tag (a stale one for the timeout test hook)
+    const uint32_t tag = act_tag(gen, P.n_layers, in.layer) - ((in.flags & F_DROP_SIGNAL) ? 1u : 0u);
+    bool ok = true;
     switch (in.op) {
         case OP_QKV: {
             const int n = tile * RT + fr;
             if (holder && n < P.qkv_rows)
 #pragma unroll
                 for (int b = 0; b < BS; ++b)
-                    if (b < nb) __stcg(P.qkv + (size_t)(in.b0 + b) * P.qkv_rows + n, v[b]);
+                    if (b < nb) ll_st(P.qkv + (size_t)(in.b0 + b) * P.qkv_rows + n, ll_pack(v[b], tag));
         } break;
-        case OP_OPROJ:
-        case OP_DOWN: {
-            const int n = tile * RT + fr;
-            if (holder && n < H)
+        case OP_OPROJ: {
+            // x_mid = x + attn . W_o^T, x being the embedding row (layer 0) or
+            // the residual leaving the previous layer
+            if (holder && n_out < H)
 #pragma unroll
                 for (int b = 0; b < BS; ++b) {
                     if (b >= nb) break;
                     const int row = in.b0 + b;
-                    float *xp = P.x + (size_t)row * H + n;
-                    if (in.flags & F_ATOMIC) {
-                        atomicAdd(xp, v[b]);
+                    float base;
+                    if (in.flags & F_EMBED_X) {
+                        base = bf2f(reinterpret_cast<const uint16_t *>(P.embed)[(size_t)token_of(P, row) * H + n_out]);
                     } else {
-                        const float base =
-                            (in.flags & F_EMBED_X)
-                                ? bf2f(reinterpret_cast<const uint16_t *>(P.embed)[(size_t)token_of(P, row) * H + n])
-                                : __ldcg(xp);
-                        __stcg(xp, base + v[b]);
+                        const uint32_t xtag = act_tag(gen, P.n_layers, in.layer - 1);
+                        const uint32_t who = who_of(in);
+                        if (ll_tag(pre[b]) == xtag) base = ll_value(pre[b]);
+                        else ok = ll_word(P, S, P.xe + (size_t)row * H + n_out, xtag, base, who) && ok;
+                        for (int k = 1; k < P.down_ranges; ++k) {
+                            float dv = 0.f;
+                            ok = ll_word(P, S, P.dpart + ((size_t)(k - 1) * P.batch + row) * H + n_out, xtag, dv, who) &&
+                                 ok;
+                            base += dv;
+                        }
+                    }
+                    ll_st(P.xm + (size_t)row * H + n_out, ll_pack(base + v[b], tag));
+                }
+        } break;
+        case OP_DOWN: {
+            // the first K range completes x_end = x_mid + its output; further
+            // ranges publish their outputs on their own
+            const int k = in.kb0 / P.down_per;
+            if (holder && n_out < H)
+#pragma unroll
+                for (int b = 0; b < BS; ++b) {
+                    if (b >= nb) break;
+                    const int row = in.b0 + b;
+                    if (k == 0) {
+                        const uint32_t mtag = act_tag(gen, P.n_layers, in.layer);
+                        float base;
+                        if (ll_tag(pre[b]) == mtag) base = ll_value(pre[b]);
+                        else ok = ll_word(P, S, P.xm + (size_t)row * H + n_out, mtag, base, who_of(in)) && ok;
+                        ll_st(P.xe + (size_t)row * H + n_out, ll_pack(base + v[b], tag));
+                    } else {
+                        ll_st(P.dpart + ((size_t)(k - 1) * P.batch + row) * H + n_out, ll_pack(v[b], tag));
                     }
                 }
         } break;
@@ -606,7 +793,8 @@ __device__ __forceinline__ void gemv_warp_tile(const KParams &P, const SmemLayou
 #pragma unroll
                 for (int b = 0; b < BS; ++b)
                     if (b < nb)
-                        __stcg(P.act_a + (size_t)(in.b0 + b) * P.i_pad + j, v[b] / (1.0f + __expf(-v[b])) * up[b]);
+                        ll_st(P.act_a + (size_t)(in.b0 + b) * P.intermediate + j,
+                              ll_pack(v[b] / (1.0f + __expf(-v[b])) * up[b], tag));
         } break;
         default: {  // OP_LMHEAD: logits, then the warp's best of this tile folded into the CTA's
             const int n = tile * RT + fr;
@@ -625,6 +813,7 @@ __device__ __forceinline__ void gemv_warp_tile(const KParams &P, const SmemLayou
             }
         } break;
     }
+    return ok;
 }
 
 // Publish this CTA's best (value, index) per sequence; the last CTA to do so
@@ -673,46 +862,68 @@ __device__ __forceinline__ void lm_publish(const KParams &P, const SmemLayout &S
 // One GEMV instruction: a run of consecutive tiles.  Tile k goes to warp
 // (tc + k) % warps (tc counts this CTA's tiles so far) and uses ring blocks
 // bc + k*nkr .. bc + (k+1)*nkr - 1 (bc counts this CTA's ring blocks so far).
+// Returns true when the CTA must stop (a wait gave up).
 template <int BS>
-__device__ __forceinline__ void gemv_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
-                                           uint64_t &act_tag, uint32_t gen, int pos, uint32_t &bc, uint32_t &tc,
+__device__ __forceinline__ bool gemv_instr(const KParams &P, const SmemLayout &S, CRing &ring, const Instr &in,
+                                           uint64_t &staged_key, uint32_t gen, int pos, uint32_t &bc, uint32_t &tc,
                                            int ii) {
     const int warp = threadIdx.x >> 5;
     const MatRef m = mat_of(P, in);
     const int nkr = in.kb1 - in.kb0, klen = nkr * m.kc;
-    const uint64_t tag = ((uint64_t)in.op << 56) | ((uint64_t)in.layer << 40) | ((uint64_t)in.b0 << 24) |
+    const uint64_t key = ((uint64_t)in.op << 56) | ((uint64_t)in.layer << 40) | ((uint64_t)in.b0 << 24) |
                          ((uint64_t)in.kb0 << 12) | (uint64_t)in.kb1;
-    if (tag != act_tag) {
+    if (key != staged_key) {
         consumer_sync();  // no warp still reads the previous activations
-        stage_act<BS>(P, S, in, m, klen, S.ssq);
-        act_tag = tag;
-        consumer_sync();
+        const bool ok = stage_act<BS>(P, S, in, m, klen, S.ssq, gen);
+        staged_key = key;
+        if (consumer_sync_or(!ok || *S.abort != 0)) return true;
     }
     if (P.trace && threadIdx.x == 0) P.trace[8 * (size_t)ii + 7] = globaltimer_ns();  // activations staged
     const int T = (int)in.ntiles;
+    bool ok = true;
     for (int k = (int)((warp - tc % kConsumerWarps + kConsumerWarps) % kConsumerWarps); k < T; k += kConsumerWarps) {
         const uint32_t bi0 = bc + (uint32_t)(k * nkr);
         switch (m.rows) {
-            case 8: gemv_warp_tile<BS, 8>(P, S, ring, in, m, (int)in.tile + k, bi0, klen); break;
-            case 4: gemv_warp_tile<BS, 4>(P, S, ring, in, m, (int)in.tile + k, bi0, klen); break;
-            case 2: gemv_warp_tile<BS, 2>(P, S, ring, in, m, (int)in.tile + k, bi0, klen); break;
-            default: gemv_warp_tile<BS, 1>(P, S, ring, in, m, (int)in.tile + k, bi0, klen); break;
+            case 8: ok = gemv_warp_tile<BS, 8>(P, S, ring, in, m, (int)in.tile + k, bi0, klen, gen) && ok; break;
+            case 4: ok = gemv_warp_tile<BS, 4>(P, S, ring, in, m, (int)in.tile + k, bi0, klen, gen) && ok; break;
+            case 2: ok = gemv_warp_tile<BS, 2>(P, S, ring, in, m, (int)in.tile + k, bi0, klen, gen) && ok; break;
+            default: ok = gemv_warp_tile<BS, 1>(P, S, ring, in, m, (int)in.tile + k, bi0, klen, gen) && ok; break;
         }
     }
     bc += (uint32_t)(T * nkr);
     tc += (uint32_t)T;
+    if ((in.op == OP_OPROJ || in.op == OP_DOWN) && consumer_sync_or(!ok || *S.abort != 0)) return true;  // epilogues read x
     if (in.op == OP_LMHEAD && (in.flags & F_LAST_LM)) lm_publish(P, S, in, gen, pos);
+    return false;
 }
 
 // ------------------------------------------------------------------ attention
 // One warp prepares one head: optional per-head RMSNorm, rotate-half RoPE at
 // `pos` (from the step's cos/sin table), scale.
-__device__ __forceinline__ void prep_head(const KParams &P, const SmemLayout &S, const float *src, const uint16_t *gain,
-                                          int pos, float scale, float *dst, uint16_t *cache_row) {
+__device__ __forceinline__ bool prep_head(const KParams &P, const SmemLayout &S, const uint64_t *src, uint32_t tag,
+                                          const uint16_t *gain, int pos, float scale, float *dst, uint16_t *cache_row) {
     const int lane = threadIdx.x & 31, d = P.head_dim, nj = d / 32, jh = nj / 2;
-    float v[4];
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    bool ok = true;
+    {
+        uint64_t w[4];
+        LlSpin sp{0ull, 0u};
+        for (;;) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = j < nj ? __ldcg(src + lane + 32 * j) : 0.f;
+            for (int j = 0; j < 4; ++j) w[j] = j < nj ? ll_ld(src + lane + 32 * j) : ll_pack(0.f, tag);
+            bool all = true;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) all = all && ll_tag(w[j]) == tag;
+            if (all) break;
+            __nanosleep(16);
+            if (!ll_spin(P, S, sp, ((uint32_t)OP_ATTN << 16), tag)) {
+                ok = false;
+                break;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = ll_value(w[j]);
+    }
     if (gain) {
         float s = 0.f;
 #pragma unroll
@@ -748,6 +959,7 @@ __device__ __forceinline__ void prep_head(const KParams &P, const SmemLayout &S,
             dst[lane + 32 * j] = o * scale;
         }
     }
+    return ok;
 }
 
 template <typename T>
@@ -769,10 +981,9 @@ __device__ __forceinline__ float ld1(const float *p) { return *p; }
 // s*32 + k*wph*32 + lane of every ring stage, one position per lane, and keeps
 // its own online-softmax state (running max m, sum l, unnormalised output o)
 // in registers, so a stage needs no CTA barrier.  The warps of a head merge at
-// the end and write the chunk's partial (o, m, l); the unit that completes its
-// (sequence, KV head) group combines the group's chunks with their
-// log-sum-exp weights into the attention output and signals the O-projection.
-constexpr int kAttnStop = 1, kAttnSignal = 2;
+// the end and write the chunk's partial (o, m, l) as tagged words; a combine
+// instruction later merges the group's chunks.
+constexpr int kAttnStop = 1;
 
 // DPL consecutive bf16 values (2 or 4) of one V row, widened.
 template <int DPL>
@@ -807,34 +1018,39 @@ __device__ __forceinline__ int attn_instr(const KParams &P, const SmemLayout &S,
     float *vpos = kpos + d;                         // [d] value of this step's position
     float *mrg = vpos + d;                          // [8 warps][d + 2] per-warp states
     float *pbuf = mrg + kConsumerWarps * (d + 2);   // [8 warps][32] probabilities
-    const float *qkv_b = P.qkv + (size_t)a.b * P.qkv_rows;
+    const uint64_t *qkv_b = P.qkv + (size_t)a.b * P.qkv_rows;
+    const uint32_t tag = act_tag(gen, P.n_layers, l);
     const LayerW *LW = P.layers + l;
     const float qscale = 1.4426950408889634f * rsqrtf((float)d);  // log2(e)/sqrt(d): scores in the exp2 domain
+    bool ok = true;
     consumer_sync();  // the previous instruction's readers of the activation region are done
     if (warp < G) {
-        prep_head(P, S, qkv_b + (a.g * G + warp) * d,
-                  P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->q_norm) : nullptr, pos, qscale, qs + warp * d,
-                  nullptr);
+        ok = prep_head(P, S, qkv_b + (a.g * G + warp) * d, tag,
+                       P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->q_norm) : nullptr, pos, qscale,
+                       qs + warp * d, nullptr);
     } else if (a.has_cur && warp == G) {
-        prep_head(P, S, qkv_b + nq * d + a.g * d, P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->k_norm) : nullptr,
-                  pos, 1.0f, kpos, P.kcache + kv_off(P, l, a.b, a.g, pos));
+        ok = prep_head(P, S, qkv_b + nq * d + a.g * d, tag,
+                       P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->k_norm) : nullptr, pos, 1.0f, kpos,
+                       P.kcache + kv_off(P, l, a.b, a.g, pos));
     }
     if (a.has_cur && warp == kConsumerWarps - 1) {
-        const float *vs = qkv_b + (nq + nkv) * d + a.g * d;
+        const uint64_t *vs = qkv_b + (nq + nkv) * d + a.g * d;
         uint16_t *vrow = P.vcache + kv_off(P, l, a.b, a.g, pos);
         for (int e = lane; e < d; e += 32) {
-            const uint16_t hv = f2bf(__ldcg(vs + e));
+            float vv = 0.f;
+            ok = ll_word(P, S, vs + e, tag, vv, (uint32_t)OP_ATTN << 16) && ok;
+            const uint16_t hv = f2bf(vv);
             vrow[e] = hv;
             vpos[e] = bf2f(hv);
         }
     }
-    consumer_sync();
+    if (consumer_sync_or(!ok || *S.abort != 0)) return kAttnStop;
     if (a.has_cur && G == kConsumerWarps) {  // every warp held a query head: the key comes now
         if (warp == 0)
-            prep_head(P, S, qkv_b + nq * d + a.g * d,
-                      P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->k_norm) : nullptr, pos, 1.0f, kpos,
-                      P.kcache + kv_off(P, l, a.b, a.g, pos));
-        consumer_sync();
+            ok = prep_head(P, S, qkv_b + nq * d + a.g * d, tag,
+                           P.qk_norm ? reinterpret_cast<const uint16_t *>(LW->k_norm) : nullptr, pos, 1.0f, kpos,
+                           P.kcache + kv_off(P, l, a.b, a.g, pos));
+        if (consumer_sync_or(!ok || *S.abort != 0)) return kAttnStop;
     }
     if (P.trace && t == 0) P.trace[8 * (size_t)ii + 7] = globaltimer_ns();  // heads prepared
     float m = -CUDART_INF_F, lsum = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
@@ -943,7 +1159,7 @@ __device__ __forceinline__ int attn_instr(const KParams &P, const SmemLayout &S,
         }
     }
     consumer_sync();
-    float *part = P.partials;
+    uint64_t *part = P.partials;
     if (active && sl == 0) {
         const int w0 = h * wph;
         float M = -CUDART_INF_F;
@@ -958,95 +1174,110 @@ __device__ __forceinline__ int attn_instr(const KParams &P, const SmemLayout &S,
                 if (e < dpl) O[e] = fmaf(wk, mrg[(w0 + k) * (d + 2) + lane * dpl + e], O[e]);
         }
         const int hg = a.g * G + h;
-        float *pd = part + (((size_t)a.b * nq + hg) * NC + a.c) * partial_stride(d);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            if (e < dpl) __stcg(pd + lane * dpl + e, O[e]);
-        if (lane == 0) {
-            __stcg(pd + d, M);
-            __stcg(pd + d + 1, L);
-        }
+        uint64_t *pd = part + (((size_t)a.b * nq + hg) * NC + a.c) * partial_stride(d);
+        const uint32_t ptag = tag - ((in.flags & F_DROP_SIGNAL) ? 1u : 0u);
+        ll_st2(pd + lane * dpl, ll_pack(O[0], ptag), ll_pack(O[1], ptag));
+        if (dpl == 4) ll_st2(pd + lane * dpl + 2, ll_pack(O[2], ptag), ll_pack(O[3], ptag));
+        if (lane == 0) ll_st2(pd + d, ll_pack(M, ptag), ll_pack(L, ptag));
     }
-    // Arrive on the group's counter; the unit that completes the group (all
-    // chunks of this sequence and KV head, this layer) combines the partials:
-    // attn[h*d + e] = sum_c 2^(m_c - M) o_c[e] / sum_c 2^(m_c - M) l_c.
-    consumer_sync();  // every partial store of this CTA is issued
-    if (t == 0) {
-        __threadfence();
-        const uint32_t target = (gen * (uint32_t)P.n_layers + (uint32_t)l + 1u) * in.arrive_count;
-        const uint32_t old = atom_acq_rel_add(P.counters + in.signal2_ctr, 1u);
-        *S.flag = (old + 1u == target) ? 1 : 0;
-    }
-    consumer_sync();
-    const bool last = *S.flag != 0;
-    if (last) {
-        // tpi threads (a power of two, same warp) share one float4 of output
-        // and take every tpi-th chunk, so each thread has at most four chunks'
-        // loads in flight; the group merges its (max, sum, vector) by shuffles
-        const int ps = partial_stride(d), items = G * d / 4;
-        int tpi = 1;
-        while (tpi < 16 && tpi < NC && 2 * tpi * items <= kConsumerThreads) tpi *= 2;
-        const int per_pass = kConsumerThreads / tpi, q = t % tpi;
-        float *dst = P.attn + (size_t)a.b * P.o_nkb * P.o_kc + (size_t)a.g * G * d;
-        for (int i0 = 0; i0 < items; i0 += per_pass) {
-            const int it = i0 + t / tpi;
-            const bool ok = it < items;
-            const int h = ok ? (4 * it) / d : 0, e = ok ? (4 * it) % d : 0;
-            const float *pc = part + (((size_t)a.b * nq + a.g * G + h) * NC) * ps;
-            float M = -CUDART_INF_F, L = 0.f;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int c0 = q; c0 < NC; c0 += 4 * tpi) {
-                float2 ml[4];
-                float4 ov[4];
+    return consumer_sync_or(*S.abort != 0) ? kAttnStop : 0;
+}
+
+// ------------------------------------------------------------------ split-KV combine
+// Merge the chunk partials of one (sequence, KV head) into its G heads'
+// attention output: attn[h*d + e] = sum_c 2^(m_c - M) o_c[e] / sum_c 2^(m_c - M) l_c,
+// M = max_c m_c (scores are in the base-2 domain).  tpi threads of one warp
+// share a float4 of output and take every tpi-th chunk, so each thread has at
+// most four chunks' loads in flight; they merge their (max, sum, vector) by
+// shuffles.  Returns true when the CTA must stop.
+__device__ __forceinline__ bool acomb_instr(const KParams &P, const SmemLayout &S, const Instr &in, uint32_t gen) {
+    const int t = threadIdx.x;
+    const int d = P.head_dim, nkv = P.n_kv_heads, G = P.n_heads / nkv, nq = P.n_heads, NC = P.chunks;
+    const int b = (int)in.tile / nkv, g = (int)in.tile % nkv;
+    const uint32_t tag = act_tag(gen, P.n_layers, in.layer);
+    const uint32_t otag = tag - ((in.flags & F_DROP_SIGNAL) ? 1u : 0u);
+    const int ps = partial_stride(d), items = G * d / 4;
+    int tpi = 1;
+    while (tpi < 16 && tpi < NC && 2 * tpi * items <= kConsumerThreads) tpi *= 2;
+    const int per_pass = kConsumerThreads / tpi, q = t % tpi;
+    uint64_t *dst = P.attn + (size_t)b * nq * d + (size_t)g * G * d;
+    bool ok = true;
+    for (int i0 = 0; i0 < items; i0 += per_pass) {
+        const int it = i0 + t / tpi;
+        const bool mine = it < items;
+        const int h = mine ? (4 * it) / d : 0, e = mine ? (4 * it) % d : 0;
+        const uint64_t *pc = P.partials + (((size_t)b * nq + g * G + h) * NC) * ps;
+        float M = -CUDART_INF_F, L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c0 = q; c0 < NC; c0 += 2 * tpi) {
+            ulonglong2 ml[2], o01[2], o23[2];
+            LlSpin sp{0ull, 0u};
+                for (;;) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     const int c = c0 + u * tpi;
-                    const bool in_range = ok && c < NC;
-                    ml[u] = in_range ? __ldcg(reinterpret_cast<const float2 *>(pc + (size_t)c * ps + d))
-                                     : make_float2(-CUDART_INF_F, 0.f);
-                    ov[u] = in_range ? __ldcg(reinterpret_cast<const float4 *>(pc + (size_t)c * ps + e))
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (mine && c < NC) {
+                        const uint64_t *r = pc + (size_t)c * ps;
+                        ml[u] = ll_ld2(r + d);
+                        o01[u] = ll_ld2(r + e);
+                        o23[u] = ll_ld2(r + e + 2);
+                    }
                 }
-                float Mn = M;
+                bool all = true;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) Mn = fmaxf(Mn, ml[u].x);
-                const float r = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mn);
-                L *= r;
-                acc.x *= r; acc.y *= r; acc.z *= r; acc.w *= r;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float w = (ml[u].x == -CUDART_INF_F) ? 0.f : exp2f(ml[u].x - Mn);
-                    L = fmaf(w, ml[u].y, L);
-                    acc.x = fmaf(w, ov[u].x, acc.x);
-                    acc.y = fmaf(w, ov[u].y, acc.y);
-                    acc.z = fmaf(w, ov[u].z, acc.z);
-                    acc.w = fmaf(w, ov[u].w, acc.w);
+                for (int u = 0; u < 2; ++u) {
+                    const int c = c0 + u * tpi;
+                    if (mine && c < NC)
+                        all = all && ll_tag(ml[u].x) == tag && ll_tag(ml[u].y) == tag && ll_tag(o01[u].x) == tag &&
+                              ll_tag(o01[u].y) == tag && ll_tag(o23[u].x) == tag && ll_tag(o23[u].y) == tag;
                 }
-                M = Mn;
+                if (all) break;
+                __nanosleep(16);
+                if (!ll_spin(P, S, sp, who_of(in), tag)) {
+                    ok = false;
+                    break;
+                }
             }
-            // merge the tpi partial states of this float4 (lanes q = 0 .. tpi-1)
-            for (int o2 = 1; o2 < tpi; o2 <<= 1) {
-                const float Mo = __shfl_xor_sync(0xFFFFFFFFu, M, o2);
-                const float Lo = __shfl_xor_sync(0xFFFFFFFFu, L, o2);
-                const float4 Ao = make_float4(__shfl_xor_sync(0xFFFFFFFFu, acc.x, o2), __shfl_xor_sync(0xFFFFFFFFu, acc.y, o2),
-                                              __shfl_xor_sync(0xFFFFFFFFu, acc.z, o2), __shfl_xor_sync(0xFFFFFFFFu, acc.w, o2));
-                const float Mn = fmaxf(M, Mo);
-                const float ra = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mn);
-                const float rb = (Mo == -CUDART_INF_F) ? 0.f : exp2f(Mo - Mn);
-                L = L * ra + Lo * rb;
-                acc = make_float4(acc.x * ra + Ao.x * rb, acc.y * ra + Ao.y * rb, acc.z * ra + Ao.z * rb,
-                                  acc.w * ra + Ao.w * rb);
-                M = Mn;
+            float Mn = M;
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                if (mine && c0 + u * tpi < NC) Mn = fmaxf(Mn, ll_value(ml[u].x));
+            const float r = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mn);
+            L *= r;
+            acc.x *= r; acc.y *= r; acc.z *= r; acc.w *= r;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                if (!(mine && c0 + u * tpi < NC)) continue;
+                const float mu = ll_value(ml[u].x);
+                const float w = (mu == -CUDART_INF_F) ? 0.f : exp2f(mu - Mn);
+                L = fmaf(w, ll_value(ml[u].y), L);
+                acc.x = fmaf(w, ll_value(o01[u].x), acc.x);
+                acc.y = fmaf(w, ll_value(o01[u].y), acc.y);
+                acc.z = fmaf(w, ll_value(o23[u].x), acc.z);
+                acc.w = fmaf(w, ll_value(o23[u].y), acc.w);
             }
-            if (ok && q == 0) {
-                const float inv = 1.0f / L;
-                __stcg(reinterpret_cast<float4 *>(dst + h * d + e),
-                       make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
-            }
+            M = Mn;
+        }
+        // merge the tpi partial states of this float4 (lanes q = 0 .. tpi-1)
+        for (int o2 = 1; o2 < tpi; o2 <<= 1) {
+            const float Mo = __shfl_xor_sync(0xFFFFFFFFu, M, o2);
+            const float Lo = __shfl_xor_sync(0xFFFFFFFFu, L, o2);
+            const float ax = __shfl_xor_sync(0xFFFFFFFFu, acc.x, o2), ay = __shfl_xor_sync(0xFFFFFFFFu, acc.y, o2);
+            const float az = __shfl_xor_sync(0xFFFFFFFFu, acc.z, o2), aw = __shfl_xor_sync(0xFFFFFFFFu, acc.w, o2);
+            const float Mn = fmaxf(M, Mo);
+            const float ra = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mn);
+            const float rb = (Mo == -CUDART_INF_F) ? 0.f : exp2f(Mo - Mn);
+            L = L * ra + Lo * rb;
+            acc = make_float4(acc.x * ra + ax * rb, acc.y * ra + ay * rb, acc.z * ra + az * rb, acc.w * ra + aw * rb);
+            M = Mn;
+        }
+        if (mine && q == 0) {
+            const float inv = 1.0f / L;
+            ll_st2(dst + h * d + e, ll_pack(acc.x * inv, otag), ll_pack(acc.y * inv, otag));
+            ll_st2(dst + h * d + e + 2, ll_pack(acc.z * inv, otag), ll_pack(acc.w * inv, otag));
         }
     }
-    const bool stop = consumer_sync_or(*S.abort != 0);
-    return (stop ? kAttnStop : 0) | (last ? kAttnSignal : 0);
+    return consumer_sync_or(!ok || *S.abort != 0);
 }
 
 // ------------------------------------------------------------------ consumer loop
@@ -1060,7 +1291,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
     const int t = threadIdx.x;
     CRing ring{0ull};
     uint32_t bc = 0, tc = 0;  // ring blocks and GEMV tiles of this CTA consumed so far
-    uint64_t act_tag = ~0ull;
+    uint64_t staged_key = ~0ull;  // which activations the shared-memory region holds
     uint32_t sat_ctr = 0xFFFFFFFFu, sat_target = 0u;
     uint32_t pend_ctr = kNoCounter, pend_n = 0u;
     bool stop = false;
@@ -1098,15 +1329,16 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
             P.trace[8 * (size_t)i + 0] = t_start;
             P.trace[8 * (size_t)i + 1] = globaltimer_ns();
         }
-        bool signal = in.op != OP_LMHEAD && !(in.flags & F_DROP_SIGNAL);
+        const bool signal = P.use_signals && in.op != OP_LMHEAD && !(in.flags & F_DROP_SIGNAL);
         if (in.op == OP_ATTN) {
             const int r = P.head_dim == 64 ? attn_instr<64>(P, S, ring, in, gen, pos, bc, i)
                                            : attn_instr<128>(P, S, ring, in, gen, pos, bc, i);
             stop = (r & kAttnStop) != 0;
-            signal = signal && (r & kAttnSignal) != 0;  // only the unit that completed its group
-            act_tag = ~0ull;
+            staged_key = ~0ull;
+        } else if (in.op == OP_ACOMB) {
+            stop = acomb_instr(P, S, in, gen);
         } else {
-            gemv_instr<BS>(P, S, ring, in, act_tag, gen, pos, bc, tc, i);
+            stop = gemv_instr<BS>(P, S, ring, in, staged_key, gen, pos, bc, tc, i);
         }
         if (!stop) {
             if (signal) {

@@ -102,7 +102,8 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     int down_split = 1;
     while ((size_t)p.bs * (((I + 255) / 256 * 256 + down_split - 1) / down_split) * 4 > (size_t)kActMax) ++down_split;
     p.down = make_mat(H, I, false, down_split);
-    p.down_ksplit = p.down.nkb;
+    p.down_ksplit = p.down.nkb;  // one K block per range: each range writes its own partial output
+    p.down_per = 1;
     p.i_pad = p.down.nkb * p.down.kc;
     const int down_blocks_per_range = 1;
     int act = 0;
@@ -125,14 +126,11 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
         --p.stages;
     if (p.stages < 2) return bad(MK_ERR_UNSUPPORTED, "not enough shared memory for the ring");
 
-    // Counters: five per layer (QKV, attention, O, gate/up, down), the LM-head
-    // arrival counter, then one split-KV arrival counter per (sequence, KV
-    // head), shared by all layers (a layer's units all arrive before the next
-    // layer's attention can start).
-    p.arr_attn = 5 * L + 1;
-    p.n_counters = p.arr_attn + B * nkv;
+    // Counters: six per layer (QKV, attention, combine, O, gate/up, down),
+    // then the LM-head arrival counter.
+    p.n_counters = kCountersPerLayer * L + 1;
     if (p.n_counters >= kNoCounter) return bad(MK_ERR_UNSUPPORTED, "too many counters");
-    const int arr_lm = 5 * L;
+    const int arr_lm = kCountersPerLayer * L;
     p.counter_count.assign(p.n_counters, 0);
 
     // ---------------------------------------------------------- instructions per phase
@@ -156,7 +154,7 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
                 for (int b0 = 0; b0 < B; b0 += bs) {
                     Instr in{};
                     in.op = op;
-                    in.flags = flags | (ksplit > 1 ? F_ATOMIC : 0);
+                    in.flags = flags;
                     in.layer = (uint16_t)l;
                     in.tile = (uint32_t)t0;
                     in.ntiles = (uint16_t)(t1 - t0);
@@ -192,22 +190,45 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
                         in.b0 = (uint16_t)b;
                         in.nb = 1;
                         in.wait_ctr = (uint16_t)counter_qkv(l);
-                        in.signal_ctr = (uint16_t)counter_att(l);  // by the last unit of (b, g) only
-                        in.signal2_ctr = (uint16_t)(p.arr_attn + b * nkv + g);
-                        in.arrive_count = (uint32_t)p.chunks;
+                        in.signal_ctr = (uint16_t)counter_att(l);
+                        in.signal2_ctr = kNoCounter;
                         v.push_back(in);
                         cost.push_back(typical_ctx / p.chunks * d * 4 + 8192.0);
                     }
-            p.counter_count[counter_att(l)] += (uint32_t)(B * nkv);
+            p.counter_count[counter_att(l)] += (uint32_t)v.size();
             phases.push_back(v);
             costs.push_back(cost);
         }
-        gemv_phase(OP_OPROJ, l, p.o, p.bs, 1, l == 0 ? F_EMBED_X : 0, counter_att(l), counter_o(l));
+        {  // one log-sum-exp combine per (sequence, KV head)
+            std::vector<Instr> v;
+            std::vector<double> cost;
+            for (int b = 0; b < B; ++b)
+                for (int g = 0; g < nkv; ++g) {
+                    Instr in{};
+                    in.op = OP_ACOMB;
+                    in.layer = (uint16_t)l;
+                    in.tile = (uint32_t)(b * nkv + g);
+                    in.b0 = (uint16_t)b;
+                    in.nb = 1;
+                    in.wait_ctr = (uint16_t)counter_att(l);
+                    in.signal_ctr = (uint16_t)counter_acomb(l);
+                    in.signal2_ctr = kNoCounter;
+                    v.push_back(in);
+                    cost.push_back((double)p.chunks * G * (d + 2) * 8 + 8192.0);
+                }
+            p.counter_count[counter_acomb(l)] += (uint32_t)v.size();
+            phases.push_back(v);
+            costs.push_back(cost);
+        }
+        gemv_phase(OP_OPROJ, l, p.o, p.bs, 1, l == 0 ? F_EMBED_X : 0, counter_acomb(l), counter_o(l));
         gemv_phase(OP_GATEUP, l, p.gu, p.gu_bs, 1, 0, counter_o(l), counter_gu(l));
         gemv_phase(OP_DOWN, l, p.down, p.bs, p.down_ksplit, 0, counter_gu(l), counter_down(l));
     }
     gemv_phase(OP_LMHEAD, L - 1, p.lm, p.bs, 1, 0, counter_down(L - 1), -1);
     p.n_phases = (int)phases.size();
+    for (int ph = 0; ph < p.n_phases; ++ph)
+        if (!phases[ph].empty() && ((phases[ph][0].flags & F_EMBED_X) || phases[ph][0].op == OP_LMHEAD))
+            p.token_phases.push_back(ph);
 
     // Fill wait counts now that every producer is known.
     for (auto &ph : phases)
@@ -277,11 +298,13 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     p.off_ranges = take((size_t)(p.n_phases + 2) * 2 * n_ctas * 4);
     p.off_layers = take((size_t)L * sizeof(LayerW));
     p.off_rope = take((size_t)(d / 2) * 8);
-    p.off_x = take((size_t)B * H * 4);
-    p.off_qkv = take((size_t)B * p.qkv_rows * 4);
-    p.off_attn = take((size_t)B * p.o.nkb * p.o.kc * 4);
-    p.off_act_a = take((size_t)B * p.i_pad * 4);
-    p.off_partials = take((size_t)B * nq * p.chunks * partial_stride(d) * 4);
+    p.off_x = take((size_t)B * H * 8);  // tagged words from here to off_lm_best
+    p.off_xe = take((size_t)B * H * 8);
+    p.off_dpart = take((size_t)(p.down_ksplit - 1) * B * H * 8);
+    p.off_qkv = take((size_t)B * p.qkv_rows * 8);
+    p.off_attn = take((size_t)B * nq * d * 8);
+    p.off_act_a = take((size_t)B * I * 8);
+    p.off_partials = take((size_t)B * nq * p.chunks * partial_stride(d) * 8);
     p.off_lm_best = take((size_t)B * n_ctas * sizeof(LmBest));
     p.off_next_scratch = take((size_t)B * 4);
     p.off_norms = take((size_t)(L * (2 * H + 2 * d) + H) * 2);
@@ -319,7 +342,8 @@ mk_status validate_plan(const Plan &p, std::string &err) {
             case OP_GATEUP: m = &p.gu; break;
             case OP_DOWN: m = &p.down; break;
             case OP_LMHEAD: m = &p.lm; break;
-            case OP_ATTN: break;
+            case OP_ATTN:
+            case OP_ACOMB: break;
             default:
                 snprintf(buf, sizeof buf, "instruction %zu: bad opcode %d", i, in.op);
                 return fail(buf);
@@ -332,9 +356,11 @@ mk_status validate_plan(const Plan &p, std::string &err) {
             if (in.nb > kMaxBatchRows) return fail("GEMV instruction carries too many batch rows");
             if ((size_t)in.nb * (in.kb1 - in.kb0) * m->kc * 4 > (size_t)p.act_bytes)
                 return fail("GEMV activation range does not fit the shared-memory region");
-            if ((in.flags & F_ATOMIC) && in.op != OP_DOWN) return fail("K-split only allowed for down");
-        } else {
+        } else if (in.op == OP_ATTN) {
             if (in.tile >= (uint32_t)(p.B * c.n_kv_heads * p.chunks)) return fail("attention unit out of range");
+        } else {
+            if (in.tile >= (uint32_t)(p.B * c.n_kv_heads) || in.b0 != in.tile / c.n_kv_heads)
+                return fail("combine unit out of range");
         }
         if (in.wait_ctr != kNoCounter && in.wait_ctr >= p.n_counters) return fail("wait counter out of range");
         if (in.signal_ctr != kNoCounter && in.signal_ctr >= p.n_counters) return fail("signal counter out of range");
@@ -357,12 +383,6 @@ mk_status validate_plan(const Plan &p, std::string &err) {
                         const uint32_t a = ++ctr[in.signal_ctr];
                         if (a > in.arrive_count) return fail("more arrivals than expected");
                     }
-                } else if (in.op == OP_ATTN) {
-                    // the unit that completes its (sequence, KV head) group signals
-                    const uint32_t a = ++ctr[in.signal2_ctr];
-                    if (in.arrive_count == 0 || a > (uint32_t)c.n_layers * in.arrive_count)
-                        return fail("more split-KV arrivals than expected");
-                    if (a % in.arrive_count == 0) ++ctr[in.signal_ctr];
                 } else if (in.signal_ctr != kNoCounter) {
                     ++ctr[in.signal_ctr];
                 }
@@ -386,11 +406,6 @@ mk_status validate_plan(const Plan &p, std::string &err) {
         if (in.wait_ctr != kNoCounter && ctr[in.wait_ctr] != in.wait_count) {
             snprintf(buf, sizeof buf, "counter %d receives %u increments per step but instruction %zu expects %u",
                      in.wait_ctr, ctr[in.wait_ctr], i, in.wait_count);
-            return fail(buf);
-        }
-        if (in.op == OP_ATTN && ctr[in.signal2_ctr] != (uint32_t)c.n_layers * in.arrive_count) {
-            snprintf(buf, sizeof buf, "split-KV arrival counter %d gets %u arrivals, expected %u", in.signal2_ctr,
-                     ctr[in.signal2_ctr], (uint32_t)c.n_layers * in.arrive_count);
             return fail(buf);
         }
         if (in.op == OP_LMHEAD && (in.flags & F_LAST_LM) && ctr[in.signal_ctr] != in.arrive_count) {

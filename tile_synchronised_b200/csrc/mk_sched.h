@@ -22,14 +22,15 @@ struct Plan {
     int chunks = 0;          // split-KV chunks per (sequence, KV head)
     int stages = 0;          // ring slots
     int act_bytes = 0;       // shared-memory activation region
-    int down_ksplit = 1;     // K ranges of the down projection (>1: atomic residual update)
-    int arr_attn = 0;        // first split-KV arrival counter (one per sequence and KV head)
+    int down_ksplit = 1;     // K ranges of the down projection (each writes its own partial output)
+    int down_per = 1;        // K blocks per down-projection range
+    std::vector<int> token_phases;  // phases that read the tokens or write the step's outputs
     int qkv_rows = 0, i_pad = 0;
     PackedMat qkv{}, o{}, gu{}, down{}, lm{};
 
     // workspace layout (byte offsets)
     size_t off_state = 0, off_counters = 0, off_instrs = 0, off_ranges = 0, off_layers = 0, off_rope = 0;
-    size_t off_x = 0, off_qkv = 0, off_attn = 0, off_act_a = 0, off_partials = 0, off_lm_best = 0;
+    size_t off_x = 0, off_xe = 0, off_dpart = 0, off_qkv = 0, off_attn = 0, off_act_a = 0, off_partials = 0, off_lm_best = 0;
     size_t off_next_scratch = 0, off_weights = 0, layer_weight_bytes = 0, off_lm = 0, off_norms = 0;
     size_t workspace_bytes = 0, kv_bytes = 0;
 
@@ -47,10 +48,13 @@ mk_status build_plan(const mk_config &cfg, int n_ctas, int swiglu_variant, Plan 
 // Simulate the schedule on the host; MK_OK or MK_ERR_STATE with a reason.
 mk_status validate_plan(const Plan &plan, std::string &err);
 
-inline int counter_qkv(int l) { return 5 * l + 0; }
-inline int counter_att(int l) { return 5 * l + 1; }
-inline int counter_o(int l) { return 5 * l + 2; }
-inline int counter_gu(int l) { return 5 * l + 3; }
-inline int counter_down(int l) { return 5 * l + 4; }
+// Tile-ready counters, six per layer, then the LM-head arrival counter.
+constexpr int kCountersPerLayer = 6;
+inline int counter_qkv(int l) { return kCountersPerLayer * l + 0; }
+inline int counter_att(int l) { return kCountersPerLayer * l + 1; }
+inline int counter_acomb(int l) { return kCountersPerLayer * l + 2; }
+inline int counter_o(int l) { return kCountersPerLayer * l + 3; }
+inline int counter_gu(int l) { return kCountersPerLayer * l + 4; }
+inline int counter_down(int l) { return kCountersPerLayer * l + 5; }
 
 }  // namespace mk

@@ -18,7 +18,7 @@ import sys
 import numpy as np
 import torch
 
-OPS = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead"}
+OPS = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "acomb"}
 
 
 def summarise(sched, base, tr):
@@ -77,6 +77,7 @@ def main(argv=None):
     ap.add_argument("--max-seq", type=int, default=None)
     ap.add_argument("--prefetch", type=int, default=None, help="L2 prefetch distance (ring blocks)")
     ap.add_argument("--time", type=int, default=0, help="also time this many steps (CUDA events)")
+    ap.add_argument("--sync", default="tags", choices=sorted(mk.SYNCS))
     a = ap.parse_args(argv)
     shape = synth.MODELS[a.workload]
     B = a.batch or shape.batch
@@ -87,6 +88,7 @@ def main(argv=None):
     tokens = synth.make_tokens(shape, prefill + a.steps, batch=B)
     if a.prefetch is not None:
         model.set_prefetch(a.prefetch)
+    model.set_sync(a.sync)
     if prefill:
         model.prefill(tokens[:, :prefill].cuda())
     d_tok = tokens[:, prefill:].t().contiguous().cuda()  # [steps, B]
@@ -102,7 +104,7 @@ def main(argv=None):
         e1.record()
         torch.cuda.synchronize()
         print(json.dumps({"timed_steps": a.time, "us_per_step": round(1e3 * e0.elapsed_time(e1) / a.time, 2),
-                          "prefetch": a.prefetch}))
+                          "prefetch": a.prefetch, "sync": a.sync}))
         model.set_position(prefill + a.steps - 1)
     tr = None
     if a.trace:
@@ -116,13 +118,13 @@ def main(argv=None):
         raise SystemExit(f"device status {st}: {model.last_error()}")
     if a.trace:
         sched, base = model.schedule()
-        summ = summarise(sched, base, tr.cpu().numpy())
-        summ.update({"workload": a.workload, "batch": B, "prefill": prefill, "variant": a.variant,
-                     "schedule": model.info()})
         stem = a.trace.replace(".json", "")
         np.save(stem + "_raw.npy", tr.cpu().numpy())
         np.save(stem + "_sched.npy", sched)
         np.save(stem + "_base.npy", base)
+        summ = summarise(sched, base, tr.cpu().numpy())
+        summ.update({"workload": a.workload, "batch": B, "prefill": prefill, "variant": a.variant,
+                     "sync": a.sync, "schedule": model.info()})
         with open(a.trace, "w") as f:
             json.dump(summ, f, indent=1)
         print(json.dumps({k: v for k, v in summ.items() if k != "phases"}, indent=1))
