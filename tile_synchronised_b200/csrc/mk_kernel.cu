@@ -507,19 +507,19 @@ __device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S,
         for (int b = 0; b < nb; ++b) {
             const uint64_t *row = src + (size_t)(in.b0 + b) * len;
             float *dst = act + (size_t)b * klen;
-            for (int c0 = t; c0 < nch; c0 += 2 * kConsumerThreads) {
-                const uint64_t *ptr[2];
+            for (int c0 = t; c0 < nch; c0 += 4 * kConsumerThreads) {
+                const uint64_t *ptr[4];
                 int mm = 0;
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
+                for (int j = 0; j < 4; ++j) {
                     const int c = c0 + j * kConsumerThreads;
                     ptr[j] = row + k0 + (size_t)c * 8;
                     if (c < nch && k0 + c * 8 < len) mm = j + 1;
                 }
-                float f[2][8];
-                ok = ll_chunks<2>(P, S, ptr, mm, tag, f, who) && ok;
+                float f[4][8];
+                ok = ll_chunks<4>(P, S, ptr, mm, tag, f, who) && ok;
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
+                for (int j = 0; j < 4; ++j) {
                     const int c = c0 + j * kConsumerThreads;
                     if (c < nch) {
                         float4 *d4 = reinterpret_cast<float4 *>(dst + (size_t)c * 8);
@@ -1017,7 +1017,7 @@ __device__ __forceinline__ int attn_instr(const KParams &P, const SmemLayout &S,
     float *kpos = qs + G * d;                       // [d] key of this step's position
     float *vpos = kpos + d;                         // [d] value of this step's position
     float *mrg = vpos + d;                          // [8 warps][d + 2] per-warp states
-    float *pbuf = mrg + kConsumerWarps * (d + 2);   // [8 warps][32] probabilities
+    float *pbuf = mrg + kConsumerWarps * (d + 2);   // [8 warps][64] probabilities
     const uint64_t *qkv_b = P.qkv + (size_t)a.b * P.qkv_rows;
     const uint32_t tag = act_tag(gen, P.n_layers, l);
     const LayerW *LW = P.layers + l;
@@ -1055,80 +1055,86 @@ __device__ __forceinline__ int attn_instr(const KParams &P, const SmemLayout &S,
     if (P.trace && t == 0) P.trace[8 * (size_t)ii + 7] = globaltimer_ns();  // heads prepared
     float m = -CUDART_INF_F, lsum = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
     const float *qh = qs + (active ? h : 0) * d;
-    float *pw = pbuf + warp * 32;  // this warp's probabilities, broadcast to all lanes for P.V
+    float *pw = pbuf + warp * 64;  // this warp's probabilities, broadcast to all lanes for P.V
     for (int st = 0; st < a.nstages; ++st) {
         const int n = min(sp, a.tma_end - (a.p0 + st * sp));
         const uint8_t *slot = ring_wait(P, S, ring, bc + st);
         if (active) {
             const uint16_t *K = reinterpret_cast<const uint16_t *>(slot);
             const uint16_t *V = reinterpret_cast<const uint16_t *>(slot + kStageBytes / 2);
-            for (int base = sl * 32; base < n; base += wph * 32) {
-                const int j = base + lane;
-                const bool valid = j < n;
-                // score of position j: two interleaved FMA chains over the
-                // head's NCH 8-column chunks, visited in a per-lane rotated
-                // order so the lanes' 16-byte reads hit different banks
-                float s0 = 0.f, s1 = 0.f;
-                if (valid) {
-                    const uint16_t *kr = K + (size_t)j * D;
+            // Each pass takes two 32-position groups of this warp's share
+            // (base and base + 32 * wph), one position of each per lane, so
+            // every q load and every reduction serves two positions.
+            for (int base = sl * 32; base < n; base += 2 * wph * 32) {
+                const int j0 = base + lane, j1 = base + wph * 32 + lane;
+                const bool v0 = j0 < n, v1 = j1 < n;
+                float a0 = 0.f, b0 = 0.f, a1 = 0.f, b1 = 0.f;
+                const uint16_t *kr0 = K + (size_t)(v0 ? j0 : 0) * D, *kr1 = K + (size_t)(v1 ? j1 : 0) * D;
 #pragma unroll
-                    for (int k = 0; k < NCH; ++k) {
-                        const int cc = (k + lane) & (NCH - 1);
-                        float kf[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(kr + cc * 8), kf);
-                        const float4 q0 = *reinterpret_cast<const float4 *>(qh + cc * 8);
-                        const float4 q1 = *reinterpret_cast<const float4 *>(qh + cc * 8 + 4);
-                        s0 = fmaf(q0.x, kf[0], s0);
-                        s1 = fmaf(q0.y, kf[1], s1);
-                        s0 = fmaf(q0.z, kf[2], s0);
-                        s1 = fmaf(q0.w, kf[3], s1);
-                        s0 = fmaf(q1.x, kf[4], s0);
-                        s1 = fmaf(q1.y, kf[5], s1);
-                        s0 = fmaf(q1.z, kf[6], s0);
-                        s1 = fmaf(q1.w, kf[7], s1);
-                    }
+                for (int k = 0; k < NCH; ++k) {
+                    // rotated chunk order: the lanes' 16-byte reads hit different banks
+                    const int cc = (k + lane) & (NCH - 1);
+                    float k0[8], k1[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(kr0 + cc * 8), k0);
+                    unpack8(*reinterpret_cast<const uint4 *>(kr1 + cc * 8), k1);
+                    const float4 q0 = *reinterpret_cast<const float4 *>(qh + cc * 8);
+                    const float4 q1 = *reinterpret_cast<const float4 *>(qh + cc * 8 + 4);
+                    a0 = fmaf(q0.x, k0[0], a0); b0 = fmaf(q0.y, k0[1], b0);
+                    a1 = fmaf(q0.x, k1[0], a1); b1 = fmaf(q0.y, k1[1], b1);
+                    a0 = fmaf(q0.z, k0[2], a0); b0 = fmaf(q0.w, k0[3], b0);
+                    a1 = fmaf(q0.z, k1[2], a1); b1 = fmaf(q0.w, k1[3], b1);
+                    a0 = fmaf(q1.x, k0[4], a0); b0 = fmaf(q1.y, k0[5], b0);
+                    a1 = fmaf(q1.x, k1[4], a1); b1 = fmaf(q1.y, k1[5], b1);
+                    a0 = fmaf(q1.z, k0[6], a0); b0 = fmaf(q1.w, k0[7], b0);
+                    a1 = fmaf(q1.z, k1[6], a1); b1 = fmaf(q1.w, k1[7], b1);
                 }
-                const float sc = valid ? s0 + s1 : -CUDART_INF_F;
-                const float mb = warp_max(sc);
+                const float sc0 = v0 ? a0 + b0 : -CUDART_INF_F, sc1 = v1 ? a1 + b1 : -CUDART_INF_F;
+                const float mb = warp_max(fmaxf(sc0, sc1));
                 const float mnew = fmaxf(m, mb);
                 const float corr = exp2f(m - mnew);
-                const float p = valid ? exp2f(sc - mnew) : 0.f;
-                lsum = lsum * corr + warp_sum(p);
+                const float p0 = v0 ? exp2f(sc0 - mnew) : 0.f, p1 = v1 ? exp2f(sc1 - mnew) : 0.f;
+                lsum = lsum * corr + warp_sum(p0 + p1);
                 m = mnew;
-                pw[lane] = p;
+                pw[lane] = p0;
+                pw[32 + lane] = p1;
                 __syncwarp();
                 // P.V: lane owns DPL dimensions; rows four at a time, two
                 // accumulator sets so consecutive FMAs do not depend on each other
-                const int cnt = min(32, n - base);
                 float oa[DPL], ob[DPL];
 #pragma unroll
                 for (int e = 0; e < DPL; ++e) oa[e] = ob[e] = 0.f;
-                const uint16_t *vb = V + (size_t)base * D + lane * DPL;
-                int jj = 0;
-                for (; jj + 4 <= cnt; jj += 4) {
-                    const float4 p4 = *reinterpret_cast<const float4 *>(pw + jj);
-                    float v0[DPL], v1[DPL], v2[DPL], v3[DPL];
-                    load_dpl<DPL>(vb + (size_t)(jj + 0) * D, v0);
-                    load_dpl<DPL>(vb + (size_t)(jj + 1) * D, v1);
-                    load_dpl<DPL>(vb + (size_t)(jj + 2) * D, v2);
-                    load_dpl<DPL>(vb + (size_t)(jj + 3) * D, v3);
 #pragma unroll
-                    for (int e = 0; e < DPL; ++e) {
-                        oa[e] = fmaf(p4.x, v0[e], oa[e]);
-                        ob[e] = fmaf(p4.y, v1[e], ob[e]);
-                        oa[e] = fmaf(p4.z, v2[e], oa[e]);
-                        ob[e] = fmaf(p4.w, v3[e], ob[e]);
+                for (int grp = 0; grp < 2; ++grp) {
+                    const int gbase = base + grp * wph * 32;
+                    const int cnt = max(0, min(32, n - gbase));
+                    const float *pg = pw + grp * 32;
+                    const uint16_t *vb = V + (size_t)gbase * D + lane * DPL;
+                    int jj = 0;
+                    for (; jj + 4 <= cnt; jj += 4) {
+                        const float4 p4 = *reinterpret_cast<const float4 *>(pg + jj);
+                        float w0[DPL], w1[DPL], w2[DPL], w3[DPL];
+                        load_dpl<DPL>(vb + (size_t)(jj + 0) * D, w0);
+                        load_dpl<DPL>(vb + (size_t)(jj + 1) * D, w1);
+                        load_dpl<DPL>(vb + (size_t)(jj + 2) * D, w2);
+                        load_dpl<DPL>(vb + (size_t)(jj + 3) * D, w3);
+#pragma unroll
+                        for (int e = 0; e < DPL; ++e) {
+                            oa[e] = fmaf(p4.x, w0[e], oa[e]);
+                            ob[e] = fmaf(p4.y, w1[e], ob[e]);
+                            oa[e] = fmaf(p4.z, w2[e], oa[e]);
+                            ob[e] = fmaf(p4.w, w3[e], ob[e]);
+                        }
                     }
-                }
-                for (; jj < cnt; ++jj) {
-                    float v0[DPL];
-                    load_dpl<DPL>(vb + (size_t)jj * D, v0);
+                    for (; jj < cnt; ++jj) {
+                        float w0[DPL];
+                        load_dpl<DPL>(vb + (size_t)jj * D, w0);
 #pragma unroll
-                    for (int e = 0; e < DPL; ++e) oa[e] = fmaf(pw[jj], v0[e], oa[e]);
+                        for (int e = 0; e < DPL; ++e) oa[e] = fmaf(pg[jj], w0[e], oa[e]);
+                    }
                 }
 #pragma unroll
                 for (int e = 0; e < DPL; ++e) o[e] = fmaf(o[e], corr, oa[e] + ob[e]);
-                __syncwarp();  // pw is rewritten by the next 32 positions
+                __syncwarp();  // pw is rewritten by the next pass
             }
         }
         __syncwarp();

@@ -118,7 +118,7 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     // last unit of a (sequence, KV head) gathers every chunk's partial.
     p.chunks = std::max(1, std::min(kMaxAttnChunks, n_ctas / (B * nkv)));
     p.chunks = std::min(p.chunks, std::max(1, c.max_seq / 16));
-    const int attn_scratch = G * d * 4 + 2 * d * 4 + kConsumerWarps * (d + 2) * 4 + kConsumerWarps * 32 * 4;
+    const int attn_scratch = G * d * 4 + 2 * d * 4 + kConsumerWarps * (d + 2) * 4 + kConsumerWarps * 64 * 4;
     act = std::max(act, attn_scratch);
     p.act_bytes = (int)align_up(act, 128);
     p.stages = kMaxStages;
