@@ -182,6 +182,13 @@ mk_status mk_tune(mk_ctx *ctx, void *stream, int *chosen);
  * an input).  Default 10; 0 disables prefetching.  0..64. */
 mk_status mk_set_prefetch(mk_ctx *ctx, int blocks);
 
+/* Shared-memory ring slots (32 KB each) the producer may fill: 0 (default)
+ * uses as many as the plan's shared memory allows, otherwise the smaller of
+ * `stages` and that.  Fewer slots keep fewer weight loads in flight per SM
+ * ahead of the consumers' activation reads.  0 or 2..8; MK_ERR_INVALID
+ * otherwise. */
+mk_status mk_set_ring_stages(mk_ctx *ctx, int stages);
+
 /* Device wait limit in nanoseconds (default 1e9).  A wait that runs out sets
  * the context's error word and makes every CTA return early. */
 mk_status mk_set_timeout_ns(mk_ctx *ctx, unsigned long long ns);

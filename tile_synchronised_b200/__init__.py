@@ -178,6 +178,10 @@ class Model(Plan):
         activations, the default) or "counters" (tile-ready counters)."""
         check(self.lib.mk_set_sync(self.ctx, SYNCS[name]), self.ctx, "mk_set_sync")
 
+    def set_ring_stages(self, stages: int) -> None:
+        """Ring slots the producer may fill (0: as many as fit)."""
+        check(self.lib.mk_set_ring_stages(self.ctx, int(stages)), self.ctx, "mk_set_ring_stages")
+
     def set_timeout_ns(self, ns: int) -> None:
         check(self.lib.mk_set_timeout_ns(self.ctx, int(ns)), self.ctx, "mk_set_timeout_ns")
 

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MK_OK", -1: "MK_ERR_INVALID", -2: "MK_ERR_CUDA", -3: "MK_ERR
 # Every symbol include/mk.h declares.
 EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk_kv_cache_bytes",
            "mk_load_weights", "mk_prefill_kv", "mk_decode_step", "mk_get_status", "mk_reset",
-           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch", "mk_set_timeout_ns", "mk_set_sync", "mk_debug_drop_signal",
+           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch", "mk_set_timeout_ns", "mk_set_sync", "mk_set_ring_stages", "mk_debug_drop_signal",
            "mk_set_trace", "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1", "mk_swiglu_tune",
            "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks",
            "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes")
@@ -86,6 +86,7 @@ def load() -> C.CDLL:
         "mk_set_prefetch": ([vp, i32], st),
         "mk_set_timeout_ns": ([vp, C.c_ulonglong], st),
         "mk_set_sync": ([vp, i32], st),
+        "mk_set_ring_stages": ([vp, i32], st),
         "mk_debug_drop_signal": ([vp, i32], st),
         "mk_set_trace": ([vp, vp, sz], st),
         "mk_get_schedule": ([vp, vp, sz, vp], st),

@@ -29,6 +29,7 @@ struct mk_ctx {
     unsigned long long *trace = nullptr;
     int prefetch = 10;  // furthest L2 prefetch distance in ring blocks
     int sync = MK_SYNC_TAGS;
+    int stages = 0;  // ring slots in use (0: all the plan's shared memory allows)
     const void *embed = nullptr;
     // captured graph of the separate-kernels variant
     cudaGraph_t graph = nullptr;
@@ -243,7 +244,7 @@ static KParams make_params(mk_ctx *c, const int32_t *tokens, int64_t tok_stride,
     P.i_pad = p.i_pad;
     P.chunks = p.chunks;
     P.n_ctas = p.n_ctas;
-    P.stages = p.stages;
+    P.stages = (c->stages > 0 && c->stages < p.stages) ? c->stages : p.stages;
     P.act_bytes = p.act_bytes;
     P.qk_norm = g.qk_norm;
     P.bs = p.bs;
@@ -567,6 +568,14 @@ mk_status mk_set_variant(mk_ctx *c, int variant) {
 mk_status mk_set_prefetch(mk_ctx *c, int blocks) {
     if (!c || blocks < 0 || blocks > 64) return MK_ERR_INVALID;
     c->prefetch = blocks;
+    drop_graph(c);
+    return MK_OK;
+}
+
+mk_status mk_set_ring_stages(mk_ctx *c, int stages) {
+    if (!c || stages < 0 || stages > kMaxStages) return MK_ERR_INVALID;
+    if (stages == 1) return fail(c, MK_ERR_INVALID, "the ring needs at least 2 slots");
+    c->stages = stages;
     drop_graph(c);
     return MK_OK;
 }

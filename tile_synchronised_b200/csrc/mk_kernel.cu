@@ -1286,6 +1286,12 @@ __device__ __forceinline__ bool acomb_instr(const KParams &P, const SmemLayout &
     return consumer_sync_or(!ok || *S.abort != 0);
 }
 
+// Counter increment after an instruction's outputs are stored: a release,
+// so a reader that acquires the counter sees the data.
+__device__ __forceinline__ void signal_counter(const KParams &P, uint32_t ctr, uint32_t n) {
+    red_release_add(P.counters + ctr, n);
+}
+
 // ------------------------------------------------------------------ consumer loop
 // Signals are batched: a CTA adds the number of instructions it finished for a
 // counter in one release when it moves on to another counter, and always
@@ -1321,7 +1327,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
             if (in.wait_ctr != sat_ctr || target != sat_target) {
                 if (pend_n) consumer_sync();  // this CTA's earlier writes are complete
                 if (t == 0) {
-                    if (pend_n) red_release_add(P.counters + pend_ctr, pend_n);
+                    if (pend_n) signal_counter(P, pend_ctr, pend_n);
                     if (!wait_counter(P, in.wait_ctr, target, (uint32_t)i)) *S.abort = 1;
                 }
                 pend_n = 0u;
@@ -1351,7 +1357,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
                 if (pend_ctr != in.signal_ctr) {
                     if (pend_n) {
                         consumer_sync();
-                        if (t == 0) red_release_add(P.counters + pend_ctr, pend_n);
+                        if (t == 0) signal_counter(P, pend_ctr, pend_n);
                     }
                     pend_ctr = in.signal_ctr;
                     pend_n = 0u;
@@ -1368,7 +1374,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
     }
     if (!stop && pend_n) {
         consumer_sync();
-        if (t == 0) red_release_add(P.counters + pend_ctr, pend_n);
+        if (t == 0) signal_counter(P, pend_ctr, pend_n);
     }
 }
 

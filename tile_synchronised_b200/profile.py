@@ -78,6 +78,7 @@ def main(argv=None):
     ap.add_argument("--prefetch", type=int, default=None, help="L2 prefetch distance (ring blocks)")
     ap.add_argument("--time", type=int, default=0, help="also time this many steps (CUDA events)")
     ap.add_argument("--sync", default="tags", choices=sorted(mk.SYNCS))
+    ap.add_argument("--stages", type=int, default=0, help="ring slots in use (0: all that fit)")
     a = ap.parse_args(argv)
     shape = synth.MODELS[a.workload]
     B = a.batch or shape.batch
@@ -89,6 +90,7 @@ def main(argv=None):
     if a.prefetch is not None:
         model.set_prefetch(a.prefetch)
     model.set_sync(a.sync)
+    model.set_ring_stages(a.stages)
     if prefill:
         model.prefill(tokens[:, :prefill].cuda())
     d_tok = tokens[:, prefill:].t().contiguous().cuda()  # [steps, B]
@@ -104,7 +106,7 @@ def main(argv=None):
         e1.record()
         torch.cuda.synchronize()
         print(json.dumps({"timed_steps": a.time, "us_per_step": round(1e3 * e0.elapsed_time(e1) / a.time, 2),
-                          "prefetch": a.prefetch, "sync": a.sync}))
+                          "prefetch": a.prefetch, "sync": a.sync, "stages": a.stages}))
         model.set_position(prefill + a.steps - 1)
     tr = None
     if a.trace:
