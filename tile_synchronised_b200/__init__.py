@@ -75,9 +75,12 @@ class Plan:
         check(self.lib.mk_validate_schedule(self.ctx), self.ctx, "mk_validate_schedule")
 
     def close(self):
-        if self.ctx:
-            self.lib.mk_destroy(self.ctx)
-            self.ctx = C.c_void_p()
+        ctx, self.ctx = self.ctx, None
+        if ctx:
+            try:
+                self.lib.mk_destroy(ctx)
+            except Exception:  # noqa: BLE001 - interpreter shutdown: the library may be gone
+                pass
 
     __del__ = close
 
