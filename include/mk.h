@@ -72,8 +72,10 @@ enum {
 };
 /* Tilings of the fused SwiGLU first stage ("Deep Kernel Fusion for
  * Transformers", Key points, "Fusion scope": row-major tiling reuses the
- * activations, column-major tiling reuses the weights). */
-enum { MK_SWIGLU_AUTO = 0, MK_SWIGLU_ROW = 1, MK_SWIGLU_COL = 2 };
+ * activations, column-major tiling reuses the weights).  MK_SWIGLU_TC runs
+ * both projections as tcgen05 MMAs with tensor-memory accumulators (batches
+ * that are multiples of 16, where the projections are dense GEMMs). */
+enum { MK_SWIGLU_AUTO = 0, MK_SWIGLU_ROW = 1, MK_SWIGLU_COL = 2, MK_SWIGLU_TC = 3 };
 
 /* Architecture and limits of one context. */
 typedef struct {
@@ -239,18 +241,22 @@ mk_status mk_validate_schedule(const mk_ctx *ctx);
  *   out[b][n] = SiLU(sum_k x[b][k] w_gate[k][n]) * sum_k x[b][k] w_up[k][n]
  * x: device fp16 [B, K] row-major; w_gate, w_up: device fp16 [K, N] row-major
  * (N contiguous); out: device fp16 [B, N].  fp32 accumulation, SiLU in fp32,
- * one rounding to fp16 at the end.  variant: MK_SWIGLU_ROW, MK_SWIGLU_COL or
- * MK_SWIGLU_AUTO (the variant mk_swiglu_tune picked for this (B, K, N), else
- * COL for B <= 8 and ROW above).  Needs K % 64 == 0, N % 64 == 0, 1 <= B <= 64,
- * all pointers 16-byte aligned; MK_ERR_INVALID otherwise.  Allocates nothing. */
+ * one rounding to fp16 at the end.  variant: MK_SWIGLU_ROW, MK_SWIGLU_COL,
+ * MK_SWIGLU_TC or MK_SWIGLU_AUTO (the variant mk_swiglu_tune picked for this
+ * (B, K, N), else MK_SWIGLU_TC where it applies, COL for B <= 8 and ROW
+ * above).  Needs K % 64 == 0, N % 64 == 0, 1 <= B <= 64, all pointers 16-byte
+ * aligned; MK_SWIGLU_TC also needs B % 16 == 0 and N % 128 == 0
+ * (MK_ERR_UNSUPPORTED otherwise).  MK_ERR_INVALID on bad arguments.
+ * Allocates nothing. */
 mk_status mk_swiglu_stage1(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K, int N,
                            int variant, void *stream);
-/* Time both variants on the given buffers (synchronous; `out` is
- * overwritten), remember the faster for (B, K, N) in a process-wide table and
- * return it in *chosen.  Per-variant mean microseconds go to us_row/us_col
- * (may be NULL). */
+/* Time every applicable variant on the given buffers (synchronous; `out` is
+ * overwritten), remember the fastest for (B, K, N) in a process-wide table
+ * and return it in *chosen.  Mean microseconds go to us_row, us_col and
+ * us_tc (each may be NULL; us_tc gets 0 when the tensor-core variant does not
+ * apply). */
 mk_status mk_swiglu_tune(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K, int N,
-                         void *stream, int *chosen, float *us_row, float *us_col);
+                         void *stream, int *chosen, float *us_row, float *us_col, float *us_tc);
 
 /* Split-KV decode attention with a log-sum-exp combine, on its own: the
  * attention of one layer of one decode step ("Look Ma, No Bubbles! Designing

@@ -10,12 +10,13 @@ import ctypes as C
 
 import torch
 
-from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW, MK_SYNC_COUNTERS,
+from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW, MK_SWIGLU_TC,
+                   MK_SYNC_COUNTERS,
                    MK_SYNC_TAGS,
                    MkConfig, MkError, MkWeights, check, load)
 
 __all__ = ["Model", "swiglu_stage1", "swiglu_tune", "MkError", "VARIANTS", "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW",
-           "MK_SWIGLU_COL", "load"]
+           "MK_SWIGLU_COL", "MK_SWIGLU_TC", "load"]
 
 VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL}
 SYNCS = {"tags": MK_SYNC_TAGS, "counters": MK_SYNC_COUNTERS}
@@ -214,14 +215,16 @@ def swiglu_stage1(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor, out
 
 
 def swiglu_tune(x, w_gate, w_up, out, stream=None):
-    """Time both tilings once and remember the faster; returns (chosen, us_row, us_col)."""
+    """Time every applicable tiling once and remember the fastest; returns
+    (chosen, us_row, us_col, us_tc) with us_tc 0 where the tensor-core variant
+    does not apply."""
     B, K = x.shape
     N = w_gate.shape[1]
-    ch, ur, uc = C.c_int(), C.c_float(), C.c_float()
+    ch, ur, uc, ut = C.c_int(), C.c_float(), C.c_float(), C.c_float()
     check(load().mk_swiglu_tune(C.c_void_p(x.data_ptr()), C.c_void_p(w_gate.data_ptr()), C.c_void_p(w_up.data_ptr()),
                                 C.c_void_p(out.data_ptr()), B, K, N, _stream(stream), C.byref(ch), C.byref(ur),
-                                C.byref(uc)), None, "mk_swiglu_tune")
-    return ch.value, ur.value, uc.value
+                                C.byref(uc), C.byref(ut)), None, "mk_swiglu_tune")
+    return ch.value, ur.value, uc.value, ut.value
 
 
 def _attn_shapes(q: torch.Tensor, k_cache: torch.Tensor):

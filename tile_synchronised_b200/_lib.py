@@ -13,7 +13,7 @@ from . import build as _build
 MK_OK, MK_ERR_INVALID, MK_ERR_CUDA, MK_ERR_TIMEOUT, MK_ERR_UNSUPPORTED, MK_ERR_STATE = 0, -1, -2, -3, -4, -5
 MK_BF16 = 0
 MK_MEGAKERNEL, MK_GRAPH, MK_GRAPH_PDL = 0, 1, 2
-MK_SWIGLU_AUTO, MK_SWIGLU_ROW, MK_SWIGLU_COL = 0, 1, 2
+MK_SWIGLU_AUTO, MK_SWIGLU_ROW, MK_SWIGLU_COL, MK_SWIGLU_TC = 0, 1, 2, 3
 MK_SYNC_TAGS, MK_SYNC_COUNTERS = 0, 1
 
 STATUS_NAMES = {0: "MK_OK", -1: "MK_ERR_INVALID", -2: "MK_ERR_CUDA", -3: "MK_ERR_TIMEOUT",
@@ -94,7 +94,7 @@ def load() -> C.CDLL:
         "mk_validate_schedule": ([vp], st),
         "mk_swiglu_stage1": ([vp, vp, vp, vp, i32, i32, i32, i32, vp], st),
         "mk_swiglu_tune": ([vp, vp, vp, vp, i32, i32, i32, vp, C.POINTER(i32), C.POINTER(C.c_float),
-                            C.POINTER(C.c_float)], st),
+                            C.POINTER(C.c_float), C.POINTER(C.c_float)], st),
         "mk_attention_decode": ([vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp, sz, vp], st),
         "mk_attention_scratch_bytes": ([i32, i32, i32, i32], sz),
         "mk_attention_chunks": ([i32, i32, i32], i32),

@@ -15,6 +15,10 @@ cudaError_t launch_set_position(State *state, int pos, cudaStream_t s);
 // Fused SwiGLU first stage (fp16): variant MK_SWIGLU_ROW or MK_SWIGLU_COL.
 cudaError_t launch_swiglu(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N, int variant,
                           cudaStream_t s);
+// The same stage on the tcgen05 tensor cores (B a multiple of 16, N of 128).
+bool swiglu_tc_supported(int B, int K, int N);
+cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N,
+                             cudaStream_t s);
 // Last error of a context-free call (the isolated operations) on this thread.
 void set_op_error(const char *msg);
 const char *op_error();

@@ -142,41 +142,56 @@ static bool swiglu_args_ok(const void *x, const void *wg, const void *wu, const 
     return true;
 }
 
+static cudaError_t run_variant(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N,
+                               int variant, cudaStream_t s) {
+    return variant == MK_SWIGLU_TC ? launch_swiglu_tc(x, wg, wu, out, B, K, N, s)
+                                   : launch_swiglu(x, wg, wu, out, B, K, N, variant, s);
+}
+
 extern "C" mk_status mk_swiglu_stage1(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K,
                                       int N, int variant, void *stream) {
     if (!swiglu_args_ok(x, w_gate, w_up, out, B, K, N)) return MK_ERR_INVALID;
     if (variant == MK_SWIGLU_AUTO) {
         std::lock_guard<std::mutex> lk(g_tune_mu);
         auto it = g_tuned.find({B, K, N});
-        variant = it != g_tuned.end() ? it->second : (B <= 8 ? MK_SWIGLU_COL : MK_SWIGLU_ROW);
+        variant = it != g_tuned.end() ? it->second
+                                      : (swiglu_tc_supported(B, K, N) ? MK_SWIGLU_TC
+                                                                      : (B <= 8 ? MK_SWIGLU_COL : MK_SWIGLU_ROW));
     }
-    if (variant != MK_SWIGLU_ROW && variant != MK_SWIGLU_COL) return MK_ERR_INVALID;
-    cudaError_t e = launch_swiglu(x, w_gate, w_up, out, B, K, N, variant, static_cast<cudaStream_t>(stream));
+    if (variant != MK_SWIGLU_ROW && variant != MK_SWIGLU_COL && variant != MK_SWIGLU_TC) return MK_ERR_INVALID;
+    if (variant == MK_SWIGLU_TC && !swiglu_tc_supported(B, K, N)) return MK_ERR_UNSUPPORTED;
+    cudaError_t e = run_variant(x, w_gate, w_up, out, B, K, N, variant, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MK_OK : MK_ERR_CUDA;
 }
 
 extern "C" mk_status mk_swiglu_tune(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K,
-                                    int N, void *stream, int *chosen, float *us_row, float *us_col) {
+                                    int N, void *stream, int *chosen, float *us_row, float *us_col, float *us_tc) {
     if (!swiglu_args_ok(x, w_gate, w_up, out, B, K, N)) return MK_ERR_INVALID;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaEvent_t e0, e1;
     if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) return MK_ERR_CUDA;
     const int reps = 20;
-    float us[2];
-    const int vs[2] = {MK_SWIGLU_ROW, MK_SWIGLU_COL};
-    for (int i = 0; i < 2; ++i) {
-        if (launch_swiglu(x, w_gate, w_up, out, B, K, N, vs[i], s) != cudaSuccess) return MK_ERR_CUDA;
+    const int vs[3] = {MK_SWIGLU_ROW, MK_SWIGLU_COL, MK_SWIGLU_TC};
+    float us[3] = {0.f, 0.f, 0.f};
+    const int nv = swiglu_tc_supported(B, K, N) ? 3 : 2;
+    int best = MK_SWIGLU_COL;
+    float best_us = 0.f;
+    for (int i = 0; i < nv; ++i) {
+        if (run_variant(x, w_gate, w_up, out, B, K, N, vs[i], s) != cudaSuccess) return MK_ERR_CUDA;
         cudaEventRecord(e0, s);
-        for (int r = 0; r < reps; ++r) launch_swiglu(x, w_gate, w_up, out, B, K, N, vs[i], s);
+        for (int r = 0; r < reps; ++r) run_variant(x, w_gate, w_up, out, B, K, N, vs[i], s);
         cudaEventRecord(e1, s);
         if (cudaEventSynchronize(e1) != cudaSuccess) return MK_ERR_CUDA;
         float ms = 0.f;
         cudaEventElapsedTime(&ms, e0, e1);
         us[i] = ms * 1000.f / reps;
+        if (i == 0 || us[i] < best_us) {
+            best_us = us[i];
+            best = vs[i];
+        }
     }
     cudaEventDestroy(e0);
     cudaEventDestroy(e1);
-    const int best = us[0] < us[1] ? MK_SWIGLU_ROW : MK_SWIGLU_COL;
     {
         std::lock_guard<std::mutex> lk(g_tune_mu);
         g_tuned[{B, K, N}] = best;
@@ -184,5 +199,6 @@ extern "C" mk_status mk_swiglu_tune(const void *x, const void *w_gate, const voi
     if (chosen) *chosen = best;
     if (us_row) *us_row = us[0];
     if (us_col) *us_col = us[1];
+    if (us_tc) *us_tc = us[2];
     return cudaGetLastError() == cudaSuccess ? MK_OK : MK_ERR_CUDA;
 }

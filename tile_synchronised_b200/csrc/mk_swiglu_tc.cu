@@ -1,0 +1,278 @@
+// mk_swiglu_tc.cu -- the fused SwiGLU first stage on the 5th-generation tensor
+// cores (tcgen05), for batches of 16 and more, where the two projections are
+// dense GEMMs ("Deep Kernel Fusion for Transformers", Key points, "Fusion
+// scope": Up and Gate GEMMs, SiLU and the product in one kernel).
+//
+//   out[b][n] = SiLU(sum_k x[b][k] Wg[k][n]) * sum_k x[b][k] Wu[k][n]
+//
+// One CTA owns 128 output features n0 .. n0+127 and the whole batch.  The
+// MMA computes D[m][b] = sum_k W[k][n0+m] x[b][k] with the weights as operand
+// A (M = 128, MN-major: n is contiguous in W) and x as operand B (N = batch,
+// K-major), both staged by TMA with 128-byte swizzling, fp32 accumulators for
+// gate and up in tensor memory.  Warp 0 lane 0 issues the TMA loads of a
+// 4..5-stage ring, warp 1 lane 0 issues the MMAs and commits each stage back
+// to its "empty" barrier, then all four warps read the accumulators out of
+// tensor memory (one row per thread) and write SiLU(g) * u as fp16.
+// Every barrier wait is bounded; a wait that runs out stops the CTA and its
+// outputs are written as NaN so that the failure cannot pass for a result.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/mk.h"
+#include "mk_device.cuh"
+#include "mk_kernel.h"
+
+namespace mk {
+
+constexpr int kTcM = 128;           // output features per CTA (MMA M)
+constexpr int kTcBK = 64;           // K per stage: one 128-byte swizzle row of fp16
+constexpr int kTcThreads = 128;
+constexpr uint64_t kTcTimeoutNs = 2000000000ull;
+
+struct TcShape {
+    int B, K, N, stages;
+    uint32_t stage_bytes, a_bytes, x_bytes;
+};
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Bounded wait for the phase `parity` of an mbarrier; false after the time
+// limit or once another role of the CTA has given up.
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_sleep(bar, parity, 10000u)) return true;
+        if ((it & 7u) == 0u) {
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > kTcTimeoutNs) {
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2,
+// descriptor version 1): start address, leading and stride byte offsets, all
+// in 16-byte units.
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void *p, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    const uint64_t start = (smem_addr(p) >> 4) & 0x3FFFu;
+    return start | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) | ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulate, fp16 A and B, A
+// MN-major, B K-major, M = 128, N = batch.
+__host__ __device__ constexpr uint32_t tc_idesc(int n) {
+    return (1u << 4)                    // D format: F32
+           | (0u << 7) | (0u << 10)     // A, B format: F16
+           | (1u << 15)                 // A MN-major
+           | (0u << 16)                 // B K-major
+           | ((uint32_t)(n >> 3) << 17) // N >> 3
+           | ((uint32_t)(kTcM >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    swiglu_tc_kernel(const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_u,
+                     const __grid_constant__ CUtensorMap map_x, __half *__restrict__ out, TcShape sh) {
+    extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
+    // stages start on a 1024-byte boundary (128-byte swizzle atoms)
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int S = sh.stages, B = sh.B;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * sh.stage_bytes);
+    uint64_t *empty = full + S;
+    uint64_t *done = empty + S;
+    volatile uint32_t *tmem_base = reinterpret_cast<volatile uint32_t *>(done + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+    const int n0 = blockIdx.x * kTcM;
+    const int nkb = sh.K / kTcBK;
+    const uint32_t ncols = B <= 16 ? 32u : (B <= 32 ? 64u : (B <= 64 ? 128u : 256u));  // gate + up, power of two
+
+    if (t == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {  // the whole warp allocates the accumulators
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(const_cast<uint32_t *>(tmem_base))),
+                     "r"(ncols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        // producer: W_gate and W_up as two 64-feature boxes each, x as one box
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % S;
+            if (kb >= S && !tc_wait(&empty[s], ((kb / S) - 1) & 1u, abort)) break;
+            uint8_t *st = smem + (size_t)s * sh.stage_bytes;
+            mbar_arrive_expect_tx(&full[s], sh.stage_bytes);
+            const int k0 = kb * kTcBK;
+            tma_load_2d(st, &map_g, n0, k0, &full[s]);
+            tma_load_2d(st + sh.a_bytes / 2, &map_g, n0 + 64, k0, &full[s]);
+            tma_load_2d(st + sh.a_bytes, &map_u, n0, k0, &full[s]);
+            tma_load_2d(st + sh.a_bytes + sh.a_bytes / 2, &map_u, n0 + 64, k0, &full[s]);
+            tma_load_2d(st + 2 * sh.a_bytes, &map_x, k0, 0, &full[s]);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer.  A (weights, MN-major): two 64-feature atoms 8 KB apart
+        // (LBO), 8 k-rows of 128 B per swizzle group (SBO 1 KB); a K step of
+        // 16 is two groups, 2 KB.  B (x, K-major): 8 rows per group (SBO
+        // 1 KB); a K step of 16 is 32 bytes along the row.
+        const uint32_t idesc = tc_idesc(B);
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % S;
+            if (!tc_wait(&full[s], (kb / S) & 1u, abort)) break;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint8_t *st = smem + (size_t)s * sh.stage_bytes;
+#pragma unroll
+            for (int ks = 0; ks < kTcBK / 16; ++ks) {
+                const uint64_t ag = smem_desc_sw128(st + ks * 2048, sh.a_bytes / 2, 1024);
+                const uint64_t au = smem_desc_sw128(st + sh.a_bytes + ks * 2048, sh.a_bytes / 2, 1024);
+                const uint64_t bx = smem_desc_sw128(st + 2 * sh.a_bytes + ks * 32, 16, 1024);
+                const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+                tc_mma(tmem, ag, bx, idesc, acc);
+                tc_mma(tmem + (uint32_t)B, au, bx, idesc, acc);
+            }
+            tc_commit(&empty[s]);
+        }
+        tc_commit(done);
+    }
+    __syncwarp();
+    // epilogue: thread t holds row m = t of both accumulators (tensor-memory
+    // lane t; warp w may read lanes 32w .. 32w+31)
+    const bool ok = tc_wait(done, 0u, abort) && !*abort;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int n = n0 + t;
+    for (int c0 = 0; c0 < B; c0 += 16) {
+        float g[16], u[16];
+        tmem_ld16(lane_addr + (uint32_t)c0, g);
+        tmem_ld16(lane_addr + (uint32_t)(B + c0), u);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float r = ok ? g[i] / (1.0f + __expf(-g[i])) * u[i] : __int_as_float(0x7fc00000);
+            out[(size_t)(c0 + i) * sh.N + n] = __float2half_rn(r);
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiled encode_fn() {
+    static std::once_flag once;
+    static EncodeTiled fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    });
+    return fn;
+}
+
+// 2-D fp16 tensor [rows][cols] (cols contiguous), box box_cols x box_rows, 128-byte swizzle.
+static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                     uint32_t box_rows) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool swiglu_tc_supported(int B, int K, int N) {
+    return B >= 16 && B <= 128 && B % 16 == 0 && K % kTcBK == 0 && N % kTcM == 0;
+}
+
+cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N,
+                             cudaStream_t s) {
+    CUtensorMap mg, mu, mx;
+    if (!make_map(&mg, wg, (uint64_t)K, (uint64_t)N, 64, kTcBK) || !make_map(&mu, wu, (uint64_t)K, (uint64_t)N, 64, kTcBK) ||
+        !make_map(&mx, x, (uint64_t)B, (uint64_t)K, kTcBK, (uint32_t)B))
+        return cudaErrorInvalidValue;
+    TcShape sh;
+    sh.B = B;
+    sh.K = K;
+    sh.N = N;
+    sh.a_bytes = (uint32_t)kTcM * kTcBK * 2;  // one matrix's stage: 2 atoms of 64 features x 64 k
+    sh.x_bytes = (uint32_t)B * kTcBK * 2;
+    sh.stage_bytes = 2 * sh.a_bytes + sh.x_bytes;
+    const int budget = 227 * 1024 - 1024 - 256;  // alignment slack and the barriers
+    sh.stages = budget / (int)sh.stage_bytes;
+    if (sh.stages > 6) sh.stages = 6;
+    if (sh.stages < 2) return cudaErrorInvalidValue;
+    const int smem = sh.stages * (int)sh.stage_bytes + 1024 + 256;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(swiglu_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    swiglu_tc_kernel<<<N / kTcM, kTcThreads, smem, s>>>(mg, mu, mx, static_cast<__half *>(out), sh);
+    return cudaGetLastError();
+}
+
+}  // namespace mk
