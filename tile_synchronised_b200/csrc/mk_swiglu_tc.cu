@@ -5,14 +5,17 @@
 //
 //   out[b][n] = SiLU(sum_k x[b][k] Wg[k][n]) * sum_k x[b][k] Wu[k][n]
 //
-// One CTA owns 128 output features n0 .. n0+127 and the whole batch.  The
-// MMA computes D[m][b] = sum_k W[k][n0+m] x[b][k] with the weights as operand
-// A (M = 128, MN-major: n is contiguous in W) and x as operand B (N = batch,
-// K-major), both staged by TMA with 128-byte swizzling, fp32 accumulators for
-// gate and up in tensor memory.  Warp 0 lane 0 issues the TMA loads of a
-// 4..5-stage ring, warp 1 lane 0 issues the MMAs and commits each stage back
-// to its "empty" barrier, then all four warps read the accumulators out of
-// tensor memory (one row per thread) and write SiLU(g) * u as fp16.
+// A cluster of two CTAs owns 128 output features n0 .. n0+127 and the whole
+// batch; each CTA of the pair takes half of K, so twice as many SMs stream
+// the weights.  The MMA computes D[m][b] = sum_k W[k][n0+m] x[b][k] with the
+// weights as operand A (M = 128, MN-major: n is contiguous in W) and x as
+// operand B (N = batch, K-major), both staged by TMA with 128-byte swizzling,
+// fp32 accumulators for gate and up in tensor memory.  Warp 0 lane 0 issues
+// the TMA loads of a 4..6-stage ring, warp 1 lane 0 issues the MMAs and
+// commits each stage back to its "empty" barrier.  Then the second CTA of the
+// pair reads its accumulators out of tensor memory (one row per thread) and
+// stores them into the first CTA's shared memory over the cluster; the first
+// adds them to its own and writes SiLU(g) * u as fp16.
 // Every barrier wait is bounded; a wait that runs out stops the CTA and its
 // outputs are written as NaN so that the failure cannot pass for a result.
 #include <cuda.h>
@@ -33,10 +36,30 @@ constexpr int kTcBK = 64;           // K per stage: one 128-byte swizzle row of 
 constexpr int kTcThreads = 128;
 constexpr uint64_t kTcTimeoutNs = 2000000000ull;
 
+constexpr int kTcSplit = 2;         // CTAs per cluster, each on its share of K
+
 struct TcShape {
     int B, K, N, stages;
     uint32_t stage_bytes, a_bytes, x_bytes;
 };
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t cluster_map(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
     asm volatile(
@@ -125,8 +148,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *done = empty + S;
     volatile uint32_t *tmem_base = reinterpret_cast<volatile uint32_t *>(done + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
-    const int n0 = blockIdx.x * kTcM;
-    const int nkb = sh.K / kTcBK;
+    const uint32_t rank = cluster_rank();
+    const int n0 = (blockIdx.x / kTcSplit) * kTcM;
+    const int nkb_all = sh.K / kTcBK;
+    const int kb_first = (int)rank * nkb_all / kTcSplit, nkb = (int)(rank + 1) * nkb_all / kTcSplit - kb_first;
     const uint32_t ncols = B <= 16 ? 32u : (B <= 32 ? 64u : (B <= 64 ? 128u : 256u));  // gate + up, power of two
 
     if (t == 0) {
@@ -157,7 +182,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (kb >= S && !tc_wait(&empty[s], ((kb / S) - 1) & 1u, abort)) break;
             uint8_t *st = smem + (size_t)s * sh.stage_bytes;
             mbar_arrive_expect_tx(&full[s], sh.stage_bytes);
-            const int k0 = kb * kTcBK;
+            const int k0 = (kb_first + kb) * kTcBK;
             tma_load_2d(st, &map_g, n0, k0, &full[s]);
             tma_load_2d(st + sh.a_bytes / 2, &map_g, n0 + 64, k0, &full[s]);
             tma_load_2d(st + sh.a_bytes, &map_u, n0, k0, &full[s]);
@@ -194,15 +219,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const bool ok = tc_wait(done, 0u, abort) && !*abort;
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    const int n = n0 + t;
-    for (int c0 = 0; c0 < B; c0 += 16) {
-        float g[16], u[16];
-        tmem_ld16(lane_addr + (uint32_t)c0, g);
-        tmem_ld16(lane_addr + (uint32_t)(B + c0), u);
+    // The first CTA's stage memory is free once both CTAs are past their
+    // final MMA; it then receives the second CTA's accumulators, column-major
+    // [2B][128], and its "ok" word after them.
+    float *part = reinterpret_cast<float *>(smem);
+    volatile int *part_ok = reinterpret_cast<volatile int *>(part + 2 * B * kTcM);
+    cluster_sync_all();
+    if (rank == 1) {
+        const uint32_t remote = cluster_map(part, 0);
+        for (int c0 = 0; c0 < 2 * B; c0 += 16) {
+            float v[16];
+            tmem_ld16(lane_addr + (uint32_t)c0, v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float r = ok ? g[i] / (1.0f + __expf(-g[i])) * u[i] : __int_as_float(0x7fc00000);
-            out[(size_t)(c0 + i) * sh.N + n] = __float2half_rn(r);
+            for (int i = 0; i < 16; ++i) st_cluster_f32(remote + (uint32_t)(((c0 + i) * kTcM + t) * 4), v[i]);
+        }
+        if (t == 0) st_cluster_f32(cluster_map((const void *)part_ok, 0), ok ? 1.f : 0.f);
+    }
+    cluster_sync_all();
+    if (rank == 0) {
+        const bool all_ok = ok && *reinterpret_cast<volatile float *>(part_ok) != 0.f;
+        const int n = n0 + t;
+        for (int c0 = 0; c0 < B; c0 += 16) {
+            float g[16], u[16];
+            tmem_ld16(lane_addr + (uint32_t)c0, g);
+            tmem_ld16(lane_addr + (uint32_t)(B + c0), u);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float gs = g[i] + part[(c0 + i) * kTcM + t], us = u[i] + part[(B + c0 + i) * kTcM + t];
+                const float r = all_ok ? gs / (1.0f + __expf(-gs)) * us : __int_as_float(0x7fc00000);
+                out[(size_t)(c0 + i) * sh.N + n] = __float2half_rn(r);
+            }
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -244,7 +290,7 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t c
 }
 
 bool swiglu_tc_supported(int B, int K, int N) {
-    return B >= 16 && B <= 128 && B % 16 == 0 && K % kTcBK == 0 && N % kTcM == 0;
+    return B >= 16 && B <= 128 && B % 16 == 0 && K % (kTcBK * kTcSplit) == 0 && N % kTcM == 0;
 }
 
 cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N,
@@ -271,8 +317,19 @@ cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    swiglu_tc_kernel<<<N / kTcM, kTcThreads, smem, s>>>(mg, mu, mx, static_cast<__half *>(out), sh);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((N / kTcM) * kTcSplit);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kTcSplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, swiglu_tc_kernel, mg, mu, mx, static_cast<__half *>(out), sh);
 }
 
 }  // namespace mk
