@@ -73,8 +73,8 @@ enum {
 /* Tilings of the fused SwiGLU first stage ("Deep Kernel Fusion for
  * Transformers", Key points, "Fusion scope": row-major tiling reuses the
  * activations, column-major tiling reuses the weights).  MK_SWIGLU_TC runs
- * both projections as tcgen05 MMAs with tensor-memory accumulators (batches
- * that are multiples of 16, where the projections are dense GEMMs). */
+ * both projections as tcgen05 MMAs with tensor-memory accumulators (the
+ * batch is the MMA's N, rounded up to 16 with zero rows in shared memory). */
 enum { MK_SWIGLU_AUTO = 0, MK_SWIGLU_ROW = 1, MK_SWIGLU_COL = 2, MK_SWIGLU_TC = 3 };
 
 /* Architecture and limits of one context. */
@@ -245,7 +245,7 @@ mk_status mk_validate_schedule(const mk_ctx *ctx);
  * MK_SWIGLU_TC or MK_SWIGLU_AUTO (the variant mk_swiglu_tune picked for this
  * (B, K, N), else MK_SWIGLU_TC where it applies, COL for B <= 8 and ROW
  * above).  Needs K % 64 == 0, N % 64 == 0, 1 <= B <= 64, all pointers 16-byte
- * aligned; MK_SWIGLU_TC also needs B % 16 == 0 and N % 128 == 0
+ * aligned; MK_SWIGLU_TC also needs K % 128 == 0 and N % 128 == 0
  * (MK_ERR_UNSUPPORTED otherwise).  MK_ERR_INVALID on bad arguments.
  * Allocates nothing. */
 mk_status mk_swiglu_stage1(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K, int N,

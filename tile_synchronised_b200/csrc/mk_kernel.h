@@ -15,8 +15,12 @@ cudaError_t launch_set_position(State *state, int pos, cudaStream_t s);
 // Fused SwiGLU first stage (fp16): variant MK_SWIGLU_ROW or MK_SWIGLU_COL.
 cudaError_t launch_swiglu(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N, int variant,
                           cudaStream_t s);
-// The same stage on the tcgen05 tensor cores (B a multiple of 16, N of 128).
+// The same stage on the tcgen05 tensor cores (K a multiple of 128, N of 128; B <= 128).
 bool swiglu_tc_supported(int B, int K, int N);
+// The column tiling on the same TMA pipeline, CUDA cores (B <= 8, N % 128 == 0).
+bool swiglu_col_tma_supported(int B, int K, int N);
+cudaError_t launch_swiglu_col_tma(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N,
+                                  cudaStream_t s);
 cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N,
                              cudaStream_t s);
 // Last error of a context-free call (the isolated operations) on this thread.

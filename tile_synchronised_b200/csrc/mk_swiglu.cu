@@ -10,7 +10,9 @@
 //       so each weight byte leaves HBM once and later groups re-read it from L2.
 //   row-tiled    (MK_SWIGLU_ROW): one CTA per (slab, batch group), so a batch
 //       group's activations stay resident while the weights are re-read per group.
-// At B <= 8 both are the same single pass.
+// At B <= 8 both are the same single pass.  For B <= 8 (N a multiple of 128)
+// the column tiling runs instead on the TMA pipeline of mk_swiglu_tc.cu, and
+// MK_SWIGLU_TC (B a multiple of 16) on the tensor cores.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -144,8 +146,10 @@ static bool swiglu_args_ok(const void *x, const void *wg, const void *wu, const 
 
 static cudaError_t run_variant(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N,
                                int variant, cudaStream_t s) {
-    return variant == MK_SWIGLU_TC ? launch_swiglu_tc(x, wg, wu, out, B, K, N, s)
-                                   : launch_swiglu(x, wg, wu, out, B, K, N, variant, s);
+    if (variant == MK_SWIGLU_TC) return launch_swiglu_tc(x, wg, wu, out, B, K, N, s);
+    if (variant == MK_SWIGLU_COL && swiglu_col_tma_supported(B, K, N))
+        return launch_swiglu_col_tma(x, wg, wu, out, B, K, N, s);
+    return launch_swiglu(x, wg, wu, out, B, K, N, variant, s);
 }
 
 extern "C" mk_status mk_swiglu_stage1(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K,
