@@ -1,4 +1,6 @@
 """Shared helpers of the GPU parity tests (comparison rules, model set-up)."""
+import os
+
 import numpy as np
 import torch
 
@@ -11,11 +13,18 @@ LOGIT_TOL = 2e-2
 
 
 def logits_close(gpu: np.ndarray, ref: np.ndarray) -> float:
-    """Returns max|delta| after asserting it is within LOGIT_TOL * max|ref| per row."""
+    """Returns max|delta| after asserting it is within LOGIT_TOL * max|ref| per row.
+    With MK_PARITY_LOG set, each row's max|delta| / max|ref| is appended to that
+    file with the running test's name (to record the margin)."""
     worst = 0.0
+    log = os.environ.get("MK_PARITY_LOG")
     for b in range(ref.shape[0]):
         d = float(np.max(np.abs(gpu[b].astype(np.float64) - ref[b])))
-        bound = LOGIT_TOL * float(np.max(np.abs(ref[b])))
+        scale = float(np.max(np.abs(ref[b])))
+        bound = LOGIT_TOL * scale
+        if log:
+            with open(log, "a") as f:
+                f.write(f"{os.environ.get('PYTEST_CURRENT_TEST', '?').split(' ')[0]}\t{d / scale:.3e}\n")
         assert d <= bound, f"row {b}: max|delta| {d:.4g} > {bound:.4g}"
         worst = max(worst, d)
     return worst

@@ -206,6 +206,38 @@ def sampled_layer0_rows(shape, tw, k, v, tokens_np, b, positions):
             assert np.max(np.abs(got_v - vv[g])) <= 2e-2 * np.max(np.abs(vv[g]))
 
 
+def host_weights(tw):
+    host = {kk: (None if tw[kk] is None else synth.to_u16(tw[kk])) for kk in ("embed", "final_norm", "lm_head")}
+    host["layers"] = [{a: (None if t is None else synth.to_u16(t)) for a, t in lw.items()} for lw in tw["layers"]]
+    return host
+
+
+def handoff_step(shape, host, model, tokens, pos, seqs):
+    """Decode the step at `pos` on the GPU with logits, then for each sequence
+    in `seqs` hand the GPU's KV cache (widened to fp32) to the oracle and
+    check that step's logits, argmax and appended K row."""
+    batch = model.batch
+    k, v = model.kv_views()
+    lg = torch.empty((batch, shape.vocab), dtype=torch.float32, device="cuda")
+    nxt = model.decode(tokens[:, pos].contiguous().cuda(), logits=lg).cpu().numpy()
+    assert model.status() == 0
+    assert model.position == pos + 1
+    g = lg.cpu().numpy()
+    tnp = tokens.numpy()
+    for b in seqs:
+        orc = oracle.OracleModel(shape, host, batch=1, max_seq=pos + 1)
+        orc.kc[:, 0, :, :pos] = k[:, b, :, :pos].float().cpu().numpy()
+        orc.vc[:, 0, :, :pos] = v[:, b, :, :pos].float().cpu().numpy()
+        orc.pos[0] = pos
+        ref, _ = orc.step([int(tnp[b, pos])])
+        d = logits_close(g[b:b + 1], ref)
+        check_argmax(nxt[b:b + 1], g[b:b + 1], ref, d)
+        # the cache row this step appended agrees with the oracle's
+        for l in (0, shape.n_layers - 1):
+            gk = k[l, b, :, pos].float().cpu().numpy()
+            assert np.max(np.abs(gk - orc.kc[l, 0, :, pos])) <= 2e-2 * np.max(np.abs(orc.kc[l, 0, :, pos]))
+
+
 def full_size_case(shape, batch, prefill, extra_steps, seqs, max_seq=None):
     import tile_synchronised_b200 as mk
     ms = max_seq or shape.max_seq
@@ -220,25 +252,9 @@ def full_size_case(shape, batch, prefill, extra_steps, seqs, max_seq=None):
     assert model.position == pos
     k, v = model.kv_views()
     sampled_layer0_rows(shape, tw, k, v, tnp, seqs[0], [0, 1, pos // 2, pos - 1])
-    lg = torch.empty((batch, shape.vocab), dtype=torch.float32, device="cuda")
-    nxt = model.decode(tokens[:, pos].contiguous().cuda(), logits=lg).cpu().numpy()
-    assert model.status() == 0
-    g = lg.cpu().numpy()
-    host = {kk: (None if tw[kk] is None else synth.to_u16(tw[kk])) for kk in ("embed", "final_norm", "lm_head")}
-    host["layers"] = [{a: (None if t is None else synth.to_u16(t)) for a, t in lw.items()} for lw in tw["layers"]]
+    host = host_weights(tw)
     del tw
-    for b in seqs:
-        orc = oracle.OracleModel(shape, host, batch=1, max_seq=pos + 1)
-        orc.kc[:, 0, :, :pos] = k[:, b, :, :pos].float().cpu().numpy()
-        orc.vc[:, 0, :, :pos] = v[:, b, :, :pos].float().cpu().numpy()
-        orc.pos[0] = pos
-        ref, _ = orc.step([int(tnp[b, pos])])
-        d = logits_close(g[b:b + 1], ref)
-        check_argmax(nxt[b:b + 1], g[b:b + 1], ref, d)
-        # the cache row this step appended agrees with the oracle's
-        for l in (0, shape.n_layers - 1):
-            gk = k[l, b, :, pos].float().cpu().numpy()
-            assert np.max(np.abs(gk - orc.kc[l, 0, :, pos])) <= 2e-2 * np.max(np.abs(orc.kc[l, 0, :, pos]))
+    handoff_step(shape, host, model, tokens, pos, seqs)
 
 
 @needs_cuda
@@ -258,6 +274,33 @@ def test_llama8b_full_size_handoff(batch, seqs):
 def test_qwen3_8b_handoff_at_1k():
     s = synth.QWEN3_8B
     full_size_case(s, 16, 1024, 2, [0, 15], max_seq=1040)
+
+
+@needs_cuda
+def test_qwen3_8b_two_layer_clone_1k_to_16k():
+    """The Qwen3-8B batch-16 trajectory from a 1024-token prefill to the last
+    slot of a 16384-position cache, on a clone cut to 2 layers (same widths,
+    heads, qk-norm, theta and vocab) so that every step runs on the GPU in
+    about a minute.  At 1k, 4k and 16k the oracle takes the GPU's cache and
+    checks one step of two sequences."""
+    import tile_synchronised_b200 as mk
+    s = synth.QWEN3_8B.replace(n_layers=2)
+    B, prefill, ms = 16, 1024, 16384
+    tw = synth.make_weights(s, device="cuda")
+    model = mk.Model(s, tw, batch=B, max_seq=ms)
+    host = host_weights(tw)
+    del tw
+    tokens = synth.make_tokens(s, ms, batch=B)
+    model.prefill(tokens[:, :prefill].cuda())
+    dev_tokens = tokens.to(dtype=torch.int32).cuda()
+    pos = prefill
+    for cp in (1024, 4096, ms - 1):
+        while pos < cp:
+            model.decode(dev_tokens[:, pos].contiguous())
+            pos += 1
+        handoff_step(s, host, model, tokens, pos, [0, B - 1])
+        pos += 1
+    assert model.position == ms
 
 
 # ---------------------------------------------------------------- the fused SwiGLU first stage

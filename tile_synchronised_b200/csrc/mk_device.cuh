@@ -116,16 +116,6 @@ __device__ __forceinline__ uint64_t ll_pack(float v, uint32_t tag) {
     return (static_cast<uint64_t>(tag) << 32) | __float_as_uint(v);
 }
 __device__ __forceinline__ float ll_value(uint64_t w) { return __uint_as_float(static_cast<uint32_t>(w)); }
-// The SwiGLU product and the attention output travel as pair words: two bf16
-// values (the lower-indexed one in bits 0-15) under one tag, half the bytes
-// of one fp32 value per word for the readers that stage a whole row.
-__device__ __forceinline__ uint64_t ll_pack2(float v0, float v1, uint32_t tag) {
-    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v0));
-    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(v1));
-    return (static_cast<uint64_t>(tag) << 32) | (hi << 16) | lo;
-}
-__device__ __forceinline__ float pair_lo(uint32_t bits) { return __uint_as_float(bits << 16); }
-__device__ __forceinline__ float pair_hi(uint32_t bits) { return __uint_as_float(bits & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t ll_tag(uint64_t w) { return static_cast<uint32_t>(w >> 32); }
 __device__ __forceinline__ void ll_st(uint64_t *p, uint64_t w) {
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");

@@ -394,7 +394,7 @@ __device__ __forceinline__ bool ll_spin(const KParams &P, const SmemLayout &S, L
 // line so the wait state costs the fast path no registers; it only runs while
 // a producer has not published yet.
 __device__ __noinline__ bool ll_spin_chunks(const KParams &P, const SmemLayout &S, const uint64_t *const *base,
-                                            int m, uint32_t pending, uint32_t tag, uint32_t *vals, uint32_t who) {
+                                            int m, uint32_t pending, uint32_t tag, float *vals, uint32_t who) {
     LlSpin sp{0ull, 0u};
     while (pending) {
         __nanosleep(16);
@@ -404,8 +404,8 @@ __device__ __noinline__ bool ll_spin_chunks(const KParams &P, const SmemLayout &
             for (int q = 0; q < 4; ++q) {
                 const ulonglong2 w = ll_ld2(base[j] + 2 * q);
                 all = all && ll_tag(w.x) == tag && ll_tag(w.y) == tag;
-                vals[8 * j + 2 * q] = static_cast<uint32_t>(w.x);
-                vals[8 * j + 2 * q + 1] = static_cast<uint32_t>(w.y);
+                vals[8 * j + 2 * q] = ll_value(w.x);
+                vals[8 * j + 2 * q + 1] = ll_value(w.y);
             }
             if (all) pending &= ~(1u << j);
         }
@@ -416,11 +416,11 @@ __device__ __noinline__ bool ll_spin_chunks(const KParams &P, const SmemLayout &
 
 // Read m <= M chunks of 8 tagged words (chunk j at ptr[j], 16-byte aligned),
 // all loads in flight together; if any word does not carry `tag` yet, spin
-// until all do.  The low 32 bits of the words (an fp32 value, or a bf16 pair)
-// go to f[j][0..7].  False when the wait gave up (f is then junk).
+// until all do.  The values go to f[j][0..7].  False when the wait gave up (f
+// is then junk).
 template <int M>
 __device__ __forceinline__ bool ll_chunks(const KParams &P, const SmemLayout &S, const uint64_t *const (&ptr)[M],
-                                          int m, uint32_t tag, uint32_t (&f)[M][8], uint32_t who) {
+                                          int m, uint32_t tag, float (&f)[M][8], uint32_t who) {
     uint32_t pending = 0;
 #pragma unroll
     for (int j = 0; j < M; ++j)
@@ -430,8 +430,8 @@ __device__ __forceinline__ bool ll_chunks(const KParams &P, const SmemLayout &S,
             for (int q = 0; q < 4; ++q) {
                 const ulonglong2 w = ll_ld2(ptr[j] + 2 * q);
                 ok = ok && ll_tag(w.x) == tag && ll_tag(w.y) == tag;
-                f[j][2 * q] = static_cast<uint32_t>(w.x);
-                f[j][2 * q + 1] = static_cast<uint32_t>(w.y);
+                f[j][2 * q] = ll_value(w.x);
+                f[j][2 * q + 1] = ll_value(w.y);
             }
             if (!ok) pending |= 1u << j;
         }
@@ -469,15 +469,15 @@ __device__ __forceinline__ bool residual8(const KParams &P, const SmemLayout &S,
                                           float (&x)[8], uint32_t who) {
     const size_t H = (size_t)P.hidden, rows = (size_t)P.batch;
     const uint64_t *ptr[1] = {P.xe + (size_t)row * H + col};
-    uint32_t f[1][8];
+    float f[1][8];
     bool ok = ll_chunks<1>(P, S, ptr, 1, tag, f, who);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) x[q] = __uint_as_float(f[0][q]);
+    for (int q = 0; q < 8; ++q) x[q] = f[0][q];
     for (int k = 1; k < P.down_ranges; ++k) {
         ptr[0] = P.dpart + ((size_t)(k - 1) * rows + row) * H + col;
         ok = ll_chunks<1>(P, S, ptr, 1, tag, f, who) && ok;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) x[q] += __uint_as_float(f[0][q]);
+        for (int q = 0; q < 8; ++q) x[q] += f[0][q];
     }
     return ok;
 }
@@ -498,15 +498,14 @@ __device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S,
     const uint32_t who = who_of(in);
     bool ok = true;
     if (in.op == OP_DOWN || in.op == OP_OPROJ) {
-        // copy of the SwiGLU product or of the attention output, both stored
-        // as bf16 pair words: a chunk is 8 words = 16 values; columns past the
-        // logical row (block padding) are zero
-        const int k0 = in.kb0 * m.kc, nch = klen / 16;
+        // copy of the SwiGLU product or of the attention output; columns past
+        // the logical row (block padding) are zero
+        const int k0 = in.kb0 * m.kc, nch = klen / 8;
         const uint64_t *src = in.op == OP_DOWN ? P.act_a : P.attn;
         const int len = in.op == OP_DOWN ? P.intermediate : P.n_heads * P.head_dim;
         const uint32_t tag = act_tag(gen, P.n_layers, in.layer);
         for (int b = 0; b < nb; ++b) {
-            const uint64_t *row = src + ((size_t)(in.b0 + b) * len + k0) / 2;
+            const uint64_t *row = src + (size_t)(in.b0 + b) * len;
             float *dst = act + (size_t)b * klen;
             for (int c0 = t; c0 < nch; c0 += 4 * kConsumerThreads) {
                 const uint64_t *ptr[4];
@@ -514,21 +513,23 @@ __device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S,
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int c = c0 + j * kConsumerThreads;
-                    ptr[j] = row + (size_t)c * 8;
-                    if (c < nch && k0 + c * 16 < len) mm = j + 1;
+                    ptr[j] = row + k0 + (size_t)c * 8;
+                    if (c < nch && k0 + c * 8 < len) mm = j + 1;
                 }
-                uint32_t f[4][8];
+                float f[4][8];
                 ok = ll_chunks<4>(P, S, ptr, mm, tag, f, who) && ok;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int c = c0 + j * kConsumerThreads;
                     if (c < nch) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dst + (size_t)c * 16);
-#pragma unroll
-                        for (int h = 0; h < 4; ++h)
-                            d4[h] = j < mm ? make_float4(pair_lo(f[j][2 * h]), pair_hi(f[j][2 * h]),
-                                                         pair_lo(f[j][2 * h + 1]), pair_hi(f[j][2 * h + 1]))
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + (size_t)c * 8);
+                        if (j < mm) {
+                            d4[0] = make_float4(f[j][0], f[j][1], f[j][2], f[j][3]);
+                            d4[1] = make_float4(f[j][4], f[j][5], f[j][6], f[j][7]);
+                        } else {
+                            d4[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            d4[1] = d4[0];
+                        }
                     }
                 }
             }
@@ -575,10 +576,10 @@ __device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S,
                 ok = residual8(P, S, row, c * 8, xtag, f, who) && ok;
             } else {
                 const uint64_t *ptr[1] = {P.xm + (size_t)row * H + c * 8};
-                uint32_t f1[1][8];
+                float f1[1][8];
                 ok = ll_chunks<1>(P, S, ptr, 1, xtag, f1, who) && ok;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) f[q] = __uint_as_float(f1[0][q]);
+                for (int q = 0; q < 8; ++q) f[q] = f1[0][q];
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q) ss[b] = fmaf(f[q], f[q], ss[b]);
@@ -783,27 +784,17 @@ __device__ __forceinline__ bool gemv_warp_tile(const KParams &P, const SmemLayou
                 }
         } break;
         case OP_GATEUP: {
-            // gate rows 0..RT/2-1, up rows RT/2..RT-1: the up partner is lane ^ 16.
-            // Outputs j and j + 1 (j even) sit on gate lanes `pl` apart; the
-            // even one stores both as one pair word.  Plans give gate/up tiles
-            // at least 4 rows, so a tile holds whole pairs.
-            if constexpr (RT >= 4) {
-                constexpr int pl = RT == 8 ? 4 : 8;
-                float a[BS], a1[BS];
+            // gate rows 0..RT/2-1, up rows RT/2..RT-1: the up partner is lane ^ 16
+            float up[BS];
 #pragma unroll
-                for (int b = 0; b < BS; ++b) {
-                    const float up = __shfl_xor_sync(0xFFFFFFFFu, v[b], 16);
-                    a[b] = v[b] / (1.0f + __expf(-v[b])) * up;
-                    a1[b] = __shfl_xor_sync(0xFFFFFFFFu, a[b], pl);
-                }
-                const int j = tile * (RT / 2) + fr;
-                if (holder && (lane & 16) == 0 && (fr & 1) == 0 && j < P.intermediate)
+            for (int b = 0; b < BS; ++b) up[b] = __shfl_xor_sync(0xFFFFFFFFu, v[b], 16);
+            const int j = tile * (RT / 2) + fr;
+            if (RT >= 2 && holder && (lane & 16) == 0 && j < P.intermediate)
 #pragma unroll
-                    for (int b = 0; b < BS; ++b)
-                        if (b < nb)
-                            ll_st(P.act_a + ((size_t)(in.b0 + b) * P.intermediate + j) / 2,
-                                  ll_pack2(a[b], a1[b], tag));
-            }
+                for (int b = 0; b < BS; ++b)
+                    if (b < nb)
+                        ll_st(P.act_a + (size_t)(in.b0 + b) * P.intermediate + j,
+                              ll_pack(v[b] / (1.0f + __expf(-v[b])) * up[b], tag));
         } break;
         default: {  // OP_LMHEAD: logits, then the warp's best of this tile folded into the CTA's
             const int n = tile * RT + fr;
@@ -1215,7 +1206,7 @@ __device__ __forceinline__ bool acomb_instr(const KParams &P, const SmemLayout &
     int tpi = 1;
     while (tpi < 16 && tpi < NC && 2 * tpi * items <= kConsumerThreads) tpi *= 2;
     const int per_pass = kConsumerThreads / tpi, q = t % tpi;
-    uint64_t *dst = P.attn + ((size_t)b * nq * d + (size_t)g * G * d) / 2;  // bf16 pair words
+    uint64_t *dst = P.attn + (size_t)b * nq * d + (size_t)g * G * d;
     bool ok = true;
     for (int i0 = 0; i0 < items; i0 += per_pass) {
         const int it = i0 + t / tpi;
@@ -1288,8 +1279,8 @@ __device__ __forceinline__ bool acomb_instr(const KParams &P, const SmemLayout &
         }
         if (mine && q == 0) {
             const float inv = 1.0f / L;
-            ll_st2(dst + (h * d + e) / 2, ll_pack2(acc.x * inv, acc.y * inv, otag),
-                   ll_pack2(acc.z * inv, acc.w * inv, otag));
+            ll_st2(dst + h * d + e, ll_pack(acc.x * inv, otag), ll_pack(acc.y * inv, otag));
+            ll_st2(dst + h * d + e + 2, ll_pack(acc.z * inv, otag), ll_pack(acc.w * inv, otag));
         }
     }
     return consumer_sync_or(!ok || *S.abort != 0);

@@ -63,8 +63,7 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     if (c.head_dim != 64 && c.head_dim != 128) return bad(MK_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
     if (c.n_heads % c.n_kv_heads) return bad(MK_ERR_UNSUPPORTED, "n_heads must be a multiple of n_kv_heads");
     if (c.n_heads / c.n_kv_heads > kMaxGroup) return bad(MK_ERR_UNSUPPORTED, "more than 8 query heads per KV head");
-    if (c.hidden % 8 || c.intermediate % 16)
-        return bad(MK_ERR_UNSUPPORTED, "hidden must be a multiple of 8 and intermediate of 16");
+    if (c.hidden % 8 || c.intermediate % 8) return bad(MK_ERR_UNSUPPORTED, "hidden and intermediate must be multiples of 8");
     if (c.hidden > 8192) return bad(MK_ERR_UNSUPPORTED, "hidden above 8192");
     if (c.batch > 64) return bad(MK_ERR_UNSUPPORTED, "batch above 64");
     if (c.max_seq > (1 << 20)) return bad(MK_ERR_UNSUPPORTED, "max_seq above 2^20");
@@ -79,16 +78,12 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     p.qkv_rows = (nq + 2 * nkv) * d;
     p.qkv = make_mat(p.qkv_rows, H);
     p.o = make_mat(H, nq * d);
-    // gate/up tiles keep at least 4 rows (2 gate + 2 up), so that every tile
-    // produces whole bf16 pairs of the SwiGLU product: above K = 4096 the
-    // tile row is cut into several ring blocks instead
-    p.gu = make_mat(2 * I, H, true, (H + 4095) / 4096);
+    p.gu = make_mat(2 * I, H, true);
     p.down = make_mat(H, I);
     p.lm = make_mat(V, H);
     if (p.qkv.rows * p.qkv.kc * 2 > kStageBytes || p.gu.rows * p.gu.kc * 2 > kStageBytes)
         return bad(MK_ERR_UNSUPPORTED, "hidden too large for one ring slot per tile row");
     if ((nq * d) % p.qkv.rows || (nkv * d) % p.qkv.rows) return bad(MK_ERR_UNSUPPORTED, "q/k/v rows not tile-aligned");
-    if (p.gu.rows < 4) return bad(MK_ERR_UNSUPPORTED, "gate/up tiles need at least 4 rows");
 
     // Batch rows per instruction and the activation region.  Activations are
     // staged in shared memory as fp32 [rows][K range]; the region is capped at
