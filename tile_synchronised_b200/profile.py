@@ -79,10 +79,13 @@ def main(argv=None):
     ap.add_argument("--time", type=int, default=0, help="also time this many steps (CUDA events)")
     ap.add_argument("--sync", default="tags", choices=sorted(mk.SYNCS))
     ap.add_argument("--stages", type=int, default=0, help="ring slots in use (0: all that fit)")
+    ap.add_argument("--synthetic-kv", type=int, default=0, metavar="C",
+                    help="timing only: instead of a prefill, fill cache positions < C with seeded N(0,1) bf16 "
+                         "values and start decoding at position C (the step's cost depends on C, not on the values)")
     a = ap.parse_args(argv)
     shape = synth.MODELS[a.workload]
     B = a.batch or shape.batch
-    prefill = shape.prefill if a.prefill is None else a.prefill
+    prefill = a.synthetic_kv or (shape.prefill if a.prefill is None else a.prefill)
     max_seq = a.max_seq or max(prefill + a.steps + 1, 16)
     tw = synth.make_weights(shape, device="cuda")
     model = mk.Model(shape, tw, batch=B, max_seq=max_seq, variant=a.variant)
@@ -91,7 +94,13 @@ def main(argv=None):
         model.set_prefetch(a.prefetch)
     model.set_sync(a.sync)
     model.set_ring_stages(a.stages)
-    if prefill:
+    if a.synthetic_kv:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(11)
+        for t in model.kv_views():
+            t[:, :, :, :prefill].normal_(generator=g)
+        model.set_position(prefill)
+    elif prefill:
         model.prefill(tokens[:, :prefill].cuda())
     d_tok = tokens[:, prefill:].t().contiguous().cuda()  # [steps, B]
     for s in range(a.steps - 1):
