@@ -67,14 +67,20 @@ def algorithmic_bytes(shape, batch, pos):
     return shape.weight_bytes() + batch * shape.hidden * 2 + batch * kv_row * pos + batch * kv_row
 
 
+# The sources that decide what the decode step launches and what it reads:
+# the megakernel, its plan and launch code, and the headers they share (not
+# the isolated SwiGLU and attention kernels).
+STEP_SOURCES = ("mk_api.cu", "mk_device.cuh", "mk_internal.h", "mk_kernel.cu", "mk_kernel.h", "mk_sched.cpp",
+                "mk_sched.h")
+
+
 def source_hash():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "tile_synchronised_b200", "csrc")
-    for n in sorted(os.listdir(d)):
-        if n.endswith((".cu", ".cuh", ".h", ".cpp")):
-            with open(os.path.join(d, n), "rb") as f:
-                h.update(n.encode())
-                h.update(f.read())
+    for n in STEP_SOURCES:
+        with open(os.path.join(d, n), "rb") as f:
+            h.update(n.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
