@@ -258,6 +258,27 @@ mk_status mk_swiglu_stage1(const void *x, const void *w_gate, const void *w_up, 
 mk_status mk_swiglu_tune(const void *x, const void *w_gate, const void *w_up, void *out, int B, int K, int N,
                          void *stream, int *chosen, float *us_row, float *us_col, float *us_tc);
 
+/* One projection of a batched decode step on the tcgen05 tensor cores (the
+ * matrix-vector products of "Look Ma, No Bubbles! Designing a Low-Latency
+ * Megakernel for Llama-1B", where a batch of B sequences makes each one a GEMM
+ * with the batch as its narrow side):
+ *   y[b][m] = sum_k w[m][k] x[b][k]
+ * w: device bf16 [M, K] row-major (the [out, in] layout of every decoder
+ * projection, as given); x: device bf16 [B, K] row-major; y: device fp32
+ * [B, M].  Swap-AB: 128 rows of w per CTA are the MMA's M, the batch
+ * (rounded up to 16 with zero rows) its N, fp32 accumulators in tensor
+ * memory; every weight byte is read once for the whole batch.  With few row
+ * tiles a cluster of 2 or 4 CTAs splits K (mk_linear_tc_split) and sums in a
+ * fixed order, so results are deterministic.  Needs 1 <= B <= 64,
+ * K % 64 == 0 (MK_ERR_UNSUPPORTED otherwise), M >= 1, all pointers 16-byte
+ * aligned (MK_ERR_INVALID).  Asynchronous on `stream`; a device-side wait
+ * that runs out (2 s) writes NaN outputs rather than hanging.  Allocates
+ * nothing. */
+mk_status mk_linear_tc(const void *x, const void *w, float *y, int B, int K, int M, void *stream);
+/* The K split (1, 2 or 4 CTAs per row tile) mk_linear_tc uses for this shape;
+ * host only.  MK_ERR_UNSUPPORTED for shapes mk_linear_tc refuses. */
+mk_status mk_linear_tc_split(int B, int K, int M, int *split);
+
 /* Split-KV decode attention with a log-sum-exp combine, on its own: the
  * attention of one layer of one decode step ("Look Ma, No Bubbles! Designing
  * a Low-Latency Megakernel for Llama-1B", introduction: generating one

@@ -155,6 +155,14 @@ def make_swiglu_inputs(batch: int, K: int = SWIGLU_K, N: int = SWIGLU_N, device=
     return x, wg, wu
 
 
+def make_linear_inputs(batch: int, K: int, M: int, device="cpu", seed: int = 21):
+    """x [B,K] ~ N(0,1) and w [M,K] ~ N(0,0.02), both bf16 (one decoder
+    projection in the [out, in] layout and a batch of input rows)."""
+    x = _randn((batch, K), seed, device, torch.bfloat16, 1.0)
+    w = _randn((M, K), seed + 1, device, torch.bfloat16, 0.02)
+    return x, w
+
+
 def to_u16(t: torch.Tensor):
     """Host numpy uint16 view of a 16-bit tensor's bytes (copies to CPU)."""
     import numpy as np

@@ -138,3 +138,27 @@ def test_noalloc_attention_refuses_oversize_without_a_device():
     st = lib.mk_attention_decode_noalloc(d, d, d, 16, 32, 8, 128, 1100, 1024, 16, d, None)
     assert st == _lib.MK_ERR_INVALID
     assert "4259840" in lib.mk_last_error(None).decode()
+
+
+def test_linear_tc_plan_and_argument_checks_need_no_device():
+    lib = _lib.load()
+    d = C.c_void_p(256)
+    # K split per row tile: a cluster of 2 or 4 CTAs while the grid stays within 148 SMs and
+    # every CTA keeps two K blocks
+    assert mkpy.linear_tc_split(16, 4096, 4096) == 4      # 32 row tiles -> 128 CTAs
+    assert mkpy.linear_tc_split(32, 4096, 6144) == 2      # 48 row tiles -> 96 CTAs
+    assert mkpy.linear_tc_split(16, 4096, 14336) == 1     # 112 row tiles
+    assert mkpy.linear_tc_split(16, 4096, 128256) == 1    # LM head: 1002 row tiles
+    assert mkpy.linear_tc_split(5, 320, 200) == 2         # 2 row tiles, 5 K blocks: 4 would leave 1 per CTA
+    assert mkpy.linear_tc_split(64, 14336, 4096) == 4
+    s = C.c_int()
+    assert lib.mk_linear_tc_split(0, 4096, 4096, C.byref(s)) == _lib.MK_ERR_UNSUPPORTED
+    assert lib.mk_linear_tc_split(65, 4096, 4096, C.byref(s)) == _lib.MK_ERR_UNSUPPORTED
+    assert lib.mk_linear_tc_split(16, 4000, 4096, C.byref(s)) == _lib.MK_ERR_UNSUPPORTED
+    assert lib.mk_linear_tc_split(16, 4096, 4096, None) == _lib.MK_ERR_INVALID
+    # refused before any launch
+    assert lib.mk_linear_tc(None, d, d, 16, 4096, 4096, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_linear_tc(C.c_void_p(8), d, d, 16, 4096, 4096, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_linear_tc(d, d, d, 0, 4096, 4096, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_linear_tc(d, d, d, 16, 4000, 4096, None) == _lib.MK_ERR_UNSUPPORTED
+    assert lib.mk_linear_tc(d, d, d, 128, 4096, 4096, None) == _lib.MK_ERR_UNSUPPORTED

@@ -1,0 +1,66 @@
+"""The tcgen05 decode projection (mk_linear_tc) against the oracle's GEMV,
+row by row, at the projection shapes of the batched decode configurations
+and at ragged shapes (row tiles and K blocks that do not divide evenly)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+SHAPES = [
+    # (B, K, M)
+    (16, 4096, 4096),     # Llama-8B / Qwen3-8B O projection, batch 16 (K split 4)
+    (32, 4096, 6144),     # Llama-8B QKV, batch 32 (K split 2)
+    (32, 14336, 4096),    # Llama-8B down projection, batch 32
+    (64, 4096, 14336),    # one half of gate/up, batch 64 (no split, 112 row tiles)
+    (1, 2048, 2048),      # batch 1 padded to 16 columns
+    (8, 4096, 4096),      # batch 8
+    (5, 320, 200),        # ragged rows (2 tiles, the second partial), 5 K blocks over a pair
+    (16, 4096, 128256),   # an LM head: 1002 row tiles, several waves
+]
+
+
+def reference(x, w):
+    """Oracle GEMV per batch row, and the matching sum of |x_k w_k| that bounds
+    any fp32 summation order."""
+    xu = x.float().cpu().numpy()
+    wu = synth.to_u16(w)
+    wabs = wu & np.uint16(0x7FFF)
+    ref = np.stack([oracle.gemv_bf16(wu, xu[b]) for b in range(xu.shape[0])])
+    mag = np.stack([oracle.gemv_bf16(wabs, np.abs(xu[b])) for b in range(xu.shape[0])])
+    return ref, mag
+
+
+@needs_cuda
+@pytest.mark.parametrize("B,K,M", SHAPES)
+def test_linear_tc_matches_oracle(B, K, M):
+    import tile_synchronised_b200 as mk
+    x, w = synth.make_linear_inputs(B, K, M, device="cuda")
+    y = mk.linear_tc(x, w)
+    torch.cuda.synchronize()
+    got = y.cpu().numpy()
+    assert got.shape == (B, M) and np.isfinite(got).all()
+    ref, mag = reference(x, w)
+    # bf16 x bf16 products are exact in fp32; any order of K fp32 additions is
+    # within K * 2^-24 * sum|x w| of the exact sum (the oracle's own rounding
+    # to fp32 adds 2^-24 |y|)
+    bound = 2.0 * K * 2.0 ** -24 * mag + 2.0 ** -23 * np.abs(ref) + 1e-30
+    assert np.all(np.abs(got.astype(np.float64) - ref) <= bound)
+
+
+@needs_cuda
+def test_linear_tc_is_deterministic_and_writes_only_its_rows():
+    import tile_synchronised_b200 as mk
+    B, K, M = 5, 320, 200
+    x, w = synth.make_linear_inputs(B, K, M, device="cuda")
+    big = torch.full((B + 2, M), 7.0, dtype=torch.float32, device="cuda")
+    y1 = mk.linear_tc(x, w, out=big[:B])
+    y2 = mk.linear_tc(x, w)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert torch.all(big[B:] == 7.0)

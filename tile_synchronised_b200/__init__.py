@@ -15,7 +15,7 @@ from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWI
                    MK_SYNC_TAGS,
                    MkConfig, MkError, MkWeights, check, load)
 
-__all__ = ["Model", "swiglu_stage1", "swiglu_tune", "MkError", "VARIANTS", "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW",
+__all__ = ["Model", "swiglu_stage1", "swiglu_tune", "linear_tc", "linear_tc_split", "MkError", "VARIANTS", "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW",
            "MK_SWIGLU_COL", "MK_SWIGLU_TC", "load"]
 
 VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL}
@@ -225,6 +225,29 @@ def swiglu_tune(x, w_gate, w_up, out, stream=None):
                                 C.c_void_p(out.data_ptr()), B, K, N, _stream(stream), C.byref(ch), C.byref(ur),
                                 C.byref(uc), C.byref(ut)), None, "mk_swiglu_tune")
     return ch.value, ur.value, uc.value, ut.value
+
+
+def linear_tc(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x @ w.T on the tcgen05 tensor cores: bf16 x [B, K], bf16 w [M, K]
+    (an [out, in] projection as given) -> fp32 y [B, M]."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16 or x.dim() != 2 or w.dim() != 2:
+        raise ValueError("x must be bf16 [B, K] and w bf16 [M, K]")
+    if not (x.is_contiguous() and w.is_contiguous()) or x.shape[1] != w.shape[1]:
+        raise ValueError("x and w must be contiguous with the same K")
+    B, K = x.shape
+    M = w.shape[0]
+    if out is None:
+        out = torch.empty((B, M), dtype=torch.float32, device=x.device)
+    check(load().mk_linear_tc(C.c_void_p(x.data_ptr()), C.c_void_p(w.data_ptr()), C.c_void_p(out.data_ptr()), B, K,
+                              M, _stream(stream)), None, "mk_linear_tc")
+    return out
+
+
+def linear_tc_split(B: int, K: int, M: int) -> int:
+    """CTAs per row tile (K split) linear_tc uses for this shape."""
+    s = C.c_int()
+    check(load().mk_linear_tc_split(B, K, M, C.byref(s)), None, "mk_linear_tc_split")
+    return s.value
 
 
 def _attn_shapes(q: torch.Tensor, k_cache: torch.Tensor):

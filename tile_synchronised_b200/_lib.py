@@ -25,7 +25,7 @@ EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk
            "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch", "mk_set_timeout_ns", "mk_set_sync", "mk_set_ring_stages", "mk_debug_drop_signal",
            "mk_set_trace", "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1", "mk_swiglu_tune",
            "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks",
-           "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes")
+           "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes", "mk_linear_tc", "mk_linear_tc_split")
 
 
 class MkConfig(C.Structure):
@@ -100,6 +100,8 @@ def load() -> C.CDLL:
         "mk_attention_chunks": ([i32, i32, i32], i32),
         "mk_attention_decode_noalloc": ([vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp], st),
         "mk_attention_noalloc_limit_bytes": ([], sz),
+        "mk_linear_tc": ([vp, vp, vp, i32, i32, i32, vp], st),
+        "mk_linear_tc_split": ([i32, i32, i32, C.POINTER(i32)], st),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)

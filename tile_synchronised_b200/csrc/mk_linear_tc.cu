@@ -1,0 +1,252 @@
+// mk_linear_tc.cu -- one decode projection on the 5th-generation tensor cores
+// (tcgen05): y[b][m] = sum_k W[m][k] x[b][k] for the batched decode, where a
+// projection of a whole batch is a dense GEMM with the batch as its narrow
+// side.  W is a model matrix as given ([out, in] row-major bf16, the layout
+// of every projection of the decoder: QKV, O, gate, up, down, LM head), x is
+// the batch of input rows (bf16, [B, in]), y is fp32 [B, out].
+//
+// Swap-AB: the weights are operand A (M = 128 output rows per CTA, K-major,
+// a row of W is contiguous in K), the batch is operand B (N = B rounded up
+// to 16, K-major), so every weight byte leaves HBM once for the whole batch
+// and the accumulator (128 lanes x N fp32 columns) lives in tensor memory.
+// Both operands are staged by TMA with 128-byte swizzling into a ring of up
+// to 6 stages; warp 0 lane 0 issues the loads, warp 1 lane 0 the MMAs, and
+// each stage goes back to the producer through tcgen05.commit.
+//
+// When there are few output tiles (a 4096-row projection has 32), a cluster
+// of 2 or 4 CTAs shares one tile and splits K, so that more SMs stream the
+// weights; the other CTAs of the cluster then store their accumulators into
+// the first one's idle stage memory over the cluster (mapa +
+// st.shared::cluster), and the first adds them in rank order and writes y.
+// Every wait is bounded; a wait that runs out stops the CTA and its outputs
+// are written as NaN so that the failure cannot pass for a result.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/mk.h"
+#include "mk_device.cuh"
+#include "mk_tc.cuh"
+
+namespace mk {
+
+constexpr int kLinM = 128;    // output rows per CTA (MMA M)
+constexpr int kLinBK = 64;    // K per stage: one 128-byte swizzle row of bf16
+constexpr int kLinThreads = 128;
+constexpr int kLinMaxSplit = 4;
+constexpr int kLinMaxB = 64;
+
+struct LinShape {
+    int Bp, rows, K, M, stages;      // Bp: the MMA's N (B rounded up to 16); rows: B
+    uint32_t stage_bytes, a_bytes;  // a stage is the W box then the x box
+};
+
+// Instruction descriptor of kind::f16: fp32 accumulate, bf16 A and B, both
+// K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t lin_idesc(int n) {
+    return (1u << 4)                     // D format: F32
+           | (1u << 7) | (1u << 10)      // A, B format: BF16
+           | (0u << 15) | (0u << 16)     // A, B K-major
+           | ((uint32_t)(n >> 3) << 17)  // N >> 3
+           | ((uint32_t)(kLinM >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(kLinThreads, 1)
+    linear_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                     float *__restrict__ y, LinShape sh) {
+    extern __shared__ __align__(1024) uint8_t lin_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(lin_smem_raw) + 1023) & ~uintptr_t(1023));
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int S = sh.stages, Bp = sh.Bp;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * sh.stage_bytes);
+    uint64_t *empty = full + S;
+    uint64_t *done = empty + S;
+    volatile uint32_t *tmem_base = reinterpret_cast<volatile uint32_t *>(done + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+    const uint32_t rank = cluster_rank(), nrank = cluster_size();
+    const int m0 = (int)(blockIdx.x / nrank) * kLinM;
+    const int nkb_all = sh.K / kLinBK;
+    const int kb_first = (int)rank * nkb_all / (int)nrank;
+    const int nkb = (int)(rank + 1) * nkb_all / (int)nrank - kb_first;
+    const uint32_t ncols = Bp <= 32 ? 32u : 64u;  // a power of two >= 32 that holds N columns
+
+    if (t == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {  // the whole warp allocates the accumulator columns
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(const_cast<uint32_t *>(tmem_base))),
+                     "r"(ncols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % S;
+            if (kb >= S && !tc_wait(&empty[s], ((kb / S) - 1) & 1u, abort)) break;
+            uint8_t *st = smem + (size_t)s * sh.stage_bytes;
+            mbar_arrive_expect_tx(&full[s], sh.stage_bytes);  // rows past M or B arrive as zeros and count
+            const int k0 = (kb_first + kb) * kLinBK;
+            tma_load_2d(st, &map_w, k0, m0, &full[s]);
+            tma_load_2d(st + sh.a_bytes, &map_x, k0, 0, &full[s]);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // Both operands K-major, 128-byte swizzle: 8 rows of 128 bytes per
+        // 1 KB group (SBO), a K step of 16 is 32 bytes along the rows.
+        const uint32_t idesc = lin_idesc(Bp);
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % S;
+            if (!tc_wait(&full[s], (kb / S) & 1u, abort)) break;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint8_t *st = smem + (size_t)s * sh.stage_bytes;
+#pragma unroll
+            for (int ks = 0; ks < kLinBK / 16; ++ks) {
+                const uint64_t a = smem_desc_sw128(st + ks * 32, 16, 1024);
+                const uint64_t b = smem_desc_sw128(st + sh.a_bytes + ks * 32, 16, 1024);
+                tc_mma(tmem, a, b, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+            }
+            tc_commit(&empty[s]);
+        }
+        tc_commit(done);
+    }
+    __syncwarp();
+    // epilogue: thread t holds output row m0 + t (tensor-memory lane t; warp w
+    // may read lanes 32w .. 32w+31), one column per batch row
+    const bool ok = tc_wait(done, 0u, abort) && !*abort;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    // Once every CTA of the cluster is past its last MMA, the first CTA's
+    // stage memory receives the others' accumulators, [rank - 1][Bp][128],
+    // and their "ok" words after them.
+    float *part = reinterpret_cast<float *>(smem);
+    float *part_ok = part + (size_t)(nrank - 1) * Bp * kLinM;
+    if (nrank > 1) cluster_sync_all();
+    if (rank != 0) {
+        const uint32_t remote = cluster_map(part, 0) + (rank - 1) * (uint32_t)(Bp * kLinM * 4);
+        for (int c0 = 0; c0 < Bp; c0 += 16) {
+            float v[16];
+            tmem_ld16(lane_addr + (uint32_t)c0, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) st_cluster_f32(remote + (uint32_t)(((c0 + i) * kLinM + t) * 4), v[i]);
+        }
+        if (t == 0) st_cluster_f32(cluster_map(part_ok + (rank - 1), 0), ok ? 1.f : 0.f);
+    }
+    if (nrank > 1) cluster_sync_all();
+    if (rank == 0) {
+        bool all_ok = ok;
+        for (uint32_t r = 1; r < nrank; ++r) all_ok = all_ok && part_ok[r - 1] != 0.f;
+        const int m = m0 + t;
+        for (int c0 = 0; c0 < Bp; c0 += 16) {
+            float v[16];
+            tmem_ld16(lane_addr + (uint32_t)c0, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int b = c0 + i;
+                float acc = v[i];
+                for (uint32_t r = 1; r < nrank; ++r) acc += part[((size_t)(r - 1) * Bp + b) * kLinM + t];
+                if (b < sh.rows && m < sh.M) y[(size_t)b * sh.M + m] = all_ok ? acc : __int_as_float(0x7fc00000);
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
+}
+
+// Launch geometry of one call, worked out on the host.
+struct LinPlan {
+    LinShape sh;
+    int split, tiles, smem;
+};
+
+static bool lin_plan(int B, int K, int M, LinPlan &p) {
+    if (B < 1 || B > kLinMaxB || K < kLinBK || K % kLinBK || M < 1) return false;
+    LinShape &sh = p.sh;
+    sh.Bp = (B + 15) / 16 * 16;
+    sh.rows = B;
+    sh.K = K;
+    sh.M = M;
+    sh.a_bytes = (uint32_t)kLinM * kLinBK * 2;                      // 16 KB of W
+    sh.stage_bytes = sh.a_bytes + (uint32_t)sh.Bp * kLinBK * 2;     // + Bp rows of x, a multiple of 2 KB
+    const int budget = 227 * 1024 - 1024 - 256;                    // alignment slack and the barriers
+    sh.stages = budget / (int)sh.stage_bytes;
+    if (sh.stages > 6) sh.stages = 6;
+    if (sh.stages < 2) return false;
+    p.tiles = (M + kLinM - 1) / kLinM;
+    const int nkb = K / kLinBK;
+    // K split across a cluster while the grid stays within one wave of SMs,
+    // every CTA keeps at least two K blocks, and the first CTA's stage
+    // memory holds the other CTAs' accumulators.
+    p.split = 1;
+    for (int s = kLinMaxSplit; s > 1; s /= 2)
+        if (p.tiles * s <= 148 && nkb >= 2 * s &&
+            (size_t)(s - 1) * sh.Bp * kLinM * 4 + 16 <= (size_t)sh.stages * sh.stage_bytes) {
+            p.split = s;
+            break;
+        }
+    p.smem = sh.stages * (int)sh.stage_bytes + 1024 + 256;
+    return true;
+}
+
+cudaError_t launch_linear_tc(const void *x, const void *w, float *y, int B, int K, int M, cudaStream_t s) {
+    LinPlan p;
+    if (!lin_plan(B, K, M, p)) return cudaErrorInvalidValue;
+    CUtensorMap mw, mx;
+    if (!tc_make_map(&mw, w, (uint64_t)M, (uint64_t)K, kLinBK, kLinM) ||
+        !tc_make_map(&mx, x, (uint64_t)B, (uint64_t)K, kLinBK, (uint32_t)p.sh.Bp))
+        return cudaErrorInvalidValue;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.tiles * p.split));
+    cfg.blockDim = dim3(kLinThreads);
+    cfg.dynamicSmemBytes = (size_t)p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, linear_tc_kernel, mw, mx, y, p.sh);
+}
+
+}  // namespace mk
+
+using namespace mk;
+
+extern "C" mk_status mk_linear_tc(const void *x, const void *w, float *y, int B, int K, int M, void *stream) {
+    if (!x || !w || !y || B < 1 || K < 1 || M < 1) return MK_ERR_INVALID;
+    for (const void *p : {x, w, static_cast<const void *>(y)})
+        if ((uintptr_t)p & 15) return MK_ERR_INVALID;
+    LinPlan p;
+    if (!lin_plan(B, K, M, p)) return MK_ERR_UNSUPPORTED;
+    const cudaError_t e = launch_linear_tc(x, w, y, B, K, M, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MK_OK : MK_ERR_CUDA;
+}
+
+extern "C" mk_status mk_linear_tc_split(int B, int K, int M, int *split) {
+    if (!split) return MK_ERR_INVALID;
+    LinPlan p;
+    if (!lin_plan(B, K, M, p)) return MK_ERR_UNSUPPORTED;
+    *split = p.split;
+    return MK_OK;
+}

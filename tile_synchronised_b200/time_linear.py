@@ -1,0 +1,54 @@
+"""Time mk_linear_tc at the projection shapes of the batched decode configurations.
+
+    python -m tile_synchronised_b200.time_linear [--reps 30]
+
+Prints one JSON list: per (B, K, M) the K split, the mean microseconds per call
+(CUDA events over back-to-back calls) and the achieved GB/s of the weights plus
+x and y.  Weight copies are rotated so that the timed set exceeds the 126 MB L2.
+"""
+import argparse
+import json
+import os
+import sys
+
+import torch
+
+SHAPES = [(1, 4096, 4096), (16, 4096, 4096), (32, 4096, 4096), (32, 4096, 6144), (32, 14336, 4096),
+          (32, 4096, 14336), (16, 4096, 128256), (64, 4096, 14336)]
+
+
+def main(argv=None):
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import synth
+    import tile_synchronised_b200 as mk
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--reps", type=int, default=30)
+    ap.add_argument("--peak-gbs", type=float, default=6550.4, help="the measured HBM copy bandwidth")
+    a = ap.parse_args(argv)
+    res = []
+    for (B, K, M) in SHAPES:
+        x, w = synth.make_linear_inputs(B, K, M, device="cuda")
+        wb = M * K * 2
+        ncopy = max(1, -(-300_000_000 // wb))
+        ws = [w] + [w.clone() for _ in range(ncopy - 1)]
+        y = torch.empty((B, M), dtype=torch.float32, device="cuda")
+        for i in range(3):
+            mk.linear_tc(x, ws[i % ncopy], out=y)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(a.reps):
+            mk.linear_tc(x, ws[i % ncopy], out=y)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / a.reps
+        gbs = (wb + B * K * 2 + B * M * 4) / us / 1e3
+        res.append({"B": B, "K": K, "M": M, "split": mk.linear_tc_split(B, K, M), "us": round(us, 2),
+                    "GBps": round(gbs, 1), "frac": round(gbs / a.peak_gbs, 3)})
+        del ws
+    print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()
