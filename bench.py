@@ -203,9 +203,18 @@ def max_over_ranks(world, v):
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, batch, steps, ms_local):
+    """Every rank decodes `batch` sequences for `steps` steps in `ms_local`
+    device milliseconds; returns (the max over ranks of those ms, ms per step,
+    whole-job tokens/s)."""
+    ms = max_over_ranks(world, ms_local)
+    return ms, ms / steps, world * batch * steps / (ms / 1e3)
 
 
 # ---------------------------------------------------------------- the product arm
@@ -257,13 +266,11 @@ def run_mk(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     ms_local = e0.elapsed_time(e1)
-    ms = max_over_ranks(world, ms_local)
+    ms, ms_per_step, value = job_throughput(world, B, args.steps, ms_local)
     st = model.status()
     if st != 0:
         raise RuntimeError(f"device status {st}: {model.last_error()}")
-    ms_per_step = ms / args.steps
     total_tokens = world * B * args.steps
-    value = total_tokens / (ms / 1e3)
 
     # roofline of the (only) kernel: algorithmic bytes per launch / launch time
     pos_list = [PREFILL + (s % WINDOW) for s in range(args.steps)]
