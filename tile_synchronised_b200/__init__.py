@@ -10,13 +10,11 @@ import ctypes as C
 
 import torch
 
-from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW, MK_SWIGLU_TC,
-                   MK_SYNC_COUNTERS,
-                   MK_SYNC_TAGS,
-                   MkConfig, MkError, MkWeights, check, load)
+from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW,
+                   MK_SWIGLU_TC, MK_SYNC_COUNTERS, MK_SYNC_TAGS, MkConfig, MkError, MkWeights, check, load)
 
-__all__ = ["Model", "swiglu_stage1", "swiglu_tune", "linear_tc", "linear_tc_split", "MkError", "VARIANTS", "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW",
-           "MK_SWIGLU_COL", "MK_SWIGLU_TC", "load"]
+__all__ = ["Model", "swiglu_stage1", "swiglu_tune", "linear_tc", "linear_tc_split", "MkError", "VARIANTS",
+           "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW", "MK_SWIGLU_COL", "MK_SWIGLU_TC", "load"]
 
 VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL}
 SYNCS = {"tags": MK_SYNC_TAGS, "counters": MK_SYNC_COUNTERS}

@@ -22,10 +22,12 @@ STATUS_NAMES = {0: "MK_OK", -1: "MK_ERR_INVALID", -2: "MK_ERR_CUDA", -3: "MK_ERR
 # Every symbol include/mk.h declares.
 EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk_kv_cache_bytes",
            "mk_load_weights", "mk_prefill_kv", "mk_decode_step", "mk_get_status", "mk_reset",
-           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch", "mk_set_timeout_ns", "mk_set_sync", "mk_set_ring_stages", "mk_debug_drop_signal",
-           "mk_set_trace", "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1", "mk_swiglu_tune",
-           "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks",
-           "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes", "mk_linear_tc", "mk_linear_tc_split")
+           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch",
+           "mk_set_timeout_ns", "mk_set_sync", "mk_set_ring_stages", "mk_debug_drop_signal", "mk_set_trace",
+           "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1",
+           "mk_swiglu_tune", "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks",
+           "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes", "mk_linear_tc",
+           "mk_linear_tc_split")
 
 
 class MkConfig(C.Structure):

@@ -365,7 +365,8 @@ cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void
     // transaction count includes.
     const int Bp = (B + 15) / 16 * 16;
     CUtensorMap mg, mu, mx;
-    if (!tc_make_map(&mg, wg, (uint64_t)K, (uint64_t)N, 64, kTcBK) || !tc_make_map(&mu, wu, (uint64_t)K, (uint64_t)N, 64, kTcBK) ||
+    if (!tc_make_map(&mg, wg, (uint64_t)K, (uint64_t)N, 64, kTcBK) ||
+        !tc_make_map(&mu, wu, (uint64_t)K, (uint64_t)N, 64, kTcBK) ||
         !tc_make_map(&mx, x, (uint64_t)B, (uint64_t)K, kTcBK, (uint32_t)Bp))
         return cudaErrorInvalidValue;
     TcShape sh;
