@@ -7,7 +7,9 @@ per-instruction device trace, and summarise where the step's time goes.
 Used as the command under ncu (small --prefill keeps the capture short) and
 for trace summaries: per phase (op, layer) the span from the first dependency
 satisfied to the last instruction done, per op the mean instruction time, the
-time spent waiting on counters, and how far the producer ran ahead.
+time spent waiting on counters, and how far the producer ran ahead, and per
+edge of a layer's chain the gap from the producer phase's end to the
+consumers' staged inputs.
 """
 from __future__ import annotations
 
@@ -19,6 +21,41 @@ import numpy as np
 import torch
 
 OPS = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "acomb"}
+
+
+# Edges of a layer's chain: (producer op, layer offset, consumer op).  The
+# consumer stamps "inputs staged" (trace slot 7) once the words it reads carry
+# the producer's tag; the gap from the producer phase's last instruction end
+# to that stamp is the cost of the edge (an L2 round trip, the staging
+# itself, and any wait for the slowest producer CTA).
+EDGES = ((5, -1, 1, "down->qkv"), (1, 0, 2, "qkv->attn"), (7, 0, 3, "acomb->oproj"), (3, 0, 4, "oproj->gateup"),
+         (4, 0, 5, "gateup->down"))
+
+
+def edge_gaps(sched, tr):
+    """Mean over the inner layers (1 .. L-2) of, per edge, the gap in µs from
+    the producer phase's last end to the first and to the last consumer
+    instruction's staged stamp."""
+    t0 = tr[:, 0].astype(np.float64)
+    origin = t0[t0 > 0].min()
+    t2 = (tr[:, 2].astype(np.float64) - origin) / 1e3
+    t7 = (tr[:, 7].astype(np.float64) - origin) / 1e3
+    ops, layers = sched["op"].astype(np.int64), sched["layer"].astype(np.int64)
+    n_layers = int(layers[ops != 6].max()) + 1
+    out = {}
+    for pop, dl, cop, name in EDGES:
+        first, last = [], []
+        for L in range(1, n_layers - 1):
+            pm = (ops == pop) & (layers == L + dl)
+            cm = (ops == cop) & (layers == L)
+            if not pm.any() or not cm.any():
+                continue
+            end = t2[pm].max()
+            first.append(t7[cm].min() - end)
+            last.append(t7[cm].max() - end)
+        if first:
+            out[name] = {"to_first_staged_us": float(np.mean(first)), "to_last_staged_us": float(np.mean(last))}
+    return out
 
 
 def summarise(sched, base, tr):
@@ -58,6 +95,7 @@ def summarise(sched, base, tr):
         if e > s:
             busy.append(float((t2[s:e] - t1[s:e]).sum() / max(1.0, t2[s:e].max())))
     out["cta_busy_frac_mean"] = float(np.mean(busy))
+    out["edges"] = edge_gaps(sched, tr)
     return out
 
 
