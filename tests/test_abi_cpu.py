@@ -158,7 +158,10 @@ def test_linear_tc_plan_and_argument_checks_need_no_device():
     assert lib.mk_linear_tc_split(16, 4096, 4096, None) == _lib.MK_ERR_INVALID
     # refused before any launch
     assert lib.mk_linear_tc(None, d, d, 16, 4096, 4096, None) == _lib.MK_ERR_INVALID
+    assert "null" in lib.mk_last_error(None).decode()
     assert lib.mk_linear_tc(C.c_void_p(8), d, d, 16, 4096, 4096, None) == _lib.MK_ERR_INVALID
+    assert "aligned" in lib.mk_last_error(None).decode()
     assert lib.mk_linear_tc(d, d, d, 0, 4096, 4096, None) == _lib.MK_ERR_INVALID
     assert lib.mk_linear_tc(d, d, d, 16, 4000, 4096, None) == _lib.MK_ERR_UNSUPPORTED
+    assert "multiple of 64" in lib.mk_last_error(None).decode()
     assert lib.mk_linear_tc(d, d, d, 128, 4096, 4096, None) == _lib.MK_ERR_UNSUPPORTED

@@ -24,9 +24,11 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdio>
 
 #include "../../include/mk.h"
 #include "mk_device.cuh"
+#include "mk_kernel.h"
 #include "mk_tc.cuh"
 
 namespace mk {
@@ -234,13 +236,32 @@ cudaError_t launch_linear_tc(const void *x, const void *w, float *y, int B, int 
 using namespace mk;
 
 extern "C" mk_status mk_linear_tc(const void *x, const void *w, float *y, int B, int K, int M, void *stream) {
-    if (!x || !w || !y || B < 1 || K < 1 || M < 1) return MK_ERR_INVALID;
+    if (!x || !w || !y) {
+        set_op_error("linear_tc: null pointer");
+        return MK_ERR_INVALID;
+    }
+    if (B < 1 || K < 1 || M < 1) {
+        set_op_error("linear_tc: B, K and M must be positive");
+        return MK_ERR_INVALID;
+    }
     for (const void *p : {x, w, static_cast<const void *>(y)})
-        if ((uintptr_t)p & 15) return MK_ERR_INVALID;
+        if ((uintptr_t)p & 15) {
+            set_op_error("linear_tc: x, w and y must be 16-byte aligned");
+            return MK_ERR_INVALID;
+        }
     LinPlan p;
-    if (!lin_plan(B, K, M, p)) return MK_ERR_UNSUPPORTED;
+    if (!lin_plan(B, K, M, p)) {
+        set_op_error("linear_tc: needs B <= 64 and K a multiple of 64");
+        return MK_ERR_UNSUPPORTED;
+    }
     const cudaError_t e = launch_linear_tc(x, w, y, B, K, M, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? MK_OK : MK_ERR_CUDA;
+    if (e != cudaSuccess) {
+        char msg[160];
+        snprintf(msg, sizeof(msg), "linear_tc: launch failed: %s", cudaGetErrorString(e));
+        set_op_error(msg);
+        return MK_ERR_CUDA;
+    }
+    return MK_OK;
 }
 
 extern "C" mk_status mk_linear_tc_split(int B, int K, int M, int *split) {
