@@ -10,9 +10,10 @@
 //       so each weight byte leaves HBM once and later groups re-read it from L2.
 //   row-tiled    (MK_SWIGLU_ROW): one CTA per (slab, batch group), so a batch
 //       group's activations stay resident while the weights are re-read per group.
-// At B <= 8 both are the same single pass.  For B <= 8 (N a multiple of 128)
-// the column tiling runs instead on the TMA pipeline of mk_swiglu_tc.cu, and
-// MK_SWIGLU_TC (B a multiple of 16) on the tensor cores.
+// At B <= 8 both are the same single pass.  For B <= 8 (K a multiple of 128,
+// N of 128) the column tiling runs instead on the TMA pipeline of
+// mk_swiglu_tc.cu, and MK_SWIGLU_TC runs on the tensor cores at any batch
+// (rounded up to 16 with zero rows).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 

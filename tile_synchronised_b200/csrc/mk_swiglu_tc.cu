@@ -1,7 +1,9 @@
 // mk_swiglu_tc.cu -- the fused SwiGLU first stage on the 5th-generation tensor
-// cores (tcgen05), for batches of 16 and more, where the two projections are
-// dense GEMMs ("Deep Kernel Fusion for Transformers", Key points, "Fusion
-// scope": Up and Gate GEMMs, SiLU and the product in one kernel).
+// cores (tcgen05) at any batch up to 128 (rounded up to 16 with zero rows:
+// the stage is bound by the weight stream, so the padding costs nothing), and
+// the CUDA-core column tiling on the same TMA pipeline for batches up to 8
+// ("Deep Kernel Fusion for Transformers", Key points, "Fusion scope": Up and
+// Gate GEMMs, SiLU and the product in one kernel).
 //
 //   out[b][n] = SiLU(sum_k x[b][k] Wg[k][n]) * sum_k x[b][k] Wu[k][n]
 //
@@ -9,8 +11,9 @@
 // batch; each CTA of the pair takes half of K, so twice as many SMs stream
 // the weights.  The MMA computes D[m][b] = sum_k W[k][n0+m] x[b][k] with the
 // weights as operand A (M = 128, MN-major: n is contiguous in W) and x as
-// operand B (N = batch, K-major), both staged by TMA with 128-byte swizzling,
-// fp32 accumulators for gate and up in tensor memory.  Warp 0 lane 0 issues
+// operand B (N = batch rounded up to 16, K-major), both staged by TMA with
+// 128-byte swizzling, fp32 accumulators for gate and up in tensor memory.
+// Warp 0 lane 0 issues
 // the TMA loads of a 4..6-stage ring, warp 1 lane 0 issues the MMAs and
 // commits each stage back to its "empty" barrier.  Then the second CTA of the
 // pair reads its accumulators out of tensor memory (one row per thread) and
