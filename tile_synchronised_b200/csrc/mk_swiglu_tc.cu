@@ -14,10 +14,10 @@
 // operand B (N = batch rounded up to 16, K-major), both staged by TMA with
 // 128-byte swizzling, fp32 accumulators for gate and up in tensor memory.
 // Warp 0 lane 0 issues the TMA loads of a 4..6-stage ring, warp 1 lane 0
-// issues the MMAs and commits each stage back to its "empty" barrier.  Then the second CTA of the
-// pair reads its accumulators out of tensor memory (one row per thread) and
-// stores them into the first CTA's shared memory over the cluster; the first
-// adds them to its own and writes SiLU(g) * u as fp16.
+// issues the MMAs and commits each stage back to its "empty" barrier.  Then
+// the second CTA of the pair reads its accumulators out of tensor memory (one
+// row per thread) and stores them into the first CTA's shared memory over the
+// cluster; the first adds them to its own and writes SiLU(g) * u as fp16.
 // Every barrier wait is bounded; a wait that runs out stops the CTA and its
 // outputs are written as NaN so that the failure cannot pass for a result.
 #include <cuda.h>
