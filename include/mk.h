@@ -279,6 +279,37 @@ mk_status mk_linear_tc(const void *x, const void *w, float *y, int B, int K, int
  * host only.  MK_ERR_UNSUPPORTED for shapes mk_linear_tc refuses. */
 mk_status mk_linear_tc_split(int B, int K, int M, int *split);
 
+/* A batched decode step whose projections all run on the tensor cores
+ * (mk_linear_tc) and whose attention is the split-KV pair of kernels above
+ * (mk_attention_decode), for the batches where the megakernel's CUDA-core
+ * GEMV becomes arithmetic-bound ("Look Ma, No Bubbles! Designing a
+ * Low-Latency Megakernel for Llama-1B" for the step; the same plain decoder
+ * math as mk_decode_step).  Every activation row enters each projection as
+ * two bf16 rows (hi = bf16(x), lo = bf16(x - hi)), so the MMA's bf16 inputs
+ * keep about 16 significant bits.
+ * mk_tcdec_create checks `cfg` (batch <= 32; hidden, intermediate and
+ * n_heads*head_dim multiples of 64; head_dim 64 or 128; at most 8 query heads
+ * per KV head) and records the weight pointers of `w`, which are READ AT EVERY
+ * STEP: they must stay alive (unlike mk_load_weights, nothing is repacked).
+ * mk_tcdec_bind gives it the caller's workspace (mk_tcdec_workspace_bytes,
+ * 256-byte aligned) and KV cache (the layout of mk_kv_cache_bytes, so a
+ * context's prefilled cache can be shared).  mk_tcdec_step decodes one token
+ * per sequence at position `pos` (all sequences share it): it writes K/V at
+ * `pos`, attends to 0 .. pos, writes d_next (device int32 [batch]) and, if
+ * d_logits is set, the fp32 logits [batch, vocab].  Asynchronous on `stream`;
+ * an out-of-range token sets the status word (mk_tcdec_status, synchronous).
+ * Errors: MK_ERR_INVALID, MK_ERR_UNSUPPORTED, MK_ERR_STATE (step before
+ * bind), MK_ERR_CUDA; the reason is in mk_tcdec_last_error. */
+typedef struct mk_tcdec mk_tcdec;
+mk_status mk_tcdec_create(const mk_config *cfg, const mk_weights *w, mk_tcdec **out);
+mk_status mk_tcdec_workspace_bytes(const mk_tcdec *dec, size_t *bytes);
+mk_status mk_tcdec_bind(mk_tcdec *dec, void *workspace, void *kv_cache);
+mk_status mk_tcdec_step(mk_tcdec *dec, const int32_t *d_tokens, int pos, int32_t *d_next, float *d_logits,
+                        void *stream);
+mk_status mk_tcdec_status(mk_tcdec *dec, int *status, void *stream);
+const char *mk_tcdec_last_error(const mk_tcdec *dec);
+mk_status mk_tcdec_destroy(mk_tcdec *dec);
+
 /* Split-KV decode attention with a log-sum-exp combine, on its own: the
  * attention of one layer of one decode step ("Look Ma, No Bubbles! Designing
  * a Low-Latency Megakernel for Llama-1B", introduction: generating one

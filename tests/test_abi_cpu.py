@@ -165,3 +165,44 @@ def test_linear_tc_plan_and_argument_checks_need_no_device():
     assert lib.mk_linear_tc(d, d, d, 16, 4000, 4096, None) == _lib.MK_ERR_UNSUPPORTED
     assert "multiple of 64" in lib.mk_last_error(None).decode()
     assert lib.mk_linear_tc(d, d, d, 128, 4096, 4096, None) == _lib.MK_ERR_UNSUPPORTED
+
+
+def _fake_weights(n_layers, keep):
+    """An mk_weights struct whose every pointer is a fake, aligned address (the
+    host-side checks never dereference them)."""
+    arrs = [(C.c_void_p * n_layers)(*([4096] * n_layers)) for _ in range(11)]
+    keep.extend(arrs)
+    return _lib.MkWeights(4096, 4096, 4096, *[C.cast(a, C.POINTER(C.c_void_p)) for a in arrs])
+
+
+def test_tcdec_host_checks_need_no_device():
+    lib = _lib.load()
+    keep = []
+    s = synth.LLAMA8B
+    cfg = mkpy.make_config(s, 8, 520, "megakernel", 148)
+    w = _fake_weights(s.n_layers, keep)
+    dec = C.c_void_p()
+    assert lib.mk_tcdec_create(C.byref(cfg), C.byref(w), C.byref(dec)) == _lib.MK_OK
+    n = C.c_size_t()
+    assert lib.mk_tcdec_workspace_bytes(dec, C.byref(n)) == _lib.MK_OK
+    # x, hi/lo rows, the projection outputs (hi and lo rows each), q, attention out, scratch for 64 chunks
+    B, H, I, V, QD, KD = 8, s.hidden, s.intermediate, s.vocab, s.n_heads * s.head_dim, s.n_kv_heads * s.head_dim
+    floor = 4 * B * H + 2 * 2 * B * max(H, QD, I) + 4 * 2 * B * (QD + 2 * KD + H + 2 * I + V) + 2 * 4 * B * QD \
+        + lib.mk_attention_scratch_bytes(B, s.n_heads, s.head_dim, 64)
+    assert floor <= n.value <= floor + 14 * 256
+    # a step before bind, and a bind with a misaligned workspace, are refused
+    d = C.c_void_p(4096)
+    assert lib.mk_tcdec_step(dec, d, 0, d, None, None) == _lib.MK_ERR_STATE
+    assert lib.mk_tcdec_bind(dec, C.c_void_p(4096 + 16), d) == _lib.MK_ERR_INVALID
+    assert "aligned" in lib.mk_tcdec_last_error(dec).decode()
+    assert lib.mk_tcdec_destroy(dec) == _lib.MK_OK
+    # shapes it does not take
+    for bad, code in ((mkpy.make_config(s, 33, 520, "megakernel", 148), _lib.MK_ERR_UNSUPPORTED),
+                      (mkpy.make_config(synth.TINY, 1, 96, "megakernel", 148), _lib.MK_ERR_UNSUPPORTED)):
+        wt = _fake_weights(bad.n_layers, keep)
+        assert lib.mk_tcdec_create(C.byref(bad), C.byref(wt), C.byref(dec)) == code
+    assert "64" in lib.mk_tcdec_last_error(None).decode()  # tiny: intermediate 688 is not a multiple of 64
+    # a null weight pointer
+    w2 = _fake_weights(s.n_layers, keep)
+    w2.final_norm = None
+    assert lib.mk_tcdec_create(C.byref(cfg), C.byref(w2), C.byref(dec)) == _lib.MK_ERR_INVALID

@@ -13,7 +13,7 @@ import torch
 from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW,
                    MK_SWIGLU_TC, MK_SYNC_COUNTERS, MK_SYNC_TAGS, MkConfig, MkError, MkWeights, check, load)
 
-__all__ = ["Model", "swiglu_stage1", "swiglu_tune", "linear_tc", "linear_tc_split", "MkError", "VARIANTS",
+__all__ = ["Model", "TcDecoder", "swiglu_stage1", "swiglu_tune", "linear_tc", "linear_tc_split", "MkError", "VARIANTS",
            "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW", "MK_SWIGLU_COL", "MK_SWIGLU_TC", "load"]
 
 VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL}
@@ -84,6 +84,22 @@ class Plan:
     __del__ = close
 
 
+def _weights_struct(weights: dict, n_layers: int, keep: list) -> MkWeights:
+    """The mk_weights struct of a ``synth.make_weights``-style dict; the host
+    pointer arrays it refers to are appended to `keep`, which must outlive it."""
+    def ptr(t):
+        return None if t is None else t.data_ptr()
+
+    def arr(name):
+        a = (C.c_void_p * n_layers)(*[ptr(lw[name]) for lw in weights["layers"]])
+        keep.append(a)
+        return C.cast(a, C.POINTER(C.c_void_p))
+
+    return MkWeights(ptr(weights["embed"]), ptr(weights["final_norm"]), ptr(weights.get("lm_head")),
+                     *[arr(n) for n in ("attn_norm", "wq", "wk", "wv", "wo", "q_norm", "k_norm", "mlp_norm",
+                                        "wg", "wu", "wd")])
+
+
 class Model(Plan):
     """A decoder bound to device weights (``synth.make_weights`` structure, bf16 on CUDA)."""
 
@@ -101,20 +117,8 @@ class Model(Plan):
         self.workspace = torch.empty(self.workspace_bytes(), dtype=torch.uint8, device=self.device)
         self.kv = torch.empty(self.kv_cache_bytes(), dtype=torch.uint8, device=self.device)
         self._weights = weights  # the embedding table must stay alive
-        L = shape.n_layers
-
-        def ptr(t):
-            return None if t is None else t.data_ptr()
-
-        def arr(name):
-            a = (C.c_void_p * L)(*[ptr(lw[name]) for lw in weights["layers"]])
-            self._keep.append(a)
-            return C.cast(a, C.POINTER(C.c_void_p))
-
         self._keep = []
-        w = MkWeights(ptr(weights["embed"]), ptr(weights["final_norm"]), ptr(weights.get("lm_head")),
-                      *[arr(n) for n in ("attn_norm", "wq", "wk", "wv", "wo", "q_norm", "k_norm", "mlp_norm",
-                                         "wg", "wu", "wd")])
+        w = _weights_struct(weights, shape.n_layers, self._keep)
         check(self.lib.mk_load_weights(self.ctx, C.byref(w), C.c_void_p(self.workspace.data_ptr()),
                                        C.c_void_p(self.kv.data_ptr()), _stream(stream)), self.ctx, "mk_load_weights")
         self._next = torch.empty(self.batch, dtype=torch.int32, device=self.device)
@@ -246,6 +250,68 @@ def linear_tc_split(B: int, K: int, M: int) -> int:
     s = C.c_int()
     check(load().mk_linear_tc_split(B, K, M, C.byref(s)), None, "mk_linear_tc_split")
     return s.value
+
+
+class TcDecoder:
+    """A batched decode step with every projection on the tensor cores
+    (mk_tcdec_*): the caller's [out, in] bf16 weights are read at every step,
+    so `weights` is kept alive here.  `kv_cache` is a uint8 CUDA tensor in the
+    layout of ``Model.kv`` (pass a model's cache to decode on from its
+    prefill), or None for a fresh one."""
+
+    def __init__(self, shape, weights: dict, batch: int, max_seq: int, kv_cache: torch.Tensor | None = None,
+                 device: int | None = None):
+        self.lib = load()
+        self.shape, self.batch, self.max_seq = shape, batch, max_seq
+        dev = torch.cuda.current_device() if device is None else device
+        self.device = torch.device("cuda", dev)
+        self.dec = C.c_void_p()
+        cfg = make_config(shape, batch, max_seq, "megakernel", 0)
+        self._weights = weights
+        self._keep = []
+        w = _weights_struct(weights, shape.n_layers, self._keep)
+        check(self.lib.mk_tcdec_create(C.byref(cfg), C.byref(w), C.byref(self.dec)), None, "mk_tcdec_create")
+        n = C.c_size_t()
+        check(self.lib.mk_tcdec_workspace_bytes(self.dec, C.byref(n)), None, "mk_tcdec_workspace_bytes")
+        self.workspace = torch.empty(n.value, dtype=torch.uint8, device=self.device)
+        if kv_cache is None:
+            kv_bytes = 2 * shape.n_layers * batch * shape.n_kv_heads * max_seq * shape.head_dim * 2
+            kv_cache = torch.zeros(kv_bytes, dtype=torch.uint8, device=self.device)
+        self.kv = kv_cache
+        self._check(self.lib.mk_tcdec_bind(self.dec, C.c_void_p(self.workspace.data_ptr()),
+                                           C.c_void_p(self.kv.data_ptr())), "mk_tcdec_bind")
+        self._next = torch.empty(batch, dtype=torch.int32, device=self.device)
+
+    def _check(self, status: int, what: str) -> None:
+        if status != 0:
+            raise MkError(status, f"{what}: {self.lib.mk_tcdec_last_error(self.dec).decode()}")
+
+    def step(self, tokens: torch.Tensor, pos: int, logits: torch.Tensor | None = None,
+             out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """Decode one token per sequence at position `pos`: int32 CUDA tokens
+        [batch] -> next tokens [batch]; fills `logits` (fp32 [batch, vocab])
+        if given."""
+        assert tokens.dtype == torch.int32 and tokens.is_cuda and tokens.is_contiguous()
+        nxt = self._next if out is None else out
+        lp = None if logits is None else C.c_void_p(logits.data_ptr())
+        self._check(self.lib.mk_tcdec_step(self.dec, C.c_void_p(tokens.data_ptr()), int(pos),
+                                           C.c_void_p(nxt.data_ptr()), lp, _stream(stream)), "mk_tcdec_step")
+        return nxt
+
+    def status(self, stream=None) -> int:
+        v = C.c_int()
+        self._check(self.lib.mk_tcdec_status(self.dec, C.byref(v), _stream(stream)), "mk_tcdec_status")
+        return v.value
+
+    def close(self):
+        dec, self.dec = getattr(self, "dec", None), None
+        if dec:
+            try:
+                self.lib.mk_tcdec_destroy(dec)
+            except Exception:  # noqa: BLE001 - interpreter shutdown: the library may be gone
+                pass
+
+    __del__ = close
 
 
 def _attn_shapes(q: torch.Tensor, k_cache: torch.Tensor):

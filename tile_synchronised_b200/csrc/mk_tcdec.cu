@@ -1,0 +1,420 @@
+// mk_tcdec.cu -- a batched decode step whose projections run on the tcgen05
+// tensor cores: every matrix of the decoder (QKV, O, gate, up, down, LM head)
+// goes through mk_linear_tc, which reads each weight byte once for the whole
+// batch, and the attention through the split-KV kernels of mk_attn.cu.  The
+// rest of the step is small kernels over [batch, width] rows: the embedding
+// gather, RMSNorm, qk-norm + RoPE + KV append, the residual adds, SiLU * up,
+// and the LM head's argmax.
+//
+// Precision.  The MMA takes bf16 operands; a row rounded to bf16 loses 8 bits
+// of every activation, which over a deep decoder moves the logits by ~1-2 % of
+// their range.  So every activation row x enters as two bf16 rows, hi =
+// bf16(x) and lo = bf16(x - hi), in batch positions b and B + b of the
+// projection's input, and the output of row b is y[b] + y[B + b]: about 16
+// significant bits per activation for twice the MMA work, on a tensor pipe
+// that these shapes leave mostly idle.
+//
+// The math is the plain decoder step (the one the megakernel computes): for
+// each layer, h = RMSNorm(x) * g1; q, k, v = h W_q^T, h W_k^T, h W_v^T;
+// optional per-head RMSNorm of q and k; rotate-half RoPE at the position;
+// append k, v to the cache; attention over positions 0 .. pos; x += o W_o^T;
+// h = RMSNorm(x) * g2; x += (SiLU(h W_g^T) * (h W_u^T)) W_d^T; then the
+// logits of RMSNorm(x) * g_f and their argmax, lowest index on ties.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "mk_device.cuh"
+#include "mk_kernel.h"
+
+namespace mk {
+namespace tcdec {
+
+constexpr int kRowThreads = 256;
+constexpr int kArgmaxThreads = 1024;
+constexpr int kMaxBatch = 32;      // 2 * batch rows must fit mk_linear_tc's 64
+constexpr int kMaxChunks = 64;     // the split-KV chunk count never exceeds this
+
+__device__ __forceinline__ void put_hilo(__nv_bfloat16 *hi, __nv_bfloat16 *lo, float v) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    *hi = h;
+    *lo = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+// Sum over the block (blockDim.x a multiple of 32, at most 1024).
+__device__ float block_sum(float v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (int)blockDim.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    __syncthreads();  // red may still be read by a previous call
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float s = 0.f;
+    for (int w = 0; w < nw; ++w) s += red[w];
+    return s;
+}
+
+// x[b][:] = E[tok[b]][:]; an out-of-range token leaves the row at zero and
+// sets the status word.
+__global__ void embed_kernel(const int32_t *tok, const uint16_t *E, float *x, int H, int V, int *status) {
+    const int b = blockIdx.x, t = tok[b];
+    const bool ok = t >= 0 && t < V;
+    if (!ok && threadIdx.x == 0) atomicOr(status, 1);
+    for (int i = threadIdx.x; i < H; i += blockDim.x) x[(size_t)b * H + i] = ok ? bf2f(E[(size_t)t * H + i]) : 0.f;
+}
+
+// out rows b (hi) and B + b (lo) = RMSNorm(x[b]) * g, epsilon inside the root.
+__global__ void norm_hilo_kernel(const float *x, const uint16_t *g, __nv_bfloat16 *out, int B, int H, float eps) {
+    __shared__ float red[32];
+    const int b = blockIdx.x;
+    const float *xr = x + (size_t)b * H;
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < H; i += blockDim.x) ss = fmaf(xr[i], xr[i], ss);
+    ss = block_sum(ss, red);
+    const float r = rsqrtf(ss / (float)H + eps);
+    for (int i = threadIdx.x; i < H; i += blockDim.x)
+        put_hilo(out + (size_t)b * H + i, out + (size_t)(B + b) * H + i, xr[i] * r * bf2f(g[i]));
+}
+
+// One block per (head, sequence), head_dim threads.  Heads 0 .. nq-1 are q,
+// then nkv k heads, then nkv v heads; y* hold the hi and lo rows of each
+// projection.  q and k get the optional per-head RMSNorm and the RoPE
+// rotation (pairs i, i + d/2, angle pos * theta^(-2i/d) in double); q goes to
+// q_out, k and v to the layer's cache at `pos` as bf16.
+__global__ void qkv_post_kernel(const float *yq, const float *yk, const float *yv, int B, int nq, int nkv, int d,
+                                const uint16_t *qn, const uint16_t *kn, int qk_norm, float eps, double theta,
+                                int pos, float *q_out, uint16_t *kc, uint16_t *vc, int max_seq) {
+    extern __shared__ float buf[];  // d values, then 32 partial sums
+    float *red = buf + d;
+    const int head = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+    const float *src;
+    int M, off;
+    if (head < nq) {
+        src = yq;
+        M = nq * d;
+        off = head * d;
+    } else if (head < nq + nkv) {
+        src = yk;
+        M = nkv * d;
+        off = (head - nq) * d;
+    } else {
+        src = yv;
+        M = nkv * d;
+        off = (head - nq - nkv) * d;
+    }
+    float v = src[(size_t)b * M + off + i] + src[(size_t)(B + b) * M + off + i];
+    const int g = head < nq ? 0 : (head < nq + nkv ? head - nq : head - nq - nkv);
+    const size_t crow = (((size_t)b * nkv + g) * max_seq + pos) * d;
+    if (head >= nq + nkv) {
+        vc[crow + i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        return;
+    }
+    if (qk_norm) {
+        const float ss = block_sum(v * v, red);
+        v = v * rsqrtf(ss / (float)d + eps) * bf2f((head < nq ? qn : kn)[i]);
+    }
+    buf[i] = v;
+    __syncthreads();
+    const int h2 = d / 2, j = i < h2 ? i : i - h2;
+    const double ang = (double)pos * pow(theta, -2.0 * (double)j / (double)d);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    const float c = (float)cd, s = (float)sd;
+    const float r = i < h2 ? buf[i] * c - buf[i + h2] * s : buf[i] * c + buf[i - h2] * s;
+    if (head < nq)
+        q_out[((size_t)b * nq + head) * d + i] = r;
+    else
+        kc[crow + i] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+}
+
+// out rows b, B + b = hi / lo of a[b][:] (n values per row).
+__global__ void cast_hilo_kernel(const float *a, __nv_bfloat16 *out, int B, int n) {
+    const int b = blockIdx.y;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        put_hilo(out + (size_t)b * n + i, out + (size_t)(B + b) * n + i, a[(size_t)b * n + i]);
+}
+
+// x[b][i] += y[b][i] + y[B + b][i]
+__global__ void residual_add_kernel(float *x, const float *y, int B, int H) {
+    const int b = blockIdx.y;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < H; i += gridDim.x * blockDim.x)
+        x[(size_t)b * H + i] += y[(size_t)b * H + i] + y[(size_t)(B + b) * H + i];
+}
+
+// out rows b, B + b = hi / lo of SiLU(g) * u, g and u summed from their hi and
+// lo rows.
+__global__ void swiglu_hilo_kernel(const float *yg, const float *yu, __nv_bfloat16 *out, int B, int I) {
+    const int b = blockIdx.y;
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < I; j += gridDim.x * blockDim.x) {
+        const float g = yg[(size_t)b * I + j] + yg[(size_t)(B + b) * I + j];
+        const float u = yu[(size_t)b * I + j] + yu[(size_t)(B + b) * I + j];
+        put_hilo(out + (size_t)b * I + j, out + (size_t)(B + b) * I + j, g / (1.0f + expf(-g)) * u);
+    }
+}
+
+// One block per sequence: logits[b][v] = y[b][v] + y[B + b][v] (written when
+// `logits` is set) and next[b] = their argmax, lowest index on ties.
+__global__ void lm_argmax_kernel(const float *y, float *logits, int32_t *next, int B, int V) {
+    __shared__ float bv_s[32];
+    __shared__ int bi_s[32];
+    const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int v = threadIdx.x; v < V; v += blockDim.x) {
+        const float l = y[(size_t)b * V + v] + y[(size_t)(B + b) * V + v];
+        if (logits) logits[(size_t)b * V + v] = l;
+        if (l > bv || (l == bv && v < bi)) {
+            bv = l;
+            bi = v;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+        }
+    }
+    if (lane == 0) {
+        bv_s[warp] = bv;
+        bi_s[warp] = bi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+            if (bv_s[w] > bv_s[0] || (bv_s[w] == bv_s[0] && bi_s[w] < bi_s[0])) {
+                bv_s[0] = bv_s[w];
+                bi_s[0] = bi_s[w];
+            }
+        next[b] = bi_s[0];
+    }
+}
+
+// Byte offsets of the workspace pieces (each 256-byte aligned).
+struct Layout {
+    size_t x, h, yq, yk, yv, ya, yg, yu, ylm, q, attn, scratch, scratch_bytes, status, total;
+};
+
+static Layout layout(const mk_config &c) {
+    Layout o{};
+    const size_t B = (size_t)c.batch, H = (size_t)c.hidden, I = (size_t)c.intermediate, V = (size_t)c.vocab;
+    const size_t QD = (size_t)c.n_heads * c.head_dim, KD = (size_t)c.n_kv_heads * c.head_dim;
+    const size_t kmax = std::max(H, std::max(QD, I));
+    size_t at = 0;
+    auto take = [&](size_t bytes) {
+        const size_t p = at;
+        at += (bytes + 255) / 256 * 256;
+        return p;
+    };
+    o.x = take(B * H * 4);
+    o.h = take(2 * B * kmax * 2);
+    o.yq = take(2 * B * QD * 4);
+    o.yk = take(2 * B * KD * 4);
+    o.yv = take(2 * B * KD * 4);
+    o.ya = take(2 * B * H * 4);
+    o.yg = take(2 * B * I * 4);
+    o.yu = take(2 * B * I * 4);
+    o.ylm = take(2 * B * V * 4);
+    o.q = take(B * QD * 4);
+    o.attn = take(B * QD * 4);
+    o.scratch_bytes = mk_attention_scratch_bytes(c.batch, c.n_heads, c.head_dim, kMaxChunks);
+    o.scratch = take(o.scratch_bytes);
+    o.status = take(4);
+    o.total = at;
+    return o;
+}
+
+}  // namespace tcdec
+}  // namespace mk
+
+using namespace mk;
+using namespace mk::tcdec;
+
+struct mk_tcdec {
+    mk_config cfg{};
+    std::string err;
+    const void *embed = nullptr, *final_norm = nullptr, *lm_head = nullptr;
+    std::vector<const void *> attn_norm, wq, wk, wv, wo, q_norm, k_norm, mlp_norm, wg, wu, wd;
+    Layout lay{};
+    uint8_t *ws = nullptr;
+    uint16_t *kv = nullptr;
+};
+
+static mk_status tc_fail(mk_tcdec *d, mk_status s, const std::string &msg) {
+    if (d)
+        d->err = msg;
+    else
+        set_op_error(msg.c_str());
+    return s;
+}
+
+static bool aligned16(const void *p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+extern "C" mk_status mk_tcdec_create(const mk_config *cfg, const mk_weights *w, mk_tcdec **out) {
+    if (!cfg || !w || !out) return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: null argument");
+    *out = nullptr;
+    const mk_config &c = *cfg;
+    if (c.n_layers < 1 || c.hidden < 1 || c.n_heads < 1 || c.n_kv_heads < 1 || c.intermediate < 1 || c.vocab < 1 ||
+        c.batch < 1 || c.max_seq < 1 || !(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f))
+        return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: sizes must be positive");
+    if (c.dtype != MK_BF16) return tc_fail(nullptr, MK_ERR_UNSUPPORTED, "tcdec: only bf16 weights");
+    if (c.batch > kMaxBatch) return tc_fail(nullptr, MK_ERR_UNSUPPORTED, "tcdec: batch above 32");
+    if (c.head_dim != 64 && c.head_dim != 128)
+        return tc_fail(nullptr, MK_ERR_UNSUPPORTED, "tcdec: head_dim must be 64 or 128");
+    if (c.n_heads % c.n_kv_heads || c.n_heads / c.n_kv_heads > 8)
+        return tc_fail(nullptr, MK_ERR_UNSUPPORTED, "tcdec: n_heads must be a multiple of n_kv_heads, at most 8x");
+    if (c.hidden % 64 || c.intermediate % 64 || (c.n_heads * c.head_dim) % 64)
+        return tc_fail(nullptr, MK_ERR_UNSUPPORTED,
+                       "tcdec: hidden, intermediate and n_heads*head_dim must be multiples of 64");
+    auto d = new mk_tcdec();
+    d->cfg = c;
+    d->embed = w->embed;
+    d->final_norm = w->final_norm;
+    d->lm_head = c.tied_embeddings ? w->embed : w->lm_head;
+    bool ok = aligned16(d->embed) && aligned16(d->final_norm) && aligned16(d->lm_head);
+    const int L = c.n_layers;
+    auto grab = [&](const void *const *src, std::vector<const void *> &dst, bool need) {
+        if (!src) {
+            if (need) ok = false;
+            dst.assign((size_t)L, nullptr);
+            return;
+        }
+        dst.assign(src, src + L);
+        if (need)
+            for (const void *p : dst) ok = ok && aligned16(p);
+    };
+    grab(w->attn_norm, d->attn_norm, true);
+    grab(w->wq, d->wq, true);
+    grab(w->wk, d->wk, true);
+    grab(w->wv, d->wv, true);
+    grab(w->wo, d->wo, true);
+    grab(w->mlp_norm, d->mlp_norm, true);
+    grab(w->wg, d->wg, true);
+    grab(w->wu, d->wu, true);
+    grab(w->wd, d->wd, true);
+    grab(w->q_norm, d->q_norm, c.qk_norm != 0);
+    grab(w->k_norm, d->k_norm, c.qk_norm != 0);
+    if (!ok) {
+        delete d;
+        return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: a weight pointer is null or not 16-byte aligned");
+    }
+    d->lay = layout(c);
+    *out = d;
+    return MK_OK;
+}
+
+extern "C" mk_status mk_tcdec_workspace_bytes(const mk_tcdec *d, size_t *bytes) {
+    if (!d || !bytes) return MK_ERR_INVALID;
+    *bytes = d->lay.total;
+    return MK_OK;
+}
+
+extern "C" mk_status mk_tcdec_bind(mk_tcdec *d, void *workspace, void *kv_cache) {
+    // the workspace and the cache belong to the caller; the status word is
+    // cleared here (synchronously) and only ever set afterwards
+    if (!d) return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: null context");
+    if (!workspace || ((uintptr_t)workspace & 255u) || !aligned16(kv_cache))
+        return tc_fail(d, MK_ERR_INVALID, "tcdec: workspace must be 256-byte and kv_cache 16-byte aligned");
+    d->ws = static_cast<uint8_t *>(workspace);
+    d->kv = static_cast<uint16_t *>(kv_cache);
+    if (cudaMemset(d->ws + d->lay.status, 0, sizeof(int)) != cudaSuccess)
+        return tc_fail(d, MK_ERR_CUDA, "tcdec: clearing the status word");
+    return MK_OK;
+}
+
+extern "C" mk_status mk_tcdec_step(mk_tcdec *d, const int32_t *d_tokens, int pos, int32_t *d_next, float *d_logits,
+                                   void *stream) {
+    if (!d) return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: null context");
+    if (!d->ws) return tc_fail(d, MK_ERR_STATE, "tcdec: mk_tcdec_step before mk_tcdec_bind");
+    const mk_config &c = d->cfg;
+    if (!d_tokens || !d_next) return tc_fail(d, MK_ERR_INVALID, "tcdec: null token buffer");
+    if (pos < 0 || pos >= c.max_seq) return tc_fail(d, MK_ERR_INVALID, "tcdec: position outside the cache");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Layout &o = d->lay;
+    const int B = c.batch, H = c.hidden, I = c.intermediate, V = c.vocab, L = c.n_layers;
+    const int nq = c.n_heads, nkv = c.n_kv_heads, hd = c.head_dim, QD = nq * hd, KD = nkv * hd;
+    float *x = reinterpret_cast<float *>(d->ws + o.x);
+    __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(d->ws + o.h);
+    float *yq = reinterpret_cast<float *>(d->ws + o.yq), *yk = reinterpret_cast<float *>(d->ws + o.yk);
+    float *yv = reinterpret_cast<float *>(d->ws + o.yv), *ya = reinterpret_cast<float *>(d->ws + o.ya);
+    float *yg = reinterpret_cast<float *>(d->ws + o.yg), *yu = reinterpret_cast<float *>(d->ws + o.yu);
+    float *ylm = reinterpret_cast<float *>(d->ws + o.ylm);
+    float *q = reinterpret_cast<float *>(d->ws + o.q), *attn = reinterpret_cast<float *>(d->ws + o.attn);
+    void *scratch = d->ws + o.scratch;
+    int *status = reinterpret_cast<int *>(d->ws + o.status);
+    const size_t layer_elems = (size_t)B * nkv * c.max_seq * hd;
+    const int n_pos = pos + 1;
+    const int chunks = mk_attention_chunks(B, nkv, n_pos);
+    mk_status st = MK_OK;
+    auto lin = [&](const void *xin, const void *wt, float *y, int K, int M) {
+        if (st == MK_OK && mk_linear_tc(xin, wt, y, 2 * B, K, M, stream) != MK_OK) {
+            st = MK_ERR_CUDA;
+            d->err = std::string("tcdec: ") + op_error();
+        }
+    };
+    const dim3 rows_grid(8, (unsigned)B);
+    embed_kernel<<<B, kRowThreads, 0, s>>>(d_tokens, static_cast<const uint16_t *>(d->embed), x, H, V, status);
+    for (int l = 0; l < L && st == MK_OK; ++l) {
+        uint16_t *kc = d->kv + (size_t)l * layer_elems, *vc = d->kv + (size_t)(L + l) * layer_elems;
+        norm_hilo_kernel<<<B, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(d->attn_norm[l]), h, B, H,
+                                                   c.rms_eps);
+        lin(h, d->wq[l], yq, H, QD);
+        lin(h, d->wk[l], yk, H, KD);
+        lin(h, d->wv[l], yv, H, KD);
+        if (st != MK_OK) break;
+        qkv_post_kernel<<<dim3((unsigned)(nq + 2 * nkv), (unsigned)B), hd, (hd + 32) * sizeof(float), s>>>(
+            yq, yk, yv, B, nq, nkv, hd, static_cast<const uint16_t *>(d->q_norm[l]),
+            static_cast<const uint16_t *>(d->k_norm[l]), c.qk_norm, c.rms_eps, (double)c.rope_theta, pos, q, kc, vc,
+            c.max_seq);
+        if (mk_attention_decode(q, kc, vc, B, nq, nkv, hd, c.max_seq, n_pos, chunks, attn, scratch, o.scratch_bytes,
+                                stream) != MK_OK) {
+            st = MK_ERR_CUDA;
+            d->err = std::string("tcdec: ") + op_error();
+            break;
+        }
+        cast_hilo_kernel<<<rows_grid, kRowThreads, 0, s>>>(attn, h, B, QD);
+        lin(h, d->wo[l], ya, QD, H);
+        residual_add_kernel<<<rows_grid, kRowThreads, 0, s>>>(x, ya, B, H);
+        norm_hilo_kernel<<<B, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(d->mlp_norm[l]), h, B, H,
+                                                   c.rms_eps);
+        lin(h, d->wg[l], yg, H, I);
+        lin(h, d->wu[l], yu, H, I);
+        swiglu_hilo_kernel<<<dim3(32, (unsigned)B), kRowThreads, 0, s>>>(yg, yu, h, B, I);
+        lin(h, d->wd[l], ya, I, H);
+        residual_add_kernel<<<rows_grid, kRowThreads, 0, s>>>(x, ya, B, H);
+    }
+    if (st != MK_OK) return st;
+    norm_hilo_kernel<<<B, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(d->final_norm), h, B, H, c.rms_eps);
+    lin(h, d->lm_head, ylm, H, V);
+    if (st != MK_OK) return st;
+    lm_argmax_kernel<<<B, kArgmaxThreads, 0, s>>>(ylm, d_logits, d_next, B, V);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: ") + cudaGetErrorString(e));
+    return MK_OK;
+}
+
+extern "C" mk_status mk_tcdec_status(mk_tcdec *d, int *status, void *stream) {
+    if (!d || !status) return MK_ERR_INVALID;
+    if (!d->ws) return tc_fail(d, MK_ERR_STATE, "tcdec: not bound");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(status, d->ws + d->lay.status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return tc_fail(d, MK_ERR_CUDA, "tcdec: reading the status word");
+    return MK_OK;
+}
+
+extern "C" const char *mk_tcdec_last_error(const mk_tcdec *d) { return d ? d->err.c_str() : op_error(); }
+
+extern "C" mk_status mk_tcdec_destroy(mk_tcdec *d) {
+    delete d;
+    return MK_OK;
+}
