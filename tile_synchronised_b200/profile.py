@@ -120,6 +120,8 @@ def main(argv=None):
     ap.add_argument("--synthetic-kv", type=int, default=0, metavar="C",
                     help="timing only: instead of a prefill, fill cache positions < C with seeded N(0,1) bf16 "
                          "values and start decoding at position C (the step's cost depends on C, not on the values)")
+    ap.add_argument("--tcdec", action="store_true",
+                    help="also time the tensor-core decode step (mk_tcdec_*) on the same cache, at the last position")
     a = ap.parse_args(argv)
     shape = synth.MODELS[a.workload]
     B = a.batch or shape.batch
@@ -155,6 +157,23 @@ def main(argv=None):
         print(json.dumps({"timed_steps": a.time, "us_per_step": round(1e3 * e0.elapsed_time(e1) / a.time, 2),
                           "prefetch": a.prefetch, "sync": a.sync, "stages": a.stages}))
         model.set_position(prefill + a.steps - 1)
+        if a.tcdec:
+            dec = mk.TcDecoder(shape, tw, B, max_seq, kv_cache=model.kv)
+            p_tc = prefill + a.steps - 1
+            tok = d_tok[a.steps - 2 if a.steps > 1 else 0]
+            for r in range(3):
+                dec.step(tok, p_tc)
+            torch.cuda.synchronize()
+            e0.record()
+            for r in range(a.time):
+                dec.step(tok, p_tc)
+            e1.record()
+            torch.cuda.synchronize()
+            if dec.status() != 0:
+                raise SystemExit("tensor-core decode step: a token out of range")
+            print(json.dumps({"tcdec_timed_steps": a.time,
+                              "tcdec_us_per_step": round(1e3 * e0.elapsed_time(e1) / a.time, 2)}))
+            dec.close()
     tr = None
     if a.trace:
         n = model.info()["n_instructions"]
