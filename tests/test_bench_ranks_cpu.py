@@ -34,7 +34,7 @@ def _rank(rank, world, port, out):
 
 def test_two_gloo_ranks_agree_on_the_slowest_time():
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:  # no fork of this multi-threaded process
         out = m.dict()
         mp.spawn(_rank, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
