@@ -47,6 +47,13 @@ def check_argmax(nxt_gpu: np.ndarray, logits_gpu: np.ndarray, logits_ref: np.nda
     return undecided
 
 
+def host_weights(tw):
+    """The same weights as host uint16 bit patterns, for the oracle."""
+    host = {kk: (None if tw[kk] is None else synth.to_u16(tw[kk])) for kk in ("embed", "final_norm", "lm_head")}
+    host["layers"] = [{a: (None if t is None else synth.to_u16(t)) for a, t in lw.items()} for lw in tw["layers"]]
+    return host
+
+
 def widen_bf16(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy()
 

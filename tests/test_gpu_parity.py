@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from gpu_common import build_pair, check_argmax, logits_close, widen_bf16
+from gpu_common import build_pair, check_argmax, host_weights, logits_close, widen_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -204,12 +204,6 @@ def sampled_layer0_rows(shape, tw, k, v, tokens_np, b, positions):
             got_v = v[0, b, g, p].float().cpu().numpy()
             assert np.max(np.abs(got_k - want_k)) <= 2e-2 * np.max(np.abs(want_k))
             assert np.max(np.abs(got_v - vv[g])) <= 2e-2 * np.max(np.abs(vv[g]))
-
-
-def host_weights(tw):
-    host = {kk: (None if tw[kk] is None else synth.to_u16(tw[kk])) for kk in ("embed", "final_norm", "lm_head")}
-    host["layers"] = [{a: (None if t is None else synth.to_u16(t)) for a, t in lw.items()} for lw in tw["layers"]]
-    return host
 
 
 def handoff_step(shape, host, model, tokens, pos, seqs):

@@ -12,8 +12,7 @@ import torch
 
 import oracle
 import synth
-from gpu_common import check_argmax, logits_close
-from test_gpu_parity import host_weights
+from gpu_common import check_argmax, host_weights, logits_close
 
 pytestmark = pytest.mark.gpu
 
