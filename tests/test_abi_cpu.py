@@ -206,3 +206,13 @@ def test_tcdec_host_checks_need_no_device():
     w2 = _fake_weights(s.n_layers, keep)
     w2.final_norm = None
     assert lib.mk_tcdec_create(C.byref(cfg), C.byref(w2), C.byref(dec)) == _lib.MK_ERR_INVALID
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/mk.h is a C header: no torch or C++ types cross the boundary."""
+    src = tmp_path / "use_mk.c"
+    src.write_text('#include "mk.h"\nint main(void) { mk_ctx *c = 0; mk_tcdec *d = 0; (void)c; (void)d;\n'
+                   '  return (int)sizeof(mk_config) + (int)sizeof(mk_weights); }\n')
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), "-c",
+                        str(src), "-o", str(tmp_path / "use_mk.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
