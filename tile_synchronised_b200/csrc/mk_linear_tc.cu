@@ -210,12 +210,9 @@ cudaError_t launch_linear_tc(const void *x, const void *w, float *y, int B, int 
     if (!tc_make_map(&mw, w, (uint64_t)M, (uint64_t)K, kLinBK, kLinM) ||
         !tc_make_map(&mx, x, (uint64_t)B, (uint64_t)K, kLinBK, (uint32_t)p.sh.Bp))
         return cudaErrorInvalidValue;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t ce = tc_allow_smem(reinterpret_cast<const void *>(linear_tc_kernel), 227 * 1024, configured);
+    if (ce != cudaSuccess) return ce;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.tiles * p.split));
     cfg.blockDim = dim3(kLinThreads);

@@ -385,12 +385,9 @@ cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void
     if (sh.stages > 6) sh.stages = 6;
     if (sh.stages < 2) return cudaErrorInvalidValue;
     const int smem = sh.stages * (int)sh.stage_bytes + 1024 + 256;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(swiglu_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t ce = tc_allow_smem(reinterpret_cast<const void *>(swiglu_tc_kernel), 227 * 1024, configured);
+    if (ce != cudaSuccess) return ce;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((N / kTcM) * kTcSplit);
     cfg.blockDim = dim3(kTcThreads);

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "mk_device.cuh"
@@ -99,6 +100,20 @@ __device__ __forceinline__ uint32_t cluster_size() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
     return r;
+}
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per device (bit d of `done` records device d; the attribute
+// is per device, so a second device gets its own call).
+inline cudaError_t tc_allow_smem(const void *fn, int bytes, std::atomic<unsigned long long> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
 }
 
 // 2-D tensor of 2-byte elements [rows][cols] (cols contiguous, row stride
