@@ -306,6 +306,77 @@ def test_qk_norm_gives_unit_rms_heads():
     np.testing.assert_allclose(nrm, math.sqrt(s.head_dim), rtol=1e-4)
 
 
+@pytest.mark.parametrize("qk_norm", [True, False])
+def test_qk_norm_makes_logits_blind_to_query_scale(qk_norm):
+    """Per-head RMSNorm of q divides out any scale of W_q, so multiplying one
+    layer's W_q by 8 (exact in bf16) leaves the logits unchanged up to the eps
+    term; without the q norm the scores grow 8x and the logits move.  A q
+    branch that is dropped, or that normalises the wrong vector, fails one of
+    the two cases."""
+    s = SMALL.replace(qk_norm=qk_norm, rms_eps=1e-6)
+    w = np_weights(s, seed=21)
+    toks = [7, 19, 3, 44]
+    base = oracle.OracleModel(s, w)
+    for t in toks:
+        ref, _ = base.step([t])
+    w["layers"][1]["wq"] = bf16_bits(widen(w["layers"][1]["wq"]) * 8.0)
+    scaled = oracle.OracleModel(s, w)
+    for t in toks:
+        got, _ = scaled.step([t])
+    rel = float(np.max(np.abs(got - ref)) / np.max(np.abs(ref)))
+    if qk_norm:
+        assert rel < 1e-5
+    else:
+        assert rel > 1e-2
+
+
+def test_qk_norm_gains_closed_form():
+    """One layer with the MLP removed (W_down = 0), two positions, distinct
+    per-element gains on the q and k head norms: the logits follow from numpy
+    alone -- RMSNorm, the projections, per-head RMSNorm times its own gain,
+    RoPE as a complex rotation of the (i, i + d/2) pairs, softmax attention
+    with KV head = q head // (nq / nkv), O-projection, final norm and head.
+    Swapping the two gain vectors, or applying one to both, fails it."""
+    s = SMALL.replace(n_layers=1, qk_norm=True, rms_eps=1e-6)
+    w = np_weights(s, seed=22)
+    L0 = w["layers"][0]
+    d, nq, nkv, eps = s.head_dim, s.n_heads, s.n_kv_heads, s.rms_eps
+    L0["q_norm"] = bf16_bits(np.linspace(0.5, 2.0, d))
+    L0["k_norm"] = bf16_bits(np.linspace(1.75, 0.25, d))
+    L0["wd"][:] = 0
+    toks = [11, 37]
+    m = oracle.OracleModel(s, w)
+    for t in toks:
+        logits, _ = m.step([t])
+
+    def rot(v, p):
+        h = d // 2
+        z = (v[..., :h] + 1j * v[..., h:]) * np.exp(1j * p * s.rope_theta ** (-2.0 * np.arange(h) / d))
+        return np.concatenate([z.real, z.imag], axis=-1)
+
+    X0 = widen(w["embed"][toks])
+    Hn = np_rms(X0, eps)
+    gq, gk = widen(L0["q_norm"]), widen(L0["k_norm"])
+    K = np.stack([rot(np_rms((widen(L0["wk"]) @ Hn[p]).reshape(nkv, d), eps) * gk, p) for p in range(2)])
+    V = np.stack([(widen(L0["wv"]) @ Hn[p]).reshape(nkv, d) for p in range(2)])
+    Q = rot(np_rms((widen(L0["wq"]) @ Hn[1]).reshape(nq, d), eps) * gq, 1)
+    o = []
+    for h in range(nq):
+        g = h // (nq // nkv)
+        sc = K[:, g] @ Q[h] / math.sqrt(d)
+        a = np.exp(sc - sc.max())
+        o.append((a / a.sum()) @ V[:, g])
+    x1 = X0[1] + widen(L0["wo"]) @ np.concatenate(o)
+    want = widen(w["lm_head"]) @ np_rms(x1, eps)
+    np.testing.assert_allclose(logits[0], want, rtol=2e-5, atol=2e-5)
+    # the two gain vectors are far enough apart that a swap is visible
+    L0["q_norm"], L0["k_norm"] = L0["k_norm"].copy(), L0["q_norm"].copy()
+    swapped = oracle.OracleModel(s, w)
+    for t in toks:
+        lsw, _ = swapped.step([t])
+    assert float(np.max(np.abs(lsw[0] - want))) > 1e-3 * float(np.max(np.abs(want)))
+
+
 def test_incremental_decode_equals_full_recompute():
     s = SMALL.replace(n_layers=2, qk_norm=False)
     w = np_weights(s, seed=16)
