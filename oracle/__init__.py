@@ -62,6 +62,7 @@ def lib():
         L.orc_forward_full.restype = C.c_int
         L.orc_swiglu_stage1_f16.argtypes = [u16p, u16p, u16p, f32p, C.c_int64, C.c_int64, C.c_int64]
         L.orc_num_threads.restype = C.c_int
+        L.orc_set_num_threads.argtypes = [C.c_int]
         _lib = L
     return _lib
 
@@ -125,6 +126,11 @@ def swiglu_stage1_f16(x_u16: np.ndarray, wg_u16: np.ndarray, wu_u16: np.ndarray)
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of later oracle calls (n < 1: all processors)."""
+    lib().orc_set_num_threads(int(n))
 
 
 # ---------------------------------------------------------------- the decoder

@@ -337,6 +337,17 @@ void orc_swiglu_stage1_f16(const uint16_t *x, const uint16_t *wg, const uint16_t
     }
 }
 
+/* Thread count of later calls (n < 1: all processors); the benchmark times
+ * the oracle on one core beside the all-core figure.  No effect on results:
+ * only the output rows of a matrix-vector product are divided among threads. */
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+    omp_set_num_threads(n > 0 ? n : omp_get_num_procs());
+#else
+    (void)n;
+#endif
+}
+
 /* Number of OpenMP threads the oracle uses (reported with its timings). */
 int orc_num_threads(void) {
     int n = 1;
