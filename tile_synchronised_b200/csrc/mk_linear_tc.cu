@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_base;
 
+    int issued = 0;  // K blocks whose copies the producer (warp 0 lane 0) has issued
     if (warp == 0 && lane == 0) {
         for (int kb = 0; kb < nkb; ++kb) {
             const int s = kb % S;
@@ -103,6 +104,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
             const int k0 = (kb_first + kb) * kLinBK;
             tma_load_2d(st, &map_w, k0, m0, &full[s]);
             tma_load_2d(st + sh.a_bytes, &map_x, k0, 0, &full[s]);
+            issued = kb + 1;
         }
     } else if (warp == 1 && lane == 0) {
         // Both operands K-major, 128-byte swizzle: 8 rows of 128 bytes per
@@ -127,6 +129,14 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     // epilogue: thread t holds output row m0 + t (tensor-memory lane t; warp w
     // may read lanes 32w .. 32w+31), one column per batch row
     const bool ok = tc_wait(done, 0u, abort) && !*abort;
+    // After an abort some copies may never have been waited for.  A stage
+    // holds at most one copy in flight, so the producer lets the last copy of
+    // every stage land before this CTA's stage memory is reused (by the
+    // cluster reduction below) or freed; the other threads wait for it at the
+    // next CTA or cluster barrier.
+    if (warp == 0 && lane == 0 && *abort)
+        for (int kb = issued > S ? issued - S : 0; kb < issued; ++kb)
+            tc_drain(&full[kb % S], (uint32_t)(kb / S) & 1u, kTcTimeoutNs);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     // Once every CTA of the cluster is past its last MMA, the first CTA's

@@ -58,6 +58,17 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile
     }
 }
 
+// After a CTA gave up: wait (bounded by `limit_ns`, ignoring the abort flag)
+// until the phase `parity` of `bar` -- the last copy issued into that stage --
+// has landed, so that no copy into this CTA's shared memory is still in
+// flight when it frees its resources and exits.  False if it did not land.
+__device__ __forceinline__ bool tc_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_sleep(bar, parity, 10000u))
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    return true;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2,
 // descriptor version 1): start address, leading and stride byte offsets, all
 // in 16-byte units.

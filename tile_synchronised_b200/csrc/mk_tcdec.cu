@@ -160,8 +160,10 @@ __global__ void swiglu_hilo_kernel(const float *yg, const float *yu, __nv_bfloat
 }
 
 // One block per sequence: logits[b][v] = y[b][v] + y[B + b][v] (written when
-// `logits` is set) and next[b] = their argmax, lowest index on ties.
-__global__ void lm_argmax_kernel(const float *y, float *logits, int32_t *next, int B, int V) {
+// `logits` is set) and next[b] = their argmax, lowest index on ties.  With no
+// finite logit to pick (a projection that gave up writes NaN), next[b] is set
+// to 0, a valid token, and bit 2 of the status word is set.
+__global__ void lm_argmax_kernel(const float *y, float *logits, int32_t *next, int B, int V, int *status) {
     __shared__ float bv_s[32];
     __shared__ int bi_s[32];
     const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -195,6 +197,10 @@ __global__ void lm_argmax_kernel(const float *y, float *logits, int32_t *next, i
                 bv_s[0] = bv_s[w];
                 bi_s[0] = bi_s[w];
             }
+        if (bi_s[0] == 0x7fffffff) {
+            atomicOr(status, 2);
+            bi_s[0] = 0;
+        }
         next[b] = bi_s[0];
     }
 }
@@ -396,7 +402,7 @@ extern "C" mk_status mk_tcdec_step(mk_tcdec *d, const int32_t *d_tokens, int pos
     norm_hilo_kernel<<<B, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(d->final_norm), h, B, H, c.rms_eps);
     lin(h, d->lm_head, ylm, H, V);
     if (st != MK_OK) return st;
-    lm_argmax_kernel<<<B, kArgmaxThreads, 0, s>>>(ylm, d_logits, d_next, B, V);
+    lm_argmax_kernel<<<B, kArgmaxThreads, 0, s>>>(ylm, d_logits, d_next, B, V, status);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: ") + cudaGetErrorString(e));
     return MK_OK;
