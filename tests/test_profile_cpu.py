@@ -45,3 +45,12 @@ def test_summary_phases_and_per_op_times():
     assert abs(s["per_op"]["gateup"]["wait_sum_us_per_cta"] - 4 * 1.0) < 1e-9
     assert s["phases"][0]["op"] == "qkv" and s["phases"][-1]["op"] == "lmhead"
     assert set(s["edges"]) == {"down->qkv", "qkv->attn", "acomb->oproj", "oproj->gateup", "gateup->down"}
+
+
+def test_sweep_table_marks_the_faster_tiling():
+    from tile_synchronised_b200 import sweep
+    md = sweep.rows_to_markdown([{"batch": 4, "kv": 1024, "row_us": 10.0, "col_us": 12.5, "tuned": "row"},
+                                 {"batch": 16, "kv": 16384, "row_us": 30.0, "col_us": 20.0, "tuned": "column"}])
+    lines = md.strip().splitlines()
+    assert len(lines) == 4
+    assert lines[2].split("|")[5].strip() == "row" and lines[3].split("|")[5].strip() == "column"
