@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
-    ap.add_argument("--variant", default="megakernel", choices=["megakernel", "graph", "graph_pdl"])
+    ap.add_argument("--variant", default="megakernel", choices=["megakernel", "graph", "graph_pdl", "tilesync"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true", help="skip timing the separate-kernel variants")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
@@ -300,7 +300,7 @@ def run_mk(args, world, rank, local):
     # the same ops as separate kernels in a CUDA graph (with and without PDL)
     variants = {}
     if not args.no_variants:
-        for v in ("megakernel", "graph", "graph_pdl"):
+        for v in ("megakernel", "graph", "graph_pdl", "tilesync"):
             if v == args.variant:
                 variants[v] = {"tokens_per_s": round(value / world, 2), "ms_per_step": round(ms_per_step, 5)}
                 continue
@@ -330,6 +330,14 @@ def run_mk(args, world, rank, local):
         cpu = {"value": round(B * n / el, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n} oracle decode steps (batch 1, positions 1024+, KV handed over from the GPU "
                          f"prefill), {el:.1f} s on {cores} OpenMP threads"}
+        import oracle
+        oracle.set_num_threads(1)
+        try:
+            n1, el1, _ = oracle_steps(shape, hw, kc, vc, tokens.numpy(), args.cpu_seconds / 3)
+        finally:
+            oracle.set_num_threads(0)
+        cpu["one_core"] = {"value": round(B * n1 / el1, 4), "unit": UNIT, "cores": 1,
+                           "sample": f"{n1} oracle decode steps, {el1:.1f} s on 1 OpenMP thread"}
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -55,8 +55,19 @@ enum { MK_BF16 = 0 };
 enum {
     MK_MEGAKERNEL = 0, /* one persistent launch, tile-ready counters between ops */
     MK_GRAPH = 1,      /* the same ops as one launch per op, replayed from a CUDA graph */
-    MK_GRAPH_PDL = 2   /* as MK_GRAPH, launches chained by programmatic dependent launch so
+    MK_GRAPH_PDL = 2,  /* as MK_GRAPH, launches chained by programmatic dependent launch so
                           each op streams its weights while the previous op finishes */
+    MK_GRAPH_TILESYNC = 3 /* the ops as separate kernels in the same CUDA graph, each
+                          launched early by programmatic dependent launch and started
+                          on the tiles it reads instead of on the previous kernel's
+                          end ("MegaOps: A Kernel Overlapping Framework ...", "In plain
+                          words" and "Keep kernels separate"): a kernel's CTAs occupy
+                          SMs as the previous kernel's CTAs leave them, stream their
+                          weights at once and wait on the tagged words (or, with
+                          MK_SYNC_COUNTERS, the tile-ready counters) of the data they
+                          read.  A kernel launches only after every CTA of the one
+                          before it has started, so what it waits for is always
+                          running; every wait is bounded. */
 };
 /* How the megakernel's dependent instructions learn that their inputs are
  * ready ("MegaOps: A Kernel Overlapping Framework ...", "In plain words": a
@@ -86,7 +97,7 @@ typedef struct {
     int batch;           /* sequences decoded together, 1..64 */
     int max_seq;         /* KV cache positions per sequence */
     int dtype;           /* MK_BF16 (the only one) */
-    int variant;         /* MK_MEGAKERNEL | MK_GRAPH | MK_GRAPH_PDL */
+    int variant;         /* MK_MEGAKERNEL | MK_GRAPH | MK_GRAPH_PDL | MK_GRAPH_TILESYNC */
     int num_sms;         /* CTAs of the persistent kernel; 0 = the device's SM count */
 } mk_config;
 
@@ -148,13 +159,18 @@ mk_status mk_prefill_kv(mk_ctx *ctx, const int32_t *d_tokens, int batch, int T, 
  * (lowest index on ties) goes to `d_next` (device int32 [batch], may be NULL).
  * If `d_logits` is not NULL it receives the fp32 logits [batch, vocab] the
  * argmax was taken over.  Advances the position.  MK_ERR_INVALID if p ==
- * max_seq.  A token outside [0, vocab) is clamped to the range on the device;
- * a device wait timeout is reported by mk_get_status. */
+ * max_seq.  The tokens live in device memory, so their range is checked on the
+ * device: a token outside [0, vocab) is recorded (the step decodes token 0 in
+ * its place so that no read leaves the embedding table) and the next
+ * mk_get_status returns MK_ERR_INVALID naming the sequence and the token; a
+ * device wait timeout is reported by mk_get_status too. */
 mk_status mk_decode_step(mk_ctx *ctx, const int32_t *d_tokens, int32_t *d_next, float *d_logits, void *stream);
 
 /* Synchronize `stream` and return MK_ERR_TIMEOUT if a device wait gave up
- * during any earlier step (the context is then poisoned until mk_reset),
- * MK_ERR_CUDA on a CUDA error, else MK_OK. */
+ * during any earlier step, MK_ERR_INVALID if an earlier step (or prefill) was
+ * given a token outside [0, vocab) -- in both cases the context is poisoned
+ * until mk_reset, and the KV rows written at the positions of those steps hold
+ * no valid result -- MK_ERR_CUDA on a CUDA error, else MK_OK. */
 mk_status mk_get_status(mk_ctx *ctx, void *stream);
 /* Clear counters, error word and position (KV cache contents are kept). */
 mk_status mk_reset(mk_ctx *ctx, void *stream);
@@ -166,7 +182,7 @@ mk_status mk_get_position(const mk_ctx *ctx, int *pos);
 mk_status mk_set_position(mk_ctx *ctx, int pos, void *stream);
 
 /* Select the execution variant for later decode steps (MK_MEGAKERNEL,
- * MK_GRAPH or MK_GRAPH_PDL). */
+ * MK_GRAPH, MK_GRAPH_PDL or MK_GRAPH_TILESYNC). */
 mk_status mk_set_variant(mk_ctx *ctx, int variant);
 
 /* One-time profiling pass ("Deep Kernel Fusion for Transformers", Summary and
@@ -177,6 +193,17 @@ mk_status mk_set_variant(mk_ctx *ctx, int variant);
  * position are restored afterwards.  Synchronous.  *chosen (may be NULL)
  * receives MK_SWIGLU_ROW or MK_SWIGLU_COL. */
 mk_status mk_tune(mk_ctx *ctx, void *stream, int *chosen);
+
+/* Select the gate/up tiling of later steps without timing it (what mk_tune
+ * would otherwise pick): MK_SWIGLU_COL, every gate/up instruction carries all
+ * of its batch rows and streams its weight tiles once; MK_SWIGLU_ROW, an
+ * instruction carries at most half of them (rounded up), so each weight tile
+ * streams once per row group.  Both give bit-identical results.  Synchronous
+ * on `stream`; the KV cache and the position are kept.  MK_ERR_INVALID for
+ * another value, MK_ERR_STATE before mk_load_weights or on a poisoned
+ * context.  mk_get_swiglu_tiling reports the active one. */
+mk_status mk_set_swiglu_tiling(mk_ctx *ctx, int variant, void *stream);
+mk_status mk_get_swiglu_tiling(const mk_ctx *ctx, int *variant);
 
 /* How far, in 32 KB ring blocks, the producer's L2 prefetches may run ahead of
  * its shared-memory loads.  It keeps min(4, blocks) ahead at all times and
@@ -204,6 +231,27 @@ mk_status mk_set_sync(mk_ctx *ctx, int mode);
  * outputs keep a stale tag), so its consumers' waits run out in either sync
  * mode; -1 clears it.  Used to test timeout reporting. */
 mk_status mk_debug_drop_signal(mk_ctx *ctx, int instr);
+
+/* Test hook: fill every buffer the step's instructions hand to each other
+ * (the tagged activation words: residual stream, q/k/v, split-KV partials,
+ * attention output, SwiGLU product, down-projection partial outputs, and the
+ * per-CTA argmax records) with 0xFF bytes -- NaN values under a tag no step
+ * writes -- so that a read of a word its producer has not written this step
+ * cannot pass for data.  Synchronous on `stream`.  MK_ERR_STATE before
+ * mk_load_weights. */
+mk_status mk_debug_poison_activations(mk_ctx *ctx, void *stream);
+
+/* Test hook: reorder the active schedule with the seeded permutation that
+ * keeps every dependency (for each phase, the CTAs' groups of instructions
+ * are dealt to the CTAs in a random order and each group is shuffled; every
+ * CTA's list stays in phase order), re-check it as mk_validate_schedule does
+ * and, when weights are loaded, upload it (synchronous).  Each instruction
+ * computes the same values wherever it runs, so results must be
+ * bit-identical to the unshuffled schedule's; a dependency the planner failed
+ * to express would show up as a difference or a timeout.  It stays in effect
+ * until the gate/up tiling is switched (mk_set_swiglu_tiling, mk_tune), which
+ * installs that tiling's unshuffled plan.  MK_ERR_STATE if the check fails. */
+mk_status mk_debug_shuffle_schedule(mk_ctx *ctx, unsigned long long seed);
 
 /* Per-instruction timing trace for the following steps: `d_trace` is a
  * device buffer of at least 8 * n_instructions uint64 (64 bytes per
@@ -296,10 +344,17 @@ mk_status mk_linear_tc_split(int B, int K, int M, int *split);
  * context's prefilled cache can be shared).  mk_tcdec_step decodes one token
  * per sequence at position `pos` (all sequences share it): it writes K/V at
  * `pos`, attends to 0 .. pos, writes d_next (device int32 [batch]) and, if
- * d_logits is set, the fp32 logits [batch, vocab].  Asynchronous on `stream`;
- * an out-of-range token sets the status word (mk_tcdec_status, synchronous).
+ * d_logits is set, the fp32 logits [batch, vocab].  Asynchronous on `stream`.
+ * Device-side failures are ORed into a status word that mk_tcdec_status reads
+ * (synchronous; 0 = none): bit 0, a token outside [0, vocab) (its row decodes
+ * from zeros); bit 1, a sequence with no finite logit, which happens when a
+ * projection's bounded wait ran out and wrote NaN (d_next then holds 0 for
+ * it).  The word is cleared by mk_tcdec_bind only.
  * Errors: MK_ERR_INVALID, MK_ERR_UNSUPPORTED, MK_ERR_STATE (step before
- * bind), MK_ERR_CUDA; the reason is in mk_tcdec_last_error. */
+ * bind), MK_ERR_CUDA; the reason is in mk_tcdec_last_error.  A step that
+ * returns an error may have queued part of its work: the K/V rows at `pos`
+ * of some layers can already be written, so the cache at `pos` is undefined
+ * until a step at the same `pos` succeeds. */
 typedef struct mk_tcdec mk_tcdec;
 mk_status mk_tcdec_create(const mk_config *cfg, const mk_weights *w, mk_tcdec **out);
 mk_status mk_tcdec_workspace_bytes(const mk_tcdec *dec, size_t *bytes);

@@ -34,7 +34,8 @@ def check_argmax(nxt_gpu: np.ndarray, logits_gpu: np.ndarray, logits_ref: np.nda
     """(i) the GPU token is the exact argmax of the GPU's own logits (lowest
     index on ties); (ii) it equals the oracle's argmax wherever the oracle's
     top-1 / top-2 margin exceeds twice the observed logit error.  Returns the
-    number of rows where (ii) was not decidable."""
+    number of rows where (ii) was not decidable (appended to MK_PARITY_LOG,
+    when set, as an "undecided" line)."""
     undecided = 0
     for b in range(logits_ref.shape[0]):
         g = logits_gpu[b]
@@ -44,6 +45,11 @@ def check_argmax(nxt_gpu: np.ndarray, logits_gpu: np.ndarray, logits_ref: np.nda
             assert int(nxt_gpu[b]) == int(np.argmax(logits_ref[b]))
         else:
             undecided += 1
+    log = os.environ.get("MK_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(f"{os.environ.get('PYTEST_CURRENT_TEST', '?').split(' ')[0]}\tundecided\t{undecided}"
+                    f"/{logits_ref.shape[0]}\n")
     return undecided
 
 

@@ -66,6 +66,39 @@ def test_plans_validate_for_any_cta_count(n_ctas):
     assert p.info()["n_ctas"] == n_ctas
 
 
+SHUFFLE_CASES = [(synth.TINY, 3, 8), (synth.LLAMA1B, 1, 148), (synth.LLAMA8B, 8, 148), (synth.QWEN3_8B, 16, 148)]
+
+
+@pytest.mark.parametrize("shape,batch,n_ctas", SHUFFLE_CASES, ids=[f"{s.name}-b{b}-c{n}" for s, b, n in SHUFFLE_CASES])
+def test_shuffled_schedules_keep_every_instruction_and_validate(shape, batch, n_ctas):
+    """The race-detection substitute: a seeded reordering of the per-SM lists
+    that keeps each list in phase order.  It must keep every instruction
+    exactly once (the same multiset), keep each CTA's phases in order, move
+    the LM head's publishing flag to the last LM instruction of every CTA that
+    has one, pass the deadlock / count simulation, and differ from the
+    planner's order."""
+    import numpy as np
+    base = mkpy.Plan(shape, batch, shape.max_seq, num_sms=n_ctas)
+    ref, ref_base = base.schedule()
+    key = lambda a: np.sort(a[["op", "layer", "tile", "kb0", "b0"]], order=["op", "layer", "tile", "kb0", "b0"])  # noqa: E731
+    phase_rank = {1: 0, 2: 1, 7: 2, 3: 3, 4: 4, 5: 5, 6: 6}
+    for seed in (1, 2, 3):
+        p = mkpy.Plan(shape, batch, shape.max_seq, num_sms=n_ctas)
+        p.shuffle_schedule(seed)
+        p.validate()
+        got, got_base = p.schedule()
+        assert len(got) == len(ref) and np.array_equal(key(got), key(ref))
+        assert not np.array_equal(got[["op", "layer", "tile", "b0"]], ref[["op", "layer", "tile", "b0"]])
+        for c in range(n_ctas):
+            lst = got[got_base[c]:got_base[c + 1]]
+            order = [(int(i["layer"]) if i["op"] != 6 else 1 << 20, phase_rank[int(i["op"])]) for i in lst]
+            assert order == sorted(order), f"CTA {c} is out of phase order"
+            lm = np.flatnonzero(lst["op"] == 6)
+            if len(lm):
+                flags = lst["flags"][lm] & 2
+                assert flags[-1] == 2 and not flags[:-1].any()
+
+
 def _create(shape, batch=1, **kw):
     lib = _lib.load()
     cfg = mkpy.make_config(shape, batch, shape.max_seq, "megakernel", 148)

@@ -46,10 +46,12 @@ def test_tiny_trajectory_and_kv_indexing(sync):
     k, v = model.kv_views()
     k.view(torch.int16).fill_(-1)  # 0xFFFF: a NaN pattern in bf16
     v.view(torch.int16).fill_(-1)
+    model.poison_activations()  # NaN words under a tag no step writes
     tokens = synth.make_tokens(s, s.prefill + s.steps)
     worst, undecided = run_trajectory(model, orc, tokens, s.prefill, s.steps)
-    # near-tie steps (oracle top-2 margin within 2x the logit error) are counted, not failed
-    assert undecided <= s.steps // 2, (undecided, worst)
+    # near-tie steps (oracle top-2 margin within 2x the logit error) are counted,
+    # not failed; at most 1 of 32 has been seen, so an eighth is allowed
+    assert undecided <= s.steps // 8, (undecided, worst)
     p_final = s.prefill + s.steps
     assert model.position == p_final
     # every written slot matches the oracle's cache; every other slot keeps the poison bits
@@ -64,10 +66,13 @@ def test_tiny_trajectory_and_kv_indexing(sync):
 
 
 @needs_cuda
-@pytest.mark.parametrize("variant,sync", [("graph", "tags"), ("graph_pdl", "tags"), ("megakernel", "counters")])
+@pytest.mark.parametrize("variant,sync", [("graph", "tags"), ("graph_pdl", "tags"), ("megakernel", "counters"),
+                                          ("tilesync", "tags"), ("tilesync", "counters")])
 def test_variants_and_sync_modes_bit_equal(variant, sync):
-    """The separate-kernel variants, and the counter-synchronised megakernel,
-    produce the same bits as the tag-synchronised megakernel."""
+    """The separate-kernel variants (plain graph, graph + PDL, and the
+    tile-synchronised separate kernels in both sync modes), and the
+    counter-synchronised megakernel, produce the same bits as the
+    tag-synchronised megakernel."""
     s = synth.TINY
     tw = synth.make_weights(s, device="cuda")
     import tile_synchronised_b200 as mk
@@ -109,7 +114,41 @@ def test_tiny_shape_variants(case):
     tw, model, orc = build_pair(s, batch=batch)
     tokens = synth.make_tokens(s, 40, batch=batch)
     worst, undecided = run_trajectory(model, orc, tokens, 24, 16)
-    assert undecided <= 8 * batch, (undecided, worst)
+    # at most 3 of 16 steps per sequence have been near ties
+    assert undecided <= 6 * batch, (undecided, worst)
+
+
+@needs_cuda
+@pytest.mark.parametrize("sync", ["tags", "counters"])
+def test_shuffled_schedule_is_bit_equal(sync):
+    """Race-detection substitute: the same step under a seeded reordering of
+    the per-SM instruction lists (every dependency kept) gives the same bits
+    as the planner's order.  8 CTAs, so that every CTA holds several
+    instructions of each phase and the reordering changes which instruction
+    waits behind which."""
+    s = synth.TINY.replace(batch=3)
+    tw = synth.make_weights(s, device="cuda")
+    import tile_synchronised_b200 as mk
+    a = mk.Model(s, tw, batch=3, num_sms=8)
+    b = mk.Model(s, tw, batch=3, num_sms=8)
+    a.set_sync(sync)
+    b.set_sync(sync)
+    b.shuffle_schedule(7)
+    tokens = synth.make_tokens(s, 28, batch=3)
+    a.prefill(tokens[:, :20].cuda())
+    b.prefill(tokens[:, :20].cuda())
+    la = torch.empty((3, s.vocab), device="cuda")
+    lb = torch.empty((3, s.vocab), device="cuda")
+    for i in range(20, 28):
+        tok = tokens[:, i].contiguous().cuda()
+        na = a.decode(tok, logits=la).clone()
+        nb = b.decode(tok, logits=lb).clone()
+        assert torch.equal(la, lb), f"step {i}: max|delta| {(la - lb).abs().max().item()}"
+        assert torch.equal(na, nb)
+    assert a.status() == 0 and b.status() == 0
+    ka, va = a.kv_views()
+    kb, vb = b.kv_views()
+    assert torch.equal(ka[:, :, :, :28], kb[:, :, :, :28]) and torch.equal(va[:, :, :, :28], vb[:, :, :, :28])
 
 
 @needs_cuda
@@ -153,6 +192,38 @@ def test_wait_timeout_is_reported_and_context_recovers(sync):
     m.drop_signal(-1)
     m.reset()
     tokens = synth.make_tokens(s, 8)
+    m.prefill(tokens[:, :7].cuda())
+    lg = torch.empty((1, s.vocab), device="cuda")
+    m.decode(tokens[:, 7].contiguous().cuda(), logits=lg)
+    assert m.status() == 0
+    orc = oracle.OracleModel.from_torch(s, tw)
+    orc.prefill(tokens[:, :7].numpy())
+    ref, _ = orc.step(tokens[:, 7].numpy())
+    logits_close(lg.cpu().numpy(), ref)
+
+
+@needs_cuda
+@pytest.mark.parametrize("variant,bad", [("megakernel", "vocab"), ("megakernel", "negative"), ("graph", "vocab")])
+def test_out_of_range_token_is_reported_and_context_recovers(variant, bad):
+    """A token outside [0, vocab) is an invalid argument that lives in device
+    memory: the step records it, mk_get_status reports MK_ERR_INVALID with the
+    sequence and the token, the context refuses further steps until mk_reset,
+    and after the reset the same context decodes correctly again."""
+    s = synth.TINY
+    tw = synth.make_weights(s, device="cuda")
+    import tile_synchronised_b200 as mk
+    from tile_synchronised_b200 import _lib
+    m = mk.Model(s, tw, variant=variant)
+    tokens = synth.make_tokens(s, 8)
+    m.prefill(tokens[:, :6].cuda())
+    assert m.status() == 0
+    value = s.vocab if bad == "vocab" else -1
+    m.decode(torch.full((1,), value, dtype=torch.int32, device="cuda"))
+    assert m.status() == _lib.MK_ERR_INVALID
+    assert f"token {value} of sequence 0" in m.last_error()
+    with pytest.raises(mk.MkError):
+        m.decode(tokens[:, 6].contiguous().cuda())  # poisoned until reset
+    m.reset()
     m.prefill(tokens[:, :7].cuda())
     lg = torch.empty((1, s.vocab), device="cuda")
     m.decode(tokens[:, 7].contiguous().cuda(), logits=lg)
@@ -252,13 +323,33 @@ def full_size_case(shape, batch, prefill, extra_steps, seqs, max_seq=None):
 
 
 @needs_cuda
-def test_llama1b_full_size_handoff():
+def test_llama1b_handoffs_across_the_benched_window():
+    """The benched workload: a 1024-token prefill, then every step of the
+    decode window with oracle handoffs at its first, middle and last positions
+    (1025, 1152, 1279 of the 1280-slot cache) and sampled layer-0 cache rows."""
+    import tile_synchronised_b200 as mk
     s = synth.LLAMA1B
-    full_size_case(s, 1, s.prefill, 8, [0])
+    tw = synth.make_weights(s, device="cuda")
+    model = mk.Model(s, tw, batch=1, max_seq=s.max_seq)
+    tokens = synth.make_tokens(s, s.max_seq)
+    model.prefill(tokens[:, :s.prefill].cuda())
+    dev_tokens = tokens.to(dtype=torch.int32).cuda()
+    k, v = model.kv_views()
+    sampled_layer0_rows(s, tw, k, v, tokens.numpy(), 0, [0, 1, 511, s.prefill - 1])
+    host = host_weights(tw)
+    del tw
+    pos = s.prefill
+    for cp in (s.prefill + 1, s.prefill + 128, s.max_seq - 1):
+        while pos < cp:
+            model.decode(dev_tokens[:, pos].contiguous())
+            pos += 1
+        handoff_step(s, host, model, tokens, pos, [0])
+        pos += 1
+    assert model.position == s.max_seq
 
 
 @needs_cuda
-@pytest.mark.parametrize("batch,seqs", [(1, [0]), (8, [0, 7])])
+@pytest.mark.parametrize("batch,seqs", [(1, [0]), (8, [0, 7]), (32, [0, 31])])
 def test_llama8b_full_size_handoff(batch, seqs):
     s = synth.LLAMA8B
     full_size_case(s, batch, s.prefill, 4, seqs)
@@ -268,6 +359,30 @@ def test_llama8b_full_size_handoff(batch, seqs):
 def test_qwen3_8b_handoff_at_1k():
     s = synth.QWEN3_8B
     full_size_case(s, 16, 1024, 2, [0, 15], max_seq=1040)
+
+
+@needs_cuda
+@pytest.mark.parametrize("C", [4096, 16383])
+def test_qwen3_8b_full_depth_handoff_on_a_seeded_cache(C):
+    """Full depth (36 layers) at the long-generation checkpoints 4k and 16k.
+    Decoding there from a prefill takes minutes, so the cache positions below
+    C are filled with seeded N(0, 1) bf16 values instead; the step at C is a
+    plain function of whatever cache it reads, so the oracle, handed the same
+    cache, checks that step for the first and last sequence of the batch."""
+    import tile_synchronised_b200 as mk
+    s = synth.QWEN3_8B
+    B = 16
+    tw = synth.make_weights(s, device="cuda")
+    model = mk.Model(s, tw, batch=B, max_seq=C + 1)
+    host = host_weights(tw)
+    del tw
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    for t in model.kv_views():
+        t[:, :, :, :C].normal_(generator=g)
+    model.set_position(C)
+    tokens = synth.make_tokens(s, C + 1, batch=B)
+    handoff_step(s, host, model, tokens, C, [0, B - 1])
 
 
 @needs_cuda
@@ -295,6 +410,68 @@ def test_qwen3_8b_two_layer_clone_1k_to_16k():
         handoff_step(s, host, model, tokens, pos, [0, B - 1])
         pos += 1
     assert model.position == ms
+
+
+# ---------------------------------------------------------------- the in-step gate/up tilings
+@needs_cuda
+@pytest.mark.parametrize("batch", [3, 8])
+def test_row_tiled_gateup_trajectory(batch):
+    """The row tiling of the fused gate/up stage inside the step (every gate/up
+    instruction carries at most half of the batch rows, so each weight tile
+    streams once per row group) against the oracle, and bit-equal to the
+    column tiling on the same tokens."""
+    import tile_synchronised_b200 as mk
+    s = synth.TINY.replace(batch=batch)
+    tw, row, orc = build_pair(s, batch=batch)
+    row.set_swiglu_tiling(mk.MK_SWIGLU_ROW)
+    assert row.swiglu_tiling() == mk.MK_SWIGLU_ROW
+    sched, _ = row.schedule()
+    gu = sched[sched["op"] == 4]
+    assert int(gu["nb"].max()) == (min(batch, 4) + 1) // 2
+    col = mk.Model(s, tw, batch=batch)
+    assert col.swiglu_tiling() == mk.MK_SWIGLU_COL
+    tokens = synth.make_tokens(s, 40, batch=batch)
+    row.prefill(tokens[:, :24].cuda())
+    col.prefill(tokens[:, :24].cuda())
+    orc.prefill(tokens[:, :24].numpy())
+    lr = torch.empty((batch, s.vocab), device="cuda")
+    lc = torch.empty((batch, s.vocab), device="cuda")
+    undecided = 0
+    for i in range(24, 40):
+        tok = tokens[:, i].contiguous()
+        nr = row.decode(tok.cuda(), logits=lr).cpu().numpy()
+        col.decode(tok.cuda(), logits=lc)
+        assert torch.equal(lr, lc), f"step {i}: row and column tilings differ"
+        ref, _ = orc.step(tok.numpy())
+        g = lr.cpu().numpy()
+        undecided += check_argmax(nr, g, ref, logits_close(g, ref))
+    assert row.status() == 0 and col.status() == 0
+    assert undecided <= 16 * batch // 4, undecided
+
+
+@needs_cuda
+def test_tune_picks_a_tiling_and_decoding_stays_within_tolerance():
+    """The one-time profiling pass inside the step times both gate/up tilings,
+    keeps the faster and restores the position; decoding then continues
+    against the oracle."""
+    import tile_synchronised_b200 as mk
+    s = synth.TINY.replace(batch=8)
+    tw, model, orc = build_pair(s, batch=8)
+    tokens = synth.make_tokens(s, 40, batch=8)
+    model.prefill(tokens[:, :24].cuda())
+    orc.prefill(tokens[:, :24].numpy())
+    chosen = model.tune()
+    assert chosen in (mk.MK_SWIGLU_ROW, mk.MK_SWIGLU_COL)
+    assert model.swiglu_tiling() == chosen
+    assert model.position == 24
+    lg = torch.empty((8, s.vocab), device="cuda")
+    for i in range(24, 32):
+        tok = tokens[:, i].contiguous()
+        nxt = model.decode(tok.cuda(), logits=lg).cpu().numpy()
+        ref, _ = orc.step(tok.numpy())
+        g = lg.cpu().numpy()
+        check_argmax(nxt, g, ref, logits_close(g, ref))
+    assert model.status() == 0
 
 
 # ---------------------------------------------------------------- the fused SwiGLU first stage

@@ -1,11 +1,7 @@
 """The tensor-core batched decode step (mk_tcdec_*) against the oracle: the
 megakernel prefills the cache, the tensor-core step decodes the next token of
 every sequence on that cache, and the oracle, handed the same cache, checks
-that step's logits, argmax and appended K row.
-
-Not yet run on a GPU: set MK_RUN_TCDEC=1 to run these tests."""
-import os
-
+that step's logits, argmax and appended K row."""
 import numpy as np
 import pytest
 import torch
@@ -17,12 +13,9 @@ from gpu_common import check_argmax, host_weights, logits_close
 pytestmark = pytest.mark.gpu
 
 needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
-opt_in = pytest.mark.skipif(os.environ.get("MK_RUN_TCDEC") != "1",
-                            reason="tensor-core decode step not yet run on a GPU (MK_RUN_TCDEC=1 runs it)")
 
 
 @needs_cuda
-@opt_in
 @pytest.mark.parametrize("name,batch,prefill,seqs", [("llama8b", 8, 512, [0, 7]), ("qwen3_8b", 16, 1024, [0, 15]),
                                                      ("llama1b", 32, 256, [0, 31])])
 def test_tcdec_step_matches_oracle(name, batch, prefill, seqs):
@@ -57,7 +50,6 @@ def test_tcdec_step_matches_oracle(name, batch, prefill, seqs):
 
 
 @needs_cuda
-@opt_in
 def test_tcdec_refuses_a_position_past_the_cache():
     import tile_synchronised_b200 as mk
     s = synth.LLAMA1B.replace(n_layers=2)

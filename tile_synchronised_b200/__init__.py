@@ -10,13 +10,13 @@ import ctypes as C
 
 import torch
 
-from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW,
+from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_GRAPH_TILESYNC, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW,
                    MK_SWIGLU_TC, MK_SYNC_COUNTERS, MK_SYNC_TAGS, MkConfig, MkError, MkWeights, check, load)
 
 __all__ = ["Model", "TcDecoder", "swiglu_stage1", "swiglu_tune", "linear_tc", "linear_tc_split", "MkError", "VARIANTS",
            "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW", "MK_SWIGLU_COL", "MK_SWIGLU_TC", "load"]
 
-VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL}
+VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL, "tilesync": MK_GRAPH_TILESYNC}
 SYNCS = {"tags": MK_SYNC_TAGS, "counters": MK_SYNC_COUNTERS}
 SCHEDULE_FIELDS = ("n_instructions", "n_ctas", "n_counters", "n_phases", "batch_rows", "attention_chunks",
                    "ring_stages", "act_bytes", "swiglu_variant", "down_k_splits")
@@ -69,6 +69,10 @@ class Plan:
         check(self.lib.mk_get_schedule(self.ctx, C.c_void_p(arr.ctypes.data), arr.nbytes,
                                        C.c_void_p(base.ctypes.data)), self.ctx, "mk_get_schedule")
         return arr, base
+
+    def shuffle_schedule(self, seed: int) -> None:
+        """Reorder the schedule with a seeded dependency-preserving permutation (test hook)."""
+        check(self.lib.mk_debug_shuffle_schedule(self.ctx, int(seed)), self.ctx, "mk_debug_shuffle_schedule")
 
     def validate(self) -> None:
         check(self.lib.mk_validate_schedule(self.ctx), self.ctx, "mk_validate_schedule")
@@ -194,10 +198,25 @@ class Model(Plan):
     def drop_signal(self, instr: int) -> None:
         check(self.lib.mk_debug_drop_signal(self.ctx, int(instr)), self.ctx, "mk_debug_drop_signal")
 
+    def poison_activations(self, stream=None) -> None:
+        """Fill the buffers instructions hand to each other with NaN words under an unused tag (test hook)."""
+        check(self.lib.mk_debug_poison_activations(self.ctx, _stream(stream)), self.ctx,
+              "mk_debug_poison_activations")
+
     def tune(self, stream=None) -> int:
         ch = C.c_int()
         check(self.lib.mk_tune(self.ctx, _stream(stream), C.byref(ch)), self.ctx, "mk_tune")
         return ch.value
+
+    def set_swiglu_tiling(self, variant: int, stream=None) -> None:
+        """Pick the gate/up tiling (MK_SWIGLU_ROW or MK_SWIGLU_COL) without timing."""
+        check(self.lib.mk_set_swiglu_tiling(self.ctx, int(variant), _stream(stream)), self.ctx,
+              "mk_set_swiglu_tiling")
+
+    def swiglu_tiling(self) -> int:
+        v = C.c_int()
+        check(self.lib.mk_get_swiglu_tiling(self.ctx, C.byref(v)), self.ctx, "mk_get_swiglu_tiling")
+        return v.value
 
     def last_error(self) -> str:
         return self.lib.mk_last_error(self.ctx).decode()

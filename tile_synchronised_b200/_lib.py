@@ -12,7 +12,7 @@ from . import build as _build
 
 MK_OK, MK_ERR_INVALID, MK_ERR_CUDA, MK_ERR_TIMEOUT, MK_ERR_UNSUPPORTED, MK_ERR_STATE = 0, -1, -2, -3, -4, -5
 MK_BF16 = 0
-MK_MEGAKERNEL, MK_GRAPH, MK_GRAPH_PDL = 0, 1, 2
+MK_MEGAKERNEL, MK_GRAPH, MK_GRAPH_PDL, MK_GRAPH_TILESYNC = 0, 1, 2, 3
 MK_SWIGLU_AUTO, MK_SWIGLU_ROW, MK_SWIGLU_COL, MK_SWIGLU_TC = 0, 1, 2, 3
 MK_SYNC_TAGS, MK_SYNC_COUNTERS = 0, 1
 
@@ -22,8 +22,10 @@ STATUS_NAMES = {0: "MK_OK", -1: "MK_ERR_INVALID", -2: "MK_ERR_CUDA", -3: "MK_ERR
 # Every symbol include/mk.h declares.
 EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk_kv_cache_bytes",
            "mk_load_weights", "mk_prefill_kv", "mk_decode_step", "mk_get_status", "mk_reset",
-           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_prefetch",
-           "mk_set_timeout_ns", "mk_set_sync", "mk_set_ring_stages", "mk_debug_drop_signal", "mk_set_trace",
+           "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_swiglu_tiling",
+           "mk_get_swiglu_tiling", "mk_set_prefetch",
+           "mk_set_timeout_ns", "mk_set_sync", "mk_set_ring_stages", "mk_debug_drop_signal",
+           "mk_debug_shuffle_schedule", "mk_debug_poison_activations", "mk_set_trace",
            "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1",
            "mk_swiglu_tune", "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks",
            "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes", "mk_linear_tc",
@@ -86,11 +88,15 @@ def load() -> C.CDLL:
         "mk_set_position": ([vp, i32, vp], st),
         "mk_set_variant": ([vp, i32], st),
         "mk_tune": ([vp, vp, C.POINTER(i32)], st),
+        "mk_set_swiglu_tiling": ([vp, i32, vp], st),
+        "mk_get_swiglu_tiling": ([vp, C.POINTER(i32)], st),
         "mk_set_prefetch": ([vp, i32], st),
         "mk_set_timeout_ns": ([vp, C.c_ulonglong], st),
         "mk_set_sync": ([vp, i32], st),
         "mk_set_ring_stages": ([vp, i32], st),
         "mk_debug_drop_signal": ([vp, i32], st),
+        "mk_debug_shuffle_schedule": ([vp, C.c_ulonglong], st),
+        "mk_debug_poison_activations": ([vp, vp], st),
         "mk_set_trace": ([vp, vp, sz], st),
         "mk_get_schedule": ([vp, vp, sz, vp], st),
         "mk_schedule_info": ([vp, C.POINTER(C.c_longlong), i32], st),

@@ -389,26 +389,31 @@ static mk_status launch_megakernel(mk_ctx *c, const int32_t *tok, int64_t stride
     return MK_OK;
 }
 
-// The separate-kernels variant: one launch of the same interpreter per phase,
-// no counter waits (the kernel boundary orders the phases).
-static KParams phase_params(mk_ctx *c, int k, const int32_t *tok, int32_t *next, float *logits, bool pdl) {
+// The separate-kernels variants: one launch of the same interpreter per
+// phase.  MK_GRAPH and MK_GRAPH_PDL wait for the whole previous kernel (its
+// end, or griddepcontrol.wait); MK_GRAPH_TILESYNC lets every kernel but the
+// first launch early (its CTAs trigger their dependents as they start) and
+// start on the tiles it reads, like the megakernel's instructions.
+static KParams phase_params(mk_ctx *c, int k, const int32_t *tok, int32_t *next, float *logits, int variant) {
     KParams P = make_params(c, tok, 1, next, logits);
     const Plan &p = c->plan;
     const int32_t *ranges = reinterpret_cast<const int32_t *>(c->ws + p.off_ranges);
-    P.use_waits = 0;
-    P.use_signals = 0;
+    const bool tiles = variant == MK_GRAPH_TILESYNC;
+    P.use_waits = tiles && c->sync == MK_SYNC_COUNTERS ? 1 : 0;
+    P.use_signals = P.use_waits;
     P.cta_begin = ranges + (size_t)(2 + k) * p.n_ctas;
     P.cta_end = ranges + (size_t)(3 + k) * p.n_ctas;
-    P.pdl = (pdl && k > 0) ? 1 : 0;
+    P.pdl = tiles ? 2 : ((variant == MK_GRAPH_PDL && k > 0) ? 1 : 0);
     return P;
 }
 
 static mk_status launch_phases(mk_ctx *c, const int32_t *tok, int32_t *next, float *logits, cudaStream_t s,
-                               bool pdl, std::vector<cudaGraphNode_t> *nodes) {
+                               int variant, std::vector<cudaGraphNode_t> *nodes) {
     const Plan &p = c->plan;
+    const bool early = variant == MK_GRAPH_PDL || variant == MK_GRAPH_TILESYNC;
     for (int k = 0; k < p.n_phases; ++k) {
-        KParams P = phase_params(c, k, tok, next, logits, pdl);
-        CK(launch_step(P, p.bs, p.n_ctas, s, false, pdl && k > 0));
+        KParams P = phase_params(c, k, tok, next, logits, variant);
+        CK(launch_step(P, p.bs, p.n_ctas, s, false, early && k > 0));
         if (nodes) {
             cudaStreamCaptureStatus cs;
             const cudaGraphNode_t *deps = nullptr;
@@ -425,10 +430,10 @@ static mk_status launch_phases(mk_ctx *c, const int32_t *tok, int32_t *next, flo
 // that read the tokens (layer-0 QKV and O-projection) or write the outputs (LM
 // head) are patched, so a new pointer costs three node updates, not a
 // re-capture.
-static mk_status retarget_graph(mk_ctx *c, const int32_t *tok, int32_t *next, float *logits, bool pdl) {
+static mk_status retarget_graph(mk_ctx *c, const int32_t *tok, int32_t *next, float *logits, int variant) {
     const Plan &p = c->plan;
     for (int k : p.token_phases) {
-        KParams P = phase_params(c, k, tok, next, logits, pdl);
+        KParams P = phase_params(c, k, tok, next, logits, variant);
         void *args[1] = {&P};
         cudaKernelNodeParams np = {};
         np.func = const_cast<void *>(step_kernel_func(P));
@@ -455,7 +460,6 @@ mk_status mk_decode_step(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, fl
     if (c->variant == MK_MEGAKERNEL) {
         st = launch_megakernel(c, d_tokens, 1, d_next, d_logits, s);
     } else {
-        const bool pdl = c->variant == MK_GRAPH_PDL;
         if (!c->gexec || c->g_variant != c->variant) {
             drop_graph(c);
             cudaStream_t cap;
@@ -465,7 +469,7 @@ mk_status mk_decode_step(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, fl
                 cudaStreamDestroy(cap);
                 return cuda_fail(c, e, "cudaStreamBeginCapture");
             }
-            st = launch_phases(c, d_tokens, d_next, d_logits, cap, pdl, &c->gnodes);
+            st = launch_phases(c, d_tokens, d_next, d_logits, cap, c->variant, &c->gnodes);
             cudaGraph_t graph = nullptr;
             e = cudaStreamEndCapture(cap, &graph);
             cudaStreamDestroy(cap);
@@ -486,7 +490,7 @@ mk_status mk_decode_step(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, fl
             c->g_logits = d_logits;
             c->g_variant = c->variant;
         } else if (c->g_tok != d_tokens || c->g_next != d_next || c->g_logits != d_logits) {
-            st = retarget_graph(c, d_tokens, d_next, d_logits, pdl);
+            st = retarget_graph(c, d_tokens, d_next, d_logits, c->variant);
             if (st != MK_OK) return st;
         }
         CK(cudaGraphLaunch(c->gexec, s));
@@ -529,6 +533,14 @@ mk_status mk_get_status(mk_ctx *c, void *stream) {
         c->err = buf;
         return MK_ERR_TIMEOUT;
     }
+    if (st.tok_err) {
+        c->poisoned = true;
+        char buf[200];
+        snprintf(buf, sizeof buf, "token %d of sequence %u is outside [0, %d): the step decoded token 0 in its place",
+                 st.tok_bad, st.tok_err - 1u, c->plan.cfg.vocab);
+        c->err = buf;
+        return MK_ERR_INVALID;
+    }
     return MK_OK;
 }
 
@@ -560,7 +572,7 @@ mk_status mk_set_position(mk_ctx *c, int pos, void *stream) {
 
 mk_status mk_set_variant(mk_ctx *c, int variant) {
     if (!c) return MK_ERR_INVALID;
-    if (variant < MK_MEGAKERNEL || variant > MK_GRAPH_PDL) return fail(c, MK_ERR_INVALID, "unknown variant");
+    if (variant < MK_MEGAKERNEL || variant > MK_GRAPH_TILESYNC) return fail(c, MK_ERR_INVALID, "unknown variant");
     c->variant = variant;
     return MK_OK;
 }
@@ -583,6 +595,7 @@ mk_status mk_set_ring_stages(mk_ctx *c, int stages) {
 mk_status mk_set_sync(mk_ctx *c, int mode) {
     if (!c) return MK_ERR_INVALID;
     if (mode != MK_SYNC_TAGS && mode != MK_SYNC_COUNTERS) return fail(c, MK_ERR_INVALID, "unknown sync mode");
+    if (mode != c->sync) drop_graph(c);  // the tile-synchronised graph captured the old waits
     c->sync = mode;
     return MK_OK;
 }
@@ -605,6 +618,28 @@ mk_status mk_debug_drop_signal(mk_ctx *c, int instr) {
     return MK_OK;
 }
 
+mk_status mk_debug_poison_activations(mk_ctx *c, void *stream) {
+    if (!c) return MK_ERR_INVALID;
+    if (!c->loaded) return fail(c, MK_ERR_STATE, "mk_debug_poison_activations before mk_load_weights");
+    const Plan &p = c->plan;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CK(cudaMemsetAsync(c->ws + p.off_x, 0xFF, p.off_lm_best - p.off_x, s));
+    CK(cudaMemsetAsync(c->ws + p.off_lm_best, 0xFF, (size_t)p.B * p.n_ctas * sizeof(LmBest), s));
+    CK(cudaStreamSynchronize(s));
+    return MK_OK;
+}
+
+mk_status mk_debug_shuffle_schedule(mk_ctx *c, unsigned long long seed) {
+    if (!c) return MK_ERR_INVALID;
+    mk_status st = shuffle_plan(c->plan, seed, c->err);
+    if (st != MK_OK) return st;
+    if (c->loaded) {
+        drop_graph(c);
+        return upload_schedule(c, nullptr);
+    }
+    return MK_OK;
+}
+
 // Swap the active gate/up tiling (same layout); counters restart.
 static mk_status switch_plan(mk_ctx *c, cudaStream_t s) {
     std::swap(c->plan, c->plan_alt);
@@ -618,6 +653,22 @@ static mk_status switch_plan(mk_ctx *c, cudaStream_t s) {
     CK(cudaMemsetAsync(c->ws + p.off_counters, 0, (size_t)p.n_counters * 4, s));
     CK(cudaMemcpyAsync(c->ws + p.off_state + offsetof(State, pos), &pos, 4, cudaMemcpyHostToDevice, s));
     CK(cudaStreamSynchronize(s));
+    return MK_OK;
+}
+
+mk_status mk_set_swiglu_tiling(mk_ctx *c, int variant, void *stream) {
+    if (!c) return MK_ERR_INVALID;
+    if (variant != MK_SWIGLU_ROW && variant != MK_SWIGLU_COL)
+        return fail(c, MK_ERR_INVALID, "mk_set_swiglu_tiling: MK_SWIGLU_ROW or MK_SWIGLU_COL");
+    if (!c->loaded) return fail(c, MK_ERR_STATE, "mk_set_swiglu_tiling before mk_load_weights");
+    if (c->poisoned) return fail(c, MK_ERR_STATE, "context poisoned by a device error; call mk_reset");
+    if (c->plan.swiglu_variant == variant) return MK_OK;
+    return switch_plan(c, static_cast<cudaStream_t>(stream));
+}
+
+mk_status mk_get_swiglu_tiling(const mk_ctx *c, int *variant) {
+    if (!c || !variant) return MK_ERR_INVALID;
+    *variant = c->plan.swiglu_variant;
     return MK_OK;
 }
 

@@ -110,7 +110,8 @@ struct State {
     uint32_t err_cta;
     uint32_t err_instr;
     uint32_t err_ctr;
-    uint32_t pad[2];
+    uint32_t tok_err;  // 0, or 1 + the first sequence whose token was outside [0, vocab)
+    int32_t tok_bad;   // that token
 };
 
 struct LmBest {
@@ -155,7 +156,7 @@ struct KParams {
     int32_t qkv_rt, o_rt, gu_rt, down_rt, lm_rt;  // rows per tile
     int32_t use_waits;          // 1: acquire-spin on the tile-ready counters before each instruction
     int32_t use_signals;        // 1: release-increment the counters after each instruction
-    int32_t pdl;                // 1: wait on the previous grid before reading activations
+    int32_t pdl;                // 1: trigger dependents, wait on the previous grid; 2: trigger only
     unsigned long long *trace;  // [n_instr][8] globaltimer stamps and waits, or null
     int32_t prefetch;           // ring blocks the L2 prefetch cursor runs ahead of the TMA loads
     double rope_inv_freq[64];   // theta^(-2i/d), i < d/2

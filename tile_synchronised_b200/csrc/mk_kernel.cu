@@ -130,9 +130,15 @@ __device__ bool wait_bar(const KParams &P, uint64_t *bar, uint32_t parity, volat
     }
 }
 
+// The token of sequence b.  One outside [0, vocab) is recorded in the step
+// state (the first such sequence and its value, reported by mk_get_status as
+// an invalid argument) and replaced by 0 so that every read stays inside the
+// embedding table; the step still runs to the end, so no wait is cut short.
 __device__ __forceinline__ int token_of(const KParams &P, int b) {
-    int t = P.tokens[(int64_t)b * P.tok_stride];
-    return min(max(t, 0), P.vocab - 1);
+    const int t = P.tokens[(int64_t)b * P.tok_stride];
+    if (t >= 0 && t < P.vocab) return t;
+    if (atomicCAS(&P.state->tok_err, 0u, (uint32_t)b + 1u) == 0u) P.state->tok_bad = t;
+    return 0;
 }
 
 struct MatRef {
@@ -1307,7 +1313,7 @@ __device__ void consumer(const KParams &P, const SmemLayout &S, int begin, int e
     uint32_t sat_ctr = 0xFFFFFFFFu, sat_target = 0u;
     uint32_t pend_ctr = kNoCounter, pend_n = 0u;
     bool stop = false;
-    if (P.pdl) pdl_wait();
+    if (P.pdl == 1) pdl_wait();  // 2: start on the tiles read, not on the previous kernel's end
     consumer_sync();
     // instructions are fetched three ahead: an L2 round trip is longer than
     // one instruction's work, and L1 is nearly all given to shared memory

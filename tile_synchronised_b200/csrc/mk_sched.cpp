@@ -68,7 +68,7 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     if (c.batch > 64) return bad(MK_ERR_UNSUPPORTED, "batch above 64");
     if (c.max_seq > (1 << 20)) return bad(MK_ERR_UNSUPPORTED, "max_seq above 2^20");
     if (n_ctas > 1024) return bad(MK_ERR_UNSUPPORTED, "more than 1024 CTAs");
-    if (c.variant < MK_MEGAKERNEL || c.variant > MK_GRAPH_PDL) return bad(MK_ERR_INVALID, "unknown variant");
+    if (c.variant < MK_MEGAKERNEL || c.variant > MK_GRAPH_TILESYNC) return bad(MK_ERR_INVALID, "unknown variant");
 
     const int L = c.n_layers, H = c.hidden, nq = c.n_heads, nkv = c.n_kv_heads, d = c.head_dim;
     const int I = c.intermediate, V = c.vocab, B = c.batch;
@@ -415,6 +415,61 @@ mk_status validate_plan(const Plan &p, std::string &err) {
         }
     }
     return MK_OK;
+}
+
+// A randomised schedule that keeps every dependency: for each phase, the
+// groups of instructions the CTAs hold are dealt out to the CTAs in a random
+// order, and each group is shuffled.  A CTA's list stays in phase order, so
+// the schedule stays deadlock-free; each instruction computes the same values
+// wherever it runs (a GEMV tile is one warp's fixed-order dot products, the
+// K ranges of the down projection are added in a fixed order, and the argmax
+// keys are order-free), so the results must be bit-identical.  A dependency
+// the plan forgot to express -- a consumer that reads data its wait does not
+// cover -- would show up here as a different result or a timeout.  The LM
+// head's "last instruction of the CTA" flag moves with the shuffle.
+mk_status shuffle_plan(Plan &p, uint64_t seed, std::string &err) {
+    uint64_t st = seed * 0x9E3779B97F4A7C15ull + 0x632BE59BD9B4E019ull;
+    auto next = [&]() {  // splitmix64
+        uint64_t z = (st += 0x9E3779B97F4A7C15ull);
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+        return z ^ (z >> 31);
+    };
+    auto shuffle = [&](auto &v) {
+        for (size_t i = v.size(); i > 1; --i) std::swap(v[i - 1], v[next() % i]);
+    };
+    const int n = p.n_ctas, np = p.n_phases;
+    std::vector<std::vector<std::vector<Instr>>> per(n, std::vector<std::vector<Instr>>(np));
+    for (int ph = 0; ph < np; ++ph)
+        for (int i = 0; i < n; ++i)
+            for (int32_t k = p.phase_begin[(size_t)ph * n + i]; k < p.phase_begin[(size_t)(ph + 1) * n + i]; ++k)
+                per[i][ph].push_back(p.instrs[k]);
+    std::vector<std::vector<std::vector<Instr>>> out(n, std::vector<std::vector<Instr>>(np));
+    std::vector<int> to(n);
+    for (int ph = 0; ph < np; ++ph) {
+        for (int i = 0; i < n; ++i) to[i] = i;
+        shuffle(to);
+        for (int i = 0; i < n; ++i) {
+            out[to[i]][ph] = per[i][ph];
+            shuffle(out[to[i]][ph]);
+        }
+    }
+    const int lm = np - 1;
+    for (int i = 0; i < n; ++i) {
+        for (auto &in : out[i][lm]) in.flags &= (uint8_t)~F_LAST_LM;
+        if (!out[i][lm].empty()) out[i][lm].back().flags |= F_LAST_LM;
+    }
+    p.instrs.clear();
+    for (int i = 0; i < n; ++i) {
+        p.cta_base[i] = (int32_t)p.instrs.size();
+        for (int ph = 0; ph < np; ++ph) {
+            p.phase_begin[(size_t)ph * n + i] = (int32_t)p.instrs.size();
+            for (auto &in : out[i][ph]) p.instrs.push_back(in);
+        }
+        p.phase_begin[(size_t)np * n + i] = (int32_t)p.instrs.size();
+    }
+    p.cta_base[n] = (int32_t)p.instrs.size();
+    return validate_plan(p, err);
 }
 
 }  // namespace mk

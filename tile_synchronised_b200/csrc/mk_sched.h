@@ -47,6 +47,9 @@ struct Plan {
 mk_status build_plan(const mk_config &cfg, int n_ctas, int swiglu_variant, Plan &plan, std::string &err);
 // Simulate the schedule on the host; MK_OK or MK_ERR_STATE with a reason.
 mk_status validate_plan(const Plan &plan, std::string &err);
+// Reorder the schedule without changing what any instruction computes (a
+// test of the dependency edges); then validate it.
+mk_status shuffle_plan(Plan &plan, uint64_t seed, std::string &err);
 
 // Tile-ready counters, six per layer, then the LM-head arrival counter.
 constexpr int kCountersPerLayer = 6;
