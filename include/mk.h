@@ -149,9 +149,24 @@ mk_status mk_kv_cache_bytes(const mk_ctx *ctx, size_t *bytes);
 mk_status mk_load_weights(mk_ctx *ctx, const mk_weights *w, void *workspace, void *kv_cache, void *stream);
 
 /* Fill the KV cache from a prompt: `d_tokens` is a device int32 [batch, T]
- * row-major array; positions restart at 0 and end at T.  Runs T decode steps
- * whose outputs are discarded.  MK_ERR_INVALID if T < 1 or T > max_seq. */
+ * row-major array; positions restart at 0 and end at T.  With the tensor-core
+ * prefill (the default where the plan allows it, see mk_set_prefill) the
+ * prompt goes through the decoder 32 positions of one sequence at a time:
+ * every projection is one tcgen05 GEMM over the packed weights, with each
+ * activation row entering as a hi/lo pair of bf16 rows, and position t
+ * attends causally to positions 0 .. t; only the KV cache is kept (the last
+ * layer stops after its K/V rows).  Otherwise it runs T decode steps whose
+ * outputs are discarded.  A token outside [0, vocab) is reported by
+ * mk_get_status as for mk_decode_step.  MK_ERR_INVALID if T < 1 or
+ * T > max_seq. */
 mk_status mk_prefill_kv(mk_ctx *ctx, const int32_t *d_tokens, int batch, int T, void *stream);
+/* How mk_prefill_kv runs: MK_PREFILL_AUTO (default: the tensor cores when every
+ * packed layer matrix is a single K block, i.e. the plan does not split a
+ * projection's K to fit its activations in shared memory; else decode steps),
+ * MK_PREFILL_STEPS (one decode step per position) or MK_PREFILL_TC
+ * (MK_ERR_UNSUPPORTED when the plan does not allow it).  Host only. */
+enum { MK_PREFILL_AUTO = 0, MK_PREFILL_STEPS = 1, MK_PREFILL_TC = 2 };
+mk_status mk_set_prefill(mk_ctx *ctx, int mode);
 
 /* One decode step at the current position p: `d_tokens` is a device int32
  * [batch]; the K/V rows of those tokens are written at position p, every
@@ -364,6 +379,16 @@ mk_status mk_tcdec_step(mk_tcdec *dec, const int32_t *d_tokens, int pos, int32_t
 mk_status mk_tcdec_status(mk_tcdec *dec, int *status, void *stream);
 const char *mk_tcdec_last_error(const mk_tcdec *dec);
 mk_status mk_tcdec_destroy(mk_tcdec *dec);
+/* Replay the step from a CUDA graph (on = 1, the default) or launch its
+ * ~16-per-layer kernels one by one (on = 0).  Every kernel of the step reads
+ * the position and the tokens from the workspace, so the first step runs
+ * eagerly and the next one captures the whole step once (once more the first
+ * time logits are asked for, or not) into a graph that every later step
+ * replays: mk_tcdec_step then queues a 4-byte-per-sequence token copy, a
+ * one-thread position write, the graph launch and the output copies.  The
+ * results are bit-identical either way (the split-KV chunk count is fixed by
+ * max_seq in both).  Rebinding drops the captured graphs.  Host only. */
+mk_status mk_tcdec_set_graph(mk_tcdec *dec, int on);
 
 /* Split-KV decode attention with a log-sum-exp combine, on its own: the
  * attention of one layer of one decode step ("Look Ma, No Bubbles! Designing

@@ -218,11 +218,12 @@ def test_tcdec_host_checks_need_no_device():
     assert lib.mk_tcdec_create(C.byref(cfg), C.byref(w), C.byref(dec)) == _lib.MK_OK
     n = C.c_size_t()
     assert lib.mk_tcdec_workspace_bytes(dec, C.byref(n)) == _lib.MK_OK
-    # x, hi/lo rows, the projection outputs (hi and lo rows each), q, attention out, scratch for 64 chunks
+    # x, hi/lo rows, the projection outputs (hi and lo rows each), q, attention out, scratch for 64 chunks,
+    # then the step's own token, argmax, position and logits buffers
     B, H, I, V, QD, KD = 8, s.hidden, s.intermediate, s.vocab, s.n_heads * s.head_dim, s.n_kv_heads * s.head_dim
     floor = 4 * B * H + 2 * 2 * B * max(H, QD, I) + 4 * 2 * B * (QD + 2 * KD + H + 2 * I + V) + 2 * 4 * B * QD \
-        + lib.mk_attention_scratch_bytes(B, s.n_heads, s.head_dim, 64)
-    assert floor <= n.value <= floor + 14 * 256
+        + lib.mk_attention_scratch_bytes(B, s.n_heads, s.head_dim, 64) + 4 * B + 4 * B + 8 + 4 * B * V
+    assert floor <= n.value <= floor + 18 * 256
     # a step before bind, and a bind with a misaligned workspace, are refused
     d = C.c_void_p(4096)
     assert lib.mk_tcdec_step(dec, d, 0, d, None, None) == _lib.MK_ERR_STATE

@@ -493,3 +493,56 @@ def test_swiglu_stage1_full_size(B):
     chosen, us_row, us_col, us_tc = mk.swiglu_tune(x, wg, wu, out)
     assert chosen in (mk.MK_SWIGLU_ROW, mk.MK_SWIGLU_COL, mk.MK_SWIGLU_TC)
     assert us_row > 0 and us_col > 0 and us_tc > 0
+
+
+# ---------------------------------------------------------------- the prefill on the tensor cores
+@needs_cuda
+@pytest.mark.parametrize("case", ["tiny_b1", "tiny_b3_qknorm", "llama1b"])
+def test_tensor_core_prefill_matches_steps_and_oracle(case):
+    """The tensor-core prefill (32 positions of a sequence per GEMM chunk,
+    causal attention within the chunk) leaves a KV cache that agrees with the
+    one the decode steps leave and with the oracle's, and the decode step that
+    follows it matches the oracle.  The prompt lengths cover one ragged chunk
+    and several chunks with a ragged tail."""
+    import tile_synchronised_b200 as mk
+    from tile_synchronised_b200 import _lib
+    if case == "llama1b":
+        s, B, T = synth.LLAMA1B, 1, 100
+    elif case == "tiny_b1":
+        s, B, T = synth.TINY, 1, 21
+    else:
+        s, B, T = synth.TINY.replace(qk_norm=True, rms_eps=1e-6), 3, 70
+    ms = T + 4
+    tw = synth.make_weights(s, device="cuda")
+    tokens = synth.make_tokens(s, T + 1, batch=B)
+    tc = mk.Model(s, tw, batch=B, max_seq=ms)
+    tc.set_prefill("tc")
+    steps = mk.Model(s, tw, batch=B, max_seq=ms)
+    steps.set_prefill("steps")
+    for m in (tc, steps):
+        m.prefill(tokens[:, :T].cuda())
+        assert m.position == T
+    assert tc.status() == 0 and steps.status() == 0
+    orc = oracle.OracleModel.from_torch(s, tw, batch=B, max_seq=ms)
+    orc.prefill(tokens[:, :T].numpy())
+    (kt, vt), (ks, vs) = tc.kv_views(), steps.kv_views()
+    for got, other, ref in ((kt, ks, orc.kc), (vt, vs, orc.vc)):
+        g = widen_bf16(got[:, :, :, :T])
+        o = widen_bf16(other[:, :, :, :T])
+        for l in range(s.n_layers):
+            scale = np.max(np.abs(ref[l, :, :, :T]))
+            assert np.max(np.abs(g[l] - ref[l, :, :, :T])) <= 2e-2 * scale, l
+            assert np.max(np.abs(g[l] - o[l])) <= 2e-2 * scale, l
+    lg = torch.empty((B, s.vocab), device="cuda")
+    nxt = tc.decode(tokens[:, T].contiguous().cuda(), logits=lg).cpu().numpy()
+    ref, _ = orc.step(tokens[:, T].numpy())
+    g = lg.cpu().numpy()
+    check_argmax(nxt, g, ref, logits_close(g, ref))
+    assert tc.status() == 0
+    # a token outside the vocabulary in the prompt is reported like a decode step's
+    bad = tokens[:, :T].clone()
+    bad[B - 1, T // 2] = s.vocab
+    tc.reset()
+    tc.prefill(bad.cuda())
+    assert tc.status() == _lib.MK_ERR_INVALID
+    assert f"sequence {B - 1}" in tc.last_error()

@@ -58,3 +58,34 @@ def test_tcdec_refuses_a_position_past_the_cache():
     tok = torch.zeros(2, dtype=torch.int32, device="cuda")
     with pytest.raises(mk.MkError):
         dec.step(tok, 8)
+
+
+@needs_cuda
+def test_tcdec_graph_replay_is_bit_equal_to_eager_launches():
+    """The step captured once in a CUDA graph replays at every position: a run
+    of consecutive steps through the graph gives the same bits (logits,
+    tokens, the K/V rows appended) as the same steps launched kernel by
+    kernel, on fresh caches."""
+    import tile_synchronised_b200 as mk
+    s = synth.LLAMA1B.replace(n_layers=2)
+    B, ms, n = 4, 64, 12
+    tw = synth.make_weights(s, device="cuda")
+    tokens = synth.make_tokens(s, n, batch=B).to(torch.int32).cuda()
+    runs = {}
+    for graph in (False, True):
+        dec = mk.TcDecoder(s, tw, B, ms)
+        dec.set_graph(graph)
+        lg = torch.empty((B, s.vocab), dtype=torch.float32, device="cuda")
+        steps = []
+        for p in range(n):
+            nxt = dec.step(tokens[:, p].contiguous(), p, logits=lg if p % 3 else None)
+            steps.append((lg.clone() if p % 3 else None, nxt.clone()))
+        torch.cuda.synchronize()
+        assert dec.status() == 0
+        runs[graph] = (steps, dec.kv.clone())
+        dec.close()
+    for p, ((la, na), (lb, nb)) in enumerate(zip(runs[False][0], runs[True][0])):
+        assert torch.equal(na, nb), p
+        if la is not None:
+            assert torch.equal(la, lb), p
+    assert torch.equal(runs[False][1], runs[True][1])

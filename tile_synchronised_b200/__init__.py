@@ -18,6 +18,7 @@ __all__ = ["Model", "TcDecoder", "swiglu_stage1", "swiglu_tune", "linear_tc", "l
 
 VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL, "tilesync": MK_GRAPH_TILESYNC}
 SYNCS = {"tags": MK_SYNC_TAGS, "counters": MK_SYNC_COUNTERS}
+PREFILLS = {"auto": 0, "steps": 1, "tc": 2}
 SCHEDULE_FIELDS = ("n_instructions", "n_ctas", "n_counters", "n_phases", "batch_rows", "attention_chunks",
                    "ring_stages", "act_bytes", "swiglu_variant", "down_k_splits")
 
@@ -160,6 +161,10 @@ class Model(Plan):
         assert t.dim() == 2 and t.shape[0] == self.batch
         check(self.lib.mk_prefill_kv(self.ctx, C.c_void_p(t.data_ptr()), self.batch, t.shape[1], _stream(stream)),
               self.ctx, "mk_prefill_kv")
+
+    def set_prefill(self, mode: str) -> None:
+        """How prefill runs: "auto" (tensor cores where the plan allows), "steps" or "tc"."""
+        check(self.lib.mk_set_prefill(self.ctx, PREFILLS[mode]), self.ctx, "mk_set_prefill")
 
     def decode(self, tokens: torch.Tensor, logits: torch.Tensor | None = None, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
@@ -316,6 +321,10 @@ class TcDecoder:
         self._check(self.lib.mk_tcdec_step(self.dec, C.c_void_p(tokens.data_ptr()), int(pos),
                                            C.c_void_p(nxt.data_ptr()), lp, _stream(stream)), "mk_tcdec_step")
         return nxt
+
+    def set_graph(self, on: bool) -> None:
+        """Replay the step from a CUDA graph (default) or launch its kernels one by one."""
+        self._check(self.lib.mk_tcdec_set_graph(self.dec, int(bool(on))), "mk_tcdec_set_graph")
 
     def status(self, stream=None) -> int:
         v = C.c_int()

@@ -15,13 +15,14 @@ MK_BF16 = 0
 MK_MEGAKERNEL, MK_GRAPH, MK_GRAPH_PDL, MK_GRAPH_TILESYNC = 0, 1, 2, 3
 MK_SWIGLU_AUTO, MK_SWIGLU_ROW, MK_SWIGLU_COL, MK_SWIGLU_TC = 0, 1, 2, 3
 MK_SYNC_TAGS, MK_SYNC_COUNTERS = 0, 1
+MK_PREFILL_AUTO, MK_PREFILL_STEPS, MK_PREFILL_TC = 0, 1, 2
 
 STATUS_NAMES = {0: "MK_OK", -1: "MK_ERR_INVALID", -2: "MK_ERR_CUDA", -3: "MK_ERR_TIMEOUT",
                 -4: "MK_ERR_UNSUPPORTED", -5: "MK_ERR_STATE"}
 
 # Every symbol include/mk.h declares.
 EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk_kv_cache_bytes",
-           "mk_load_weights", "mk_prefill_kv", "mk_decode_step", "mk_get_status", "mk_reset",
+           "mk_load_weights", "mk_prefill_kv", "mk_set_prefill", "mk_decode_step", "mk_get_status", "mk_reset",
            "mk_get_position", "mk_set_position", "mk_set_variant", "mk_tune", "mk_set_swiglu_tiling",
            "mk_get_swiglu_tiling", "mk_set_prefetch",
            "mk_set_timeout_ns", "mk_set_sync", "mk_set_ring_stages", "mk_debug_drop_signal",
@@ -30,7 +31,7 @@ EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk
            "mk_swiglu_tune", "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks",
            "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes", "mk_linear_tc",
            "mk_linear_tc_split", "mk_tcdec_create", "mk_tcdec_workspace_bytes", "mk_tcdec_bind", "mk_tcdec_step",
-           "mk_tcdec_status", "mk_tcdec_last_error", "mk_tcdec_destroy")
+           "mk_tcdec_status", "mk_tcdec_last_error", "mk_tcdec_destroy", "mk_tcdec_set_graph")
 
 
 class MkConfig(C.Structure):
@@ -81,6 +82,7 @@ def load() -> C.CDLL:
         "mk_kv_cache_bytes": ([vp, C.POINTER(sz)], st),
         "mk_load_weights": ([vp, C.POINTER(MkWeights), vp, vp, vp], st),
         "mk_prefill_kv": ([vp, vp, i32, i32, vp], st),
+        "mk_set_prefill": ([vp, i32], st),
         "mk_decode_step": ([vp, vp, vp, vp, vp], st),
         "mk_get_status": ([vp, vp], st),
         "mk_reset": ([vp, vp], st),
@@ -118,6 +120,7 @@ def load() -> C.CDLL:
         "mk_tcdec_status": ([vp, C.POINTER(i32), vp], st),
         "mk_tcdec_last_error": ([vp], C.c_char_p),
         "mk_tcdec_destroy": ([vp], st),
+        "mk_tcdec_set_graph": ([vp, i32], st),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)

@@ -31,6 +31,8 @@ struct mk_ctx {
     int sync = MK_SYNC_TAGS;
     int stages = 0;  // ring slots in use (0: all the plan's shared memory allows)
     const void *embed = nullptr;
+    std::vector<LayerW> lw;  // host copy of the per-layer device pointers (packed weights, norms)
+    int prefill = MK_PREFILL_AUTO;
     // captured graph of the separate-kernels variant
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t gexec = nullptr;
@@ -77,7 +79,7 @@ static mk_status plan_both(mk_ctx *c, const mk_config &cfg, int n_ctas, int acti
         if (grow) {
             for (size_t *o : {&p->off_ranges, &p->off_layers, &p->off_rope, &p->off_x, &p->off_xe, &p->off_dpart, &p->off_qkv, &p->off_attn,
                               &p->off_act_a, &p->off_partials, &p->off_lm_best, &p->off_next_scratch, &p->off_norms,
-                              &p->off_weights, &p->off_lm, &p->workspace_bytes})
+                              &p->off_weights, &p->off_lm, &p->off_prefill, &p->workspace_bytes})
                 *o += grow;
             p->lm.offset = p->off_lm;
         }
@@ -91,6 +93,7 @@ static mk_status plan_both(mk_ctx *c, const mk_config &cfg, int n_ctas, int acti
         small.off_act_a = big.off_act_a; small.off_partials = big.off_partials; small.off_lm_best = big.off_lm_best;
         small.off_next_scratch = big.off_next_scratch; small.off_norms = big.off_norms;
         small.off_weights = big.off_weights; small.off_lm = big.off_lm; small.lm.offset = big.lm.offset;
+        small.off_prefill = big.off_prefill;
         small.workspace_bytes = big.workspace_bytes;
     }
     s = validate_plan(a, c->err);
@@ -350,6 +353,7 @@ mk_status mk_load_weights(mk_ctx *c, const mk_weights *w, void *workspace, void 
     CK(cudaMemcpyAsync(norms + (size_t)L * (2 * H + 2 * d) * 2, w->final_norm, (size_t)H * 2,
                        cudaMemcpyDeviceToDevice, s));
     CK(cudaMemcpyAsync(c->ws + p.off_layers, lw.data(), lw.size() * sizeof(LayerW), cudaMemcpyHostToDevice, s));
+    c->lw = lw;
     std::vector<double> inv(d / 2);
     for (int i = 0; i < d / 2; ++i) inv[i] = std::pow((double)g.rope_theta, -2.0 * i / d);
     CK(cudaMemcpyAsync(c->ws + p.off_rope, inv.data(), inv.size() * 8, cudaMemcpyHostToDevice, s));
@@ -500,6 +504,34 @@ mk_status mk_decode_step(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, fl
     return st;
 }
 
+// The prefill on the tensor cores: every position of the prompt of every
+// sequence goes through the decoder in chunks of kPrefillRows positions, each
+// projection one GEMM over the packed weights (mk_tcdec.cu, prefill_tc).
+static mk_status prefill_tensor_cores(mk_ctx *c, const int32_t *d_tokens, int T, cudaStream_t s) {
+    const Plan &p = c->plan;
+    const mk_config &g = p.cfg;
+    PrefillTc a{};
+    a.L = g.n_layers; a.H = g.hidden; a.nq = g.n_heads; a.nkv = g.n_kv_heads; a.d = g.head_dim;
+    a.I = g.intermediate; a.V = g.vocab; a.B = g.batch; a.max_seq = g.max_seq; a.qk_norm = g.qk_norm;
+    a.eps = g.rms_eps;
+    a.theta = (double)g.rope_theta;
+    a.embed = c->embed;
+    a.layers = c->lw.data();
+    a.qkv_kc = p.qkv.kc; a.qkv_M = p.qkv.tiles * p.qkv.rows;
+    a.o_kc = p.o.kc; a.o_M = p.o.tiles * p.o.rows;
+    a.gu_kc = p.gu.kc; a.gu_M = p.gu.tiles * p.gu.rows; a.gu_rows = p.gu.rows;
+    a.down_kc = p.down.kc; a.down_M = p.down.tiles * p.down.rows;
+    a.kcache = reinterpret_cast<uint16_t *>(c->kv);
+    a.vcache = reinterpret_cast<uint16_t *>(c->kv + p.kv_bytes / 2);
+    a.state = reinterpret_cast<State *>(c->ws + p.off_state);
+    a.scratch = c->ws + p.off_prefill;
+    a.scratch_bytes = p.prefill_bytes;
+    const std::string err = prefill_tc(a, d_tokens, T, s);
+    if (!err.empty()) return fail(c, MK_ERR_CUDA, "mk_prefill_kv (tensor cores): " + err);
+    CK(launch_set_position(reinterpret_cast<State *>(c->ws + p.off_state), T, s));
+    return MK_OK;
+}
+
 mk_status mk_prefill_kv(mk_ctx *c, const int32_t *d_tokens, int batch, int T, void *stream) {
     if (!c) return MK_ERR_INVALID;
     if (!c->loaded) return fail(c, MK_ERR_STATE, "mk_prefill_kv before mk_load_weights");
@@ -508,6 +540,16 @@ mk_status mk_prefill_kv(mk_ctx *c, const int32_t *d_tokens, int batch, int T, vo
         return fail(c, MK_ERR_INVALID, "mk_prefill_kv: bad tokens, batch or length");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const Plan &p = c->plan;
+    if (c->prefill != MK_PREFILL_STEPS && p.prefill_tc) {
+        c->pos = 0;
+        mk_status st = prefill_tensor_cores(c, d_tokens, T, s);
+        if (st != MK_OK) return st;
+        c->pos = T;
+        return MK_OK;
+    }
+    if (c->prefill == MK_PREFILL_TC)
+        return fail(c, MK_ERR_UNSUPPORTED, "mk_prefill_kv: this plan splits a projection's K, so the tensor-core "
+                                           "prefill cannot read its packed weights");
     CK(cudaMemsetAsync(c->ws + p.off_state + offsetof(State, pos), 0, 4, s));
     c->pos = 0;
     int32_t *scratch = reinterpret_cast<int32_t *>(c->ws + p.off_next_scratch);
@@ -516,6 +558,16 @@ mk_status mk_prefill_kv(mk_ctx *c, const int32_t *d_tokens, int batch, int T, vo
         if (st != MK_OK) return st;
         c->pos += 1;
     }
+    return MK_OK;
+}
+
+mk_status mk_set_prefill(mk_ctx *c, int mode) {
+    if (!c) return MK_ERR_INVALID;
+    if (mode != MK_PREFILL_AUTO && mode != MK_PREFILL_STEPS && mode != MK_PREFILL_TC)
+        return fail(c, MK_ERR_INVALID, "unknown prefill mode");
+    if (mode == MK_PREFILL_TC && !c->plan.prefill_tc)
+        return fail(c, MK_ERR_UNSUPPORTED, "mk_set_prefill: this plan splits a projection's K (no tensor-core prefill)");
+    c->prefill = mode;
     return MK_OK;
 }
 

@@ -44,6 +44,11 @@ struct AttnArgs {
     const uint16_t *k, *v;
     float *out, *part;
     int B, nq, nkv, d, max_seq, n_pos, chunks;
+    const int *n_pos_dev;  // if set, the attended length is read here (a captured graph's step)
+    // if set, row b of q / out is a query of sequence row_seq[b] over its
+    // positions 0 .. row_len[b] - 1 (a prefill chunk: several positions of one
+    // sequence, each attending causally); else row b is sequence b
+    const int *row_seq, *row_len;
 };
 
 // One CTA = one (chunk, KV head, sequence).  Warps split the G heads
@@ -65,11 +70,13 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
     uint16_t *kt = reinterpret_cast<uint16_t *>(qs + G * d);        // [TP][d]
     uint16_t *vt = kt + TP * d;                                     // [TP][d]
     float *mrg = reinterpret_cast<float *>(vt + TP * d);            // [warps][d + 2]
-    const long long p0 = (long long)c * a.n_pos / a.chunks, p1 = (long long)(c + 1) * a.n_pos / a.chunks;
+    const int n_pos = a.row_len ? a.row_len[b] : (a.n_pos_dev ? *a.n_pos_dev : a.n_pos);  // empty chunks write empty records
+    const int seq = a.row_seq ? a.row_seq[b] : b;
+    const long long p0 = (long long)c * n_pos / a.chunks, p1 = (long long)(c + 1) * n_pos / a.chunks;
     const float qscale = 1.4426950408889634f * rsqrtf((float)d);
     const float *qb = a.q + ((size_t)b * a.nq + (size_t)g * G) * d;
     for (int i = t; i < G * d; i += kAttnThreads) qs[i] = qb[i] * qscale;
-    const size_t head = ((size_t)b * a.nkv + g) * (size_t)a.max_seq;
+    const size_t head = ((size_t)seq * a.nkv + g) * (size_t)a.max_seq;
     float m = -CUDART_INF_F, l = 0.f, o[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) o[e] = 0.f;
@@ -167,6 +174,29 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// The decode attention with the attended length read from device memory at
+// run time (n_pos_dev, between 1 and max_seq) over a fixed number of chunks,
+// for a step that is captured once in a CUDA graph and replayed at every
+// position.  `part` holds batch * nq * chunks * (d + 2) floats.
+cudaError_t launch_attention_dev(const float *q, const void *k, const void *v, int B, int nq, int nkv, int d,
+                                 int max_seq, const int *n_pos_dev, int chunks, float *out, float *part,
+                                 cudaStream_t s) {
+    AttnArgs a{q, static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), out, part, B, nq, nkv, d,
+               max_seq, max_seq, chunks, n_pos_dev, nullptr, nullptr};
+    return launch_attention(a, s);
+}
+
+// Causal attention of `rows` query rows over one layer's cache: row r is a
+// query of sequence row_seq[r] over its positions 0 .. row_len[r] - 1 (the
+// rows of a prefill chunk), `chunks` split-KV chunks per row.
+cudaError_t launch_attention_rows(const float *q, const void *k, const void *v, int rows, int nq, int nkv, int d,
+                                  int max_seq, const int *row_seq, const int *row_len, int chunks, float *out,
+                                  float *part, cudaStream_t s) {
+    AttnArgs a{q, static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), out, part, rows, nq, nkv, d,
+               max_seq, max_seq, chunks, nullptr, row_seq, row_len};
+    return launch_attention(a, s);
+}
+
 // ------------------------------------------------------------------ host side
 static thread_local char g_op_error[256] = "";
 
@@ -240,7 +270,7 @@ extern "C" mk_status mk_attention_decode(const float *q, const void *k_cache, co
                                          int chunks, float *out, void *scratch, size_t scratch_bytes,
                                          void *stream) {
     AttnArgs a{q, static_cast<const uint16_t *>(k_cache), static_cast<const uint16_t *>(v_cache), out, nullptr,
-               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks};
+               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks, nullptr, nullptr, nullptr};
     mk_status st = attention_args(a, q, k_cache, v_cache, out);
     if (st != MK_OK) return st;
     const size_t need = mk_attention_scratch_bytes(batch, n_heads, head_dim, a.chunks);
@@ -283,7 +313,7 @@ extern "C" mk_status mk_attention_decode_noalloc(const float *q, const void *k_c
                                                  int n_heads, int n_kv_heads, int head_dim, int max_seq, int n_pos,
                                                  int chunks, float *out, void *stream) {
     AttnArgs a{q, static_cast<const uint16_t *>(k_cache), static_cast<const uint16_t *>(v_cache), out, nullptr,
-               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks};
+               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks, nullptr, nullptr, nullptr};
     const bool auto_chunks = chunks == 0;
     mk_status st = attention_args(a, q, k_cache, v_cache, out);
     if (st != MK_OK) return st;

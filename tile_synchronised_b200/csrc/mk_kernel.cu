@@ -130,15 +130,23 @@ __device__ bool wait_bar(const KParams &P, uint64_t *bar, uint32_t parity, volat
     }
 }
 
-// The token of sequence b.  One outside [0, vocab) is recorded in the step
-// state (the first such sequence and its value, reported by mk_get_status as
-// an invalid argument) and replaced by 0 so that every read stays inside the
-// embedding table; the step still runs to the end, so no wait is cut short.
+// The token of sequence b, with one outside [0, vocab) replaced by 0 so that
+// every read stays inside the embedding table (check_tokens has recorded it;
+// the step still runs to the end, so no wait is cut short).
 __device__ __forceinline__ int token_of(const KParams &P, int b) {
     const int t = P.tokens[(int64_t)b * P.tok_stride];
-    if (t >= 0 && t < P.vocab) return t;
-    if (atomicCAS(&P.state->tok_err, 0u, (uint32_t)b + 1u) == 0u) P.state->tok_bad = t;
-    return 0;
+    return (unsigned)t < (unsigned)P.vocab ? t : 0;
+}
+
+// At the start of a launch, thread b of CTA 0 checks the token of sequence b
+// and records one outside [0, vocab) in the step state (the first such
+// sequence and its value; mk_get_status reports it as an invalid argument).
+__device__ __forceinline__ void check_tokens(const KParams &P) {
+    const int b = threadIdx.x;
+    if (blockIdx.x != 0 || b >= P.batch) return;
+    const int t = P.tokens[(int64_t)b * P.tok_stride];
+    if ((unsigned)t >= (unsigned)P.vocab && atomicCAS(&P.state->tok_err, 0u, (uint32_t)b + 1u) == 0u)
+        P.state->tok_bad = t;
 }
 
 struct MatRef {
@@ -489,8 +497,18 @@ __device__ __forceinline__ bool residual8(const KParams &P, const SmemLayout &S,
 }
 
 // ------------------------------------------------------------------ activation staging
+// Shared-memory position of the first of the 8 values of chunk c (values
+// c*8 .. c*8+7 of a staged row); the other four sit 128 floats further.  A
+// lane multiplies 8 consecutive columns of a 256-column chunk by the
+// activations staged here: split into two float4 that the warp's 32 lanes
+// read as two contiguous 512-byte runs, those reads are free of shared-memory
+// bank conflicts (8 consecutive floats per lane would be 32 bytes apart,
+// two lanes per bank group).
+__device__ __forceinline__ int act_slot(int c) { return (c >> 5) * 256 + (c & 31) * 4; }
+
 // Writes the instruction's activations for batch rows [b0, b0+nb) as fp32
-// [nb][klen] into shared memory: RMSNorm(x) * gain for QKV / gate-up / LM head,
+// [nb][klen] into shared memory (each 256-value group in the act_slot order):
+// RMSNorm(x) * gain for QKV / gate-up / LM head,
 // a plain copy of the attention output or of the SwiGLU product otherwise.
 // Each thread reads tagged words and spins until they carry the producing
 // layer's tag.  Returns false if a wait gave up; every thread still reaches
@@ -528,13 +546,14 @@ __device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S,
                 for (int j = 0; j < 4; ++j) {
                     const int c = c0 + j * kConsumerThreads;
                     if (c < nch) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dst + (size_t)c * 8);
+                        float4 *d0 = reinterpret_cast<float4 *>(dst + act_slot(c));
+                        float4 *d1 = reinterpret_cast<float4 *>(dst + act_slot(c) + 128);
                         if (j < mm) {
-                            d4[0] = make_float4(f[j][0], f[j][1], f[j][2], f[j][3]);
-                            d4[1] = make_float4(f[j][4], f[j][5], f[j][6], f[j][7]);
+                            *d0 = make_float4(f[j][0], f[j][1], f[j][2], f[j][3]);
+                            *d1 = make_float4(f[j][4], f[j][5], f[j][6], f[j][7]);
                         } else {
-                            d4[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            d4[1] = d4[0];
+                            *d0 = make_float4(0.f, 0.f, 0.f, 0.f);
+                            *d1 = *d0;
                         }
                     }
                 }
@@ -568,10 +587,11 @@ __device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S,
         if (b >= nb) break;
         const int row = in.b0 + b;
         for (int c = t; c < nch; c += kConsumerThreads) {
-            float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen + c * 8);
+            float4 *d0 = reinterpret_cast<float4 *>(act + (size_t)b * klen + act_slot(c));
+            float4 *d1 = reinterpret_cast<float4 *>(act + (size_t)b * klen + act_slot(c) + 128);
             if (c * 8 >= H) {
-                dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-                dst[1] = dst[0];
+                *d0 = make_float4(0.f, 0.f, 0.f, 0.f);
+                *d1 = *d0;
                 continue;
             }
             float f[8], g[8];
@@ -589,8 +609,8 @@ __device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S,
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q) ss[b] = fmaf(f[q], f[q], ss[b]);
-            dst[0] = make_float4(f[0] * g[0], f[1] * g[1], f[2] * g[2], f[3] * g[3]);
-            dst[1] = make_float4(f[4] * g[4], f[5] * g[5], f[6] * g[6], f[7] * g[7]);
+            *d0 = make_float4(f[0] * g[0], f[1] * g[1], f[2] * g[2], f[3] * g[3]);
+            *d1 = make_float4(f[4] * g[4], f[5] * g[5], f[6] * g[6], f[7] * g[7]);
         }
     }
 #pragma unroll
@@ -611,11 +631,12 @@ __device__ __forceinline__ bool stage_act(const KParams &P, const SmemLayout &S,
 #pragma unroll
         for (int b = 0; b < BS; ++b) {
             if (b < nb) {
-                float4 *dst = reinterpret_cast<float4 *>(act + (size_t)b * klen + c * 8);
-                const float4 x0 = dst[0], x1 = dst[1];
+                float4 *d0 = reinterpret_cast<float4 *>(act + (size_t)b * klen + act_slot(c));
+                float4 *d1 = reinterpret_cast<float4 *>(act + (size_t)b * klen + act_slot(c) + 128);
+                const float4 x0 = *d0, x1 = *d1;
                 const float r = rs[b];
-                dst[0] = make_float4(x0.x * r, x0.y * r, x0.z * r, x0.w * r);
-                dst[1] = make_float4(x1.x * r, x1.y * r, x1.z * r, x1.w * r);
+                *d0 = make_float4(x0.x * r, x0.y * r, x0.z * r, x0.w * r);
+                *d1 = make_float4(x1.x * r, x1.y * r, x1.z * r, x1.w * r);
             }
         }
     }
@@ -696,8 +717,9 @@ __device__ __forceinline__ bool gemv_warp_tile(const KParams &P, const SmemLayou
 #pragma unroll
             for (int b = 0; b < BS; ++b) {
                 if (b < nb) {
-                    const float4 *a4 = reinterpret_cast<const float4 *>(act + (size_t)b * klen + j * kc + col);
-                    const float4 x0 = a4[0], x1 = a4[1];
+                    const float *ab = act + (size_t)b * klen + j * kc + c * 256 + lane * 4;
+                    const float4 x0 = *reinterpret_cast<const float4 *>(ab);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(ab + 128);
                     af[b][0] = x0.x; af[b][1] = x0.y; af[b][2] = x0.z; af[b][3] = x0.w;
                     af[b][4] = x1.x; af[b][5] = x1.y; af[b][6] = x1.z; af[b][7] = x1.w;
                 } else {
@@ -1040,15 +1062,34 @@ __device__ __forceinline__ int attn_instr(const KParams &P, const SmemLayout &S,
                        P.kcache + kv_off(P, l, a.b, a.g, pos));
     }
     if (a.has_cur && warp == kConsumerWarps - 1) {
+        // this step's V row: a lane's d/32 words are loaded together and
+        // re-read together until all carry the tag (one round trip, not one
+        // per word)
         const uint64_t *vs = qkv_b + (nq + nkv) * d + a.g * d;
         uint16_t *vrow = P.vcache + kv_off(P, l, a.b, a.g, pos);
-        for (int e = lane; e < d; e += 32) {
-            float vv = 0.f;
-            ok = ll_word(P, S, vs + e, tag, vv, (uint32_t)OP_ATTN << 16) && ok;
-            const uint16_t hv = f2bf(vv);
-            vrow[e] = hv;
-            vpos[e] = bf2f(hv);
+        const int nj = d / 32;
+        uint64_t w[4];
+        LlSpin sp{0ull, 0u};
+        for (;;) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = j < nj ? ll_ld(vs + lane + 32 * j) : ll_pack(0.f, tag);
+            bool all = true;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) all = all && ll_tag(w[j]) == tag;
+            if (all) break;
+            __nanosleep(16);
+            if (!ll_spin(P, S, sp, (uint32_t)OP_ATTN << 16, tag)) {
+                ok = false;
+                break;
+            }
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (j < nj) {
+                const uint16_t hv = f2bf(ll_value(w[j]));
+                vrow[lane + 32 * j] = hv;
+                vpos[lane + 32 * j] = bf2f(hv);
+            }
     }
     if (consumer_sync_or(!ok || *S.abort != 0)) return kAttnStop;
     if (a.has_cur && G == kConsumerWarps) {  // every warp held a query head: the key comes now
@@ -1414,6 +1455,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
         S.rope[i] = make_float2(cs, sn);
     }
     if (t < 64) S.best[t] = argmax_key(-CUDART_INF_F, 0x7fffffff);
+    check_tokens(P);
     __syncthreads();
     const int begin = P.cta_begin[blockIdx.x], end = P.cta_end[blockIdx.x];
     if (t >= kConsumerThreads) {

@@ -2,6 +2,8 @@
 #pragma once
 #include <cuda_runtime.h>
 
+#include <string>
+
 #include "mk_internal.h"
 
 namespace mk {
@@ -23,6 +25,36 @@ cudaError_t launch_swiglu_col_tma(const void *x, const void *wg, const void *wu,
                                   cudaStream_t s);
 cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void *out, int B, int K, int N,
                              cudaStream_t s);
+// Split-KV decode attention whose attended length is read from device memory
+// (mk_attn.cu); the caller has checked the shapes.
+cudaError_t launch_attention_dev(const float *q, const void *k, const void *v, int B, int nq, int nkv, int d,
+                                 int max_seq, const int *n_pos_dev, int chunks, float *out, float *part,
+                                 cudaStream_t s);
+// Causal attention of prefill rows (mk_attn.cu): row r of q / out attends
+// positions 0 .. row_len[r] - 1 of sequence row_seq[r] of one layer's cache.
+cudaError_t launch_attention_rows(const float *q, const void *k, const void *v, int rows, int nq, int nkv, int d,
+                                  int max_seq, const int *row_seq, const int *row_len, int chunks, float *out,
+                                  float *part, cudaStream_t s);
+// The tensor-core prefill of a megakernel context (mk_tcdec.cu): positions
+// 0 .. T-1 of every sequence through the decoder in chunks of kPrefillRows,
+// every projection one mk_linear_tc call over the packed weights, which must
+// each be a single K block (plain row-major [rows, kc]).  Fills the KV cache
+// only.
+struct PrefillTc {
+    int L, H, nq, nkv, d, I, V, B, max_seq, qk_norm;
+    float eps;
+    double theta;
+    const void *embed;
+    const LayerW *layers;  // host array of the L layers' device pointers
+    int qkv_kc, qkv_M, o_kc, o_M, gu_kc, gu_M, gu_rows, down_kc, down_M;
+    uint16_t *kcache, *vcache;
+    State *state;
+    uint8_t *scratch;
+    size_t scratch_bytes;
+};
+size_t prefill_scratch_bytes(int H, int nq, int d, int kmax, int mmax);
+// Returns an empty string, or the reason it stopped.
+std::string prefill_tc(const PrefillTc &a, const int32_t *tokens, int T, cudaStream_t s);
 // Last error of a context-free call (the isolated operations) on this thread.
 void set_op_error(const char *msg);
 const char *op_error();

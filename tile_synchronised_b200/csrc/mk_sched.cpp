@@ -312,6 +312,14 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
                            align_up(mat_bytes(p.gu), 256) + align_up(mat_bytes(p.down), 256);
     p.off_weights = take((size_t)L * p.layer_weight_bytes);
     p.off_lm = take(mat_bytes(p.lm));
+    p.prefill_tc = p.qkv.nkb == 1 && p.o.nkb == 1 && p.gu.nkb == 1 && p.down.nkb == 1;
+    if (p.prefill_tc) {
+        const int kmax = std::max({p.qkv.kc, p.o.kc, p.gu.kc, p.down.kc});
+        const int mmax = std::max({p.qkv.tiles * p.qkv.rows, p.o.tiles * p.o.rows, p.gu.tiles * p.gu.rows,
+                                   p.down.tiles * p.down.rows});
+        p.prefill_bytes = prefill_scratch_bytes(H, nq, d, kmax, mmax);
+        p.off_prefill = take(p.prefill_bytes);
+    }
     p.qkv.offset = 0;
     p.o.offset = align_up(mat_bytes(p.qkv), 256);
     p.gu.offset = p.o.offset + align_up(mat_bytes(p.o), 256);

@@ -32,6 +32,10 @@ struct Plan {
     size_t off_state = 0, off_counters = 0, off_instrs = 0, off_ranges = 0, off_layers = 0, off_rope = 0;
     size_t off_x = 0, off_xe = 0, off_dpart = 0, off_qkv = 0, off_attn = 0, off_act_a = 0, off_partials = 0, off_lm_best = 0;
     size_t off_next_scratch = 0, off_weights = 0, layer_weight_bytes = 0, off_lm = 0, off_norms = 0;
+    // tensor-core prefill: possible when every packed layer matrix is one K
+    // block (then a plain row-major [rows, kc] matrix); its scratch region
+    bool prefill_tc = false;
+    size_t off_prefill = 0, prefill_bytes = 0;
     size_t workspace_bytes = 0, kv_bytes = 0;
 
     // schedule
@@ -43,6 +47,8 @@ struct Plan {
     std::vector<uint32_t> counter_count; // increments each counter receives per step (0 = arrival counter)
 };
 
+// Bytes of the tensor-core prefill's scratch (mk_tcdec.cu).
+size_t prefill_scratch_bytes(int H, int nq, int d, int kmax, int mmax);
 // Build a plan; returns MK_OK or an error code with a reason in `err`.
 mk_status build_plan(const mk_config &cfg, int n_ctas, int swiglu_variant, Plan &plan, std::string &err);
 // Simulate the schedule on the host; MK_OK or MK_ERR_STATE with a reason.

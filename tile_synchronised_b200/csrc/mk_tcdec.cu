@@ -87,13 +87,15 @@ __global__ void norm_hilo_kernel(const float *x, const uint16_t *g, __nv_bfloat1
 // then nkv k heads, then nkv v heads; y* hold the hi and lo rows of each
 // projection.  q and k get the optional per-head RMSNorm and the RoPE
 // rotation (pairs i, i + d/2, angle pos * theta^(-2i/d) in double); q goes to
-// q_out, k and v to the layer's cache at `pos` as bf16.
+// q_out, k and v to the layer's cache at `pos` as bf16.  The position is read
+// from device memory (posw[0]), so a captured step replays at any position.
 __global__ void qkv_post_kernel(const float *yq, const float *yk, const float *yv, int B, int nq, int nkv, int d,
                                 const uint16_t *qn, const uint16_t *kn, int qk_norm, float eps, double theta,
-                                int pos, float *q_out, uint16_t *kc, uint16_t *vc, int max_seq) {
+                                const int *posw, float *q_out, uint16_t *kc, uint16_t *vc, int max_seq) {
     extern __shared__ float buf[];  // d values, then 32 partial sums
     float *red = buf + d;
     const int head = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+    const int pos = posw[0];
     const float *src;
     int M, off;
     if (head < nq) {
@@ -159,6 +161,12 @@ __global__ void swiglu_hilo_kernel(const float *yg, const float *yu, __nv_bfloat
     }
 }
 
+// posw[0] = the position of the step, posw[1] = the attended length.
+__global__ void set_pos_kernel(int *posw, int pos) {
+    posw[0] = pos;
+    posw[1] = pos + 1;
+}
+
 // One block per sequence: logits[b][v] = y[b][v] + y[B + b][v] (written when
 // `logits` is set) and next[b] = their argmax, lowest index on ties.  With no
 // finite logit to pick (a projection that gave up writes NaN), next[b] is set
@@ -205,9 +213,124 @@ __global__ void lm_argmax_kernel(const float *y, float *logits, int32_t *next, i
     }
 }
 
+// ------------------------------------------------------------------ prefill rows
+// The prefill of a megakernel context on the tensor cores: R <= 32
+// consecutive positions t0 .. t0 + R - 1 of one sequence b go through the
+// decoder together, every projection one mk_linear_tc call over the
+// context's packed weights (which are plain row-major [rows, kc] matrices
+// when each has a single K block), activations as hi/lo bf16 row pairs as in
+// the batched step, and attention causal per row (position t0 + r attends to
+// 0 .. t0 + r).  Only the KV cache is kept: the last layer stops after its
+// K/V rows.
+
+// x[r][:] = E[tok(b, t0 + r)][:]; a token outside [0, V) decodes from token 0
+// and is recorded in the context's state (first one wins), as the megakernel
+// does.
+__global__ void prefill_embed_kernel(const int32_t *tok, int64_t tok_stride, int b, int t0, const uint16_t *E,
+                                     float *x, int H, int V, State *state) {
+    const int r = blockIdx.x;
+    int t = tok[(int64_t)b * tok_stride + t0 + r];
+    if (t < 0 || t >= V) {
+        if (threadIdx.x == 0 && atomicCAS(&state->tok_err, 0u, (uint32_t)b + 1u) == 0u) state->tok_bad = t;
+        t = 0;
+    }
+    for (int i = threadIdx.x; i < H; i += blockDim.x) x[(size_t)r * H + i] = bf2f(E[(size_t)t * H + i]);
+}
+
+// out rows r (hi) and R + r (lo), Kp wide = RMSNorm(x[r]) * g, zero past H.
+__global__ void prefill_norm_kernel(const float *x, const uint16_t *g, __nv_bfloat16 *out, int R, int H, int Kp,
+                                    float eps) {
+    __shared__ float red[32];
+    const int r = blockIdx.x;
+    const float *xr = x + (size_t)r * H;
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < H; i += blockDim.x) ss = fmaf(xr[i], xr[i], ss);
+    ss = block_sum(ss, red);
+    const float rs = rsqrtf(ss / (float)H + eps);
+    for (int i = threadIdx.x; i < Kp; i += blockDim.x)
+        put_hilo(out + (size_t)r * Kp + i, out + (size_t)(R + r) * Kp + i, i < H ? xr[i] * rs * bf2f(g[i]) : 0.f);
+}
+
+// One block per (head, row), head_dim threads, over the packed QKV output y
+// [2R][M] (q heads, then k, then v): the optional per-head RMSNorm and RoPE at
+// position t0 + r; q to q_out [R][nq][d], k and v to the layer's cache rows of
+// sequence b at t0 + r.
+__global__ void prefill_qkv_kernel(const float *y, int R, int M, int nq, int nkv, int d, const uint16_t *qn,
+                                   const uint16_t *kn, int qk_norm, float eps, double theta, int b, int t0,
+                                   float *q_out, uint16_t *kc, uint16_t *vc, int max_seq) {
+    extern __shared__ float buf[];
+    float *red = buf + d;
+    const int head = blockIdx.x, r = blockIdx.y, i = threadIdx.x;
+    const int pos = t0 + r;
+    float v = y[(size_t)r * M + head * d + i] + y[(size_t)(R + r) * M + head * d + i];
+    const int g = head < nq ? 0 : (head < nq + nkv ? head - nq : head - nq - nkv);
+    const size_t crow = (((size_t)b * nkv + g) * max_seq + pos) * d;
+    if (head >= nq + nkv) {
+        vc[crow + i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        return;
+    }
+    if (qk_norm) {
+        const float ss = block_sum(v * v, red);
+        v = v * rsqrtf(ss / (float)d + eps) * bf2f((head < nq ? qn : kn)[i]);
+    }
+    buf[i] = v;
+    __syncthreads();
+    const int h2 = d / 2, j = i < h2 ? i : i - h2;
+    const double ang = (double)pos * pow(theta, -2.0 * (double)j / (double)d);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    const float c = (float)cd, sn = (float)sd;
+    const float o = i < h2 ? buf[i] * c - buf[i + h2] * sn : buf[i] * c + buf[i - h2] * sn;
+    if (head < nq)
+        q_out[((size_t)r * nq + head) * d + i] = o;
+    else
+        kc[crow + i] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+}
+
+// row_seq[r] = b, row_len[r] = t0 + r + 1: the rows' sequence and attended length.
+__global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, int t0) {
+    const int r = threadIdx.x;
+    if (r < R) {
+        row_seq[r] = b;
+        row_len[r] = t0 + r + 1;
+    }
+}
+
+// out rows r, R + r (Kp wide) = hi / lo of a[r][0 .. n), zero past n.
+__global__ void prefill_cast_kernel(const float *a, __nv_bfloat16 *out, int R, int n, int Kp) {
+    const int r = blockIdx.y;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < Kp; i += gridDim.x * blockDim.x)
+        put_hilo(out + (size_t)r * Kp + i, out + (size_t)(R + r) * Kp + i, i < n ? a[(size_t)r * n + i] : 0.f);
+}
+
+// x[r][i] += y[r][i] + y[R + r][i], y rows M wide.
+__global__ void prefill_residual_kernel(float *x, const float *y, int R, int H, int M) {
+    const int r = blockIdx.y;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < H; i += gridDim.x * blockDim.x)
+        x[(size_t)r * H + i] += y[(size_t)r * M + i] + y[(size_t)(R + r) * M + i];
+}
+
+// The packed gate/up output y [2R][M] interleaves them tile by tile: packed
+// row t*rows + k is gate row t*rows/2 + k for k < rows/2, else up row
+// t*rows/2 + k - rows/2.  out rows r, R + r (Kp wide) = hi / lo of
+// SiLU(gate) * up, zero past I.
+__global__ void prefill_swiglu_kernel(const float *y, __nv_bfloat16 *out, int R, int I, int M, int rows, int Kp) {
+    const int r = blockIdx.y, half = rows / 2;
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < Kp; j += gridDim.x * blockDim.x) {
+        float val = 0.f;
+        if (j < I) {
+            const size_t gi = (size_t)(j / half) * rows + j % half, ui = gi + half;
+            const float gt = y[(size_t)r * M + gi] + y[(size_t)(R + r) * M + gi];
+            const float up = y[(size_t)r * M + ui] + y[(size_t)(R + r) * M + ui];
+            val = gt / (1.0f + expf(-gt)) * up;
+        }
+        put_hilo(out + (size_t)r * Kp + j, out + (size_t)(R + r) * Kp + j, val);
+    }
+}
+
 // Byte offsets of the workspace pieces (each 256-byte aligned).
 struct Layout {
-    size_t x, h, yq, yk, yv, ya, yg, yu, ylm, q, attn, scratch, scratch_bytes, status, total;
+    size_t x, h, yq, yk, yv, ya, yg, yu, ylm, q, attn, scratch, scratch_bytes, status, tok, nxt, posw, lg, total;
 };
 
 static Layout layout(const mk_config &c) {
@@ -235,11 +358,91 @@ static Layout layout(const mk_config &c) {
     o.scratch_bytes = mk_attention_scratch_bytes(c.batch, c.n_heads, c.head_dim, kMaxChunks);
     o.scratch = take(o.scratch_bytes);
     o.status = take(4);
+    o.tok = take(B * 4);   // the step's tokens, copied in from the caller
+    o.nxt = take(B * 4);   // its argmax, copied out to the caller
+    o.posw = take(8);      // position and attended length
+    o.lg = take(B * V * 4);  // its logits, copied out when the caller asks for them
     o.total = at;
     return o;
 }
 
 }  // namespace tcdec
+
+size_t prefill_scratch_bytes(int H, int nq, int d, int kmax, int mmax) {
+    const size_t R = kPrefillRows;
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    return up(R * H * 4) + up(2 * R * kmax * 2) + up(2 * R * (size_t)mmax * 4) + 2 * up(R * nq * d * 4) +
+           up(R * nq * kPrefillChunks * (size_t)(d + 2) * 4) + up(2 * R * 4);
+}
+
+std::string prefill_tc(const PrefillTc &a, const int32_t *tokens, int T, cudaStream_t s) {
+    using namespace tcdec;
+    const int R = kPrefillRows;
+    const int kmax = std::max(std::max(a.qkv_kc, a.o_kc), std::max(a.gu_kc, a.down_kc));
+    const int mmax = std::max(std::max(a.qkv_M, a.o_M), std::max(a.gu_M, a.down_M));
+    if (a.scratch_bytes < prefill_scratch_bytes(a.H, a.nq, a.d, kmax, mmax)) return "prefill scratch too small";
+    uint8_t *p = a.scratch;
+    auto take = [&](size_t bytes) {
+        uint8_t *q = p;
+        p += (bytes + 255) / 256 * 256;
+        return q;
+    };
+    float *x = reinterpret_cast<float *>(take((size_t)R * a.H * 4));
+    __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(take((size_t)2 * R * kmax * 2));
+    float *y = reinterpret_cast<float *>(take((size_t)2 * R * mmax * 4));
+    float *q = reinterpret_cast<float *>(take((size_t)R * a.nq * a.d * 4));
+    float *attn = reinterpret_cast<float *>(take((size_t)R * a.nq * a.d * 4));
+    float *part = reinterpret_cast<float *>(take((size_t)R * a.nq * kPrefillChunks * (a.d + 2) * 4));
+    int *rows = reinterpret_cast<int *>(take((size_t)2 * R * 4));
+    const size_t layer_elems = (size_t)a.B * a.nkv * a.max_seq * a.d;
+    std::string err;
+    auto lin = [&](const void *w, int K, int M, int n) {
+        if (err.empty() && mk_linear_tc(h, w, y, 2 * n, K, M, s) != MK_OK) err = op_error();
+    };
+    for (int b = 0; b < a.B && err.empty(); ++b)
+        for (int t0 = 0; t0 < T && err.empty(); t0 += R) {
+            const int n = std::min(R, T - t0);
+            prefill_embed_kernel<<<n, kRowThreads, 0, s>>>(tokens, T, b, t0, static_cast<const uint16_t *>(a.embed),
+                                                          x, a.H, a.V, a.state);
+            prefill_rows_kernel<<<1, 32, 0, s>>>(rows, rows + R, n, b, t0);
+            const int chunks = std::max(1, std::min(kPrefillChunks, (t0 + n) / 128));
+            for (int l = 0; l < a.L && err.empty(); ++l) {
+                const LayerW &W = a.layers[l];
+                uint16_t *kc = a.kcache + (size_t)l * layer_elems, *vc = a.vcache + (size_t)l * layer_elems;
+                prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(W.attn_norm), h, n,
+                                                             a.H, a.qkv_kc, a.eps);
+                lin(W.qkv, a.qkv_kc, a.qkv_M, n);
+                if (!err.empty()) break;
+                prefill_qkv_kernel<<<dim3((unsigned)(a.nq + 2 * a.nkv), (unsigned)n), a.d, (a.d + 32) * sizeof(float),
+                                     s>>>(y, n, a.qkv_M, a.nq, a.nkv, a.d, static_cast<const uint16_t *>(W.q_norm),
+                                          static_cast<const uint16_t *>(W.k_norm), a.qk_norm, a.eps, a.theta, b, t0,
+                                          q, kc, vc, a.max_seq);
+                if (l == a.L - 1) break;  // the cache is all the prefill keeps: the last layer ends at its K/V
+                const cudaError_t e = launch_attention_rows(q, kc, vc, n, a.nq, a.nkv, a.d, a.max_seq, rows,
+                                                            rows + R, chunks, attn, part, s);
+                if (e != cudaSuccess) {
+                    err = std::string("prefill attention: ") + cudaGetErrorString(e);
+                    break;
+                }
+                prefill_cast_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(attn, h, n, a.nq * a.d, a.o_kc);
+                lin(W.o, a.o_kc, a.o_M, n);
+                prefill_residual_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(x, y, n, a.H, a.o_M);
+                prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(W.mlp_norm), h, n,
+                                                             a.H, a.gu_kc, a.eps);
+                lin(W.gu, a.gu_kc, a.gu_M, n);
+                prefill_swiglu_kernel<<<dim3(32, (unsigned)n), kRowThreads, 0, s>>>(y, h, n, a.I, a.gu_M, a.gu_rows,
+                                                                                  a.down_kc);
+                lin(W.down, a.down_kc, a.down_M, n);
+                prefill_residual_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(x, y, n, a.H, a.down_M);
+            }
+        }
+    if (err.empty()) {
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) err = cudaGetErrorString(e);
+    }
+    return err;
+}
+
 }  // namespace mk
 
 using namespace mk;
@@ -253,7 +456,19 @@ struct mk_tcdec {
     Layout lay{};
     uint8_t *ws = nullptr;
     uint16_t *kv = nullptr;
+    int chunks = 1;                                // split-KV chunks, fixed for every position
+    bool use_graph = true;
+    bool warmed = false;                           // one eager step ran (kernel attributes are set)
+    cudaGraphExec_t exec[2] = {nullptr, nullptr};  // the captured step without / with logits
 };
+
+static void drop_graphs(mk_tcdec *d) {
+    for (auto &e : d->exec)
+        if (e) {
+            cudaGraphExecDestroy(e);
+            e = nullptr;
+        }
+}
 
 static mk_status tc_fail(mk_tcdec *d, mk_status s, const std::string &msg) {
     if (d)
@@ -314,6 +529,9 @@ extern "C" mk_status mk_tcdec_create(const mk_config *cfg, const mk_weights *w, 
         return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: a weight pointer is null or not 16-byte aligned");
     }
     d->lay = layout(c);
+    d->chunks = mk_attention_chunks(c.batch, c.n_kv_heads, c.max_seq);
+    if (d->chunks < 1) d->chunks = 1;
+    if (d->chunks > kMaxChunks) d->chunks = kMaxChunks;
     *out = d;
     return MK_OK;
 }
@@ -330,6 +548,7 @@ extern "C" mk_status mk_tcdec_bind(mk_tcdec *d, void *workspace, void *kv_cache)
     if (!d) return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: null context");
     if (!workspace || ((uintptr_t)workspace & 255u) || !aligned16(kv_cache))
         return tc_fail(d, MK_ERR_INVALID, "tcdec: workspace must be 256-byte and kv_cache 16-byte aligned");
+    drop_graphs(d);  // the captured steps point at the old buffers
     d->ws = static_cast<uint8_t *>(workspace);
     d->kv = static_cast<uint16_t *>(kv_cache);
     if (cudaMemset(d->ws + d->lay.status, 0, sizeof(int)) != cudaSuccess)
@@ -337,15 +556,14 @@ extern "C" mk_status mk_tcdec_bind(mk_tcdec *d, void *workspace, void *kv_cache)
     return MK_OK;
 }
 
-extern "C" mk_status mk_tcdec_step(mk_tcdec *d, const int32_t *d_tokens, int pos, int32_t *d_next, float *d_logits,
-                                   void *stream) {
-    if (!d) return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: null context");
-    if (!d->ws) return tc_fail(d, MK_ERR_STATE, "tcdec: mk_tcdec_step before mk_tcdec_bind");
+// Queue one whole step on `s`: tokens from the workspace's token row, the
+// position from its position words, the argmax (and the logits if `logits`)
+// into the workspace.  Every launch reads its varying inputs from device
+// memory, so the same sequence of launches, captured once, serves every step.
+static mk_status enqueue_step(mk_tcdec *d, cudaStream_t s, bool logits) {
     const mk_config &c = d->cfg;
-    if (!d_tokens || !d_next) return tc_fail(d, MK_ERR_INVALID, "tcdec: null token buffer");
-    if (pos < 0 || pos >= c.max_seq) return tc_fail(d, MK_ERR_INVALID, "tcdec: position outside the cache");
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const Layout &o = d->lay;
+    void *stream = s;
     const int B = c.batch, H = c.hidden, I = c.intermediate, V = c.vocab, L = c.n_layers;
     const int nq = c.n_heads, nkv = c.n_kv_heads, hd = c.head_dim, QD = nq * hd, KD = nkv * hd;
     float *x = reinterpret_cast<float *>(d->ws + o.x);
@@ -355,11 +573,12 @@ extern "C" mk_status mk_tcdec_step(mk_tcdec *d, const int32_t *d_tokens, int pos
     float *yg = reinterpret_cast<float *>(d->ws + o.yg), *yu = reinterpret_cast<float *>(d->ws + o.yu);
     float *ylm = reinterpret_cast<float *>(d->ws + o.ylm);
     float *q = reinterpret_cast<float *>(d->ws + o.q), *attn = reinterpret_cast<float *>(d->ws + o.attn);
-    void *scratch = d->ws + o.scratch;
+    float *scratch = reinterpret_cast<float *>(d->ws + o.scratch);
     int *status = reinterpret_cast<int *>(d->ws + o.status);
+    const int32_t *tok = reinterpret_cast<const int32_t *>(d->ws + o.tok);
+    int32_t *nxt = reinterpret_cast<int32_t *>(d->ws + o.nxt);
+    const int *posw = reinterpret_cast<const int *>(d->ws + o.posw);
     const size_t layer_elems = (size_t)B * nkv * c.max_seq * hd;
-    const int n_pos = pos + 1;
-    const int chunks = mk_attention_chunks(B, nkv, n_pos);
     mk_status st = MK_OK;
     auto lin = [&](const void *xin, const void *wt, float *y, int K, int M) {
         if (st == MK_OK && mk_linear_tc(xin, wt, y, 2 * B, K, M, stream) != MK_OK) {
@@ -368,7 +587,7 @@ extern "C" mk_status mk_tcdec_step(mk_tcdec *d, const int32_t *d_tokens, int pos
         }
     };
     const dim3 rows_grid(8, (unsigned)B);
-    embed_kernel<<<B, kRowThreads, 0, s>>>(d_tokens, static_cast<const uint16_t *>(d->embed), x, H, V, status);
+    embed_kernel<<<B, kRowThreads, 0, s>>>(tok, static_cast<const uint16_t *>(d->embed), x, H, V, status);
     for (int l = 0; l < L && st == MK_OK; ++l) {
         uint16_t *kc = d->kv + (size_t)l * layer_elems, *vc = d->kv + (size_t)(L + l) * layer_elems;
         norm_hilo_kernel<<<B, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(d->attn_norm[l]), h, B, H,
@@ -379,12 +598,13 @@ extern "C" mk_status mk_tcdec_step(mk_tcdec *d, const int32_t *d_tokens, int pos
         if (st != MK_OK) break;
         qkv_post_kernel<<<dim3((unsigned)(nq + 2 * nkv), (unsigned)B), hd, (hd + 32) * sizeof(float), s>>>(
             yq, yk, yv, B, nq, nkv, hd, static_cast<const uint16_t *>(d->q_norm[l]),
-            static_cast<const uint16_t *>(d->k_norm[l]), c.qk_norm, c.rms_eps, (double)c.rope_theta, pos, q, kc, vc,
+            static_cast<const uint16_t *>(d->k_norm[l]), c.qk_norm, c.rms_eps, (double)c.rope_theta, posw, q, kc, vc,
             c.max_seq);
-        if (mk_attention_decode(q, kc, vc, B, nq, nkv, hd, c.max_seq, n_pos, chunks, attn, scratch, o.scratch_bytes,
-                                stream) != MK_OK) {
+        const cudaError_t ea =
+            launch_attention_dev(q, kc, vc, B, nq, nkv, hd, c.max_seq, posw + 1, d->chunks, attn, scratch, s);
+        if (ea != cudaSuccess) {
             st = MK_ERR_CUDA;
-            d->err = std::string("tcdec: ") + op_error();
+            d->err = std::string("tcdec: attention: ") + cudaGetErrorString(ea);
             break;
         }
         cast_hilo_kernel<<<rows_grid, kRowThreads, 0, s>>>(attn, h, B, QD);
@@ -402,9 +622,68 @@ extern "C" mk_status mk_tcdec_step(mk_tcdec *d, const int32_t *d_tokens, int pos
     norm_hilo_kernel<<<B, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(d->final_norm), h, B, H, c.rms_eps);
     lin(h, d->lm_head, ylm, H, V);
     if (st != MK_OK) return st;
-    lm_argmax_kernel<<<B, kArgmaxThreads, 0, s>>>(ylm, d_logits, d_next, B, V, status);
+    lm_argmax_kernel<<<B, kArgmaxThreads, 0, s>>>(ylm, logits ? reinterpret_cast<float *>(d->ws + o.lg) : nullptr,
+                                                  nxt, B, V, status);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: ") + cudaGetErrorString(e));
+    return MK_OK;
+}
+
+// Capture enqueue_step once (per logits / no-logits) into an executable graph.
+static mk_status capture_step(mk_tcdec *d, bool logits) {
+    cudaStream_t cap;
+    cudaError_t e = cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: ") + cudaGetErrorString(e));
+    e = cudaStreamBeginCapture(cap, cudaStreamCaptureModeRelaxed);
+    if (e != cudaSuccess) {
+        cudaStreamDestroy(cap);
+        return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: begin capture: ") + cudaGetErrorString(e));
+    }
+    const mk_status st = enqueue_step(d, cap, logits);
+    cudaGraph_t g = nullptr;
+    e = cudaStreamEndCapture(cap, &g);
+    cudaStreamDestroy(cap);
+    if (st != MK_OK || e != cudaSuccess) {
+        if (g) cudaGraphDestroy(g);
+        return st != MK_OK ? st : tc_fail(d, MK_ERR_CUDA, std::string("tcdec: end capture: ") + cudaGetErrorString(e));
+    }
+    e = cudaGraphInstantiate(&d->exec[logits ? 1 : 0], g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: instantiate: ") + cudaGetErrorString(e));
+    return MK_OK;
+}
+
+extern "C" mk_status mk_tcdec_step(mk_tcdec *d, const int32_t *d_tokens, int pos, int32_t *d_next, float *d_logits,
+                                   void *stream) {
+    if (!d) return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: null context");
+    if (!d->ws) return tc_fail(d, MK_ERR_STATE, "tcdec: mk_tcdec_step before mk_tcdec_bind");
+    const mk_config &c = d->cfg;
+    if (!d_tokens || !d_next) return tc_fail(d, MK_ERR_INVALID, "tcdec: null token buffer");
+    if (pos < 0 || pos >= c.max_seq) return tc_fail(d, MK_ERR_INVALID, "tcdec: position outside the cache");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Layout &o = d->lay;
+    const int B = c.batch;
+    const bool logits = d_logits != nullptr;
+    cudaError_t e = cudaMemcpyAsync(d->ws + o.tok, d_tokens, (size_t)B * 4, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: tokens: ") + cudaGetErrorString(e));
+    set_pos_kernel<<<1, 1, 0, s>>>(reinterpret_cast<int *>(d->ws + o.posw), pos);
+    mk_status st;
+    if (d->use_graph && d->warmed) {
+        if (!d->exec[logits ? 1 : 0]) {
+            st = capture_step(d, logits);
+            if (st != MK_OK) return st;
+        }
+        e = cudaGraphLaunch(d->exec[logits ? 1 : 0], s);
+        if (e != cudaSuccess) return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: graph launch: ") + cudaGetErrorString(e));
+    } else {
+        st = enqueue_step(d, s, logits);  // the first step runs eagerly: it sets the kernels' attributes
+        if (st != MK_OK) return st;
+        d->warmed = true;
+    }
+    e = cudaMemcpyAsync(d_next, d->ws + o.nxt, (size_t)B * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess && logits)
+        e = cudaMemcpyAsync(d_logits, d->ws + o.lg, (size_t)B * c.vocab * 4, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return tc_fail(d, MK_ERR_CUDA, std::string("tcdec: outputs: ") + cudaGetErrorString(e));
     return MK_OK;
 }
 
@@ -421,6 +700,14 @@ extern "C" mk_status mk_tcdec_status(mk_tcdec *d, int *status, void *stream) {
 extern "C" const char *mk_tcdec_last_error(const mk_tcdec *d) { return d ? d->err.c_str() : op_error(); }
 
 extern "C" mk_status mk_tcdec_destroy(mk_tcdec *d) {
+    if (d) drop_graphs(d);
     delete d;
+    return MK_OK;
+}
+
+extern "C" mk_status mk_tcdec_set_graph(mk_tcdec *d, int on) {
+    if (!d) return tc_fail(nullptr, MK_ERR_INVALID, "tcdec: null context");
+    d->use_graph = on != 0;
+    if (!d->use_graph) drop_graphs(d);
     return MK_OK;
 }

@@ -120,6 +120,9 @@ def main(argv=None):
     ap.add_argument("--synthetic-kv", type=int, default=0, metavar="C",
                     help="timing only: instead of a prefill, fill cache positions < C with seeded N(0,1) bf16 "
                          "values and start decoding at position C (the step's cost depends on C, not on the values)")
+    ap.add_argument("--prefill-mode", default="auto", choices=["auto", "steps", "tc"],
+                    help="how the prompt fills the cache: the tensor cores where the plan allows (auto), decode "
+                         "steps, or the tensor cores (tc); the prefill is timed")
     ap.add_argument("--tcdec", action="store_true",
                     help="also time the tensor-core decode step (mk_tcdec_*) on the same cache, at the last position")
     a = ap.parse_args(argv)
@@ -141,7 +144,16 @@ def main(argv=None):
             t[:, :, :, :prefill].normal_(generator=g)
         model.set_position(prefill)
     elif prefill:
-        model.prefill(tokens[:, :prefill].cuda())
+        model.set_prefill(a.prefill_mode)
+        dev_prompt = tokens[:, :prefill].cuda()
+        torch.cuda.synchronize()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record()
+        model.prefill(dev_prompt)
+        p1.record()
+        torch.cuda.synchronize()
+        print(json.dumps({"prefill_tokens": prefill, "batch": B, "prefill_mode": a.prefill_mode,
+                          "prefill_ms": round(p0.elapsed_time(p1), 3)}))
     d_tok = tokens[:, prefill:].t().contiguous().cuda()  # [steps, B]
     for s in range(a.steps - 1):
         model.decode(d_tok[s])

@@ -1,10 +1,14 @@
 """Time mk_linear_tc at the projection shapes of the batched decode configurations.
 
-    python -m tile_synchronised_b200.time_linear [--reps 30]
+    python -m tile_synchronised_b200.time_linear [--reps 30] [--shape B K M ...]
+        [--swiglu-batch B]
 
 Prints one JSON list: per (B, K, M) the K split, the mean microseconds per call
 (CUDA events over back-to-back calls) and the achieved GB/s of the weights plus
 x and y.  Weight copies are rotated so that the timed set exceeds the 126 MB L2.
+--shape (repeatable) replaces the default shapes; --swiglu-batch also times the
+tensor-core fused SwiGLU first stage (MK_SWIGLU_TC) at the 70B-shard shape.
+Also the command that ncu profiles the tensor-core kernels under.
 """
 import argparse
 import json
@@ -25,9 +29,12 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--reps", type=int, default=30)
     ap.add_argument("--peak-gbs", type=float, default=6550.4, help="the measured HBM copy bandwidth")
+    ap.add_argument("--shape", type=int, nargs=3, action="append", metavar=("B", "K", "M"),
+                    help="time this (batch, K, M) instead of the default shapes (repeatable)")
+    ap.add_argument("--swiglu-batch", type=int, default=0, help="also time MK_SWIGLU_TC at this batch")
     a = ap.parse_args(argv)
     res = []
-    for (B, K, M) in SHAPES:
+    for (B, K, M) in (a.shape or SHAPES):
         x, w = synth.make_linear_inputs(B, K, M, device="cuda")
         wb = M * K * 2
         ncopy = max(1, -(-300_000_000 // wb))
@@ -47,6 +54,24 @@ def main(argv=None):
         res.append({"B": B, "K": K, "M": M, "split": mk.linear_tc_split(B, K, M), "us": round(us, 2),
                     "GBps": round(gbs, 1), "frac": round(gbs / a.peak_gbs, 3)})
         del ws
+    if a.swiglu_batch:
+        B = a.swiglu_batch
+        x, wg, wu = synth.make_swiglu_inputs(B, device="cuda")
+        out = torch.empty((B, wg.shape[1]), dtype=torch.float16, device="cuda")
+        for i in range(3):
+            mk.swiglu_stage1(x, wg, wu, out=out, variant=mk.MK_SWIGLU_TC)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(a.reps):
+            mk.swiglu_stage1(x, wg, wu, out=out, variant=mk.MK_SWIGLU_TC)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / a.reps
+        K, N = wg.shape
+        gbs = (2 * K * N * 2 + B * K * 2 + B * N * 2) / us / 1e3
+        res.append({"swiglu_tc_B": B, "K": K, "N": N, "us": round(us, 2), "GBps": round(gbs, 1),
+                    "frac": round(gbs / a.peak_gbs, 3)})
     print(json.dumps(res))
 
 
