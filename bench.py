@@ -43,7 +43,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
-    ap.add_argument("--variant", default="megakernel", choices=["megakernel", "graph", "graph_pdl", "tilesync"])
+    ap.add_argument("--variant", default="megakernel",
+                    choices=["megakernel", "graph", "graph_pdl", "tilesync", "tensor_cores"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true", help="skip timing the separate-kernel variants")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
@@ -232,7 +233,15 @@ def run_mk(args, world, rank, local):
     model.prefill(tokens[:, :PREFILL].cuda())
     win = tokens[0, PREFILL:].contiguous().cuda()  # teacher-forced inputs, resident in HBM
     stream = torch.cuda.current_stream()
-    launches_per_step = {"megakernel": 1}.get(args.variant, model.info()["n_phases"])
+    if args.variant == "megakernel":
+        launches_per_step = 1
+    elif args.variant == "tensor_cores":
+        # per pass of up to 32 sequences: embed, rows, 13 per layer (norm, QKV GEMM, q/k/v post, 2 attention,
+        # cast, O GEMM, residual, norm, gate/up GEMM, SiLU*mul, down GEMM, residual), final norm, LM GEMM,
+        # argmax; then the position advance
+        launches_per_step = ((B + 31) // 32) * (2 + 13 * shape.n_layers + 3) + 1
+    else:
+        launches_per_step = model.info()["n_phases"]
 
     def run_steps(n, start, e2e=None):
         rewinds = 0
@@ -300,7 +309,7 @@ def run_mk(args, world, rank, local):
     # the same ops as separate kernels in a CUDA graph (with and without PDL)
     variants = {}
     if not args.no_variants:
-        for v in ("megakernel", "graph", "graph_pdl", "tilesync"):
+        for v in ("megakernel", "graph", "graph_pdl", "tilesync", "tensor_cores"):
             if v == args.variant:
                 variants[v] = {"tokens_per_s": round(value / world, 2), "ms_per_step": round(ms_per_step, 5)}
                 continue

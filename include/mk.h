@@ -57,7 +57,7 @@ enum {
     MK_GRAPH = 1,      /* the same ops as one launch per op, replayed from a CUDA graph */
     MK_GRAPH_PDL = 2,  /* as MK_GRAPH, launches chained by programmatic dependent launch so
                           each op streams its weights while the previous op finishes */
-    MK_GRAPH_TILESYNC = 3 /* the ops as separate kernels in the same CUDA graph, each
+    MK_GRAPH_TILESYNC = 3, /* the ops as separate kernels in the same CUDA graph, each
                           launched early by programmatic dependent launch and started
                           on the tiles it reads instead of on the previous kernel's
                           end ("MegaOps: A Kernel Overlapping Framework ...", "In plain
@@ -68,6 +68,12 @@ enum {
                           read.  A kernel launches only after every CTA of the one
                           before it has started, so what it waits for is always
                           running; every wait is bounded. */
+    MK_TENSOR_CORES = 4   /* the same step with every projection a tcgen05 GEMM over the
+                          packed weights (up to 32 sequences a pass, each activation row
+                          a hi/lo pair of bf16 rows), attention per sequence, the LM
+                          head and the argmax; replayed from a CUDA graph.  The batched
+                          counterpart of the megakernel, whose CUDA-core GEMVs turn
+                          arithmetic-bound as the batch grows. */
 };
 /* How the megakernel's dependent instructions learn that their inputs are
  * ready ("MegaOps: A Kernel Overlapping Framework ...", "In plain words": a
@@ -97,7 +103,7 @@ typedef struct {
     int batch;           /* sequences decoded together, 1..64 */
     int max_seq;         /* KV cache positions per sequence */
     int dtype;           /* MK_BF16 (the only one) */
-    int variant;         /* MK_MEGAKERNEL | MK_GRAPH | MK_GRAPH_PDL | MK_GRAPH_TILESYNC */
+    int variant;         /* MK_MEGAKERNEL | MK_GRAPH | MK_GRAPH_PDL | MK_GRAPH_TILESYNC | MK_TENSOR_CORES */
     int num_sms;         /* CTAs of the persistent kernel; 0 = the device's SM count */
 } mk_config;
 
@@ -150,21 +156,18 @@ mk_status mk_load_weights(mk_ctx *ctx, const mk_weights *w, void *workspace, voi
 
 /* Fill the KV cache from a prompt: `d_tokens` is a device int32 [batch, T]
  * row-major array; positions restart at 0 and end at T.  With the tensor-core
- * prefill (the default where the plan allows it, see mk_set_prefill) the
- * prompt goes through the decoder 32 positions of one sequence at a time:
- * every projection is one tcgen05 GEMM over the packed weights, with each
- * activation row entering as a hi/lo pair of bf16 rows, and position t
- * attends causally to positions 0 .. t; only the KV cache is kept (the last
- * layer stops after its K/V rows).  Otherwise it runs T decode steps whose
- * outputs are discarded.  A token outside [0, vocab) is reported by
+ * prefill (the default, see mk_set_prefill) the prompt goes through the
+ * decoder 32 positions of one sequence at a time: every projection is one
+ * tcgen05 GEMM reading the packed weight tiles of mk_load_weights in place,
+ * with each activation row entering as a hi/lo pair of bf16 rows, and
+ * position t attends causally to positions 0 .. t; only the KV cache is kept
+ * (the last layer stops after its K/V rows).  Otherwise it runs T decode
+ * steps whose outputs are discarded.  A token outside [0, vocab) is reported by
  * mk_get_status as for mk_decode_step.  MK_ERR_INVALID if T < 1 or
  * T > max_seq. */
 mk_status mk_prefill_kv(mk_ctx *ctx, const int32_t *d_tokens, int batch, int T, void *stream);
-/* How mk_prefill_kv runs: MK_PREFILL_AUTO (default: the tensor cores when every
- * packed layer matrix is a single K block, i.e. the plan does not split a
- * projection's K to fit its activations in shared memory; else decode steps),
- * MK_PREFILL_STEPS (one decode step per position) or MK_PREFILL_TC
- * (MK_ERR_UNSUPPORTED when the plan does not allow it).  Host only. */
+/* How mk_prefill_kv runs: MK_PREFILL_AUTO (default) and MK_PREFILL_TC, the
+ * tensor cores; MK_PREFILL_STEPS, one decode step per position.  Host only. */
 enum { MK_PREFILL_AUTO = 0, MK_PREFILL_STEPS = 1, MK_PREFILL_TC = 2 };
 mk_status mk_set_prefill(mk_ctx *ctx, int mode);
 
@@ -197,7 +200,7 @@ mk_status mk_get_position(const mk_ctx *ctx, int *pos);
 mk_status mk_set_position(mk_ctx *ctx, int pos, void *stream);
 
 /* Select the execution variant for later decode steps (MK_MEGAKERNEL,
- * MK_GRAPH, MK_GRAPH_PDL or MK_GRAPH_TILESYNC). */
+ * MK_GRAPH, MK_GRAPH_PDL, MK_GRAPH_TILESYNC or MK_TENSOR_CORES). */
 mk_status mk_set_variant(mk_ctx *ctx, int variant);
 
 /* One-time profiling pass ("Deep Kernel Fusion for Transformers", Summary and

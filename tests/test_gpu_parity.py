@@ -303,11 +303,11 @@ def handoff_step(shape, host, model, tokens, pos, seqs):
             assert np.max(np.abs(gk - orc.kc[l, 0, :, pos])) <= 2e-2 * np.max(np.abs(orc.kc[l, 0, :, pos]))
 
 
-def full_size_case(shape, batch, prefill, extra_steps, seqs, max_seq=None):
+def full_size_case(shape, batch, prefill, extra_steps, seqs, max_seq=None, variant="megakernel"):
     import tile_synchronised_b200 as mk
     ms = max_seq or shape.max_seq
     tw = synth.make_weights(shape, device="cuda")
-    model = mk.Model(shape, tw, batch=batch, max_seq=ms)
+    model = mk.Model(shape, tw, batch=batch, max_seq=ms, variant=variant)
     tokens = synth.make_tokens(shape, prefill + extra_steps + 1, batch=batch)
     tnp = tokens.numpy()
     model.prefill(tokens[:, :prefill].cuda())
@@ -353,6 +353,29 @@ def test_llama1b_handoffs_across_the_benched_window():
 def test_llama8b_full_size_handoff(batch, seqs):
     s = synth.LLAMA8B
     full_size_case(s, batch, s.prefill, 4, seqs)
+
+
+@needs_cuda
+@pytest.mark.parametrize("name,batch,prefill,seqs", [("llama8b", 32, 512, [0, 31]), ("qwen3_8b", 16, 1024, [0, 15]),
+                                                     ("llama1b", 1, 1024, [0])])
+def test_tensor_core_variant_full_size_handoff(name, batch, prefill, seqs):
+    """The decode step with every projection on the tensor cores over the
+    packed weights (MK_TENSOR_CORES), after a tensor-core prefill: a few steps
+    (the first launched directly, the second captured, the rest replayed from
+    the graph), then a full-depth oracle handoff of the first and last
+    sequence."""
+    s = synth.MODELS[name]
+    full_size_case(s, batch, prefill, 3, seqs, max_seq=prefill + 8, variant="tensor_cores")
+
+
+@needs_cuda
+@pytest.mark.parametrize("batch", [1, 3])
+def test_tensor_core_variant_trajectory(batch):
+    s = synth.TINY.replace(batch=batch)
+    tw, model, orc = build_pair(s, batch=batch, variant="tensor_cores")
+    tokens = synth.make_tokens(s, 40, batch=batch)
+    worst, undecided = run_trajectory(model, orc, tokens, 24, 16)
+    assert undecided <= 6 * batch, (undecided, worst)
 
 
 @needs_cuda
@@ -497,19 +520,24 @@ def test_swiglu_stage1_full_size(B):
 
 # ---------------------------------------------------------------- the prefill on the tensor cores
 @needs_cuda
-@pytest.mark.parametrize("case", ["tiny_b1", "tiny_b3_qknorm", "llama1b"])
+@pytest.mark.parametrize("case", ["tiny_b1", "tiny_b3_qknorm", "tiny_b4_ksplit", "llama1b"])
 def test_tensor_core_prefill_matches_steps_and_oracle(case):
     """The tensor-core prefill (32 positions of a sequence per GEMM chunk,
     causal attention within the chunk) leaves a KV cache that agrees with the
     one the decode steps leave and with the oracle's, and the decode step that
     follows it matches the oracle.  The prompt lengths cover one ragged chunk
-    and several chunks with a ragged tail."""
+    and several chunks with a ragged tail; one plan packs a matrix as several
+    K blocks."""
     import tile_synchronised_b200 as mk
     from tile_synchronised_b200 import _lib
     if case == "llama1b":
         s, B, T = synth.LLAMA1B, 1, 100
     elif case == "tiny_b1":
         s, B, T = synth.TINY, 1, 21
+    elif case == "tiny_b4_ksplit":
+        # 4 rows x 5120 fp32 exceed the 64 KB activation region: the plan
+        # packs the down projection as two K blocks, read by a 4-D tensor map
+        s, B, T = synth.TINY.replace(intermediate=5120), 4, 40
     else:
         s, B, T = synth.TINY.replace(qk_norm=True, rms_eps=1e-6), 3, 70
     ms = T + 4

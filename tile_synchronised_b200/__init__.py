@@ -10,13 +10,14 @@ import ctypes as C
 
 import torch
 
-from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_GRAPH_TILESYNC, MK_MEGAKERNEL, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW,
+from ._lib import (MK_GRAPH, MK_GRAPH_PDL, MK_GRAPH_TILESYNC, MK_MEGAKERNEL, MK_TENSOR_CORES, MK_SWIGLU_AUTO, MK_SWIGLU_COL, MK_SWIGLU_ROW,
                    MK_SWIGLU_TC, MK_SYNC_COUNTERS, MK_SYNC_TAGS, MkConfig, MkError, MkWeights, check, load)
 
 __all__ = ["Model", "TcDecoder", "swiglu_stage1", "swiglu_tune", "linear_tc", "linear_tc_split", "MkError", "VARIANTS",
            "MK_SWIGLU_AUTO", "MK_SWIGLU_ROW", "MK_SWIGLU_COL", "MK_SWIGLU_TC", "load"]
 
-VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL, "tilesync": MK_GRAPH_TILESYNC}
+VARIANTS = {"megakernel": MK_MEGAKERNEL, "graph": MK_GRAPH, "graph_pdl": MK_GRAPH_PDL, "tilesync": MK_GRAPH_TILESYNC,
+            "tensor_cores": MK_TENSOR_CORES}
 SYNCS = {"tags": MK_SYNC_TAGS, "counters": MK_SYNC_COUNTERS}
 PREFILLS = {"auto": 0, "steps": 1, "tc": 2}
 SCHEDULE_FIELDS = ("n_instructions", "n_ctas", "n_counters", "n_phases", "batch_rows", "attention_chunks",

@@ -12,7 +12,7 @@ from . import build as _build
 
 MK_OK, MK_ERR_INVALID, MK_ERR_CUDA, MK_ERR_TIMEOUT, MK_ERR_UNSUPPORTED, MK_ERR_STATE = 0, -1, -2, -3, -4, -5
 MK_BF16 = 0
-MK_MEGAKERNEL, MK_GRAPH, MK_GRAPH_PDL, MK_GRAPH_TILESYNC = 0, 1, 2, 3
+MK_MEGAKERNEL, MK_GRAPH, MK_GRAPH_PDL, MK_GRAPH_TILESYNC, MK_TENSOR_CORES = 0, 1, 2, 3, 4
 MK_SWIGLU_AUTO, MK_SWIGLU_ROW, MK_SWIGLU_COL, MK_SWIGLU_TC = 0, 1, 2, 3
 MK_SYNC_TAGS, MK_SYNC_COUNTERS = 0, 1
 MK_PREFILL_AUTO, MK_PREFILL_STEPS, MK_PREFILL_TC = 0, 1, 2

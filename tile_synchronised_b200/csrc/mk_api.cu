@@ -39,6 +39,10 @@ struct mk_ctx {
     std::vector<cudaGraphNode_t> gnodes;  // kernel node of each phase
     const void *g_tok = nullptr, *g_next = nullptr, *g_logits = nullptr;
     int g_variant = -1;
+    // captured decode step on the tensor cores (MK_TENSOR_CORES)
+    cudaGraphExec_t tc_exec = nullptr;
+    const float *tc_logits = nullptr;
+    bool tc_warmed = false;
 };
 
 static mk_status fail(mk_ctx *c, mk_status s, const std::string &msg) {
@@ -55,6 +59,8 @@ static mk_status cuda_fail(mk_ctx *c, cudaError_t e, const char *where) {
     } while (0)
 
 static void drop_graph(mk_ctx *c) {
+    if (c->tc_exec) cudaGraphExecDestroy(c->tc_exec);
+    c->tc_exec = nullptr;
     if (c->gexec) cudaGraphExecDestroy(c->gexec);
     if (c->graph) cudaGraphDestroy(c->graph);
     c->gexec = nullptr;
@@ -453,6 +459,9 @@ static mk_status retarget_graph(mk_ctx *c, const int32_t *tok, int32_t *next, fl
     return MK_OK;
 }
 
+static mk_status decode_tensor_cores(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, float *d_logits,
+                                     cudaStream_t s);
+
 mk_status mk_decode_step(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, float *d_logits, void *stream) {
     if (!c) return MK_ERR_INVALID;
     if (!c->loaded) return fail(c, MK_ERR_STATE, "mk_decode_step before mk_load_weights");
@@ -463,6 +472,8 @@ mk_status mk_decode_step(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, fl
     mk_status st;
     if (c->variant == MK_MEGAKERNEL) {
         st = launch_megakernel(c, d_tokens, 1, d_next, d_logits, s);
+    } else if (c->variant == MK_TENSOR_CORES) {
+        st = decode_tensor_cores(c, d_tokens, d_next, d_logits, s);
     } else {
         if (!c->gexec || c->g_variant != c->variant) {
             drop_graph(c);
@@ -504,10 +515,9 @@ mk_status mk_decode_step(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, fl
     return st;
 }
 
-// The prefill on the tensor cores: every position of the prompt of every
-// sequence goes through the decoder in chunks of kPrefillRows positions, each
-// projection one GEMM over the packed weights (mk_tcdec.cu, prefill_tc).
-static mk_status prefill_tensor_cores(mk_ctx *c, const int32_t *d_tokens, int T, cudaStream_t s) {
+// The row passes on the tensor cores (mk_tcdec.cu) over this context's
+// packed weights, cache and scratch region.
+static PrefillTc tc_args(mk_ctx *c) {
     const Plan &p = c->plan;
     const mk_config &g = p.cfg;
     PrefillTc a{};
@@ -517,18 +527,81 @@ static mk_status prefill_tensor_cores(mk_ctx *c, const int32_t *d_tokens, int T,
     a.theta = (double)g.rope_theta;
     a.embed = c->embed;
     a.layers = c->lw.data();
-    a.qkv_kc = p.qkv.kc; a.qkv_M = p.qkv.tiles * p.qkv.rows;
-    a.o_kc = p.o.kc; a.o_M = p.o.tiles * p.o.rows;
-    a.gu_kc = p.gu.kc; a.gu_M = p.gu.tiles * p.gu.rows; a.gu_rows = p.gu.rows;
-    a.down_kc = p.down.kc; a.down_M = p.down.tiles * p.down.rows;
+    a.qkv = p.qkv;
+    a.o = p.o;
+    a.gu = p.gu;
+    a.down = p.down;
+    a.lm = p.lm;
+    a.lm_w = c->ws + p.lm.offset;
+    a.final_norm = c->ws + p.off_norms + (size_t)g.n_layers * (2 * g.hidden + 2 * g.head_dim) * 2;
     a.kcache = reinterpret_cast<uint16_t *>(c->kv);
     a.vcache = reinterpret_cast<uint16_t *>(c->kv + p.kv_bytes / 2);
     a.state = reinterpret_cast<State *>(c->ws + p.off_state);
     a.scratch = c->ws + p.off_prefill;
     a.scratch_bytes = p.prefill_bytes;
+    return a;
+}
+
+// The prefill on the tensor cores: every position of the prompt of every
+// sequence goes through the decoder in chunks of kPrefillRows positions, each
+// projection one GEMM over the packed weights (mk_tcdec.cu, prefill_tc).
+static mk_status prefill_tensor_cores(mk_ctx *c, const int32_t *d_tokens, int T, cudaStream_t s) {
+    const Plan &p = c->plan;
+    const PrefillTc a = tc_args(c);
     const std::string err = prefill_tc(a, d_tokens, T, s);
     if (!err.empty()) return fail(c, MK_ERR_CUDA, "mk_prefill_kv (tensor cores): " + err);
     CK(launch_set_position(reinterpret_cast<State *>(c->ws + p.off_state), T, s));
+    return MK_OK;
+}
+
+// One decode step on the tensor cores (MK_TENSOR_CORES).  The step's launches
+// read the position from the device state and the tokens from the scratch's
+// token row, so the first call runs them directly (setting the kernels'
+// attributes) and the next captures them once into a CUDA graph that every
+// later call replays: a token copy in, the graph, the argmax copy out.  The
+// logits pointer is part of the capture; a different one captures again.
+static mk_status decode_tensor_cores(mk_ctx *c, const int32_t *d_tokens, int32_t *d_next, float *d_logits,
+                                     cudaStream_t s) {
+    const PrefillTc a = tc_args(c);
+    const int B = c->plan.cfg.batch;
+    int32_t *tok = decode_tc_tokens(a), *nxt = decode_tc_next(a);
+    if (!tok || !nxt) return fail(c, MK_ERR_STATE, "tensor-core decode: no scratch region");
+    CK(cudaMemcpyAsync(tok, d_tokens, (size_t)B * 4, cudaMemcpyDeviceToDevice, s));
+    if (!c->tc_warmed || c->tc_exec == nullptr || c->tc_logits != d_logits) {
+        if (c->tc_exec) {
+            cudaGraphExecDestroy(c->tc_exec);
+            c->tc_exec = nullptr;
+        }
+        if (!c->tc_warmed) {
+            const std::string err = decode_tc(a, tok, nxt, d_logits, s);
+            if (!err.empty()) return fail(c, MK_ERR_CUDA, "tensor-core decode: " + err);
+            c->tc_warmed = true;
+        } else {
+            cudaStream_t cap;
+            CK(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
+            cudaError_t e = cudaStreamBeginCapture(cap, cudaStreamCaptureModeRelaxed);
+            if (e != cudaSuccess) {
+                cudaStreamDestroy(cap);
+                return cuda_fail(c, e, "cudaStreamBeginCapture");
+            }
+            const std::string err = decode_tc(a, tok, nxt, d_logits, cap);
+            cudaGraph_t graph = nullptr;
+            e = cudaStreamEndCapture(cap, &graph);
+            cudaStreamDestroy(cap);
+            if (!err.empty() || e != cudaSuccess) {
+                if (graph) cudaGraphDestroy(graph);
+                return fail(c, MK_ERR_CUDA, "tensor-core decode capture: " + (err.empty() ? std::string(cudaGetErrorString(e)) : err));
+            }
+            e = cudaGraphInstantiate(&c->tc_exec, graph, 0);
+            cudaGraphDestroy(graph);
+            if (e != cudaSuccess) return cuda_fail(c, e, "cudaGraphInstantiate");
+            c->tc_logits = d_logits;
+            CK(cudaGraphLaunch(c->tc_exec, s));
+        }
+    } else {
+        CK(cudaGraphLaunch(c->tc_exec, s));
+    }
+    if (d_next) CK(cudaMemcpyAsync(d_next, nxt, (size_t)B * 4, cudaMemcpyDeviceToDevice, s));
     return MK_OK;
 }
 
@@ -547,9 +620,6 @@ mk_status mk_prefill_kv(mk_ctx *c, const int32_t *d_tokens, int batch, int T, vo
         c->pos = T;
         return MK_OK;
     }
-    if (c->prefill == MK_PREFILL_TC)
-        return fail(c, MK_ERR_UNSUPPORTED, "mk_prefill_kv: this plan splits a projection's K, so the tensor-core "
-                                           "prefill cannot read its packed weights");
     CK(cudaMemsetAsync(c->ws + p.off_state + offsetof(State, pos), 0, 4, s));
     c->pos = 0;
     int32_t *scratch = reinterpret_cast<int32_t *>(c->ws + p.off_next_scratch);
@@ -565,8 +635,6 @@ mk_status mk_set_prefill(mk_ctx *c, int mode) {
     if (!c) return MK_ERR_INVALID;
     if (mode != MK_PREFILL_AUTO && mode != MK_PREFILL_STEPS && mode != MK_PREFILL_TC)
         return fail(c, MK_ERR_INVALID, "unknown prefill mode");
-    if (mode == MK_PREFILL_TC && !c->plan.prefill_tc)
-        return fail(c, MK_ERR_UNSUPPORTED, "mk_set_prefill: this plan splits a projection's K (no tensor-core prefill)");
     c->prefill = mode;
     return MK_OK;
 }
@@ -624,7 +692,7 @@ mk_status mk_set_position(mk_ctx *c, int pos, void *stream) {
 
 mk_status mk_set_variant(mk_ctx *c, int variant) {
     if (!c) return MK_ERR_INVALID;
-    if (variant < MK_MEGAKERNEL || variant > MK_GRAPH_TILESYNC) return fail(c, MK_ERR_INVALID, "unknown variant");
+    if (variant < MK_MEGAKERNEL || variant > MK_TENSOR_CORES) return fail(c, MK_ERR_INVALID, "unknown variant");
     c->variant = variant;
     return MK_OK;
 }

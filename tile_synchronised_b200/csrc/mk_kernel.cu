@@ -414,12 +414,16 @@ __device__ __noinline__ bool ll_spin_chunks(const KParams &P, const SmemLayout &
         __nanosleep(16);
         for (int j = 0; j < m; ++j) {
             if (!((pending >> j) & 1u)) continue;
+            // the chunk's four loads go out together, before any value is kept
+            ulonglong2 w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) w[q] = ll_ld2(base[j] + 2 * q);
             bool all = true;
+#pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const ulonglong2 w = ll_ld2(base[j] + 2 * q);
-                all = all && ll_tag(w.x) == tag && ll_tag(w.y) == tag;
-                vals[8 * j + 2 * q] = ll_value(w.x);
-                vals[8 * j + 2 * q + 1] = ll_value(w.y);
+                all = all && ll_tag(w[q].x) == tag && ll_tag(w[q].y) == tag;
+                vals[8 * j + 2 * q] = ll_value(w[q].x);
+                vals[8 * j + 2 * q + 1] = ll_value(w[q].y);
             }
             if (all) pending &= ~(1u << j);
         }

@@ -30,6 +30,11 @@ cudaError_t launch_swiglu_tc(const void *x, const void *wg, const void *wu, void
 cudaError_t launch_attention_dev(const float *q, const void *k, const void *v, int B, int nq, int nkv, int d,
                                  int max_seq, const int *n_pos_dev, int chunks, float *out, float *part,
                                  cudaStream_t s);
+// y[b][m] = sum_k W[m][k] x[b][k] on the tensor cores (mk_linear_tc.cu) with W
+// one of the megakernel's packed matrices, [tiles][K / kc][rows][kc] bf16, and
+// x bf16 [B][K] (K = the packed width, zero past the logical one).
+cudaError_t launch_linear_tc_packed(const void *x, const void *w, float *y, int B, int K, int M, int kc, int rows,
+                                    cudaStream_t s);
 // Causal attention of prefill rows (mk_attn.cu): row r of q / out attends
 // positions 0 .. row_len[r] - 1 of sequence row_seq[r] of one layer's cache.
 cudaError_t launch_attention_rows(const float *q, const void *k, const void *v, int rows, int nq, int nkv, int d,
@@ -37,16 +42,16 @@ cudaError_t launch_attention_rows(const float *q, const void *k, const void *v, 
                                   float *part, cudaStream_t s);
 // The tensor-core prefill of a megakernel context (mk_tcdec.cu): positions
 // 0 .. T-1 of every sequence through the decoder in chunks of kPrefillRows,
-// every projection one mk_linear_tc call over the packed weights, which must
-// each be a single K block (plain row-major [rows, kc]).  Fills the KV cache
-// only.
+// every projection one tensor-core GEMM over the packed weights.  Fills the KV
+// cache only.
 struct PrefillTc {
     int L, H, nq, nkv, d, I, V, B, max_seq, qk_norm;
     float eps;
     double theta;
     const void *embed;
     const LayerW *layers;  // host array of the L layers' device pointers
-    int qkv_kc, qkv_M, o_kc, o_M, gu_kc, gu_M, gu_rows, down_kc, down_M;
+    PackedMat qkv, o, gu, down, lm;  // the packed matrices' geometry
+    const void *lm_w, *final_norm;  // the packed LM head and the final norm gains
     uint16_t *kcache, *vcache;
     State *state;
     uint8_t *scratch;
@@ -55,6 +60,14 @@ struct PrefillTc {
 size_t prefill_scratch_bytes(int H, int nq, int d, int kmax, int mmax);
 // Returns an empty string, or the reason it stopped.
 std::string prefill_tc(const PrefillTc &a, const int32_t *tokens, int T, cudaStream_t s);
+// One decode step of every sequence at the context's current position (read
+// on the device from a.state, then advanced) through the same row pass, plus
+// the final norm, the LM head and the argmax: the megakernel's step on the
+// tensor cores.  tokens [B] in; next [B] (and logits [B][V] if set) out.
+std::string decode_tc(const PrefillTc &a, const int32_t *tokens, int32_t *next, float *logits, cudaStream_t s);
+// The scratch's own token and argmax rows (a captured step copies through them).
+int32_t *decode_tc_tokens(const PrefillTc &a);
+int32_t *decode_tc_next(const PrefillTc &a);
 // Last error of a context-free call (the isolated operations) on this thread.
 void set_op_error(const char *msg);
 const char *op_error();

@@ -42,6 +42,7 @@ constexpr int kLinMaxB = 64;
 struct LinShape {
     int Bp, rows, K, M, stages;      // Bp: the MMA's N (B rounded up to 16); rows: B
     uint32_t stage_bytes, a_bytes;  // a stage is the W box then the x box
+    int w_kc, w_rows;               // W packed as [tiles][K / w_kc][w_rows][w_kc] (4-D map), or w_kc = 0: row-major
 };
 
 // Instruction descriptor of kind::f16: fp32 accumulate, bf16 A and B, both
@@ -102,7 +103,10 @@ __global__ void __launch_bounds__(kLinThreads, 1)
             uint8_t *st = smem + (size_t)s * sh.stage_bytes;
             mbar_arrive_expect_tx(&full[s], sh.stage_bytes);  // rows past M or B arrive as zeros and count
             const int k0 = (kb_first + kb) * kLinBK;
-            tma_load_2d(st, &map_w, k0, m0, &full[s]);
+            if (sh.w_kc)
+                tma_load_4d(st, &map_w, k0 % sh.w_kc, 0, k0 / sh.w_kc, m0 / sh.w_rows, &full[s]);
+            else
+                tma_load_2d(st, &map_w, k0, m0, &full[s]);
             tma_load_2d(st + sh.a_bytes, &map_x, k0, 0, &full[s]);
             issued = kb + 1;
         }
@@ -213,12 +217,20 @@ static bool lin_plan(int B, int K, int M, LinPlan &p) {
     return true;
 }
 
-cudaError_t launch_linear_tc(const void *x, const void *w, float *y, int B, int K, int M, cudaStream_t s) {
+// w_kc > 0: W is packed as [tiles][K / w_kc][w_rows][w_kc] (tiles = M / w_rows
+// rounded up), read through a 4-D tensor map; else W is row-major [M, K].
+static cudaError_t launch_linear(const void *x, const void *w, float *y, int B, int K, int M, int w_kc, int w_rows,
+                                 cudaStream_t s) {
     LinPlan p;
     if (!lin_plan(B, K, M, p)) return cudaErrorInvalidValue;
+    if (w_kc && (w_kc % kLinBK || K % w_kc || w_rows < 1 || kLinM % w_rows)) return cudaErrorInvalidValue;
+    p.sh.w_kc = w_kc;
+    p.sh.w_rows = w_rows;
     CUtensorMap mw, mx;
-    if (!tc_make_map(&mw, w, (uint64_t)M, (uint64_t)K, kLinBK, kLinM) ||
-        !tc_make_map(&mx, x, (uint64_t)B, (uint64_t)K, kLinBK, (uint32_t)p.sh.Bp))
+    const bool wmap = w_kc ? tc_make_map_packed(&mw, w, (uint64_t)((M + w_rows - 1) / w_rows), (uint32_t)(K / w_kc),
+                                                (uint32_t)w_rows, (uint32_t)w_kc)
+                           : tc_make_map(&mw, w, (uint64_t)M, (uint64_t)K, kLinBK, kLinM);
+    if (!wmap || !tc_make_map(&mx, x, (uint64_t)B, (uint64_t)K, kLinBK, (uint32_t)p.sh.Bp))
         return cudaErrorInvalidValue;
     static std::atomic<unsigned long long> configured{0};
     const cudaError_t ce = tc_allow_smem(reinterpret_cast<const void *>(linear_tc_kernel), 227 * 1024, configured);
@@ -236,6 +248,15 @@ cudaError_t launch_linear_tc(const void *x, const void *w, float *y, int B, int 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, linear_tc_kernel, mw, mx, y, p.sh);
+}
+
+cudaError_t launch_linear_tc(const void *x, const void *w, float *y, int B, int K, int M, cudaStream_t s) {
+    return launch_linear(x, w, y, B, K, M, 0, 0, s);
+}
+
+cudaError_t launch_linear_tc_packed(const void *x, const void *w, float *y, int B, int K, int M, int kc, int rows,
+                                    cudaStream_t s) {
+    return launch_linear(x, w, y, B, K, M, kc, rows, s);
 }
 
 }  // namespace mk

@@ -68,7 +68,7 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
     if (c.batch > 64) return bad(MK_ERR_UNSUPPORTED, "batch above 64");
     if (c.max_seq > (1 << 20)) return bad(MK_ERR_UNSUPPORTED, "max_seq above 2^20");
     if (n_ctas > 1024) return bad(MK_ERR_UNSUPPORTED, "more than 1024 CTAs");
-    if (c.variant < MK_MEGAKERNEL || c.variant > MK_GRAPH_TILESYNC) return bad(MK_ERR_INVALID, "unknown variant");
+    if (c.variant < MK_MEGAKERNEL || c.variant > MK_TENSOR_CORES) return bad(MK_ERR_INVALID, "unknown variant");
 
     const int L = c.n_layers, H = c.hidden, nq = c.n_heads, nkv = c.n_kv_heads, d = c.head_dim;
     const int I = c.intermediate, V = c.vocab, B = c.batch;
@@ -312,11 +312,14 @@ mk_status build_plan(const mk_config &c, int n_ctas, int swiglu_variant, Plan &p
                            align_up(mat_bytes(p.gu), 256) + align_up(mat_bytes(p.down), 256);
     p.off_weights = take((size_t)L * p.layer_weight_bytes);
     p.off_lm = take(mat_bytes(p.lm));
-    p.prefill_tc = p.qkv.nkb == 1 && p.o.nkb == 1 && p.gu.nkb == 1 && p.down.nkb == 1;
+    p.prefill_tc = true;  // the tensor cores read every packed matrix (4-D tensor map over its tiles)
     if (p.prefill_tc) {
-        const int kmax = std::max({p.qkv.kc, p.o.kc, p.gu.kc, p.down.kc});
+        // (also the buffers of the decode step on the tensor cores, whose LM
+        // head is the widest GEMM output)
+        const int kmax = std::max({p.qkv.nkb * p.qkv.kc, p.o.nkb * p.o.kc, p.gu.nkb * p.gu.kc, p.down.nkb * p.down.kc,
+                                   p.lm.nkb * p.lm.kc});
         const int mmax = std::max({p.qkv.tiles * p.qkv.rows, p.o.tiles * p.o.rows, p.gu.tiles * p.gu.rows,
-                                   p.down.tiles * p.down.rows});
+                                   p.down.tiles * p.down.rows, p.lm.tiles * p.lm.rows});
         p.prefill_bytes = prefill_scratch_bytes(H, nq, d, kmax, mmax);
         p.off_prefill = take(p.prefill_bytes);
     }

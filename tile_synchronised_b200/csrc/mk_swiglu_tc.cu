@@ -356,6 +356,18 @@ bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool tc_make_map_packed(CUtensorMap *m, const void *base, uint64_t tiles, uint32_t nkb, uint32_t rows, uint32_t kc) {
+    EncodeTiled enc = encode_fn();
+    if (!enc || rows < 1 || rows > 128 || 128 % rows || kc % 64) return false;
+    const cuuint64_t dims[4] = {kc, rows, nkb, tiles};
+    const cuuint64_t strides[3] = {(cuuint64_t)kc * 2, (cuuint64_t)rows * kc * 2, (cuuint64_t)nkb * rows * kc * 2};
+    const cuuint32_t box[4] = {64, rows, 1, 128 / rows};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool swiglu_tc_supported(int B, int K, int N) {
     return B >= 1 && B <= 128 && K % (kTcBK * kTcSplit) == 0 && N % kTcM == 0;
 }

@@ -41,6 +41,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// 4-D tile of a tensor map: coordinates innermost first.
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];" ::"r"(smem_addr(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_addr(bar))
+        : "memory");
+}
+
 // Bounded wait for the phase `parity` of an mbarrier; false after the time
 // limit or once another role of the CTA has given up.
 __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
@@ -133,5 +143,12 @@ inline cudaError_t tc_allow_smem(const void *fn, int bytes, std::atomic<unsigned
 // missing or refuses the map.
 bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                  uint32_t box_rows, bool swizzle = true);
+// A matrix packed as [tiles][nkb][rows][kc] 2-byte elements (the decode
+// megakernel's weight tiles: `rows` rows of K block kb of tile t contiguous)
+// as a 4-D tensor (kc, rows, nkb, tiles), with a box of 64 columns of 128 /
+// rows consecutive tiles, i.e. 128 consecutive matrix rows x 64 columns laid
+// out in shared memory exactly as a 2-D box of a row-major matrix, 128-byte
+// swizzled.  kc a multiple of 64, rows a power of two <= 128.
+bool tc_make_map_packed(CUtensorMap *m, const void *base, uint64_t tiles, uint32_t nkb, uint32_t rows, uint32_t kc);
 
 }  // namespace mk

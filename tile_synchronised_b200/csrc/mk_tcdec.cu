@@ -223,15 +223,17 @@ __global__ void lm_argmax_kernel(const float *y, float *logits, int32_t *next, i
 // 0 .. t0 + r).  Only the KV cache is kept: the last layer stops after its
 // K/V rows.
 
-// x[r][:] = E[tok(b, t0 + r)][:]; a token outside [0, V) decodes from token 0
-// and is recorded in the context's state (first one wins), as the megakernel
-// does.
+// x[r][:] = E[tok][:] with tok = tok[b * tok_stride + t0 + r] (a prefill
+// chunk: positions t0 + r of sequence b) or, for b < 0, tok[r] of sequence r
+// (a decode step); a token outside [0, V) decodes from token 0 and is
+// recorded in the context's state (first one wins), as the megakernel does.
 __global__ void prefill_embed_kernel(const int32_t *tok, int64_t tok_stride, int b, int t0, const uint16_t *E,
-                                     float *x, int H, int V, State *state) {
+                                     float *x, int H, int V, State *state, int seq0) {
     const int r = blockIdx.x;
-    int t = tok[(int64_t)b * tok_stride + t0 + r];
+    const int seq = b < 0 ? seq0 + r : b;
+    int t = b < 0 ? tok[r] : tok[(int64_t)b * tok_stride + t0 + r];
     if (t < 0 || t >= V) {
-        if (threadIdx.x == 0 && atomicCAS(&state->tok_err, 0u, (uint32_t)b + 1u) == 0u) state->tok_bad = t;
+        if (threadIdx.x == 0 && atomicCAS(&state->tok_err, 0u, (uint32_t)seq + 1u) == 0u) state->tok_bad = t;
         t = 0;
     }
     for (int i = threadIdx.x; i < H; i += blockDim.x) x[(size_t)r * H + i] = bf2f(E[(size_t)t * H + i]);
@@ -253,15 +255,15 @@ __global__ void prefill_norm_kernel(const float *x, const uint16_t *g, __nv_bflo
 
 // One block per (head, row), head_dim threads, over the packed QKV output y
 // [2R][M] (q heads, then k, then v): the optional per-head RMSNorm and RoPE at
-// position t0 + r; q to q_out [R][nq][d], k and v to the layer's cache rows of
-// sequence b at t0 + r.
+// the row's position row_len[r] - 1; q to q_out [R][nq][d], k and v to the
+// layer's cache rows of sequence row_seq[r] at that position.
 __global__ void prefill_qkv_kernel(const float *y, int R, int M, int nq, int nkv, int d, const uint16_t *qn,
-                                   const uint16_t *kn, int qk_norm, float eps, double theta, int b, int t0,
-                                   float *q_out, uint16_t *kc, uint16_t *vc, int max_seq) {
+                                   const uint16_t *kn, int qk_norm, float eps, double theta, const int *row_seq,
+                                   const int *row_len, float *q_out, uint16_t *kc, uint16_t *vc, int max_seq) {
     extern __shared__ float buf[];
     float *red = buf + d;
     const int head = blockIdx.x, r = blockIdx.y, i = threadIdx.x;
-    const int pos = t0 + r;
+    const int b = row_seq[r], pos = row_len[r] - 1;
     float v = y[(size_t)r * M + head * d + i] + y[(size_t)(R + r) * M + head * d + i];
     const int g = head < nq ? 0 : (head < nq + nkv ? head - nq : head - nq - nkv);
     const size_t crow = (((size_t)b * nkv + g) * max_seq + pos) * d;
@@ -287,14 +289,68 @@ __global__ void prefill_qkv_kernel(const float *y, int R, int M, int nq, int nkv
         kc[crow + i] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
 }
 
-// row_seq[r] = b, row_len[r] = t0 + r + 1: the rows' sequence and attended length.
-__global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, int t0) {
+// row_seq[r] = b, row_len[r] = t0 + r + 1: the rows' sequence and attended
+// length (a prefill chunk); for b < 0, row r is sequence r at the context's
+// current position (a decode step; read on the device, so a captured step
+// replays at any position).
+__global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, int t0, const State *state, int seq0) {
     const int r = threadIdx.x;
     if (r < R) {
-        row_seq[r] = b;
-        row_len[r] = t0 + r + 1;
+        row_seq[r] = b < 0 ? seq0 + r : b;
+        row_len[r] = b < 0 ? state->pos + 1 : t0 + r + 1;
     }
 }
+
+// One block per row of a decode pass: logits[seq0 + r][v] = y[r][v] + y[n + r][v]
+// (y rows ldy wide; written when `logits` is set) and next[seq0 + r] = their
+// argmax, lowest index on ties.  With no finite logit (a projection whose
+// bounded wait ran out writes NaN) next is 0 and the state's error word gets
+// code 5.
+__global__ void rows_argmax_kernel(const float *y, int ldy, int n, float *logits, int32_t *next, int V, int seq0,
+                                   State *state) {
+    __shared__ float bv_s[32];
+    __shared__ int bi_s[32];
+    const int r = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int v = threadIdx.x; v < V; v += blockDim.x) {
+        const float l = y[(size_t)r * ldy + v] + y[(size_t)(n + r) * ldy + v];
+        if (logits) logits[(size_t)(seq0 + r) * V + v] = l;
+        if (l > bv || (l == bv && v < bi)) {
+            bv = l;
+            bi = v;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+        }
+    }
+    if (lane == 0) {
+        bv_s[warp] = bv;
+        bi_s[warp] = bi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+            if (bv_s[w] > bv_s[0] || (bv_s[w] == bv_s[0] && bi_s[w] < bi_s[0])) {
+                bv_s[0] = bv_s[w];
+                bi_s[0] = bi_s[w];
+            }
+        if (bi_s[0] == 0x7fffffff) {
+            atomicCAS(&state->err, 0u, 5u);
+            bi_s[0] = 0;
+        }
+        next[seq0 + r] = bi_s[0];
+    }
+}
+
+// After a decode step on the tensor cores: the context's position advances.
+__global__ void advance_pos_kernel(State *state) { state->pos += 1; }
 
 // out rows r, R + r (Kp wide) = hi / lo of a[r][0 .. n), zero past n.
 __global__ void prefill_cast_kernel(const float *a, __nv_bfloat16 *out, int R, int n, int Kp) {
@@ -372,75 +428,157 @@ size_t prefill_scratch_bytes(int H, int nq, int d, int kmax, int mmax) {
     const size_t R = kPrefillRows;
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     return up(R * H * 4) + up(2 * R * kmax * 2) + up(2 * R * (size_t)mmax * 4) + 2 * up(R * nq * d * 4) +
-           up(R * nq * kPrefillChunks * (size_t)(d + 2) * 4) + up(2 * R * 4);
+           up(R * nq * kPrefillChunks * (size_t)(d + 2) * 4) + up(2 * R * 4) + 2 * up(64 * 4);
 }
 
-std::string prefill_tc(const PrefillTc &a, const int32_t *tokens, int T, cudaStream_t s) {
-    using namespace tcdec;
+namespace {
+
+// The row pass's buffers, carved out of the context's scratch region.
+struct RowsScratch {
+    float *x, *y, *q, *attn, *part;
+    __nv_bfloat16 *h;
+    int *rows;           // row_seq [kPrefillRows], then row_len [kPrefillRows]
+    int32_t *tok, *nxt;  // a decode step's tokens and argmax (64 each)
+};
+
+int pk(const PackedMat &m) { return m.nkb * m.kc; }    // a packed matrix's width as a GEMM operand
+int pm(const PackedMat &m) { return m.tiles * m.rows; }  // and its height
+
+bool carve(const PrefillTc &a, RowsScratch &sc) {
     const int R = kPrefillRows;
-    const int kmax = std::max(std::max(a.qkv_kc, a.o_kc), std::max(a.gu_kc, a.down_kc));
-    const int mmax = std::max(std::max(a.qkv_M, a.o_M), std::max(a.gu_M, a.down_M));
-    if (a.scratch_bytes < prefill_scratch_bytes(a.H, a.nq, a.d, kmax, mmax)) return "prefill scratch too small";
+    const int kmax = std::max(std::max(pk(a.qkv), pk(a.o)), std::max(pk(a.gu), std::max(pk(a.down), pk(a.lm))));
+    const int mmax = std::max(std::max(pm(a.qkv), pm(a.o)), std::max(pm(a.gu), std::max(pm(a.down), pm(a.lm))));
+    if (a.scratch_bytes < prefill_scratch_bytes(a.H, a.nq, a.d, kmax, mmax)) return false;
     uint8_t *p = a.scratch;
     auto take = [&](size_t bytes) {
         uint8_t *q = p;
         p += (bytes + 255) / 256 * 256;
         return q;
     };
-    float *x = reinterpret_cast<float *>(take((size_t)R * a.H * 4));
-    __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(take((size_t)2 * R * kmax * 2));
-    float *y = reinterpret_cast<float *>(take((size_t)2 * R * mmax * 4));
-    float *q = reinterpret_cast<float *>(take((size_t)R * a.nq * a.d * 4));
-    float *attn = reinterpret_cast<float *>(take((size_t)R * a.nq * a.d * 4));
-    float *part = reinterpret_cast<float *>(take((size_t)R * a.nq * kPrefillChunks * (a.d + 2) * 4));
-    int *rows = reinterpret_cast<int *>(take((size_t)2 * R * 4));
+    sc.x = reinterpret_cast<float *>(take((size_t)R * a.H * 4));
+    sc.h = reinterpret_cast<__nv_bfloat16 *>(take((size_t)2 * R * kmax * 2));
+    sc.y = reinterpret_cast<float *>(take((size_t)2 * R * mmax * 4));
+    sc.q = reinterpret_cast<float *>(take((size_t)R * a.nq * a.d * 4));
+    sc.attn = reinterpret_cast<float *>(take((size_t)R * a.nq * a.d * 4));
+    sc.part = reinterpret_cast<float *>(take((size_t)R * a.nq * kPrefillChunks * (a.d + 2) * 4));
+    sc.rows = reinterpret_cast<int *>(take((size_t)2 * R * 4));
+    sc.tok = reinterpret_cast<int32_t *>(take(64 * 4));
+    sc.nxt = reinterpret_cast<int32_t *>(take(64 * 4));
+    return true;
+}
+
+// n rows (their sequence and attended length in sc.rows, their embeddings in
+// sc.x) through every layer; without `full` the last layer stops after its
+// K/V rows (a prefill keeps only the cache).
+std::string rows_through_layers(const PrefillTc &a, const RowsScratch &sc, int n, int chunks, bool full,
+                                cudaStream_t s) {
+    using namespace tcdec;
+    const int R = kPrefillRows;
     const size_t layer_elems = (size_t)a.B * a.nkv * a.max_seq * a.d;
     std::string err;
-    auto lin = [&](const void *w, int K, int M, int n) {
-        if (err.empty() && mk_linear_tc(h, w, y, 2 * n, K, M, s) != MK_OK) err = op_error();
+    auto lin = [&](const void *w, const PackedMat &m) {
+        if (!err.empty()) return;
+        const cudaError_t e = launch_linear_tc_packed(sc.h, w, sc.y, 2 * n, pk(m), pm(m), m.kc, m.rows, s);
+        if (e != cudaSuccess) err = std::string("projection: ") + cudaGetErrorString(e);
     };
-    for (int b = 0; b < a.B && err.empty(); ++b)
-        for (int t0 = 0; t0 < T && err.empty(); t0 += R) {
-            const int n = std::min(R, T - t0);
-            prefill_embed_kernel<<<n, kRowThreads, 0, s>>>(tokens, T, b, t0, static_cast<const uint16_t *>(a.embed),
-                                                          x, a.H, a.V, a.state);
-            prefill_rows_kernel<<<1, 32, 0, s>>>(rows, rows + R, n, b, t0);
-            const int chunks = std::max(1, std::min(kPrefillChunks, (t0 + n) / 128));
-            for (int l = 0; l < a.L && err.empty(); ++l) {
-                const LayerW &W = a.layers[l];
-                uint16_t *kc = a.kcache + (size_t)l * layer_elems, *vc = a.vcache + (size_t)l * layer_elems;
-                prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(W.attn_norm), h, n,
-                                                             a.H, a.qkv_kc, a.eps);
-                lin(W.qkv, a.qkv_kc, a.qkv_M, n);
-                if (!err.empty()) break;
-                prefill_qkv_kernel<<<dim3((unsigned)(a.nq + 2 * a.nkv), (unsigned)n), a.d, (a.d + 32) * sizeof(float),
-                                     s>>>(y, n, a.qkv_M, a.nq, a.nkv, a.d, static_cast<const uint16_t *>(W.q_norm),
-                                          static_cast<const uint16_t *>(W.k_norm), a.qk_norm, a.eps, a.theta, b, t0,
-                                          q, kc, vc, a.max_seq);
-                if (l == a.L - 1) break;  // the cache is all the prefill keeps: the last layer ends at its K/V
-                const cudaError_t e = launch_attention_rows(q, kc, vc, n, a.nq, a.nkv, a.d, a.max_seq, rows,
-                                                            rows + R, chunks, attn, part, s);
-                if (e != cudaSuccess) {
-                    err = std::string("prefill attention: ") + cudaGetErrorString(e);
-                    break;
-                }
-                prefill_cast_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(attn, h, n, a.nq * a.d, a.o_kc);
-                lin(W.o, a.o_kc, a.o_M, n);
-                prefill_residual_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(x, y, n, a.H, a.o_M);
-                prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(x, static_cast<const uint16_t *>(W.mlp_norm), h, n,
-                                                             a.H, a.gu_kc, a.eps);
-                lin(W.gu, a.gu_kc, a.gu_M, n);
-                prefill_swiglu_kernel<<<dim3(32, (unsigned)n), kRowThreads, 0, s>>>(y, h, n, a.I, a.gu_M, a.gu_rows,
-                                                                                  a.down_kc);
-                lin(W.down, a.down_kc, a.down_M, n);
-                prefill_residual_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(x, y, n, a.H, a.down_M);
-            }
+    for (int l = 0; l < a.L && err.empty(); ++l) {
+        const LayerW &W = a.layers[l];
+        uint16_t *kc = a.kcache + (size_t)l * layer_elems, *vc = a.vcache + (size_t)l * layer_elems;
+        prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(sc.x, static_cast<const uint16_t *>(W.attn_norm), sc.h, n,
+                                                     a.H, pk(a.qkv), a.eps);
+        lin(W.qkv, a.qkv);
+        if (!err.empty()) break;
+        prefill_qkv_kernel<<<dim3((unsigned)(a.nq + 2 * a.nkv), (unsigned)n), a.d, (a.d + 32) * sizeof(float), s>>>(
+            sc.y, n, pm(a.qkv), a.nq, a.nkv, a.d, static_cast<const uint16_t *>(W.q_norm),
+            static_cast<const uint16_t *>(W.k_norm), a.qk_norm, a.eps, a.theta, sc.rows, sc.rows + R, sc.q, kc, vc,
+            a.max_seq);
+        if (!full && l == a.L - 1) break;  // a prefill keeps only the cache: the last layer ends at its K/V
+        const cudaError_t e = launch_attention_rows(sc.q, kc, vc, n, a.nq, a.nkv, a.d, a.max_seq, sc.rows,
+                                                    sc.rows + R, chunks, sc.attn, sc.part, s);
+        if (e != cudaSuccess) {
+            err = std::string("attention: ") + cudaGetErrorString(e);
+            break;
         }
+        prefill_cast_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(sc.attn, sc.h, n, a.nq * a.d, pk(a.o));
+        lin(W.o, a.o);
+        prefill_residual_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(sc.x, sc.y, n, a.H, pm(a.o));
+        prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(sc.x, static_cast<const uint16_t *>(W.mlp_norm), sc.h, n,
+                                                     a.H, pk(a.gu), a.eps);
+        lin(W.gu, a.gu);
+        prefill_swiglu_kernel<<<dim3(32, (unsigned)n), kRowThreads, 0, s>>>(sc.y, sc.h, n, a.I, pm(a.gu), a.gu.rows,
+                                                                          pk(a.down));
+        lin(W.down, a.down);
+        prefill_residual_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(sc.x, sc.y, n, a.H, pm(a.down));
+    }
+    return err;
+}
+
+std::string last_error(std::string err) {
     if (err.empty()) {
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) err = cudaGetErrorString(e);
     }
     return err;
+}
+
+}  // namespace
+
+std::string prefill_tc(const PrefillTc &a, const int32_t *tokens, int T, cudaStream_t s) {
+    using namespace tcdec;
+    const int R = kPrefillRows;
+    RowsScratch sc;
+    if (!carve(a, sc)) return "prefill scratch too small";
+    std::string err;
+    for (int b = 0; b < a.B && err.empty(); ++b)
+        for (int t0 = 0; t0 < T && err.empty(); t0 += R) {
+            const int n = std::min(R, T - t0);
+            prefill_embed_kernel<<<n, kRowThreads, 0, s>>>(tokens, T, b, t0, static_cast<const uint16_t *>(a.embed),
+                                                          sc.x, a.H, a.V, a.state, 0);
+            prefill_rows_kernel<<<1, 32, 0, s>>>(sc.rows, sc.rows + R, n, b, t0, a.state, 0);
+            const int chunks = std::max(1, std::min(kPrefillChunks, (t0 + n) / 128));
+            err = rows_through_layers(a, sc, n, chunks, false, s);
+        }
+    return last_error(err);
+}
+
+std::string decode_tc(const PrefillTc &a, const int32_t *tokens, int32_t *next, float *logits, cudaStream_t s) {
+    using namespace tcdec;
+    const int R = kPrefillRows;
+    RowsScratch sc;
+    if (!carve(a, sc)) return "scratch too small";
+    // the attended length is read on the device; split the positions so that
+    // a long cache still spreads over the SMs, a fixed count so that the same
+    // launches serve every position
+    const int chunks = std::max(1, std::min(kPrefillChunks, a.max_seq / 256));
+    std::string err;
+    for (int b0 = 0; b0 < a.B && err.empty(); b0 += R) {
+        const int n = std::min(R, a.B - b0);
+        prefill_embed_kernel<<<n, kRowThreads, 0, s>>>(tokens + b0, 0, -1, 0, static_cast<const uint16_t *>(a.embed),
+                                                      sc.x, a.H, a.V, a.state, b0);
+        prefill_rows_kernel<<<1, 32, 0, s>>>(sc.rows, sc.rows + R, n, -1, 0, a.state, b0);
+        err = rows_through_layers(a, sc, n, chunks, true, s);
+        if (!err.empty()) break;
+        prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(sc.x, static_cast<const uint16_t *>(a.final_norm), sc.h, n, a.H,
+                                                     pk(a.lm), a.eps);
+        const cudaError_t e = launch_linear_tc_packed(sc.h, a.lm_w, sc.y, 2 * n, pk(a.lm), pm(a.lm), a.lm.kc,
+                                                      a.lm.rows, s);
+        if (e != cudaSuccess) {
+            err = std::string("LM head: ") + cudaGetErrorString(e);
+            break;
+        }
+        rows_argmax_kernel<<<n, 1024, 0, s>>>(sc.y, pm(a.lm), n, logits, next, a.V, b0, a.state);
+    }
+    if (err.empty()) advance_pos_kernel<<<1, 1, 0, s>>>(a.state);
+    return last_error(err);
+}
+
+int32_t *decode_tc_tokens(const PrefillTc &a) {
+    RowsScratch sc;
+    return carve(a, sc) ? sc.tok : nullptr;
+}
+int32_t *decode_tc_next(const PrefillTc &a) {
+    RowsScratch sc;
+    return carve(a, sc) ? sc.nxt : nullptr;
 }
 
 }  // namespace mk
