@@ -423,7 +423,9 @@ mk_status mk_attention_decode(const float *q, const void *k_cache, const void *v
 size_t mk_attention_scratch_bytes(int batch, int n_heads, int head_dim, int chunks);
 /* The chunk count mk_attention_decode picks for chunks = 0 on the current
  * device: about one CTA per SM over (sequence, KV head) pairs, at most 64, and
- * at least 16 positions per chunk. */
+ * at least 16 positions per chunk; for caches of 1024 positions and more, as
+ * many chunks of at least 512 positions as fill two CTAs per SM in whole
+ * waves (the first count whose last wave is 90 % full), when that is more. */
 int mk_attention_chunks(int batch, int n_kv_heads, int n_pos);
 
 /* mk_attention_decode without a scratch argument: the partial records live in

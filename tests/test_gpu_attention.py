@@ -42,6 +42,10 @@ CASES = [  # batch, nq, nkv, d, max_seq, n_pos, chunks
     (2, 12, 4, 256, 64, 33, 3),       # group 3, d = 256
     (1, 8, 8, 128, 100, 100, 100),    # MHA, one position per chunk
     (16, 32, 8, 128, 1100, 1024, 0),  # Qwen3-8B batch 16 at 1k
+    (2, 16, 2, 64, 3000, 2777, 0),    # group 8 at d = 64, ragged last stage
+    (1, 16, 8, 128, 9000, 8191, 5),   # group 2, chunks of 1638 / 1639 positions
+    (2, 32, 8, 128, 16400, 16384, 0),  # Qwen3-8B layer at 16k: long chunks over the stage ring
+    (3, 8, 4, 64, 700, 129, 2),       # group 2 at d = 64: one full stage + one position
 ]
 
 

@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 
@@ -49,6 +50,7 @@ struct AttnArgs {
     // positions 0 .. row_len[b] - 1 (a prefill chunk: several positions of one
     // sequence, each attending causally); else row b is sequence b
     const int *row_seq, *row_len;
+    int pdl;  // launch both kernels with programmatic dependent launch (a step's chain of kernels)
 };
 
 // One CTA = one (chunk, KV head, sequence).  Warps split the G heads
@@ -57,6 +59,8 @@ struct AttnArgs {
 // l*DPL .. l*DPL + DPL - 1.  The warps' states are merged in shared memory.
 template <int DPL>
 __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) {
+    pdl_wait();  // no-ops unless launched with programmatic dependent launch
+    pdl_launch_dependents();
     constexpr int d = 32 * DPL;
     constexpr int TP = attn_tile_positions(d);
     const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -142,8 +146,257 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
     }
 }
 
+// Raise a kernel's dynamic shared-memory limit once per device (bit d of
+// `done` records device d).
+static cudaError_t allow_smem(const void *fn, int bytes, std::atomic<unsigned long long> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
+// ------------------------------------------------------------------ tiles through a TMA ring
+// The same partials for head_dim 64 and 128 and G = 2, 4 or 8 query heads per
+// KV head, with the cache streamed by 1-D bulk copies (TMA) through a ring of
+// kTileStages shared-memory stages, so that the next tiles are in flight
+// while one is consumed.  A stage holds the K rows and then the V rows of
+// kTileBytes / (2 d) consecutive positions.
+//
+// Every warp serves all G heads, so each K and V row is read from shared
+// memory once per CTA.  Lane l owns dimensions l*DPL .. l*DPL + DPL - 1 and
+// keeps q and the output of every head for them in registers.  A warp takes
+// 32 / G positions at a time (32 (position, head) pairs): each lane forms its
+// partial dot products for all 32 pairs, and a transposing butterfly over the
+// lanes (16 + 8 + 4 + 2 + 1 shuffles) leaves lane l with the whole score of
+// pair l (position l / G, head l % G).  The online softmax runs on those
+// lanes; the probabilities go through shared memory to the lanes that apply
+// them to the V rows.  The eight warps take alternate groups of positions and
+// merge at the end, through the drained ring.
+constexpr int kTileStages = 3;
+constexpr int kTileBytes = 16384;  // one stage's K rows; its V rows as many
+
+__host__ __device__ inline int attn_tile_smem_bytes() {
+    return kTileStages * 2 * kTileBytes + kAttnWarps * 40 * 4 + kTileStages * 8;
+}
+
+__device__ __forceinline__ void load_bf16_row_part(const uint16_t *p, float *f, int n) {
+    if (n == 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        f[0] = __uint_as_float(u.x << 16);
+        f[1] = __uint_as_float(u.x & 0xffff0000u);
+        f[2] = __uint_as_float(u.y << 16);
+        f[3] = __uint_as_float(u.y & 0xffff0000u);
+    } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+        f[0] = __uint_as_float(u << 16);
+        f[1] = __uint_as_float(u & 0xffff0000u);
+    }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kAttnThreads, 2) attn_tile_kernel(AttnArgs a) {
+    pdl_wait();  // no-ops unless launched with programmatic dependent launch
+    pdl_launch_dependents();
+    static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(G == 2 || G == 4 || G == 8, "query heads per KV head");
+    constexpr int TP = kTileBytes / (2 * D);  // positions per stage
+    constexpr int DPL = D / 32;               // dimensions per lane
+    constexpr int P = 32 / G;                 // positions per warp group
+    constexpr unsigned FULL = 0xffffffffu;
+    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t *ring = smem;                                                            // [stages][K | V]
+    float *pw = reinterpret_cast<float *>(smem + kTileStages * 2 * kTileBytes) + warp * 40;  // [32] p, [8] corr
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTileStages * 2 * kTileBytes + kAttnWarps * 40 * 4);
+    const int n_pos = a.row_len ? a.row_len[b] : (a.n_pos_dev ? *a.n_pos_dev : a.n_pos);  // empty chunks write empty records
+    const int seq = a.row_seq ? a.row_seq[b] : b;
+    const int p0 = (int)((long long)c * n_pos / a.chunks), p1 = (int)((long long)(c + 1) * n_pos / a.chunks);
+    const int ntiles = p1 > p0 ? (p1 - p0 + TP - 1) / TP : 0;
+    const size_t head = ((size_t)seq * a.nkv + g) * (size_t)a.max_seq;
+    if (t == 0) {
+        for (int s = 0; s < kTileStages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const uint64_t pol = policy_evict_first();
+    auto issue = [&](int i) {
+        const int s = i % kTileStages, pos = p0 + i * TP, n = min(TP, p1 - pos);
+        const uint32_t bytes = (uint32_t)(n * D * 2);
+        uint8_t *dst = ring + (size_t)s * 2 * kTileBytes;
+        mbar_arrive_expect_tx(&full[s], 2 * bytes);
+        bulk_g2s(dst, a.k + (head + pos) * D, bytes, &full[s], pol);
+        bulk_g2s(dst + kTileBytes, a.v + (head + pos) * D, bytes, &full[s], pol);
+    };
+    if (t == 0)
+        for (int i = 0; i < ntiles && i < kTileStages; ++i) issue(i);
+
+    // q of the G heads for this lane's dimensions, scaled by log2(e)/sqrt(d)
+    const float qscale = 1.4426950408889634f * rsqrtf((float)D);
+    float q[G][DPL], o[G][DPL];
+    {
+        const float *qb = a.q + ((size_t)b * a.nq + (size_t)g * G) * D + lane * DPL;
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) {
+                q[h][e] = qb[h * D + e] * qscale;
+                o[h][e] = 0.f;
+            }
+    }
+    float m = -CUDART_INF_F, l = 0.f;  // running max and sum of head lane % G
+    bool bad = false;
+    int i = 0;
+    for (; i < ntiles; ++i) {
+        const int s = i % kTileStages;
+        const uint32_t par = (uint32_t)(i / kTileStages) & 1u;
+        if (!mbar_try_wait(&full[s], par)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait_sleep(&full[s], par, 10000u))
+                if (globaltimer_ns() - t0 > 2000000000ull) {
+                    bad = true;
+                    break;
+                }
+        }
+        if (!bad) {
+            const int n = min(TP, p1 - (p0 + i * TP));
+            const uint16_t *K = reinterpret_cast<const uint16_t *>(ring + (size_t)s * 2 * kTileBytes);
+            const uint16_t *V = K + kTileBytes / 2;
+            for (int base = warp * P; base < n; base += kAttnWarps * P) {
+                const int cnt = min(P, n - base);
+                float acc[32];
+#pragma unroll
+                for (int j = 0; j < P; ++j) {
+                    float kf[DPL];
+                    load_bf16_row_part(K + (size_t)(base + min(j, cnt - 1)) * D + lane * DPL, kf, DPL);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        float x = q[h][0] * kf[0];
+#pragma unroll
+                        for (int e = 1; e < DPL; ++e) x = fmaf(q[h][e], kf[e], x);
+                        acc[j * G + h] = x;
+                    }
+                }
+                // transposing butterfly: lane l ends with the full sum of pair l
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) {
+                    const bool up = lane & off;
+#pragma unroll
+                    for (int r = 0; r < off; ++r) {
+                        const float send = up ? acc[r] : acc[r + off];
+                        const float keep = up ? acc[r + off] : acc[r];
+                        acc[r] = keep + __shfl_xor_sync(FULL, send, off);
+                    }
+                }
+                const bool valid = lane / G < cnt;
+                const float sc = valid ? acc[0] : -CUDART_INF_F;
+                float gm = sc;
+#pragma unroll
+                for (int off = G; off < 32; off <<= 1) gm = fmaxf(gm, __shfl_xor_sync(FULL, gm, off));
+                const float mnew = fmaxf(m, gm);
+                const float corr = exp2f(m - mnew);
+                const float p = valid ? exp2f(sc - mnew) : 0.f;
+                float ps = p;
+#pragma unroll
+                for (int off = G; off < 32; off <<= 1) ps += __shfl_xor_sync(FULL, ps, off);
+                l = l * corr + ps;
+                m = mnew;
+                pw[lane] = p;
+                if (lane < G) pw[32 + lane] = corr;
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float cr = pw[32 + h];
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) o[h][e] *= cr;
+                }
+#pragma unroll
+                for (int j = 0; j < P; ++j) {
+                    if (j < cnt) {
+                        float vf[DPL];
+                        load_bf16_row_part(V + (size_t)(base + j) * D + lane * DPL, vf, DPL);
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float pj = pw[j * G + h];
+#pragma unroll
+                            for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(pj, vf[e], o[h][e]);
+                        }
+                    }
+                }
+                __syncwarp();  // pw is rewritten by the next group
+            }
+        }
+        if (__syncthreads_or(bad)) break;  // every warp is done with stage s (or some wait gave up)
+        if (t == 0 && i + kTileStages < ntiles) issue(i + kTileStages);
+    }
+    const bool aborted = i < ntiles;
+    if (aborted) {
+        // never leave with a copy into this CTA's shared memory in flight
+        if (t == 0)
+            for (int k = i; k < ntiles && k < i + kTileStages; ++k) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait_sleep(&full[k % kTileStages], (uint32_t)(k / kTileStages) & 1u, 10000u))
+                    if (globaltimer_ns() - t0 > 2000000000ull) break;
+            }
+        for (int x = t; x < G * D; x += kAttnThreads) {
+            const int hh = x / D, e = x % D;
+            float *rec = a.part + (((size_t)b * a.nq + (size_t)g * G + hh) * a.chunks + c) * (D + 2);
+            rec[e] = CUDART_NAN_F;
+            if (e == 0) rec[D] = rec[D + 1] = CUDART_NAN_F;
+        }
+        return;
+    }
+    // merge the warps through the ring (every copy into it has landed and been read)
+    float *mo = reinterpret_cast<float *>(ring);         // [warp][G][D]
+    float *ml = mo + kAttnWarps * G * D;                 // [warp][G][2]
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) mo[(warp * G + h) * D + lane * DPL + e] = o[h][e];
+    if (lane < G) {
+        ml[(warp * G + lane) * 2] = m;
+        ml[(warp * G + lane) * 2 + 1] = l;
+    }
+    __syncthreads();
+    for (int x = t; x < G * D; x += kAttnThreads) {
+        const int hh = x / D, e = x % D;
+        float M = -CUDART_INF_F;
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, ml[(w * G + hh) * 2]);
+        float O = 0.f, L = 0.f;
+        if (M != -CUDART_INF_F)
+            for (int w = 0; w < kAttnWarps; ++w) {
+                const float mw = ml[(w * G + hh) * 2];
+                if (mw == -CUDART_INF_F) continue;
+                const float f = exp2f(mw - M);
+                O = fmaf(f, mo[(w * G + hh) * D + e], O);
+                L = fmaf(f, ml[(w * G + hh) * 2 + 1], L);
+            }
+        float *rec = a.part + (((size_t)b * a.nq + (size_t)g * G + hh) * a.chunks + c) * (D + 2);
+        rec[e] = O;
+        if (e == 0) {
+            rec[D] = M;
+            rec[D + 1] = L;
+        }
+    }
+}
+
+template <int D, int G>
+static cudaError_t launch_tile(cudaLaunchConfig_t &cfg, const AttnArgs &a) {
+    static std::atomic<unsigned long long> configured{0};
+    const int smem = attn_tile_smem_bytes();
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(attn_tile_kernel<D, G>), smem, configured);
+    return e == cudaSuccess ? cudaLaunchKernelEx(&cfg, attn_tile_kernel<D, G>, a) : e;
+}
+
 // One CTA per (query head, sequence), one thread per output dimension.
 __global__ void attn_combine_kernel(AttnArgs a) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x, d = a.d;
     const float *rec = a.part + ((size_t)b * a.nq + h) * a.chunks * (size_t)(d + 2);
     float M = -CUDART_INF_F;
@@ -161,17 +414,36 @@ __global__ void attn_combine_kernel(AttnArgs a) {
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s) {
     const int G = a.nq / a.nkv;
-    const dim3 grid(a.chunks, a.nkv, a.B);
-    const int smem = attn_smem_bytes(G, a.d);
-    switch (a.d) {
-        case 64: attn_partial_kernel<2><<<grid, kAttnThreads, smem, s>>>(a); break;
-        case 128: attn_partial_kernel<4><<<grid, kAttnThreads, smem, s>>>(a); break;
-        default: attn_partial_kernel<8><<<grid, kAttnThreads, smem, s>>>(a); break;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.chunks, a.nkv, a.B);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = (size_t)attn_smem_bytes(G, a.d);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    cudaError_t e;
+    if ((a.d == 64 || a.d == 128) && (G == 2 || G == 4 || G == 8)) {
+        // the TMA-ring kernel (~97 KB of shared memory, two CTAs per SM)
+        if (a.d == 64)
+            e = G == 2 ? launch_tile<64, 2>(cfg, a) : G == 4 ? launch_tile<64, 4>(cfg, a) : launch_tile<64, 8>(cfg, a);
+        else
+            e = G == 2 ? launch_tile<128, 2>(cfg, a) : G == 4 ? launch_tile<128, 4>(cfg, a)
+                                                           : launch_tile<128, 8>(cfg, a);
+    } else {
+        switch (a.d) {
+            case 64: e = cudaLaunchKernelEx(&cfg, attn_partial_kernel<2>, a); break;
+            case 128: e = cudaLaunchKernelEx(&cfg, attn_partial_kernel<4>, a); break;
+            default: e = cudaLaunchKernelEx(&cfg, attn_partial_kernel<8>, a); break;
+        }
     }
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<<<dim3(a.nq, a.B), a.d, 0, s>>>(a);
-    return cudaGetLastError();
+    cfg.gridDim = dim3(a.nq, a.B);
+    cfg.blockDim = dim3(a.d);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, attn_combine_kernel, a);
 }
 
 // The decode attention with the attended length read from device memory at
@@ -182,7 +454,7 @@ cudaError_t launch_attention_dev(const float *q, const void *k, const void *v, i
                                  int max_seq, const int *n_pos_dev, int chunks, float *out, float *part,
                                  cudaStream_t s) {
     AttnArgs a{q, static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), out, part, B, nq, nkv, d,
-               max_seq, max_seq, chunks, n_pos_dev, nullptr, nullptr};
+               max_seq, max_seq, chunks, n_pos_dev, nullptr, nullptr, 0};
     return launch_attention(a, s);
 }
 
@@ -191,9 +463,9 @@ cudaError_t launch_attention_dev(const float *q, const void *k, const void *v, i
 // rows of a prefill chunk), `chunks` split-KV chunks per row.
 cudaError_t launch_attention_rows(const float *q, const void *k, const void *v, int rows, int nq, int nkv, int d,
                                   int max_seq, const int *row_seq, const int *row_len, int chunks, float *out,
-                                  float *part, cudaStream_t s) {
+                                  float *part, cudaStream_t s, bool pdl) {
     AttnArgs a{q, static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), out, part, rows, nq, nkv, d,
-               max_seq, max_seq, chunks, nullptr, row_seq, row_len};
+               max_seq, max_seq, chunks, nullptr, row_seq, row_len, pdl ? 1 : 0};
     return launch_attention(a, s);
 }
 
@@ -204,11 +476,29 @@ void set_op_error(const char *msg) { snprintf(g_op_error, sizeof(g_op_error), "%
 const char *op_error() { return g_op_error[0] ? g_op_error : "null context"; }
 
 int attention_auto_chunks(int B, int nkv, int n_pos, int sms) {
+    // about one CTA per SM over the (sequence, KV head) pairs, at least 16 positions per chunk
     int c = sms / (B * nkv);
     if (c < 1) c = 1;
     if (c > 64) c = 64;
-    const int by_len = n_pos / 16 > 0 ? n_pos / 16 : 1;  // at least 16 positions per chunk
-    return c < by_len ? c : by_len;
+    const int by_len = n_pos / 16 > 0 ? n_pos / 16 : 1;
+    if (c > by_len) c = by_len;
+    // long caches: chunks of at least 512 positions, as many as fill the
+    // two-per-SM slots in whole waves (the first count reaching 90 % of its
+    // last wave, else the best one)
+    const long long pairs = (long long)B * nkv, slots = 2LL * (sms > 0 ? sms : 1);
+    const int hi = n_pos / 512 < 64 ? n_pos / 512 : 64;
+    int best = 0;
+    double best_eff = 0.0;
+    for (int k = 1; k <= hi; ++k) {
+        const long long ctas = pairs * k, waves = (ctas + slots - 1) / slots;
+        const double eff = (double)ctas / (double)(waves * slots);
+        if (eff > best_eff + 1e-9) {
+            best = k;
+            best_eff = eff;
+        }
+        if (eff >= 0.9) break;
+    }
+    return best > c ? best : c;
 }
 
 // Checks shared by every attention entry point; fills a.chunks when it is 0.
@@ -270,7 +560,7 @@ extern "C" mk_status mk_attention_decode(const float *q, const void *k_cache, co
                                          int chunks, float *out, void *scratch, size_t scratch_bytes,
                                          void *stream) {
     AttnArgs a{q, static_cast<const uint16_t *>(k_cache), static_cast<const uint16_t *>(v_cache), out, nullptr,
-               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks, nullptr, nullptr, nullptr};
+               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks, nullptr, nullptr, nullptr, 0};
     mk_status st = attention_args(a, q, k_cache, v_cache, out);
     if (st != MK_OK) return st;
     const size_t need = mk_attention_scratch_bytes(batch, n_heads, head_dim, a.chunks);
@@ -313,7 +603,7 @@ extern "C" mk_status mk_attention_decode_noalloc(const float *q, const void *k_c
                                                  int n_heads, int n_kv_heads, int head_dim, int max_seq, int n_pos,
                                                  int chunks, float *out, void *stream) {
     AttnArgs a{q, static_cast<const uint16_t *>(k_cache), static_cast<const uint16_t *>(v_cache), out, nullptr,
-               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks, nullptr, nullptr, nullptr};
+               batch, n_heads, n_kv_heads, head_dim, max_seq, n_pos, chunks, nullptr, nullptr, nullptr, 0};
     const bool auto_chunks = chunks == 0;
     mk_status st = attention_args(a, q, k_cache, v_cache, out);
     if (st != MK_OK) return st;

@@ -34,12 +34,12 @@ cudaError_t launch_attention_dev(const float *q, const void *k, const void *v, i
 // one of the megakernel's packed matrices, [tiles][K / kc][rows][kc] bf16, and
 // x bf16 [B][K] (K = the packed width, zero past the logical one).
 cudaError_t launch_linear_tc_packed(const void *x, const void *w, float *y, int B, int K, int M, int kc, int rows,
-                                    cudaStream_t s);
+                                    cudaStream_t s, bool pdl = false);
 // Causal attention of prefill rows (mk_attn.cu): row r of q / out attends
 // positions 0 .. row_len[r] - 1 of sequence row_seq[r] of one layer's cache.
 cudaError_t launch_attention_rows(const float *q, const void *k, const void *v, int rows, int nq, int nkv, int d,
                                   int max_seq, const int *row_seq, const int *row_len, int chunks, float *out,
-                                  float *part, cudaStream_t s);
+                                  float *part, cudaStream_t s, bool pdl = false);
 // The tensor-core prefill of a megakernel context (mk_tcdec.cu): positions
 // 0 .. T-1 of every sequence through the decoder in chunks of kPrefillRows,
 // every projection one tensor-core GEMM over the packed weights.  Fills the KV

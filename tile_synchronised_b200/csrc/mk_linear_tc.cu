@@ -94,20 +94,37 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_base;
+    // Launched with programmatic dependent launch (a step's chain of kernels),
+    // the next kernel may now start its own set-up; without it this is a no-op.
+    pdl_launch_dependents();
 
     int issued = 0;  // K blocks whose copies the producer (warp 0 lane 0) has issued
     if (warp == 0 && lane == 0) {
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int s = kb % S;
-            if (kb >= S && !tc_wait(&empty[s], ((kb / S) - 1) & 1u, abort)) break;
+        auto load_w = [&](int kb) {
+            const int s = kb % S, k0 = (kb_first + kb) * kLinBK;
             uint8_t *st = smem + (size_t)s * sh.stage_bytes;
             mbar_arrive_expect_tx(&full[s], sh.stage_bytes);  // rows past M or B arrive as zeros and count
-            const int k0 = (kb_first + kb) * kLinBK;
             if (sh.w_kc)
                 tma_load_4d(st, &map_w, k0 % sh.w_kc, 0, k0 / sh.w_kc, m0 / sh.w_rows, &full[s]);
             else
                 tma_load_2d(st, &map_w, k0, m0, &full[s]);
-            tma_load_2d(st + sh.a_bytes, &map_x, k0, 0, &full[s]);
+        };
+        auto load_x = [&](int kb) {
+            const int s = kb % S, k0 = (kb_first + kb) * kLinBK;
+            tma_load_2d(smem + (size_t)s * sh.stage_bytes + sh.a_bytes, &map_x, k0, 0, &full[s]);
+        };
+        // The weights do not depend on the kernel before this one: the first
+        // stages' weight boxes go out before the wait for its results (x).
+        const int pre = nkb < S ? nkb : S;
+        for (int kb = 0; kb < pre; ++kb) load_w(kb);
+        pdl_wait();
+        for (int kb = 0; kb < pre; ++kb) load_x(kb);
+        issued = pre;
+        for (int kb = pre; kb < nkb; ++kb) {
+            const int s = kb % S;
+            if (!tc_wait(&empty[s], ((kb / S) - 1) & 1u, abort)) break;
+            load_w(kb);
+            load_x(kb);
             issued = kb + 1;
         }
     } else if (warp == 1 && lane == 0) {
@@ -220,7 +237,7 @@ static bool lin_plan(int B, int K, int M, LinPlan &p) {
 // w_kc > 0: W is packed as [tiles][K / w_kc][w_rows][w_kc] (tiles = M / w_rows
 // rounded up), read through a 4-D tensor map; else W is row-major [M, K].
 static cudaError_t launch_linear(const void *x, const void *w, float *y, int B, int K, int M, int w_kc, int w_rows,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, bool pdl) {
     LinPlan p;
     if (!lin_plan(B, K, M, p)) return cudaErrorInvalidValue;
     if (w_kc && (w_kc % kLinBK || K % w_kc || w_rows < 1 || kLinM % w_rows)) return cudaErrorInvalidValue;
@@ -240,23 +257,25 @@ static cudaError_t launch_linear(const void *x, const void *w, float *y, int B, 
     cfg.blockDim = dim3(kLinThreads);
     cfg.dynamicSmemBytes = (size_t)p.smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)p.split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, linear_tc_kernel, mw, mx, y, p.sh);
 }
 
 cudaError_t launch_linear_tc(const void *x, const void *w, float *y, int B, int K, int M, cudaStream_t s) {
-    return launch_linear(x, w, y, B, K, M, 0, 0, s);
+    return launch_linear(x, w, y, B, K, M, 0, 0, s, false);
 }
 
 cudaError_t launch_linear_tc_packed(const void *x, const void *w, float *y, int B, int K, int M, int kc, int rows,
-                                    cudaStream_t s) {
-    return launch_linear(x, w, y, B, K, M, kc, rows, s);
+                                    cudaStream_t s, bool pdl) {
+    return launch_linear(x, w, y, B, K, M, kc, rows, s, pdl);
 }
 
 }  // namespace mk

@@ -214,6 +214,32 @@ __global__ void lm_argmax_kernel(const float *y, float *logits, int32_t *next, i
 }
 
 // ------------------------------------------------------------------ prefill rows
+// Every kernel of the row pass is launched with programmatic dependent launch:
+// it first waits for the kernel before it (griddepcontrol.wait: that kernel
+// has finished and its writes are visible), then lets the next one launch, so
+// the next kernel's launch and set-up overlap this one.  Without the launch
+// attribute both instructions return at once.
+__device__ __forceinline__ void row_pass_prologue() {
+    pdl_wait();
+    pdl_launch_dependents();
+}
+
+// Launch `k` on `s` with programmatic dependent launch allowed.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
+}
 // The prefill of a megakernel context on the tensor cores: R <= 32
 // consecutive positions t0 .. t0 + R - 1 of one sequence b go through the
 // decoder together, every projection one mk_linear_tc call over the
@@ -229,6 +255,7 @@ __global__ void lm_argmax_kernel(const float *y, float *logits, int32_t *next, i
 // recorded in the context's state (first one wins), as the megakernel does.
 __global__ void prefill_embed_kernel(const int32_t *tok, int64_t tok_stride, int b, int t0, const uint16_t *E,
                                      float *x, int H, int V, State *state, int seq0) {
+    row_pass_prologue();
     const int r = blockIdx.x;
     const int seq = b < 0 ? seq0 + r : b;
     int t = b < 0 ? tok[r] : tok[(int64_t)b * tok_stride + t0 + r];
@@ -242,6 +269,7 @@ __global__ void prefill_embed_kernel(const int32_t *tok, int64_t tok_stride, int
 // out rows r (hi) and R + r (lo), Kp wide = RMSNorm(x[r]) * g, zero past H.
 __global__ void prefill_norm_kernel(const float *x, const uint16_t *g, __nv_bfloat16 *out, int R, int H, int Kp,
                                     float eps) {
+    row_pass_prologue();
     __shared__ float red[32];
     const int r = blockIdx.x;
     const float *xr = x + (size_t)r * H;
@@ -260,6 +288,7 @@ __global__ void prefill_norm_kernel(const float *x, const uint16_t *g, __nv_bflo
 __global__ void prefill_qkv_kernel(const float *y, int R, int M, int nq, int nkv, int d, const uint16_t *qn,
                                    const uint16_t *kn, int qk_norm, float eps, double theta, const int *row_seq,
                                    const int *row_len, float *q_out, uint16_t *kc, uint16_t *vc, int max_seq) {
+    row_pass_prologue();
     extern __shared__ float buf[];
     float *red = buf + d;
     const int head = blockIdx.x, r = blockIdx.y, i = threadIdx.x;
@@ -294,6 +323,7 @@ __global__ void prefill_qkv_kernel(const float *y, int R, int M, int nq, int nkv
 // current position (a decode step; read on the device, so a captured step
 // replays at any position).
 __global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, int t0, const State *state, int seq0) {
+    row_pass_prologue();
     const int r = threadIdx.x;
     if (r < R) {
         row_seq[r] = b < 0 ? seq0 + r : b;
@@ -308,6 +338,7 @@ __global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, in
 // code 5.
 __global__ void rows_argmax_kernel(const float *y, int ldy, int n, float *logits, int32_t *next, int V, int seq0,
                                    State *state) {
+    row_pass_prologue();
     __shared__ float bv_s[32];
     __shared__ int bi_s[32];
     const int r = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -350,10 +381,14 @@ __global__ void rows_argmax_kernel(const float *y, int ldy, int n, float *logits
 }
 
 // After a decode step on the tensor cores: the context's position advances.
-__global__ void advance_pos_kernel(State *state) { state->pos += 1; }
+__global__ void advance_pos_kernel(State *state) {
+    row_pass_prologue();
+    state->pos += 1;
+}
 
 // out rows r, R + r (Kp wide) = hi / lo of a[r][0 .. n), zero past n.
 __global__ void prefill_cast_kernel(const float *a, __nv_bfloat16 *out, int R, int n, int Kp) {
+    row_pass_prologue();
     const int r = blockIdx.y;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < Kp; i += gridDim.x * blockDim.x)
         put_hilo(out + (size_t)r * Kp + i, out + (size_t)(R + r) * Kp + i, i < n ? a[(size_t)r * n + i] : 0.f);
@@ -361,6 +396,7 @@ __global__ void prefill_cast_kernel(const float *a, __nv_bfloat16 *out, int R, i
 
 // x[r][i] += y[r][i] + y[R + r][i], y rows M wide.
 __global__ void prefill_residual_kernel(float *x, const float *y, int R, int H, int M) {
+    row_pass_prologue();
     const int r = blockIdx.y;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < H; i += gridDim.x * blockDim.x)
         x[(size_t)r * H + i] += y[(size_t)r * M + i] + y[(size_t)(R + r) * M + i];
@@ -371,6 +407,7 @@ __global__ void prefill_residual_kernel(float *x, const float *y, int R, int H, 
 // t*rows/2 + k - rows/2.  out rows r, R + r (Kp wide) = hi / lo of
 // SiLU(gate) * up, zero past I.
 __global__ void prefill_swiglu_kernel(const float *y, __nv_bfloat16 *out, int R, int I, int M, int rows, int Kp) {
+    row_pass_prologue();
     const int r = blockIdx.y, half = rows / 2;
     for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < Kp; j += gridDim.x * blockDim.x) {
         float val = 0.f;
@@ -478,37 +515,39 @@ std::string rows_through_layers(const PrefillTc &a, const RowsScratch &sc, int n
     std::string err;
     auto lin = [&](const void *w, const PackedMat &m) {
         if (!err.empty()) return;
-        const cudaError_t e = launch_linear_tc_packed(sc.h, w, sc.y, 2 * n, pk(m), pm(m), m.kc, m.rows, s);
+        const cudaError_t e = launch_linear_tc_packed(sc.h, w, sc.y, 2 * n, pk(m), pm(m), m.kc, m.rows, s, true);
         if (e != cudaSuccess) err = std::string("projection: ") + cudaGetErrorString(e);
     };
     for (int l = 0; l < a.L && err.empty(); ++l) {
         const LayerW &W = a.layers[l];
         uint16_t *kc = a.kcache + (size_t)l * layer_elems, *vc = a.vcache + (size_t)l * layer_elems;
-        prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(sc.x, static_cast<const uint16_t *>(W.attn_norm), sc.h, n,
-                                                     a.H, pk(a.qkv), a.eps);
+        launch_pdl(prefill_norm_kernel, dim3(n), dim3(kRowThreads), 0, s, sc.x,
+                   static_cast<const uint16_t *>(W.attn_norm), sc.h, n, a.H, pk(a.qkv), a.eps);
         lin(W.qkv, a.qkv);
         if (!err.empty()) break;
-        prefill_qkv_kernel<<<dim3((unsigned)(a.nq + 2 * a.nkv), (unsigned)n), a.d, (a.d + 32) * sizeof(float), s>>>(
-            sc.y, n, pm(a.qkv), a.nq, a.nkv, a.d, static_cast<const uint16_t *>(W.q_norm),
-            static_cast<const uint16_t *>(W.k_norm), a.qk_norm, a.eps, a.theta, sc.rows, sc.rows + R, sc.q, kc, vc,
-            a.max_seq);
+        launch_pdl(prefill_qkv_kernel, dim3((unsigned)(a.nq + 2 * a.nkv), (unsigned)n), dim3(a.d),
+                   (a.d + 32) * sizeof(float), s, sc.y, n, pm(a.qkv), a.nq, a.nkv, a.d,
+                   static_cast<const uint16_t *>(W.q_norm), static_cast<const uint16_t *>(W.k_norm), a.qk_norm, a.eps,
+                   a.theta, sc.rows, sc.rows + R, sc.q, kc, vc, a.max_seq);
         if (!full && l == a.L - 1) break;  // a prefill keeps only the cache: the last layer ends at its K/V
         const cudaError_t e = launch_attention_rows(sc.q, kc, vc, n, a.nq, a.nkv, a.d, a.max_seq, sc.rows,
-                                                    sc.rows + R, chunks, sc.attn, sc.part, s);
+                                                    sc.rows + R, chunks, sc.attn, sc.part, s, true);
         if (e != cudaSuccess) {
             err = std::string("attention: ") + cudaGetErrorString(e);
             break;
         }
-        prefill_cast_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(sc.attn, sc.h, n, a.nq * a.d, pk(a.o));
+        launch_pdl(prefill_cast_kernel, dim3(8, (unsigned)n), dim3(kRowThreads), 0, s, sc.attn, sc.h, n, a.nq * a.d,
+                   pk(a.o));
         lin(W.o, a.o);
-        prefill_residual_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(sc.x, sc.y, n, a.H, pm(a.o));
-        prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(sc.x, static_cast<const uint16_t *>(W.mlp_norm), sc.h, n,
-                                                     a.H, pk(a.gu), a.eps);
+        launch_pdl(prefill_residual_kernel, dim3(8, (unsigned)n), dim3(kRowThreads), 0, s, sc.x, sc.y, n, a.H, pm(a.o));
+        launch_pdl(prefill_norm_kernel, dim3(n), dim3(kRowThreads), 0, s, sc.x,
+                   static_cast<const uint16_t *>(W.mlp_norm), sc.h, n, a.H, pk(a.gu), a.eps);
         lin(W.gu, a.gu);
-        prefill_swiglu_kernel<<<dim3(32, (unsigned)n), kRowThreads, 0, s>>>(sc.y, sc.h, n, a.I, pm(a.gu), a.gu.rows,
-                                                                          pk(a.down));
+        launch_pdl(prefill_swiglu_kernel, dim3(32, (unsigned)n), dim3(kRowThreads), 0, s, sc.y, sc.h, n, a.I,
+                   pm(a.gu), a.gu.rows, pk(a.down));
         lin(W.down, a.down);
-        prefill_residual_kernel<<<dim3(8, (unsigned)n), kRowThreads, 0, s>>>(sc.x, sc.y, n, a.H, pm(a.down));
+        launch_pdl(prefill_residual_kernel, dim3(8, (unsigned)n), dim3(kRowThreads), 0, s, sc.x, sc.y, n, a.H,
+                   pm(a.down));
     }
     return err;
 }
@@ -532,9 +571,10 @@ std::string prefill_tc(const PrefillTc &a, const int32_t *tokens, int T, cudaStr
     for (int b = 0; b < a.B && err.empty(); ++b)
         for (int t0 = 0; t0 < T && err.empty(); t0 += R) {
             const int n = std::min(R, T - t0);
-            prefill_embed_kernel<<<n, kRowThreads, 0, s>>>(tokens, T, b, t0, static_cast<const uint16_t *>(a.embed),
-                                                          sc.x, a.H, a.V, a.state, 0);
-            prefill_rows_kernel<<<1, 32, 0, s>>>(sc.rows, sc.rows + R, n, b, t0, a.state, 0);
+            launch_pdl(prefill_embed_kernel, dim3(n), dim3(kRowThreads), 0, s, tokens, (int64_t)T, b, t0,
+                       static_cast<const uint16_t *>(a.embed), sc.x, a.H, a.V, a.state, 0);
+            launch_pdl(prefill_rows_kernel, dim3(1), dim3(32), 0, s, sc.rows, sc.rows + R, n, b, t0,
+                       static_cast<const State *>(a.state), 0);
             const int chunks = std::max(1, std::min(kPrefillChunks, (t0 + n) / 128));
             err = rows_through_layers(a, sc, n, chunks, false, s);
         }
@@ -553,22 +593,24 @@ std::string decode_tc(const PrefillTc &a, const int32_t *tokens, int32_t *next, 
     std::string err;
     for (int b0 = 0; b0 < a.B && err.empty(); b0 += R) {
         const int n = std::min(R, a.B - b0);
-        prefill_embed_kernel<<<n, kRowThreads, 0, s>>>(tokens + b0, 0, -1, 0, static_cast<const uint16_t *>(a.embed),
-                                                      sc.x, a.H, a.V, a.state, b0);
-        prefill_rows_kernel<<<1, 32, 0, s>>>(sc.rows, sc.rows + R, n, -1, 0, a.state, b0);
+        launch_pdl(prefill_embed_kernel, dim3(n), dim3(kRowThreads), 0, s, tokens + b0, (int64_t)0, -1, 0,
+                   static_cast<const uint16_t *>(a.embed), sc.x, a.H, a.V, a.state, b0);
+        launch_pdl(prefill_rows_kernel, dim3(1), dim3(32), 0, s, sc.rows, sc.rows + R, n, -1, 0,
+                   static_cast<const State *>(a.state), b0);
         err = rows_through_layers(a, sc, n, chunks, true, s);
         if (!err.empty()) break;
-        prefill_norm_kernel<<<n, kRowThreads, 0, s>>>(sc.x, static_cast<const uint16_t *>(a.final_norm), sc.h, n, a.H,
-                                                     pk(a.lm), a.eps);
+        launch_pdl(prefill_norm_kernel, dim3(n), dim3(kRowThreads), 0, s, sc.x,
+                   static_cast<const uint16_t *>(a.final_norm), sc.h, n, a.H, pk(a.lm), a.eps);
         const cudaError_t e = launch_linear_tc_packed(sc.h, a.lm_w, sc.y, 2 * n, pk(a.lm), pm(a.lm), a.lm.kc,
-                                                      a.lm.rows, s);
+                                                      a.lm.rows, s, true);
         if (e != cudaSuccess) {
             err = std::string("LM head: ") + cudaGetErrorString(e);
             break;
         }
-        rows_argmax_kernel<<<n, 1024, 0, s>>>(sc.y, pm(a.lm), n, logits, next, a.V, b0, a.state);
+        launch_pdl(rows_argmax_kernel, dim3(n), dim3(1024), 0, s, static_cast<const float *>(sc.y), pm(a.lm), n, logits,
+                   next, a.V, b0, a.state);
     }
-    if (err.empty()) advance_pos_kernel<<<1, 1, 0, s>>>(a.state);
+    if (err.empty()) launch_pdl(advance_pos_kernel, dim3(1), dim3(1), 0, s, a.state);
     return last_error(err);
 }
 
