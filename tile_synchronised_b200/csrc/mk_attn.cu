@@ -51,6 +51,9 @@ struct AttnArgs {
     // sequence, each attending causally); else row b is sequence b
     const int *row_seq, *row_len;
     int pdl;  // launch both kernels with programmatic dependent launch (a step's chain of kernels)
+    // if set, the combine writes bf16 hi / lo pairs here (rows b and B + b,
+    // nq * d wide) instead of fp32 to out
+    uint16_t *hilo;
 };
 
 // One CTA = one (chunk, KV head, sequence).  Warps split the G heads
@@ -409,7 +412,14 @@ __global__ void attn_combine_kernel(AttnArgs a) {
         O = fmaf(f, rec[(size_t)c * (d + 2) + e], O);
         L = fmaf(f, rec[(size_t)c * (d + 2) + d + 1], L);
     }
-    a.out[((size_t)b * a.nq + h) * d + e] = O / L;
+    const float o = O / L;
+    if (a.hilo) {
+        const uint16_t hi = f2bf(o);
+        a.hilo[((size_t)b * a.nq + h) * d + e] = hi;
+        a.hilo[((size_t)(a.B + b) * a.nq + h) * d + e] = f2bf(o - bf2f(hi));
+    } else {
+        a.out[((size_t)b * a.nq + h) * d + e] = o;
+    }
 }
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s) {
@@ -463,9 +473,9 @@ cudaError_t launch_attention_dev(const float *q, const void *k, const void *v, i
 // rows of a prefill chunk), `chunks` split-KV chunks per row.
 cudaError_t launch_attention_rows(const float *q, const void *k, const void *v, int rows, int nq, int nkv, int d,
                                   int max_seq, const int *row_seq, const int *row_len, int chunks, float *out,
-                                  float *part, cudaStream_t s, bool pdl) {
+                                  float *part, cudaStream_t s, bool pdl, void *hilo) {
     AttnArgs a{q, static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), out, part, rows, nq, nkv, d,
-               max_seq, max_seq, chunks, nullptr, row_seq, row_len, pdl ? 1 : 0};
+               max_seq, max_seq, chunks, nullptr, row_seq, row_len, pdl ? 1 : 0, static_cast<uint16_t *>(hilo)};
     return launch_attention(a, s);
 }
 

@@ -37,9 +37,12 @@ cudaError_t launch_linear_tc_packed(const void *x, const void *w, float *y, int 
                                     cudaStream_t s, bool pdl = false);
 // Causal attention of prefill rows (mk_attn.cu): row r of q / out attends
 // positions 0 .. row_len[r] - 1 of sequence row_seq[r] of one layer's cache.
+// With `hilo` set, the output goes there instead of `out`, as the bf16 pair
+// hi = bf16(o), lo = bf16(o - hi) in rows r and rows + r (ld columns apart,
+// ld = nq * d): the tensor cores' input form.
 cudaError_t launch_attention_rows(const float *q, const void *k, const void *v, int rows, int nq, int nkv, int d,
                                   int max_seq, const int *row_seq, const int *row_len, int chunks, float *out,
-                                  float *part, cudaStream_t s, bool pdl = false);
+                                  float *part, cudaStream_t s, bool pdl = false, void *hilo = nullptr);
 // The tensor-core prefill of a megakernel context (mk_tcdec.cu): positions
 // 0 .. T-1 of every sequence through the decoder in chunks of kPrefillRows,
 // every projection one tensor-core GEMM over the packed weights.  Fills the KV

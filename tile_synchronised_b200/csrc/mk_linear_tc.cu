@@ -38,6 +38,7 @@ constexpr int kLinBK = 64;    // K per stage: one 128-byte swizzle row of bf16
 constexpr int kLinThreads = 128;
 constexpr int kLinMaxSplit = 4;
 constexpr int kLinMaxB = 64;
+constexpr int kLinMaxStages = 6;
 
 struct LinShape {
     int Bp, rows, K, M, stages;      // Bp: the MMA's N (B rounded up to 16); rows: B
@@ -215,11 +216,14 @@ static bool lin_plan(int B, int K, int M, LinPlan &p) {
     sh.a_bytes = (uint32_t)kLinM * kLinBK * 2;                      // 16 KB of W
     sh.stage_bytes = sh.a_bytes + (uint32_t)sh.Bp * kLinBK * 2;     // + Bp rows of x, a multiple of 2 KB
     const int budget = 227 * 1024 - 1024 - 256;                    // alignment slack and the barriers
-    sh.stages = budget / (int)sh.stage_bytes;
-    if (sh.stages > 6) sh.stages = 6;
-    if (sh.stages < 2) return false;
     p.tiles = (M + kLinM - 1) / kLinM;
     const int nkb = K / kLinBK;
+    // up to 6 stages (96 KB of weights in flight; 12 measured slower, the LM
+    // head at 0.76 of HBM against 0.96), never more than the K blocks there are
+    sh.stages = budget / (int)sh.stage_bytes;
+    if (sh.stages > kLinMaxStages) sh.stages = kLinMaxStages;
+    if (sh.stages > nkb) sh.stages = nkb;
+    if (sh.stages < 2) return false;
     // K split across a cluster while the grid stays within one wave of SMs,
     // every CTA keeps at least two K blocks, and the first CTA's stage
     // memory holds the other CTAs' accumulators.

@@ -38,7 +38,10 @@ namespace mk {
 namespace tcdec {
 
 constexpr int kRowThreads = 256;
-constexpr int kArgmaxThreads = 1024;
+constexpr int kArgmaxThreads = 512;
+constexpr int kArgParts = 32;     // slices of a row's logits in the first argmax pass (one warp reduces them)
+constexpr int kNormThreads = 1024;
+constexpr int kNormPer = 8;       // RMSNorm rows up to kNormThreads * kNormPer = 8192 wide
 constexpr int kMaxBatch = 32;      // 2 * batch rows must fit mk_linear_tc's 64
 constexpr int kMaxChunks = 64;     // the split-KV chunk count never exceeds this
 
@@ -266,19 +269,44 @@ __global__ void prefill_embed_kernel(const int32_t *tok, int64_t tok_stride, int
     for (int i = threadIdx.x; i < H; i += blockDim.x) x[(size_t)r * H + i] = bf2f(E[(size_t)t * H + i]);
 }
 
-// out rows r (hi) and R + r (lo), Kp wide = RMSNorm(x[r]) * g, zero past H.
-__global__ void prefill_norm_kernel(const float *x, const uint16_t *g, __nv_bfloat16 *out, int R, int H, int Kp,
-                                    float eps) {
+// x[r] += y[r][:H] + y[R + r][:H] when y is given (the residual add of a
+// projection's hi and lo outputs, y rows M wide), then out rows r and R + r
+// (Kp wide) = hi / lo of RMSNorm(x[r]) * g, zero past H.  One block per row
+// with the whole row in registers (H <= kNormThreads * kNormPer): every load
+// of the row is in flight at once, and x is read and written once.
+__global__ void __launch_bounds__(kNormThreads) residual_norm_kernel(float *x, const float *y, int M,
+                                                                     const uint16_t *g, __nv_bfloat16 *out, int R,
+                                                                     int H, int Kp, float eps) {
     row_pass_prologue();
     __shared__ float red[32];
-    const int r = blockIdx.x;
-    const float *xr = x + (size_t)r * H;
+    const int r = blockIdx.x, t = threadIdx.x;
+    float *xr = x + (size_t)r * H;
+    float v[kNormPer];
     float ss = 0.f;
-    for (int i = threadIdx.x; i < H; i += blockDim.x) ss = fmaf(xr[i], xr[i], ss);
+#pragma unroll
+    for (int j = 0; j < kNormPer; ++j) {
+        const int i = t + j * kNormThreads;
+        float xv = 0.f;
+        if (i < H) {
+            xv = xr[i];
+            if (y) xv += y[(size_t)r * M + i] + y[(size_t)(R + r) * M + i];
+        }
+        v[j] = xv;
+        ss = fmaf(xv, xv, ss);
+    }
+    if (y)
+#pragma unroll
+        for (int j = 0; j < kNormPer; ++j)
+            if (t + j * kNormThreads < H) xr[t + j * kNormThreads] = v[j];
     ss = block_sum(ss, red);
     const float rs = rsqrtf(ss / (float)H + eps);
-    for (int i = threadIdx.x; i < Kp; i += blockDim.x)
-        put_hilo(out + (size_t)r * Kp + i, out + (size_t)(R + r) * Kp + i, i < H ? xr[i] * rs * bf2f(g[i]) : 0.f);
+#pragma unroll
+    for (int j = 0; j < kNormPer; ++j) {
+        const int i = t + j * kNormThreads;
+        if (i < Kp) put_hilo(out + (size_t)r * Kp + i, out + (size_t)(R + r) * Kp + i, i < H ? v[j] * rs * bf2f(g[i]) : 0.f);
+    }
+    for (int i = t + kNormPer * kNormThreads; i < Kp; i += kNormThreads)
+        put_hilo(out + (size_t)r * Kp + i, out + (size_t)(R + r) * Kp + i, 0.f);
 }
 
 // One block per (head, row), head_dim threads, over the packed QKV output y
@@ -331,52 +359,75 @@ __global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, in
     }
 }
 
-// One block per row of a decode pass: logits[seq0 + r][v] = y[r][v] + y[n + r][v]
-// (y rows ldy wide; written when `logits` is set) and next[seq0 + r] = their
-// argmax, lowest index on ties.  With no finite logit (a projection whose
-// bounded wait ran out writes NaN) next is 0 and the state's error word gets
-// code 5.
-__global__ void rows_argmax_kernel(const float *y, int ldy, int n, float *logits, int32_t *next, int V, int seq0,
-                                   State *state) {
+// The argmax of each row's logits y[r] + y[n + r] (hi and lo outputs, ldy
+// apart), lowest index on ties, NaN never chosen, in two passes: block (p, r)
+// reduces the p-th of kArgParts slices of row r (and copies its logits out
+// when asked), then argmax_final_kernel reduces the slices' winners.  The
+// rule is a total order on (value, index), so the result does not depend on
+// the order of the reductions.
+__device__ __forceinline__ void arg_better(float &bv, int &bi, float ov, int oi) {
+    if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+    }
+}
+
+__global__ void __launch_bounds__(kArgmaxThreads) argmax_part_kernel(const float *y, int ldy, int n, float *logits,
+                                                                     int V, int seq0, float *pv, int *pi) {
     row_pass_prologue();
     __shared__ float bv_s[32];
     __shared__ int bi_s[32];
-    const int r = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int p = blockIdx.x, r = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int v0 = (int)((long long)p * V / kArgParts), v1 = (int)((long long)(p + 1) * V / kArgParts);
     float bv = -INFINITY;
     int bi = 0x7fffffff;
-    for (int v = threadIdx.x; v < V; v += blockDim.x) {
-        const float l = y[(size_t)r * ldy + v] + y[(size_t)(n + r) * ldy + v];
-        if (logits) logits[(size_t)(seq0 + r) * V + v] = l;
-        if (l > bv || (l == bv && v < bi)) {
-            bv = l;
-            bi = v;
+    for (int base = v0 + (int)threadIdx.x; base < v1; base += 4 * kArgmaxThreads) {
+        float l[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int v = base + u * kArgmaxThreads;
+            l[u] = v < v1 ? y[(size_t)r * ldy + v] + y[(size_t)(n + r) * ldy + v] : -INFINITY;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int v = base + u * kArgmaxThreads;
+            if (v < v1) {
+                if (logits) logits[(size_t)(seq0 + r) * V + v] = l[u];
+                arg_better(bv, bi, l[u], v);
+            }
         }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
-        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-            bv = ov;
-            bi = oi;
-        }
-    }
+    for (int o = 16; o > 0; o >>= 1)
+        arg_better(bv, bi, __shfl_xor_sync(0xFFFFFFFFu, bv, o), __shfl_xor_sync(0xFFFFFFFFu, bi, o));
     if (lane == 0) {
         bv_s[warp] = bv;
         bi_s[warp] = bi;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
-            if (bv_s[w] > bv_s[0] || (bv_s[w] == bv_s[0] && bi_s[w] < bi_s[0])) {
-                bv_s[0] = bv_s[w];
-                bi_s[0] = bi_s[w];
-            }
-        if (bi_s[0] == 0x7fffffff) {
+        for (int w = 1; w < kArgmaxThreads / 32; ++w) arg_better(bv, bi, bv_s[w], bi_s[w]);
+        pv[r * kArgParts + p] = bv;
+        pi[r * kArgParts + p] = bi;
+    }
+}
+
+// One warp per row over its kArgParts slice winners; a row without a finite
+// or infinite logit (all NaN) decodes token 0 and sets the state's error.
+__global__ void argmax_final_kernel(const float *pv, const int *pi, int32_t *next, int seq0, State *state) {
+    row_pass_prologue();
+    const int r = blockIdx.x, lane = threadIdx.x;
+    float bv = pv[r * kArgParts + lane];
+    int bi = pi[r * kArgParts + lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        arg_better(bv, bi, __shfl_xor_sync(0xFFFFFFFFu, bv, o), __shfl_xor_sync(0xFFFFFFFFu, bi, o));
+    if (lane == 0) {
+        if (bi == 0x7fffffff) {
             atomicCAS(&state->err, 0u, 5u);
-            bi_s[0] = 0;
+            bi = 0;
         }
-        next[seq0 + r] = bi_s[0];
+        next[seq0 + r] = bi;
     }
 }
 
@@ -392,14 +443,6 @@ __global__ void prefill_cast_kernel(const float *a, __nv_bfloat16 *out, int R, i
     const int r = blockIdx.y;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < Kp; i += gridDim.x * blockDim.x)
         put_hilo(out + (size_t)r * Kp + i, out + (size_t)(R + r) * Kp + i, i < n ? a[(size_t)r * n + i] : 0.f);
-}
-
-// x[r][i] += y[r][i] + y[R + r][i], y rows M wide.
-__global__ void prefill_residual_kernel(float *x, const float *y, int R, int H, int M) {
-    row_pass_prologue();
-    const int r = blockIdx.y;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < H; i += gridDim.x * blockDim.x)
-        x[(size_t)r * H + i] += y[(size_t)r * M + i] + y[(size_t)(R + r) * M + i];
 }
 
 // The packed gate/up output y [2R][M] interleaves them tile by tile: packed
@@ -521,8 +564,9 @@ std::string rows_through_layers(const PrefillTc &a, const RowsScratch &sc, int n
     for (int l = 0; l < a.L && err.empty(); ++l) {
         const LayerW &W = a.layers[l];
         uint16_t *kc = a.kcache + (size_t)l * layer_elems, *vc = a.vcache + (size_t)l * layer_elems;
-        launch_pdl(prefill_norm_kernel, dim3(n), dim3(kRowThreads), 0, s, sc.x,
-                   static_cast<const uint16_t *>(W.attn_norm), sc.h, n, a.H, pk(a.qkv), a.eps);
+        if (l == 0)  // later layers get their normalised input from the previous layer's last residual add
+            launch_pdl(residual_norm_kernel, dim3(n), dim3(kNormThreads), 0, s, sc.x, static_cast<const float *>(nullptr),
+                       0, static_cast<const uint16_t *>(W.attn_norm), sc.h, n, a.H, pk(a.qkv), a.eps);
         lin(W.qkv, a.qkv);
         if (!err.empty()) break;
         launch_pdl(prefill_qkv_kernel, dim3((unsigned)(a.nq + 2 * a.nkv), (unsigned)n), dim3(a.d),
@@ -530,24 +574,33 @@ std::string rows_through_layers(const PrefillTc &a, const RowsScratch &sc, int n
                    static_cast<const uint16_t *>(W.q_norm), static_cast<const uint16_t *>(W.k_norm), a.qk_norm, a.eps,
                    a.theta, sc.rows, sc.rows + R, sc.q, kc, vc, a.max_seq);
         if (!full && l == a.L - 1) break;  // a prefill keeps only the cache: the last layer ends at its K/V
+        // the attention output goes straight into the O projection's hi / lo
+        // input rows when their width is the logical one (no padding to clear)
+        const bool direct = pk(a.o) == a.nq * a.d;
         const cudaError_t e = launch_attention_rows(sc.q, kc, vc, n, a.nq, a.nkv, a.d, a.max_seq, sc.rows,
-                                                    sc.rows + R, chunks, sc.attn, sc.part, s, true);
+                                                    sc.rows + R, chunks, sc.attn, sc.part, s, true,
+                                                    direct ? static_cast<void *>(sc.h) : nullptr);
         if (e != cudaSuccess) {
             err = std::string("attention: ") + cudaGetErrorString(e);
             break;
         }
-        launch_pdl(prefill_cast_kernel, dim3(8, (unsigned)n), dim3(kRowThreads), 0, s, sc.attn, sc.h, n, a.nq * a.d,
-                   pk(a.o));
+        if (!direct)
+            launch_pdl(prefill_cast_kernel, dim3(8, (unsigned)n), dim3(kRowThreads), 0, s, sc.attn, sc.h, n,
+                       a.nq * a.d, pk(a.o));
         lin(W.o, a.o);
-        launch_pdl(prefill_residual_kernel, dim3(8, (unsigned)n), dim3(kRowThreads), 0, s, sc.x, sc.y, n, a.H, pm(a.o));
-        launch_pdl(prefill_norm_kernel, dim3(n), dim3(kRowThreads), 0, s, sc.x,
-                   static_cast<const uint16_t *>(W.mlp_norm), sc.h, n, a.H, pk(a.gu), a.eps);
+        launch_pdl(residual_norm_kernel, dim3(n), dim3(kNormThreads), 0, s, sc.x, static_cast<const float *>(sc.y),
+                   pm(a.o), static_cast<const uint16_t *>(W.mlp_norm), sc.h, n, a.H, pk(a.gu), a.eps);
         lin(W.gu, a.gu);
         launch_pdl(prefill_swiglu_kernel, dim3(32, (unsigned)n), dim3(kRowThreads), 0, s, sc.y, sc.h, n, a.I,
                    pm(a.gu), a.gu.rows, pk(a.down));
         lin(W.down, a.down);
-        launch_pdl(prefill_residual_kernel, dim3(8, (unsigned)n), dim3(kRowThreads), 0, s, sc.x, sc.y, n, a.H,
-                   pm(a.down));
+        // the residual add, then the next layer's input norm (after the last
+        // layer, the final norm ahead of the LM head)
+        const bool last = l + 1 == a.L;
+        launch_pdl(residual_norm_kernel, dim3(n), dim3(kNormThreads), 0, s, sc.x, static_cast<const float *>(sc.y),
+                   pm(a.down),
+                   static_cast<const uint16_t *>(last ? a.final_norm : a.layers[l + 1].attn_norm), sc.h, n, a.H,
+                   last ? pk(a.lm) : pk(a.qkv), a.eps);
     }
     return err;
 }
@@ -597,18 +650,20 @@ std::string decode_tc(const PrefillTc &a, const int32_t *tokens, int32_t *next, 
                    static_cast<const uint16_t *>(a.embed), sc.x, a.H, a.V, a.state, b0);
         launch_pdl(prefill_rows_kernel, dim3(1), dim3(32), 0, s, sc.rows, sc.rows + R, n, -1, 0,
                    static_cast<const State *>(a.state), b0);
-        err = rows_through_layers(a, sc, n, chunks, true, s);
+        err = rows_through_layers(a, sc, n, chunks, true, s);  // ends with the final norm
         if (!err.empty()) break;
-        launch_pdl(prefill_norm_kernel, dim3(n), dim3(kRowThreads), 0, s, sc.x,
-                   static_cast<const uint16_t *>(a.final_norm), sc.h, n, a.H, pk(a.lm), a.eps);
         const cudaError_t e = launch_linear_tc_packed(sc.h, a.lm_w, sc.y, 2 * n, pk(a.lm), pm(a.lm), a.lm.kc,
                                                       a.lm.rows, s, true);
         if (e != cudaSuccess) {
             err = std::string("LM head: ") + cudaGetErrorString(e);
             break;
         }
-        launch_pdl(rows_argmax_kernel, dim3(n), dim3(1024), 0, s, static_cast<const float *>(sc.y), pm(a.lm), n, logits,
-                   next, a.V, b0, a.state);
+        float *pv = sc.part;  // the attention partials are free again
+        int *pi = reinterpret_cast<int *>(sc.part + kPrefillRows * kArgParts);
+        launch_pdl(argmax_part_kernel, dim3(kArgParts, (unsigned)n), dim3(kArgmaxThreads), 0, s,
+                   static_cast<const float *>(sc.y), pm(a.lm), n, logits, a.V, b0, pv, pi);
+        launch_pdl(argmax_final_kernel, dim3(n), dim3(kArgParts), 0, s, static_cast<const float *>(pv),
+                   static_cast<const int *>(pi), next, b0, a.state);
     }
     if (err.empty()) launch_pdl(advance_pos_kernel, dim3(1), dim3(1), 0, s, a.state);
     return last_error(err);
