@@ -344,6 +344,27 @@ mk_status mk_linear_tc(const void *x, const void *w, float *y, int B, int K, int
 /* The K split (1, 2 or 4 CTAs per row tile) mk_linear_tc uses for this shape;
  * host only.  MK_ERR_UNSUPPORTED for shapes mk_linear_tc refuses. */
 mk_status mk_linear_tc_split(int B, int K, int M, int *split);
+/* The same product as stream-K work sharing, for projections whose row tiles
+ * do not fill the SMs evenly (a 4096-row projection has 32 tiles of 128
+ * rows, a 28672-row one 224, one and a half waves): the tiles x K/64 units
+ * are cut into one contiguous range per CTA, at most one CTA per SM, so
+ * every SM streams the same number of weight bytes.  A tile split between
+ * CTAs is finished by the CTA holding its first K block, which adds the
+ * other CTAs' partial sums in CTA order after they raise a flag (the sum is
+ * deterministic).  `workspace` is device memory of
+ * mk_linear_tc_streamk_workspace_bytes() bytes, 16-byte aligned, zero-filled
+ * before its first use; every call that completes leaves it as it found it
+ * (zero flags); after a call whose device-side wait ran out (NaN outputs)
+ * zero it again.  Calls sharing a workspace must not run concurrently.  Falls
+ * back to mk_linear_tc's launch where one tile per CTA already fills the
+ * SMs (mk_linear_tc_streamk_grid returns 0 then).  Arguments and errors as
+ * mk_linear_tc; NULL or short workspace: MK_ERR_INVALID. */
+size_t mk_linear_tc_streamk_workspace_bytes(void);
+mk_status mk_linear_tc_streamk(const void *x, const void *w, float *y, int B, int K, int M, void *workspace,
+                               size_t workspace_bytes, void *stream);
+/* CTAs the stream-K launch of (B, K, M) uses on the current device, 0 when
+ * mk_linear_tc_streamk runs the one-tile-per-CTA kernel instead. */
+int mk_linear_tc_streamk_grid(int B, int K, int M);
 
 /* A batched decode step whose projections all run on the tensor cores
  * (mk_linear_tc) and whose attention is the split-KV pair of kernels above

@@ -200,6 +200,28 @@ def test_linear_tc_plan_and_argument_checks_need_no_device():
     assert lib.mk_linear_tc(d, d, d, 128, 4096, 4096, None) == _lib.MK_ERR_UNSUPPORTED
 
 
+def test_linear_tc_streamk_plan_and_argument_checks_need_no_device():
+    lib = _lib.load()
+    d = C.c_void_p(256)
+    need = mkpy.linear_tc_streamk_workspace_bytes()
+    assert need == 256 * 64 * 128 * 4 + 256 * 4  # contributions of up to 256 CTAs x 64 columns, then the flags
+    # one CTA per SM (148 without a device) whenever each gets at least 4 units of 128 rows x 64 K
+    assert mkpy.linear_tc_streamk_grid(16, 4096, 4096) == 148    # 32 tiles x 64 K blocks
+    assert mkpy.linear_tc_streamk_grid(32, 4096, 24576) == 148   # 192 tiles: 1.3 waves of the plain kernel
+    assert mkpy.linear_tc_streamk_grid(32, 4096, 28672) == 0     # 224 tiles: 1.5 waves, plain does as well
+    assert mkpy.linear_tc_streamk_grid(5, 320, 200) == 2         # 10 units
+    assert mkpy.linear_tc_streamk_grid(1, 128, 128) == 0         # 2 units: too few to share
+    assert mkpy.linear_tc_streamk_grid(16, 4096, 128256) == 0    # 1002 tiles: many waves already
+    assert mkpy.linear_tc_streamk_grid(16, 4096, 18944) == 0     # 148 tiles: exactly one wave
+    assert lib.mk_linear_tc_streamk(None, d, d, 16, 4096, 4096, d, need, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_linear_tc_streamk(d, d, d, 16, 4096, 4096, None, need, None) == _lib.MK_ERR_INVALID
+    assert lib.mk_linear_tc_streamk(d, d, d, 16, 4096, 4096, C.c_void_p(264), need, None) == _lib.MK_ERR_INVALID
+    assert "aligned" in lib.mk_last_error(None).decode()
+    assert lib.mk_linear_tc_streamk(d, d, d, 16, 4096, 4096, d, need - 1, None) == _lib.MK_ERR_INVALID
+    assert "workspace needs" in lib.mk_last_error(None).decode()
+    assert lib.mk_linear_tc_streamk(d, d, d, 16, 4000, 4096, d, need, None) == _lib.MK_ERR_UNSUPPORTED
+
+
 def _fake_weights(n_layers, keep):
     """An mk_weights struct whose every pointer is a fake, aligned address (the
     host-side checks never dereference them)."""

@@ -270,6 +270,44 @@ def linear_tc(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
     return out
 
 
+_streamk_ws = {}
+
+
+def linear_tc_streamk(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """linear_tc with stream-K work sharing (equal weight bytes per SM where
+    the row tiles alone would not fill the SMs).  `workspace`: a zero-filled
+    uint8 CUDA tensor of linear_tc_streamk_workspace_bytes() bytes, or None
+    for one kept per device (calls sharing it must not overlap)."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16 or x.dim() != 2 or w.dim() != 2:
+        raise ValueError("x must be bf16 [B, K] and w bf16 [M, K]")
+    if not (x.is_contiguous() and w.is_contiguous()) or x.shape[1] != w.shape[1]:
+        raise ValueError("x and w must be contiguous with the same K")
+    B, K = x.shape
+    M = w.shape[0]
+    if out is None:
+        out = torch.empty((B, M), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        key = x.device.index
+        if key not in _streamk_ws:
+            _streamk_ws[key] = torch.zeros(linear_tc_streamk_workspace_bytes(), dtype=torch.uint8, device=x.device)
+        workspace = _streamk_ws[key]
+    check(load().mk_linear_tc_streamk(C.c_void_p(x.data_ptr()), C.c_void_p(w.data_ptr()),
+                                      C.c_void_p(out.data_ptr()), B, K, M, C.c_void_p(workspace.data_ptr()),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+          None, "mk_linear_tc_streamk", op=True)
+    return out
+
+
+def linear_tc_streamk_workspace_bytes() -> int:
+    return int(load().mk_linear_tc_streamk_workspace_bytes())
+
+
+def linear_tc_streamk_grid(B: int, K: int, M: int) -> int:
+    """CTAs of the stream-K launch for this shape, 0 where it falls back."""
+    return int(load().mk_linear_tc_streamk_grid(B, K, M))
+
+
 def linear_tc_split(B: int, K: int, M: int) -> int:
     """CTAs per row tile (K split) linear_tc uses for this shape."""
     s = C.c_int()

@@ -30,7 +30,8 @@ EXPORTS = ("mk_create", "mk_destroy", "mk_last_error", "mk_workspace_bytes", "mk
            "mk_get_schedule", "mk_schedule_info", "mk_validate_schedule", "mk_swiglu_stage1",
            "mk_swiglu_tune", "mk_attention_decode", "mk_attention_scratch_bytes", "mk_attention_chunks",
            "mk_attention_decode_noalloc", "mk_attention_noalloc_limit_bytes", "mk_linear_tc",
-           "mk_linear_tc_split", "mk_tcdec_create", "mk_tcdec_workspace_bytes", "mk_tcdec_bind", "mk_tcdec_step",
+           "mk_linear_tc_split", "mk_linear_tc_streamk", "mk_linear_tc_streamk_workspace_bytes",
+           "mk_linear_tc_streamk_grid", "mk_tcdec_create", "mk_tcdec_workspace_bytes", "mk_tcdec_bind", "mk_tcdec_step",
            "mk_tcdec_status", "mk_tcdec_last_error", "mk_tcdec_destroy", "mk_tcdec_set_graph")
 
 
@@ -113,6 +114,9 @@ def load() -> C.CDLL:
         "mk_attention_noalloc_limit_bytes": ([], sz),
         "mk_linear_tc": ([vp, vp, vp, i32, i32, i32, vp], st),
         "mk_linear_tc_split": ([i32, i32, i32, C.POINTER(i32)], st),
+        "mk_linear_tc_streamk": ([vp, vp, vp, i32, i32, i32, vp, sz, vp], st),
+        "mk_linear_tc_streamk_workspace_bytes": ([], sz),
+        "mk_linear_tc_streamk_grid": ([i32, i32, i32], i32),
         "mk_tcdec_create": ([C.POINTER(MkConfig), C.POINTER(MkWeights), C.POINTER(vp)], st),
         "mk_tcdec_workspace_bytes": ([vp, C.POINTER(sz)], st),
         "mk_tcdec_bind": ([vp, vp, vp], st),

@@ -35,6 +35,14 @@ cudaError_t launch_attention_dev(const float *q, const void *k, const void *v, i
 // x bf16 [B][K] (K = the packed width, zero past the logical one).
 cudaError_t launch_linear_tc_packed(const void *x, const void *w, float *y, int B, int K, int M, int kc, int rows,
                                     cudaStream_t s, bool pdl = false);
+// The same as a stream-K launch when the tiles would not fill the SMs evenly
+// (mk_linear_tc.cu): ws holds kSkWorkspaceFloats floats and flags
+// kSkWorkspaceFlags words, zero before the first launch (every launch leaves
+// them zero); falls back to the launch above otherwise.
+constexpr size_t kSkWorkspaceFloats = (size_t)256 * 64 * 128;
+constexpr size_t kSkWorkspaceFlags = 256;
+cudaError_t launch_linear_tc_packed_sk(const void *x, const void *w, float *y, int B, int K, int M, int kc, int rows,
+                                       float *ws, uint32_t *flags, cudaStream_t s, bool pdl);
 // Causal attention of prefill rows (mk_attn.cu): row r of q / out attends
 // positions 0 .. row_len[r] - 1 of sequence row_seq[r] of one layer's cache.
 // With `hilo` set, the output goes there instead of `out`, as the bf16 pair

@@ -39,6 +39,9 @@ constexpr int kLinThreads = 128;
 constexpr int kLinMaxSplit = 4;
 constexpr int kLinMaxB = 64;
 constexpr int kLinMaxStages = 6;
+constexpr int kSkMaxCtas = 256;  // stream-K CTAs at most (the workspace is sized for this many)
+static_assert(kSkWorkspaceFloats >= (size_t)kSkMaxCtas * kLinMaxB * kLinM && kSkWorkspaceFlags >= kSkMaxCtas,
+              "stream-K workspace");
 
 struct LinShape {
     int Bp, rows, K, M, stages;      // Bp: the MMA's N (B rounded up to 16); rows: B
@@ -200,6 +203,203 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
 }
 
+// ------------------------------------------------------------------ stream-K
+// The same product for projections with too few 128-row tiles to give every
+// SM an equal share (a 4096-row projection has 32 tiles, a 28672-row one 224,
+// i.e. 1.5 waves): the work is cut into units of one tile x one K block,
+// tiles x K/64 of them, and CTA i of G (G <= the SM count, all resident)
+// takes the contiguous units [i U / G, (i + 1) U / G).  A CTA's range
+// therefore covers at most kSkMaxSeg pieces (segments) of consecutive tiles:
+// possibly the tail of one tile, whole tiles, and the head of a last one,
+// each accumulated in its own tensor-memory columns.  A segment that holds
+// its tile's first K block belongs to that CTA (the tile's owner); a segment
+// without it (at most one per CTA, its first) is a contribution: after the
+// main loop the CTA stores that accumulator in its slot of `ws` and raises
+// its flag, before it waits for anyone.  The owner then adds the
+// contributions of the CTAs after it that hold the rest of its tile, in CTA
+// order (deterministic), writes y and lowers their flags for the next
+// launch.  Waits only run towards higher CTA indices and every CTA publishes
+// before it waits, so they always end.  The roles are the plain kernel's:
+// warp 0 lane 0 issues the copies, warp 1 lane 0 the MMAs, and all four
+// warps run the epilogue.
+constexpr int kSkMaxSeg = 4;
+
+struct SkArgs {
+    int G, U, nkb;    // CTAs, units (tiles x K blocks), K blocks per tile
+    float *ws;        // [G][Bp][128]: a CTA's contribution, row-contiguous
+    uint32_t *flags;  // [G]: 1 while CTA i's contribution waits in ws; zero between launches
+};
+
+__host__ __device__ inline int sk_first(const SkArgs &k, int i) { return (int)((long long)i * k.U / k.G); }
+
+__global__ void __launch_bounds__(kLinThreads, 1)
+    linear_sk_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                     float *__restrict__ y, LinShape sh, SkArgs sk) {
+    extern __shared__ __align__(1024) uint8_t lin_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(lin_smem_raw) + 1023) & ~uintptr_t(1023));
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int S = sh.stages, Bp = sh.Bp, nkb = sk.nkb;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * sh.stage_bytes);
+    uint64_t *empty = full + S;
+    uint64_t *done = empty + S;
+    volatile uint32_t *tmem_base = reinterpret_cast<volatile uint32_t *>(done + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+    const int i = blockIdx.x;
+    const int u0 = sk_first(sk, i), u1 = sk_first(sk, i + 1), n = u1 - u0;
+    const int t_first = u0 / nkb, nseg = (u1 - 1) / nkb - t_first + 1;
+    uint32_t ncols = 32;
+    while (ncols < (uint32_t)(nseg * Bp)) ncols <<= 1;
+
+    if (t == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(const_cast<uint32_t *>(tmem_base))),
+                     "r"(ncols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_base;
+    pdl_launch_dependents();
+
+    int issued = 0;
+    if (warp == 0 && lane == 0) {
+        // unit j of this CTA: tile (u0 + j) / nkb, K block (u0 + j) % nkb,
+        // stepped without divisions
+        int tile = t_first, kb = u0 - t_first * nkb;
+        auto load = [&](int j, int tl, int k, bool w_only, bool x_only) {
+            const int s = j % S, k0 = k * kLinBK;
+            uint8_t *st = smem + (size_t)s * sh.stage_bytes;
+            if (!x_only) {
+                mbar_arrive_expect_tx(&full[s], sh.stage_bytes);
+                if (sh.w_kc)
+                    tma_load_4d(st, &map_w, k0 % sh.w_kc, 0, k0 / sh.w_kc, tl * kLinM / sh.w_rows, &full[s]);
+                else
+                    tma_load_2d(st, &map_w, k0, tl * kLinM, &full[s]);
+            }
+            if (!w_only) tma_load_2d(st + sh.a_bytes, &map_x, k0, 0, &full[s]);
+        };
+        const int pre = n < S ? n : S;
+        {
+            int tl = tile, k = kb;
+            for (int j = 0; j < pre; ++j) {
+                load(j, tl, k, true, false);
+                if (++k == nkb) k = 0, ++tl;
+            }
+        }
+        pdl_wait();
+        for (int j = 0; j < pre; ++j) {
+            load(j, tile, kb, false, true);
+            if (++kb == nkb) kb = 0, ++tile;
+        }
+        issued = pre;
+        for (int j = pre; j < n; ++j) {
+            const int s = j % S;
+            if (!tc_wait(&empty[s], ((j / S) - 1) & 1u, abort)) break;
+            load(j, tile, kb, false, false);
+            if (++kb == nkb) kb = 0, ++tile;
+            issued = j + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t idesc = lin_idesc(Bp);
+        int seg = 0, kb = u0 - t_first * nkb;
+        for (int j = 0; j < n; ++j) {
+            const int s = j % S;
+            if (!tc_wait(&full[s], (j / S) & 1u, abort)) break;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint8_t *st = smem + (size_t)s * sh.stage_bytes;
+            const bool first = j == 0 || kb == 0;
+            const uint32_t d = tmem + (uint32_t)(seg * Bp);
+#pragma unroll
+            for (int ks = 0; ks < kLinBK / 16; ++ks) {
+                const uint64_t a = smem_desc_sw128(st + ks * 32, 16, 1024);
+                const uint64_t b = smem_desc_sw128(st + sh.a_bytes + ks * 32, 16, 1024);
+                tc_mma(d, a, b, idesc, (!first || ks > 0) ? 1u : 0u);
+            }
+            tc_commit(&empty[s]);
+            if (++kb == nkb) kb = 0, ++seg;
+        }
+        tc_commit(done);
+    }
+    __syncwarp();
+    bool ok = tc_wait(done, 0u, abort) && !*abort;
+    if (warp == 0 && lane == 0 && *abort)
+        for (int j = issued > S ? issued - S : 0; j < issued; ++j)
+            tc_drain(&full[j % S], (uint32_t)(j / S) & 1u, kTcTimeoutNs);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    // epilogue: thread t holds row t of a tile (tensor-memory lane t)
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const float nan = __int_as_float(0x7fc00000);
+    for (int seg = 0; seg < nseg; ++seg) {
+        const int T = t_first + seg, tu0 = T * nkb, tu1 = tu0 + nkb;
+        const bool head = u0 <= tu0, whole = head && u1 >= tu1;
+        const int m = T * kLinM + t;
+        if (!head) {  // a contribution to tile T, this CTA's first segment
+            float *slot = sk.ws + (size_t)i * Bp * kLinM + t;
+            for (int c0 = 0; c0 < Bp; c0 += 16) {
+                float v[16];
+                tmem_ld16(lane_addr + (uint32_t)(seg * Bp + c0), v);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) slot[(size_t)(c0 + c) * kLinM] = ok ? v[c] : nan;
+            }
+            __threadfence();
+            __syncthreads();
+            if (t == 0) red_release_add(&sk.flags[i], 1u);
+            continue;
+        }
+        // the owner: contributions from CTAs i+1, i+2, ... while they start inside T
+        int jend = i + 1;
+        if (!whole)
+            while (jend < sk.G && sk_first(sk, jend) < tu1) ++jend;
+        bool got = ok;
+        for (int j = i + 1; j < jend && got; ++j) {
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t it = 0;
+            while (ld_acquire_gpu(&sk.flags[j]) == 0u) {
+                __nanosleep(32);
+                if ((++it & 15u) == 0u && globaltimer_ns() - t0 > kTcTimeoutNs) {
+                    got = false;
+                    break;
+                }
+            }
+        }
+        for (int c0 = 0; c0 < Bp; c0 += 16) {
+            float v[16];
+            tmem_ld16(lane_addr + (uint32_t)(seg * Bp + c0), v);
+            if (got)
+                for (int j = i + 1; j < jend; ++j) {
+                    const float *slot = sk.ws + (size_t)j * Bp * kLinM + t;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) v[c] += slot[(size_t)(c0 + c) * kLinM];
+                }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const int b = c0 + c;
+                if (b < sh.rows && m < sh.M) y[(size_t)b * sh.M + m] = got ? v[c] : nan;
+            }
+        }
+        if (jend > i + 1) {
+            __syncthreads();  // every thread has read the contributions
+            if (t == 0)
+                for (int j = i + 1; j < jend; ++j) sk.flags[j] = 0u;
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
+}
+
 // Launch geometry of one call, worked out on the host.
 struct LinPlan {
     LinShape sh;
@@ -282,6 +482,72 @@ cudaError_t launch_linear_tc_packed(const void *x, const void *w, float *y, int 
     return launch_linear(x, w, y, B, K, M, kc, rows, s, pdl);
 }
 
+// Stream-K geometry: G CTAs (at most the SM count, at least 4 units each)
+// over tiles x K blocks; false when a CTA's range would span more than
+// kSkMaxSeg tiles (many tiles: the one-tile-per-CTA kernel then already
+// fills the SMs in several waves).
+static bool sk_plan(int B, int K, int M, int sms, LinPlan &p, SkArgs &sk) {
+    if (!lin_plan(B, K, M, p)) return false;
+    sk.nkb = K / kLinBK;
+    sk.U = p.tiles * sk.nkb;
+    sk.G = sms < sk.U / 4 ? sms : sk.U / 4;
+    if (sk.G > kSkMaxCtas) sk.G = kSkMaxCtas;
+    if (sk.G < 2) return false;
+    const int per = (sk.U + sk.G - 1) / sk.G;  // the longest range
+    if ((per + sk.nkb - 1) / sk.nkb + 1 > kSkMaxSeg) return false;
+    p.smem = p.sh.stages * (int)p.sh.stage_bytes + 1024 + 256;
+    return true;
+}
+
+static int device_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+// The stream-K grid for (B, K, M), or 0 where the one-tile-per-CTA kernel
+// does as well: one full wave with its K split, or 1.5 waves of tiles and
+// more (its later CTAs then start out of step with the first ones; a
+// 28672-row projection of 224 tiles measured 46 us plain, 48 us stream-K).
+static int sk_grid(int B, int K, int M, int sms, LinPlan &p, SkArgs &sk) {
+    if (!lin_plan(B, K, M, p)) return 0;
+    if (p.tiles * p.split == sms || 2 * p.tiles >= 3 * sms) return 0;
+    return sk_plan(B, K, M, sms, p, sk) ? sk.G : 0;
+}
+
+cudaError_t launch_linear_tc_packed_sk(const void *x, const void *w, float *y, int B, int K, int M, int kc, int rows,
+                                       float *ws, uint32_t *flags, cudaStream_t s, bool pdl) {
+    LinPlan p;
+    SkArgs sk{};
+    if (!ws || !flags || sk_grid(B, K, M, device_sms(), p, sk) == 0)
+        return launch_linear(x, w, y, B, K, M, kc, rows, s, pdl);
+    if (kc && (kc % kLinBK || K % kc || rows < 1 || kLinM % rows)) return cudaErrorInvalidValue;
+    p.sh.w_kc = kc;
+    p.sh.w_rows = rows;
+    sk.ws = ws;
+    sk.flags = flags;
+    CUtensorMap mw, mx;
+    const bool wmap = kc ? tc_make_map_packed(&mw, w, (uint64_t)((M + rows - 1) / rows), (uint32_t)(K / kc),
+                                              (uint32_t)rows, (uint32_t)kc)
+                         : tc_make_map(&mw, w, (uint64_t)M, (uint64_t)K, kLinBK, kLinM);
+    if (!wmap || !tc_make_map(&mx, x, (uint64_t)B, (uint64_t)K, kLinBK, (uint32_t)p.sh.Bp))
+        return cudaErrorInvalidValue;
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t ce = tc_allow_smem(reinterpret_cast<const void *>(linear_sk_kernel), 227 * 1024, configured);
+    if (ce != cudaSuccess) return ce;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sk.G);
+    cfg.blockDim = dim3(kLinThreads);
+    cfg.dynamicSmemBytes = (size_t)p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, linear_sk_kernel, mw, mx, y, p.sh, sk);
+}
+
 }  // namespace mk
 
 using namespace mk;
@@ -320,5 +586,55 @@ extern "C" mk_status mk_linear_tc_split(int B, int K, int M, int *split) {
     LinPlan p;
     if (!lin_plan(B, K, M, p)) return MK_ERR_UNSUPPORTED;
     *split = p.split;
+    return MK_OK;
+}
+
+extern "C" size_t mk_linear_tc_streamk_workspace_bytes(void) {
+    return kSkWorkspaceFloats * sizeof(float) + kSkWorkspaceFlags * sizeof(uint32_t);
+}
+
+extern "C" int mk_linear_tc_streamk_grid(int B, int K, int M) {
+    LinPlan p;
+    SkArgs sk{};
+    return sk_grid(B, K, M, device_sms(), p, sk);
+}
+
+extern "C" mk_status mk_linear_tc_streamk(const void *x, const void *w, float *y, int B, int K, int M,
+                                          void *workspace, size_t workspace_bytes, void *stream) {
+    if (!x || !w || !y || !workspace) {
+        set_op_error("linear_tc_streamk: null pointer");
+        return MK_ERR_INVALID;
+    }
+    if (B < 1 || K < 1 || M < 1) {
+        set_op_error("linear_tc_streamk: B, K and M must be positive");
+        return MK_ERR_INVALID;
+    }
+    for (const void *p : {x, w, static_cast<const void *>(y), static_cast<const void *>(workspace)})
+        if ((uintptr_t)p & 15) {
+            set_op_error("linear_tc_streamk: x, w, y and the workspace must be 16-byte aligned");
+            return MK_ERR_INVALID;
+        }
+    if (workspace_bytes < mk_linear_tc_streamk_workspace_bytes()) {
+        char msg[160];
+        snprintf(msg, sizeof(msg), "linear_tc_streamk: the workspace needs %zu bytes (got %zu)",
+                 mk_linear_tc_streamk_workspace_bytes(), workspace_bytes);
+        set_op_error(msg);
+        return MK_ERR_INVALID;
+    }
+    LinPlan p;
+    if (!lin_plan(B, K, M, p)) {
+        set_op_error("linear_tc_streamk: needs B <= 64 and K a multiple of 64");
+        return MK_ERR_UNSUPPORTED;
+    }
+    float *ws = static_cast<float *>(workspace);
+    uint32_t *flags = reinterpret_cast<uint32_t *>(ws + kSkWorkspaceFloats);
+    const cudaError_t e =
+        launch_linear_tc_packed_sk(x, w, y, B, K, M, 0, 0, ws, flags, static_cast<cudaStream_t>(stream), false);
+    if (e != cudaSuccess) {
+        char msg[160];
+        snprintf(msg, sizeof(msg), "linear_tc_streamk: launch failed: %s", cudaGetErrorString(e));
+        set_op_error(msg);
+        return MK_ERR_CUDA;
+    }
     return MK_OK;
 }

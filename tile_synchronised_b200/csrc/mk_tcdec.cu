@@ -349,14 +349,18 @@ __global__ void prefill_qkv_kernel(const float *y, int R, int M, int nq, int nkv
 // row_seq[r] = b, row_len[r] = t0 + r + 1: the rows' sequence and attended
 // length (a prefill chunk); for b < 0, row r is sequence r at the context's
 // current position (a decode step; read on the device, so a captured step
-// replays at any position).
-__global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, int t0, const State *state, int seq0) {
+// replays at any position).  Also clears the stream-K projections' flags
+// (left zero by every launch that completes; this heals a pass after one
+// that gave up).
+__global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, int t0, const State *state, int seq0,
+                                    uint32_t *sk_flags) {
     row_pass_prologue();
     const int r = threadIdx.x;
     if (r < R) {
         row_seq[r] = b < 0 ? seq0 + r : b;
         row_len[r] = b < 0 ? state->pos + 1 : t0 + r + 1;
     }
+    for (int i = r; i < (int)kSkWorkspaceFlags; i += blockDim.x) sk_flags[i] = 0u;
 }
 
 // The argmax of each row's logits y[r] + y[n + r] (hi and lo outputs, ldy
@@ -508,7 +512,8 @@ size_t prefill_scratch_bytes(int H, int nq, int d, int kmax, int mmax) {
     const size_t R = kPrefillRows;
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     return up(R * H * 4) + up(2 * R * kmax * 2) + up(2 * R * (size_t)mmax * 4) + 2 * up(R * nq * d * 4) +
-           up(R * nq * kPrefillChunks * (size_t)(d + 2) * 4) + up(2 * R * 4) + 2 * up(64 * 4);
+           up(R * nq * kPrefillChunks * (size_t)(d + 2) * 4) + up(2 * R * 4) + 2 * up(64 * 4) +
+           up(kSkWorkspaceFloats * 4) + up(kSkWorkspaceFlags * 4);
 }
 
 namespace {
@@ -519,6 +524,8 @@ struct RowsScratch {
     __nv_bfloat16 *h;
     int *rows;           // row_seq [kPrefillRows], then row_len [kPrefillRows]
     int32_t *tok, *nxt;  // a decode step's tokens and argmax (64 each)
+    float *skws;         // the stream-K projections' contributions
+    uint32_t *skflags;   // and their flags
 };
 
 int pk(const PackedMat &m) { return m.nkb * m.kc; }    // a packed matrix's width as a GEMM operand
@@ -544,6 +551,8 @@ bool carve(const PrefillTc &a, RowsScratch &sc) {
     sc.rows = reinterpret_cast<int *>(take((size_t)2 * R * 4));
     sc.tok = reinterpret_cast<int32_t *>(take(64 * 4));
     sc.nxt = reinterpret_cast<int32_t *>(take(64 * 4));
+    sc.skws = reinterpret_cast<float *>(take(kSkWorkspaceFloats * 4));
+    sc.skflags = reinterpret_cast<uint32_t *>(take(kSkWorkspaceFlags * 4));
     return true;
 }
 
@@ -558,7 +567,8 @@ std::string rows_through_layers(const PrefillTc &a, const RowsScratch &sc, int n
     std::string err;
     auto lin = [&](const void *w, const PackedMat &m) {
         if (!err.empty()) return;
-        const cudaError_t e = launch_linear_tc_packed(sc.h, w, sc.y, 2 * n, pk(m), pm(m), m.kc, m.rows, s, true);
+        const cudaError_t e =
+            launch_linear_tc_packed_sk(sc.h, w, sc.y, 2 * n, pk(m), pm(m), m.kc, m.rows, sc.skws, sc.skflags, s, true);
         if (e != cudaSuccess) err = std::string("projection: ") + cudaGetErrorString(e);
     };
     for (int l = 0; l < a.L && err.empty(); ++l) {
@@ -627,7 +637,7 @@ std::string prefill_tc(const PrefillTc &a, const int32_t *tokens, int T, cudaStr
             launch_pdl(prefill_embed_kernel, dim3(n), dim3(kRowThreads), 0, s, tokens, (int64_t)T, b, t0,
                        static_cast<const uint16_t *>(a.embed), sc.x, a.H, a.V, a.state, 0);
             launch_pdl(prefill_rows_kernel, dim3(1), dim3(32), 0, s, sc.rows, sc.rows + R, n, b, t0,
-                       static_cast<const State *>(a.state), 0);
+                       static_cast<const State *>(a.state), 0, sc.skflags);
             const int chunks = std::max(1, std::min(kPrefillChunks, (t0 + n) / 128));
             err = rows_through_layers(a, sc, n, chunks, false, s);
         }
@@ -649,11 +659,11 @@ std::string decode_tc(const PrefillTc &a, const int32_t *tokens, int32_t *next, 
         launch_pdl(prefill_embed_kernel, dim3(n), dim3(kRowThreads), 0, s, tokens + b0, (int64_t)0, -1, 0,
                    static_cast<const uint16_t *>(a.embed), sc.x, a.H, a.V, a.state, b0);
         launch_pdl(prefill_rows_kernel, dim3(1), dim3(32), 0, s, sc.rows, sc.rows + R, n, -1, 0,
-                   static_cast<const State *>(a.state), b0);
+                   static_cast<const State *>(a.state), b0, sc.skflags);
         err = rows_through_layers(a, sc, n, chunks, true, s);  // ends with the final norm
         if (!err.empty()) break;
-        const cudaError_t e = launch_linear_tc_packed(sc.h, a.lm_w, sc.y, 2 * n, pk(a.lm), pm(a.lm), a.lm.kc,
-                                                      a.lm.rows, s, true);
+        const cudaError_t e = launch_linear_tc_packed_sk(sc.h, a.lm_w, sc.y, 2 * n, pk(a.lm), pm(a.lm), a.lm.kc,
+                                                         a.lm.rows, sc.skws, sc.skflags, s, true);
         if (e != cudaSuccess) {
             err = std::string("LM head: ") + cudaGetErrorString(e);
             break;

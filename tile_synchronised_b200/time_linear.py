@@ -1,13 +1,14 @@
 """Time mk_linear_tc at the projection shapes of the batched decode configurations.
 
     python -m tile_synchronised_b200.time_linear [--reps 30] [--shape B K M ...]
-        [--swiglu-batch B]
+        [--streamk] [--swiglu-batch B]
 
 Prints one JSON list: per (B, K, M) the K split, the mean microseconds per call
 (CUDA events over back-to-back calls) and the achieved GB/s of the weights plus
 x and y.  Weight copies are rotated so that the timed set exceeds the 126 MB L2.
---shape (repeatable) replaces the default shapes; --swiglu-batch also times the
-tensor-core fused SwiGLU first stage (MK_SWIGLU_TC) at the 70B-shard shape.
+--shape (repeatable) replaces the default shapes; --streamk also times the
+stream-K launch (mk_linear_tc_streamk) of each shape; --swiglu-batch also times
+the tensor-core fused SwiGLU first stage (MK_SWIGLU_TC) at the 70B-shard shape.
 Also the command that ncu profiles the tensor-core kernels under.
 """
 import argparse
@@ -32,6 +33,7 @@ def main(argv=None):
     ap.add_argument("--shape", type=int, nargs=3, action="append", metavar=("B", "K", "M"),
                     help="time this (batch, K, M) instead of the default shapes (repeatable)")
     ap.add_argument("--swiglu-batch", type=int, default=0, help="also time MK_SWIGLU_TC at this batch")
+    ap.add_argument("--streamk", action="store_true", help="also time mk_linear_tc_streamk on each shape")
     a = ap.parse_args(argv)
     res = []
     for (B, K, M) in (a.shape or SHAPES):
@@ -40,19 +42,27 @@ def main(argv=None):
         ncopy = max(1, -(-300_000_000 // wb))
         ws = [w] + [w.clone() for _ in range(ncopy - 1)]
         y = torch.empty((B, M), dtype=torch.float32, device="cuda")
-        for i in range(3):
-            mk.linear_tc(x, ws[i % ncopy], out=y)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for i in range(a.reps):
-            mk.linear_tc(x, ws[i % ncopy], out=y)
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / a.reps
-        gbs = (wb + B * K * 2 + B * M * 4) / us / 1e3
-        res.append({"B": B, "K": K, "M": M, "split": mk.linear_tc_split(B, K, M), "us": round(us, 2),
-                    "GBps": round(gbs, 1), "frac": round(gbs / a.peak_gbs, 3)})
+        calls = [("plain", lambda wi: mk.linear_tc(x, wi, out=y))]
+        if a.streamk:
+            calls.append(("streamk", lambda wi: mk.linear_tc_streamk(x, wi, out=y)))
+        for kind, call in calls:
+            for i in range(3):
+                call(ws[i % ncopy])
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(a.reps):
+                call(ws[i % ncopy])
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / a.reps
+            gbs = (wb + B * K * 2 + B * M * 4) / us / 1e3
+            r = {"B": B, "K": K, "M": M, "split": mk.linear_tc_split(B, K, M), "us": round(us, 2),
+                 "GBps": round(gbs, 1), "frac": round(gbs / a.peak_gbs, 3)}
+            if a.streamk:
+                r["kind"] = kind
+                r["streamk_ctas"] = mk.linear_tc_streamk_grid(B, K, M)
+            res.append(r)
         del ws
     if a.swiglu_batch:
         B = a.swiglu_batch
