@@ -70,9 +70,9 @@ def algorithmic_bytes(shape, batch, pos):
 
 # The sources that decide what the decode step launches and what it reads:
 # the megakernel, its plan and launch code, and the headers they share (not
-# the isolated SwiGLU and attention kernels).
-STEP_SOURCES = ("mk_api.cu", "mk_device.cuh", "mk_internal.h", "mk_kernel.cu", "mk_kernel.h", "mk_sched.cpp",
-                "mk_sched.h")
+# the isolated SwiGLU, attention and tensor-core kernels, nor mk_kernel.h,
+# which only declares their entry points).
+STEP_SOURCES = ("mk_api.cu", "mk_device.cuh", "mk_internal.h", "mk_kernel.cu", "mk_sched.cpp", "mk_sched.h")
 
 
 def source_hash():
