@@ -387,13 +387,232 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_tile_kernel(AttnArgs a) 
     }
 }
 
+// The same partials with 8 dimensions per lane, for G <= 4: a cache row is
+// read by d / 8 lanes (16 bytes each, one load), so a warp reads 32 / (d / 8)
+// rows at once (its sub-warps).  Each sub-warp forms the partial dot
+// products of its positions for all G heads, and a transposing butterfly
+// over its d / 8 lanes leaves lane l of the sub-warp with the whole score of
+// pair l (position l / G of the sub-warp, head l % G); the online softmax
+// runs over the whole warp as above, each sub-warp applies the probabilities
+// of its own positions to their V rows, and the sub-warps' outputs are added
+// once at the end.  About two thirds of the instructions of the 4-dimension
+// layout per cache byte (that kernel is issue-bound).
+template <int D, int G>
+__global__ void __launch_bounds__(kAttnThreads, 2) attn_wide_kernel(AttnArgs a) {
+    pdl_wait();  // no-ops unless launched with programmatic dependent launch
+    pdl_launch_dependents();
+    static_assert(D == 64 || D == 128, "head_dim");
+    constexpr int TP = kTileBytes / (2 * D);  // positions per stage
+    constexpr int LPR = D / 8;                // lanes per cache row
+    constexpr int SUBS = 32 / LPR;            // sub-warps (rows read at once)
+    static_assert(LPR % G == 0, "G must divide d / 8");
+    constexpr int PPS = LPR / G;              // positions per sub-warp per group
+    constexpr int P = SUBS * PPS;             // positions per warp per group (32 / G)
+    constexpr unsigned FULL = 0xffffffffu;
+    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31, sub = lane / LPR, li = lane % LPR;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t *ring = smem;
+    float *pw = reinterpret_cast<float *>(smem + kTileStages * 2 * kTileBytes) + warp * 40;  // [32] p, [8] corr
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTileStages * 2 * kTileBytes + kAttnWarps * 40 * 4);
+    const int n_pos = a.row_len ? a.row_len[b] : (a.n_pos_dev ? *a.n_pos_dev : a.n_pos);
+    const int seq = a.row_seq ? a.row_seq[b] : b;
+    const int p0 = (int)((long long)c * n_pos / a.chunks), p1 = (int)((long long)(c + 1) * n_pos / a.chunks);
+    const int ntiles = p1 > p0 ? (p1 - p0 + TP - 1) / TP : 0;
+    const size_t head = ((size_t)seq * a.nkv + g) * (size_t)a.max_seq;
+    if (t == 0) {
+        for (int s = 0; s < kTileStages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const uint64_t pol = policy_evict_first();
+    auto issue = [&](int i) {
+        const int s = i % kTileStages, pos = p0 + i * TP, n = min(TP, p1 - pos);
+        const uint32_t bytes = (uint32_t)(n * D * 2);
+        uint8_t *dst = ring + (size_t)s * 2 * kTileBytes;
+        mbar_arrive_expect_tx(&full[s], 2 * bytes);
+        bulk_g2s(dst, a.k + (head + pos) * D, bytes, &full[s], pol);
+        bulk_g2s(dst + kTileBytes, a.v + (head + pos) * D, bytes, &full[s], pol);
+    };
+    if (t == 0)
+        for (int i = 0; i < ntiles && i < kTileStages; ++i) issue(i);
+
+    const float qscale = 1.4426950408889634f * rsqrtf((float)D);
+    float q[G][8], o[G][8];
+    {
+        const float *qb = a.q + ((size_t)b * a.nq + (size_t)g * G) * D + li * 8;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float4 x0 = *reinterpret_cast<const float4 *>(qb + h * D);
+            const float4 x1 = *reinterpret_cast<const float4 *>(qb + h * D + 4);
+            q[h][0] = x0.x * qscale; q[h][1] = x0.y * qscale; q[h][2] = x0.z * qscale; q[h][3] = x0.w * qscale;
+            q[h][4] = x1.x * qscale; q[h][5] = x1.y * qscale; q[h][6] = x1.z * qscale; q[h][7] = x1.w * qscale;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[h][e] = 0.f;
+        }
+    }
+    float m = -CUDART_INF_F, l = 0.f;  // running max and sum of head lane % G
+    bool bad = false;
+    int i = 0;
+    for (; i < ntiles; ++i) {
+        const int s = i % kTileStages;
+        const uint32_t par = (uint32_t)(i / kTileStages) & 1u;
+        if (!mbar_try_wait(&full[s], par)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait_sleep(&full[s], par, 10000u))
+                if (globaltimer_ns() - t0 > 2000000000ull) {
+                    bad = true;
+                    break;
+                }
+        }
+        if (!bad) {
+            const int n = min(TP, p1 - (p0 + i * TP));
+            const uint16_t *K = reinterpret_cast<const uint16_t *>(ring + (size_t)s * 2 * kTileBytes);
+            const uint16_t *V = K + kTileBytes / 2;
+            for (int base = warp * P; base < n; base += kAttnWarps * P) {
+                const int cnt = min(P, n - base);
+                float acc[LPR];
+#pragma unroll
+                for (int jj = 0; jj < PPS; ++jj) {
+                    const int row = base + min(sub * PPS + jj, cnt - 1);
+                    float kf[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(K + (size_t)row * D + li * 8), kf);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        float x = q[h][0] * kf[0];
+#pragma unroll
+                        for (int e = 1; e < 8; ++e) x = fmaf(q[h][e], kf[e], x);
+                        acc[jj * G + h] = x;
+                    }
+                }
+                // transposing butterfly within the sub-warp: lane li ends with pair li
+#pragma unroll
+                for (int off = LPR / 2; off >= 1; off >>= 1) {
+                    const bool up = li & off;
+#pragma unroll
+                    for (int r = 0; r < off; ++r) {
+                        const float send = up ? acc[r] : acc[r + off];
+                        const float keep = up ? acc[r + off] : acc[r];
+                        acc[r] = keep + __shfl_xor_sync(FULL, send, off);
+                    }
+                }
+                const int mypos = sub * PPS + li / G;  // this lane's position in the group
+                const bool valid = mypos < cnt;
+                const float sc = valid ? acc[0] : -CUDART_INF_F;
+                float gm = sc;
+#pragma unroll
+                for (int off = G; off < 32; off <<= 1) gm = fmaxf(gm, __shfl_xor_sync(FULL, gm, off));
+                const float mnew = fmaxf(m, gm);
+                const float corr = exp2f(m - mnew);
+                const float p = valid ? exp2f(sc - mnew) : 0.f;
+                float ps = p;
+#pragma unroll
+                for (int off = G; off < 32; off <<= 1) ps += __shfl_xor_sync(FULL, ps, off);
+                l = l * corr + ps;
+                m = mnew;
+                pw[sub * PPS * G + li] = p;  // index = position * G + head
+                if (lane < G) pw[32 + lane] = corr;
+                __syncwarp();
+                if (__any_sync(FULL, corr != 1.0f)) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float cr = pw[32 + h];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o[h][e] *= cr;
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < PPS; ++jj) {
+                    const int pos = sub * PPS + jj;
+                    if (pos < cnt) {
+                        float vf[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(V + (size_t)(base + pos) * D + li * 8), vf);
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float pj = pw[pos * G + h];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pj, vf[e], o[h][e]);
+                        }
+                    }
+                }
+                __syncwarp();  // pw is rewritten by the next group
+            }
+        }
+        if (__syncthreads_or(bad)) break;  // every warp is done with stage s (or some wait gave up)
+        if (t == 0 && i + kTileStages < ntiles) issue(i + kTileStages);
+    }
+    if (i < ntiles) {
+        // never leave with a copy into this CTA's shared memory in flight
+        if (t == 0)
+            for (int k = i; k < ntiles && k < i + kTileStages; ++k) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait_sleep(&full[k % kTileStages], (uint32_t)(k / kTileStages) & 1u, 10000u))
+                    if (globaltimer_ns() - t0 > 2000000000ull) break;
+            }
+        for (int x = t; x < G * D; x += kAttnThreads) {
+            const int hh = x / D, e = x % D;
+            float *rec = a.part + (((size_t)b * a.nq + (size_t)g * G + hh) * a.chunks + c) * (D + 2);
+            rec[e] = CUDART_NAN_F;
+            if (e == 0) rec[D] = rec[D + 1] = CUDART_NAN_F;
+        }
+        return;
+    }
+    // the sub-warps hold the same running max per head: their outputs add
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[h][e] += __shfl_xor_sync(FULL, o[h][e], off);
+    // merge the warps through the ring (every copy into it has landed and been read)
+    float *mo = reinterpret_cast<float *>(ring);  // [warp][G][D]
+    float *ml = mo + kAttnWarps * G * D;          // [warp][G][2]
+    if (sub == 0)
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mo[(warp * G + h) * D + li * 8 + e] = o[h][e];
+    if (lane < G) {
+        ml[(warp * G + lane) * 2] = m;
+        ml[(warp * G + lane) * 2 + 1] = l;
+    }
+    __syncthreads();
+    for (int x = t; x < G * D; x += kAttnThreads) {
+        const int hh = x / D, e = x % D;
+        float M = -CUDART_INF_F;
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, ml[(w * G + hh) * 2]);
+        float O = 0.f, L = 0.f;
+        if (M != -CUDART_INF_F)
+            for (int w = 0; w < kAttnWarps; ++w) {
+                const float mw = ml[(w * G + hh) * 2];
+                if (mw == -CUDART_INF_F) continue;
+                const float f = exp2f(mw - M);
+                O = fmaf(f, mo[(w * G + hh) * D + e], O);
+                L = fmaf(f, ml[(w * G + hh) * 2 + 1], L);
+            }
+        float *rec = a.part + (((size_t)b * a.nq + (size_t)g * G + hh) * a.chunks + c) * (D + 2);
+        rec[e] = O;
+        if (e == 0) {
+            rec[D] = M;
+            rec[D + 1] = L;
+        }
+    }
+}
+
 template <int D, int G>
 static cudaError_t launch_tile(cudaLaunchConfig_t &cfg, const AttnArgs &a) {
     static std::atomic<unsigned long long> configured{0};
     const int smem = attn_tile_smem_bytes();
     cfg.dynamicSmemBytes = (size_t)smem;
-    cudaError_t e = allow_smem(reinterpret_cast<const void *>(attn_tile_kernel<D, G>), smem, configured);
-    return e == cudaSuccess ? cudaLaunchKernelEx(&cfg, attn_tile_kernel<D, G>, a) : e;
+    // 8 dimensions per lane where q and the outputs of the G heads fit the
+    // registers of two CTAs per SM; 4 per lane for G = 8
+    constexpr bool wide = G <= 4;
+    const void *fn = wide ? reinterpret_cast<const void *>(attn_wide_kernel<D, (wide ? G : 4)>)
+                          : reinterpret_cast<const void *>(attn_tile_kernel<D, G>);
+    cudaError_t e = allow_smem(fn, smem, configured);
+    if (e != cudaSuccess) return e;
+    return wide ? cudaLaunchKernelEx(&cfg, attn_wide_kernel<D, (wide ? G : 4)>, a)
+                : cudaLaunchKernelEx(&cfg, attn_tile_kernel<D, G>, a);
 }
 
 // One CTA per (query head, sequence), one thread per output dimension.
