@@ -163,8 +163,9 @@ static cudaError_t allow_smem(const void *fn, int bytes, std::atomic<unsigned lo
 }
 
 // ------------------------------------------------------------------ tiles through a TMA ring
-// The same partials for head_dim 64 and 128 and G = 2, 4 or 8 query heads per
-// KV head, with the cache streamed by 1-D bulk copies (TMA) through a ring of
+// The same partials for head_dim 64 and 128 and G = 8 query heads per KV head
+// (attn_wide_kernel below serves G = 2 and 4 with the same ring and
+// records), with the cache streamed by 1-D bulk copies (TMA) through a ring of
 // kTileStages shared-memory stages, so that the next tiles are in flight
 // while one is consumed.  A stage holds the K rows and then the V rows of
 // kTileBytes / (2 d) consecutive positions.
@@ -606,13 +607,13 @@ static cudaError_t launch_tile(cudaLaunchConfig_t &cfg, const AttnArgs &a) {
     cfg.dynamicSmemBytes = (size_t)smem;
     // 8 dimensions per lane where q and the outputs of the G heads fit the
     // registers of two CTAs per SM; 4 per lane for G = 8
-    constexpr bool wide = G <= 4;
-    const void *fn = wide ? reinterpret_cast<const void *>(attn_wide_kernel<D, (wide ? G : 4)>)
-                          : reinterpret_cast<const void *>(attn_tile_kernel<D, G>);
-    cudaError_t e = allow_smem(fn, smem, configured);
-    if (e != cudaSuccess) return e;
-    return wide ? cudaLaunchKernelEx(&cfg, attn_wide_kernel<D, (wide ? G : 4)>, a)
-                : cudaLaunchKernelEx(&cfg, attn_tile_kernel<D, G>, a);
+    if constexpr (G <= 4) {
+        const cudaError_t e = allow_smem(reinterpret_cast<const void *>(attn_wide_kernel<D, G>), smem, configured);
+        return e == cudaSuccess ? cudaLaunchKernelEx(&cfg, attn_wide_kernel<D, G>, a) : e;
+    } else {
+        const cudaError_t e = allow_smem(reinterpret_cast<const void *>(attn_tile_kernel<D, G>), smem, configured);
+        return e == cudaSuccess ? cudaLaunchKernelEx(&cfg, attn_tile_kernel<D, G>, a) : e;
+    }
 }
 
 // One CTA per (query head, sequence), one thread per output dimension.
