@@ -157,7 +157,7 @@ mk_status mk_load_weights(mk_ctx *ctx, const mk_weights *w, void *workspace, voi
 /* Fill the KV cache from a prompt: `d_tokens` is a device int32 [batch, T]
  * row-major array; positions restart at 0 and end at T.  With the tensor-core
  * prefill (the default, see mk_set_prefill) the prompt goes through the
- * decoder 32 positions of one sequence at a time: every projection is one
+ * decoder 128 positions of one sequence at a time: every projection is one
  * tcgen05 GEMM reading the packed weight tiles of mk_load_weights in place,
  * with each activation row entering as a hi/lo pair of bf16 rows, and
  * position t attends causally to positions 0 .. t; only the KV cache is kept
@@ -333,9 +333,10 @@ mk_status mk_swiglu_tune(const void *x, const void *w_gate, const void *w_up, vo
  * projection, as given); x: device bf16 [B, K] row-major; y: device fp32
  * [B, M].  Swap-AB: 128 rows of w per CTA are the MMA's M, the batch
  * (rounded up to 16 with zero rows) its N, fp32 accumulators in tensor
- * memory; every weight byte is read once for the whole batch.  With few row
- * tiles a cluster of 2 or 4 CTAs splits K (mk_linear_tc_split) and sums in a
- * fixed order, so results are deterministic.  Needs 1 <= B <= 64,
+ * memory (up to 256 columns); every weight byte is read once for the whole
+ * batch.  With few row tiles a cluster of 2 or 4 CTAs splits K
+ * (mk_linear_tc_split) and sums in a
+ * fixed order, so results are deterministic.  Needs 1 <= B <= 256,
  * K % 64 == 0 (MK_ERR_UNSUPPORTED otherwise), M >= 1, all pointers 16-byte
  * aligned (MK_ERR_INVALID).  Asynchronous on `stream`; a device-side wait
  * that runs out (2 s) writes NaN outputs rather than hanging.  Allocates

@@ -186,7 +186,8 @@ def test_linear_tc_plan_and_argument_checks_need_no_device():
     assert mkpy.linear_tc_split(64, 14336, 4096) == 4
     s = C.c_int()
     assert lib.mk_linear_tc_split(0, 4096, 4096, C.byref(s)) == _lib.MK_ERR_UNSUPPORTED
-    assert lib.mk_linear_tc_split(65, 4096, 4096, C.byref(s)) == _lib.MK_ERR_UNSUPPORTED
+    assert lib.mk_linear_tc_split(257, 4096, 4096, C.byref(s)) == _lib.MK_ERR_UNSUPPORTED
+    assert mkpy.linear_tc_split(256, 2048, 2048) == 2     # 256 columns: the partials of 4 CTAs would not fit
     assert lib.mk_linear_tc_split(16, 4000, 4096, C.byref(s)) == _lib.MK_ERR_UNSUPPORTED
     assert lib.mk_linear_tc_split(16, 4096, 4096, None) == _lib.MK_ERR_INVALID
     # refused before any launch
@@ -197,14 +198,14 @@ def test_linear_tc_plan_and_argument_checks_need_no_device():
     assert lib.mk_linear_tc(d, d, d, 0, 4096, 4096, None) == _lib.MK_ERR_INVALID
     assert lib.mk_linear_tc(d, d, d, 16, 4000, 4096, None) == _lib.MK_ERR_UNSUPPORTED
     assert "multiple of 64" in lib.mk_last_error(None).decode()
-    assert lib.mk_linear_tc(d, d, d, 128, 4096, 4096, None) == _lib.MK_ERR_UNSUPPORTED
+    assert lib.mk_linear_tc(d, d, d, 257, 4096, 4096, None) == _lib.MK_ERR_UNSUPPORTED
 
 
 def test_linear_tc_streamk_plan_and_argument_checks_need_no_device():
     lib = _lib.load()
     d = C.c_void_p(256)
     need = mkpy.linear_tc_streamk_workspace_bytes()
-    assert need == 256 * 64 * 128 * 4 + 256 * 4  # contributions of up to 256 CTAs x 64 columns, then the flags
+    assert need == 256 * 256 * 128 * 4 + 256 * 4  # contributions of up to 256 CTAs x 256 columns, then the flags
     # one CTA per SM (148 without a device) whenever each gets at least 4 units of 128 rows x 64 K
     assert mkpy.linear_tc_streamk_grid(16, 4096, 4096) == 148    # 32 tiles x 64 K blocks
     assert mkpy.linear_tc_streamk_grid(32, 4096, 24576) == 148   # 192 tiles: 1.3 waves of the plain kernel

@@ -22,6 +22,7 @@ SHAPES = [
     (8, 4096, 4096),      # batch 8
     (5, 320, 200),        # ragged rows (2 tiles, the second partial), 5 K blocks over a pair
     (16, 4096, 128256),   # an LM head: 1002 row tiles, several waves
+    (256, 1024, 1024),    # 256 columns (a 128-position prefill chunk as hi/lo pairs), K split 2
 ]
 
 
@@ -77,6 +78,7 @@ STREAMK_SHAPES = [
     (64, 4096, 4096),     # batch 64: N = 64 accumulator columns per segment
     (3, 8192, 1000),      # ragged rows: the last tile is partial
     (5, 320, 200),        # 2 tiles x 5 K blocks over 2 CTAs
+    (256, 2048, 2048),    # 256 columns: at most 2 segments of a CTA in tensor memory
 ]
 
 

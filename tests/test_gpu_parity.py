@@ -522,12 +522,12 @@ def test_swiglu_stage1_full_size(B):
 @needs_cuda
 @pytest.mark.parametrize("case", ["tiny_b1", "tiny_b3_qknorm", "tiny_b4_ksplit", "llama1b"])
 def test_tensor_core_prefill_matches_steps_and_oracle(case):
-    """The tensor-core prefill (32 positions of a sequence per GEMM chunk,
+    """The tensor-core prefill (128 positions of a sequence per GEMM chunk,
     causal attention within the chunk) leaves a KV cache that agrees with the
     one the decode steps leave and with the oracle's, and the decode step that
     follows it matches the oracle.  The prompt lengths cover one ragged chunk
-    and several chunks with a ragged tail; one plan packs a matrix as several
-    K blocks."""
+    and two and three chunks with a ragged tail; one plan packs a matrix as
+    several K blocks."""
     import tile_synchronised_b200 as mk
     from tile_synchronised_b200 import _lib
     if case == "llama1b":
@@ -537,9 +537,9 @@ def test_tensor_core_prefill_matches_steps_and_oracle(case):
     elif case == "tiny_b4_ksplit":
         # 4 rows x 5120 fp32 exceed the 64 KB activation region: the plan
         # packs the down projection as two K blocks, read by a 4-D tensor map
-        s, B, T = synth.TINY.replace(intermediate=5120), 4, 40
+        s, B, T = synth.TINY.replace(intermediate=5120), 4, 140
     else:
-        s, B, T = synth.TINY.replace(qk_norm=True, rms_eps=1e-6), 3, 70
+        s, B, T = synth.TINY.replace(qk_norm=True, rms_eps=1e-6), 3, 300
     ms = T + 4
     tw = synth.make_weights(s, device="cuda")
     tokens = synth.make_tokens(s, T + 1, batch=B)

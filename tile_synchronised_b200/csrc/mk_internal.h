@@ -26,7 +26,7 @@ constexpr int kMaxAttnChunks = 16;  // split-KV chunks per (sequence, KV head); 
 // Tagged words per split-KV partial record: o[d], m, l.
 constexpr int partial_stride(int head_dim) { return head_dim + 2; }
 constexpr int kMaxGroup = 8;                            // query heads per KV head
-constexpr int kPrefillRows = 32;      // positions of one sequence per tensor-core prefill chunk (hi/lo: 64 MMA rows)
+constexpr int kPrefillRows = 128;     // positions of one sequence per tensor-core prefill chunk (hi/lo: 256 MMA columns)
 constexpr int kPrefillChunks = 16;    // most split-KV chunks per row in the prefill's causal attention
 constexpr uint16_t kNoCounter = 0xFFFF;
 

@@ -39,7 +39,7 @@ cudaError_t launch_linear_tc_packed(const void *x, const void *w, float *y, int 
 // (mk_linear_tc.cu): ws holds kSkWorkspaceFloats floats and flags
 // kSkWorkspaceFlags words, zero before the first launch (every launch leaves
 // them zero); falls back to the launch above otherwise.
-constexpr size_t kSkWorkspaceFloats = (size_t)256 * 64 * 128;
+constexpr size_t kSkWorkspaceFloats = (size_t)256 * 256 * 128;
 constexpr size_t kSkWorkspaceFlags = 256;
 cudaError_t launch_linear_tc_packed_sk(const void *x, const void *w, float *y, int B, int K, int M, int kc, int rows,
                                        float *ws, uint32_t *flags, cudaStream_t s, bool pdl);

@@ -37,7 +37,7 @@ constexpr int kLinM = 128;    // output rows per CTA (MMA M)
 constexpr int kLinBK = 64;    // K per stage: one 128-byte swizzle row of bf16
 constexpr int kLinThreads = 128;
 constexpr int kLinMaxSplit = 4;
-constexpr int kLinMaxB = 64;
+constexpr int kLinMaxB = 256;  // the MMA's N limit at M = 128
 constexpr int kLinMaxStages = 6;
 constexpr int kSkMaxCtas = 256;  // stream-K CTAs at most (the workspace is sized for this many)
 static_assert(kSkWorkspaceFloats >= (size_t)kSkMaxCtas * kLinMaxB * kLinM && kSkWorkspaceFlags >= kSkMaxCtas,
@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     const int nkb_all = sh.K / kLinBK;
     const int kb_first = (int)rank * nkb_all / (int)nrank;
     const int nkb = (int)(rank + 1) * nkb_all / (int)nrank - kb_first;
-    const uint32_t ncols = Bp <= 32 ? 32u : 64u;  // a power of two >= 32 that holds N columns
+    uint32_t ncols = 32;  // a power of two >= 32 that holds N columns
+    while (ncols < (uint32_t)Bp) ncols <<= 1;
 
     if (t == 0) {
         for (int s = 0; s < S; ++s) {
@@ -494,7 +495,8 @@ static bool sk_plan(int B, int K, int M, int sms, LinPlan &p, SkArgs &sk) {
     if (sk.G > kSkMaxCtas) sk.G = kSkMaxCtas;
     if (sk.G < 2) return false;
     const int per = (sk.U + sk.G - 1) / sk.G;  // the longest range
-    if ((per + sk.nkb - 1) / sk.nkb + 1 > kSkMaxSeg) return false;
+    const int segs = (per + sk.nkb - 1) / sk.nkb + 1;
+    if (segs > kSkMaxSeg || segs * p.sh.Bp > 512) return false;  // every segment's columns in tensor memory
     p.smem = p.sh.stages * (int)p.sh.stage_bytes + 1024 + 256;
     return true;
 }
@@ -568,7 +570,7 @@ extern "C" mk_status mk_linear_tc(const void *x, const void *w, float *y, int B,
         }
     LinPlan p;
     if (!lin_plan(B, K, M, p)) {
-        set_op_error("linear_tc: needs B <= 64 and K a multiple of 64");
+        set_op_error("linear_tc: needs B <= 256 and K a multiple of 64");
         return MK_ERR_UNSUPPORTED;
     }
     const cudaError_t e = launch_linear_tc(x, w, y, B, K, M, static_cast<cudaStream_t>(stream));
@@ -623,7 +625,7 @@ extern "C" mk_status mk_linear_tc_streamk(const void *x, const void *w, float *y
     }
     LinPlan p;
     if (!lin_plan(B, K, M, p)) {
-        set_op_error("linear_tc_streamk: needs B <= 64 and K a multiple of 64");
+        set_op_error("linear_tc_streamk: needs B <= 256 and K a multiple of 64");
         return MK_ERR_UNSUPPORTED;
     }
     float *ws = static_cast<float *>(workspace);

@@ -243,7 +243,7 @@ static cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
 }
-// The prefill of a megakernel context on the tensor cores: R <= 32
+// The prefill of a megakernel context on the tensor cores: R <= 128
 // consecutive positions t0 .. t0 + R - 1 of one sequence b go through the
 // decoder together, every projection one mk_linear_tc call over the
 // context's packed weights (which are plain row-major [rows, kc] matrices
@@ -355,12 +355,11 @@ __global__ void prefill_qkv_kernel(const float *y, int R, int M, int nq, int nkv
 __global__ void prefill_rows_kernel(int *row_seq, int *row_len, int R, int b, int t0, const State *state, int seq0,
                                     uint32_t *sk_flags) {
     row_pass_prologue();
-    const int r = threadIdx.x;
-    if (r < R) {
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
         row_seq[r] = b < 0 ? seq0 + r : b;
         row_len[r] = b < 0 ? state->pos + 1 : t0 + r + 1;
     }
-    for (int i = r; i < (int)kSkWorkspaceFlags; i += blockDim.x) sk_flags[i] = 0u;
+    for (int i = threadIdx.x; i < (int)kSkWorkspaceFlags; i += blockDim.x) sk_flags[i] = 0u;
 }
 
 // The argmax of each row's logits y[r] + y[n + r] (hi and lo outputs, ldy
@@ -636,7 +635,7 @@ std::string prefill_tc(const PrefillTc &a, const int32_t *tokens, int T, cudaStr
             const int n = std::min(R, T - t0);
             launch_pdl(prefill_embed_kernel, dim3(n), dim3(kRowThreads), 0, s, tokens, (int64_t)T, b, t0,
                        static_cast<const uint16_t *>(a.embed), sc.x, a.H, a.V, a.state, 0);
-            launch_pdl(prefill_rows_kernel, dim3(1), dim3(32), 0, s, sc.rows, sc.rows + R, n, b, t0,
+            launch_pdl(prefill_rows_kernel, dim3(1), dim3(128), 0, s, sc.rows, sc.rows + R, n, b, t0,
                        static_cast<const State *>(a.state), 0, sc.skflags);
             const int chunks = std::max(1, std::min(kPrefillChunks, (t0 + n) / 128));
             err = rows_through_layers(a, sc, n, chunks, false, s);
@@ -658,7 +657,7 @@ std::string decode_tc(const PrefillTc &a, const int32_t *tokens, int32_t *next, 
         const int n = std::min(R, a.B - b0);
         launch_pdl(prefill_embed_kernel, dim3(n), dim3(kRowThreads), 0, s, tokens + b0, (int64_t)0, -1, 0,
                    static_cast<const uint16_t *>(a.embed), sc.x, a.H, a.V, a.state, b0);
-        launch_pdl(prefill_rows_kernel, dim3(1), dim3(32), 0, s, sc.rows, sc.rows + R, n, -1, 0,
+        launch_pdl(prefill_rows_kernel, dim3(1), dim3(128), 0, s, sc.rows, sc.rows + R, n, -1, 0,
                    static_cast<const State *>(a.state), b0, sc.skflags);
         err = rows_through_layers(a, sc, n, chunks, true, s);  // ends with the final norm
         if (!err.empty()) break;
