@@ -214,6 +214,8 @@ def test_linear_tc_streamk_plan_and_argument_checks_need_no_device():
     assert mkpy.linear_tc_streamk_grid(1, 128, 128) == 0         # 2 units: too few to share
     assert mkpy.linear_tc_streamk_grid(16, 4096, 128256) == 0    # 1002 tiles: many waves already
     assert mkpy.linear_tc_streamk_grid(16, 4096, 18944) == 0     # 148 tiles: exactly one wave
+    assert mkpy.linear_tc_streamk_grid(256, 2048, 16384) == 0    # 256 columns, 128 tiles: plain
+    assert mkpy.linear_tc_streamk_grid(256, 2048, 2048) == 128   # 256 columns, 16 tiles: stream-K
     assert lib.mk_linear_tc_streamk(None, d, d, 16, 4096, 4096, d, need, None) == _lib.MK_ERR_INVALID
     assert lib.mk_linear_tc_streamk(d, d, d, 16, 4096, 4096, None, need, None) == _lib.MK_ERR_INVALID
     assert lib.mk_linear_tc_streamk(d, d, d, 16, 4096, 4096, C.c_void_p(264), need, None) == _lib.MK_ERR_INVALID

@@ -514,6 +514,10 @@ static int device_sms() {
 static int sk_grid(int B, int K, int M, int sms, LinPlan &p, SkArgs &sk) {
     if (!lin_plan(B, K, M, p)) return 0;
     if (p.tiles * p.split == sms || 2 * p.tiles >= 3 * sms) return 0;
+    // above 64 columns a contribution (128 rows x Bp fp32) costs more than an
+    // uneven wave unless the tiles fill at most half the SMs (at 256 columns
+    // the 128-tile gate/up of a 1B model took 34 us plain, 46 us stream-K)
+    if (p.sh.Bp > 64 && 2 * p.tiles * p.split > sms) return 0;
     return sk_plan(B, K, M, sms, p, sk) ? sk.G : 0;
 }
 
