@@ -649,9 +649,11 @@ std::string decode_tc(const PrefillTc &a, const int32_t *tokens, int32_t *next, 
     RowsScratch sc;
     if (!carve(a, sc)) return "scratch too small";
     // the attended length is read on the device; split the positions so that
-    // a long cache still spreads over the SMs, a fixed count so that the same
-    // launches serve every position
-    const int chunks = std::max(1, std::min(kPrefillChunks, a.max_seq / 256));
+    // a long cache still spreads over the SMs, a fixed count (the isolated
+    // attention's rule at max_seq) so that the same launches serve every
+    // position
+    const int chunks =
+        std::max(1, std::min(kPrefillChunks, mk_attention_chunks(std::min(a.B, R), a.nkv, a.max_seq)));
     std::string err;
     for (int b0 = 0; b0 < a.B && err.empty(); b0 += R) {
         const int n = std::min(R, a.B - b0);
