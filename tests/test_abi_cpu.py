@@ -275,3 +275,16 @@ def test_header_is_plain_c(tmp_path):
     r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), "-c",
                         str(src), "-o", str(tmp_path / "use_mk.o")], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_attention_chunk_rule_needs_no_device():
+    # without a device the rule assumes 148 SMs
+    ch = mkpy.attention_chunks
+    assert ch(1, 8, 1025) == 18       # about one CTA per SM over the 8 (sequence, KV head) pairs
+    assert ch(1, 8, 100) == 6         # at least 16 positions a chunk
+    assert ch(3, 4, 1) == 1
+    assert ch(16, 8, 1024) == 2       # 1024 positions: 2 chunks of 512 fill the slots best
+    assert ch(16, 8, 16384) == 9      # long cache: 1152 CTAs, 97 % of the last of 4 waves of 2 per SM
+    assert ch(4, 8, 32768) == 9       # 288 CTAs, one wave of 2 per SM
+    assert ch(1, 8, 32768) == 34      # the first count whose wave is 90 % full: 272 of 296 slots
+    assert ch(0, 8, 1024) == 0 and ch(1, 0, 1024) == 0 and ch(1, 8, 0) == 0
